@@ -1,0 +1,403 @@
+"""CPU oracle of the learned product-hash routed-attention forward.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's
+CPU-baseline leg may import this module.  It shares no code with the CUDA
+library and imports nothing from it.
+
+It is written to be read against the two pages that describe the method:
+
+  Report  = "Monodratic: a reproducible sparse attention mixer" (D. Todorov,
+            technical report summary), sections Mixer, Learned sparse route,
+            Capacity, Finite-range scaling, Evidence, Limits, Figures 1-4.
+  Article = "Monodratic Claims Learned Routing Can Make Sparse Causal Attention
+            More Selective" (remio.ai), section "Monodratic Turns Sparse
+            Attention Into a Retrieval Decision" unless stated.
+
+The forward is index -> route -> attend:
+  1. rotary embedding of queries and keys (Report, Mixer; Article);
+  2. per-block summaries of the rotated queries and keys;
+  3. a product address per source block from P codebooks (Article: "each
+     product address combines decisions from multiple learned code
+     components"; Report, Capacity: "spherical codebook");
+  4. bounded causal posting lists, overflow counted (Report, Mixer: "writes
+     keys into bounded causal posting lists"; Report, Capacity and Evidence:
+     overflow, maximum assigned load);
+  5. probe -> candidates in fixed slots -> rerank -> R remote blocks, plus L
+     local blocks added separately (Article; Report, Mixer; Report,
+     Finite-range scaling: "fixed candidate-slot checks");
+  6. ordinary causal softmax over the tokens of the selected blocks, no value
+     summary (Report, Mixer; Article).
+And the independent dense selected-mask form of step 6 (Report, Evidence:
+"Selected-mask oracle error"; Article, "Why Learned Product-Hash Routing
+Matters Now").
+
+Precision.  Every value is computed in float64 from the stored inputs.  Two
+readings fix what the pages leave open (both recorded with the others in the
+design notes):
+  * the rotary angle is the float32 product fp32(t) * fp32(base**(-2i/D)),
+    the way a float32 PyTorch rotary table is built; its cosine and sine are
+    then taken in float64;
+  * a routing decision (an argmax, a top-p, a top-R) is taken on the deciding
+    quantities rounded to float32, the precision the routing kernels decide
+    in.  Equal float32 scores go to the lower index.  ``margin`` outputs give
+    the float32 gap at each decision boundary so callers can tell a near tie.
+Attention outputs stay in float64.
+"""
+from __future__ import annotations
+
+import itertools
+from dataclasses import dataclass, field
+
+import numpy as np
+
+TIE_REL = 1e-6   # a decision whose float32 margin is below 1e-6*max(1,|s|) is a near tie
+
+
+def f32(x):
+    """Round to float32 and return as float64 (the values a float32 kernel holds)."""
+    return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------- 1. rotary
+def rope_inv_freq(D: int, base: float) -> np.ndarray:
+    """omega_i = base**(-2i/D), i < D/2, rounded to float32."""
+    i = np.arange(D // 2, dtype=np.float64)
+    return np.array([base ** (-2.0 * ii / D) for ii in i]).astype(np.float32)
+
+
+def rope_angles(S: int, D: int, base: float) -> np.ndarray:
+    """Angle of pair i at position t: the float32 product fp32(t) * omega_i. [S, D/2]"""
+    t = np.arange(S, dtype=np.float32)
+    return (t[:, None] * rope_inv_freq(D, base)[None, :]).astype(np.float32)
+
+
+def rope(x: np.ndarray, base: float) -> np.ndarray:
+    """Rotary embedding of x [B,S,H,D] at absolute positions 0..S-1.
+
+    Rotate-half pairing: coordinate i is paired with i + D/2 and the pair is
+    rotated by the angle of position t and frequency i.  Applied to queries and
+    keys, never to values (Report, Mixer: "After rotary position embedding").
+    """
+    B, S, H, D = x.shape
+    th = rope_angles(S, D, base).astype(np.float64)
+    c = np.cos(th)[None, :, None, :]
+    s = np.sin(th)[None, :, None, :]
+    x1 = x[..., : D // 2]
+    x2 = x[..., D // 2:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+# ------------------------------------------------------------- 2. summaries
+def block_means(xr: np.ndarray, bs: int) -> np.ndarray:
+    """Mean of the rotated vectors over each block of bs tokens.
+
+    [B,S,H,D] -> [B,H,nb,D].  Source blocks and query blocks are both
+    summarised this way (Article: "source blocks receive learned product
+    addresses"; the query of a block is its mean rotated query).
+    """
+    B, S, H, D = xr.shape
+    nb = S // bs
+    return xr.reshape(B, nb, bs, H, D).mean(axis=2).transpose(0, 2, 1, 3)
+
+
+# ------------------------------------------------------------------ 3. codes
+def codeword_scores(xbar: np.ndarray, codebooks: np.ndarray) -> np.ndarray:
+    """<xbar_s, C[s,k]> for every subspace s and codeword k, rounded to float32.
+
+    xbar [..., D] is split into P contiguous subvectors of D/P.  The summary is
+    not normalised: dividing by a positive norm does not change which codeword
+    wins.  -> [..., P, K]
+    """
+    P, K, d = codebooks.shape
+    sub = f32(xbar).reshape(*xbar.shape[:-1], P, d)
+    return f32(np.einsum("...pd,pkd->...pk", sub, codebooks.astype(np.float64)))
+
+
+def assign_codes(kbar: np.ndarray, codebooks: np.ndarray):
+    """Product address of each source block.
+
+    Per subspace the code is the codeword of largest score (lowest index on
+    equal scores); the address is sum_s code_s * K**(P-1-s), the first
+    subspace most significant.  Returns (addr [...], codes [..., P],
+    margin [..., P] = best - second best score).
+    """
+    P, K, _ = codebooks.shape
+    sc = codeword_scores(kbar, codebooks)
+    codes = np.argmax(sc, axis=-1)                   # first maximum -> lowest index
+    srt = -np.sort(-sc, axis=-1)
+    margin = srt[..., 0] - srt[..., 1] if K > 1 else np.full(sc.shape[:-1], np.inf)
+    weights = K ** np.arange(P - 1, -1, -1)
+    addr = (codes * weights).sum(axis=-1)
+    return addr.astype(np.int64), codes.astype(np.int64), margin
+
+
+def probe_codes(qbar: np.ndarray, codebooks: np.ndarray, p: int):
+    """The p best codewords per subspace for each query block.
+
+    Ordered by score, highest first, lower index first on equal scores.
+    Returns (codes [..., P, p], margin [..., P] = gap between ranks p and p+1).
+    """
+    P, K, _ = codebooks.shape
+    sc = codeword_scores(qbar, codebooks)
+    order = np.argsort(-sc, axis=-1, kind="stable")
+    codes = order[..., :p]
+    srt = np.take_along_axis(sc, order, axis=-1)
+    margin = srt[..., p - 1] - srt[..., p] if p < K else np.full(sc.shape[:-1], np.inf)
+    return codes.astype(np.int64), margin
+
+
+def probe_addresses(codes_row: np.ndarray, K: int) -> np.ndarray:
+    """Addresses probed by one query block: the product of its per-subspace
+    codeword choices, enumerated with the first subspace's rank slowest.
+    codes_row [P, p] -> [p**P]."""
+    P, p = codes_row.shape
+    weights = K ** np.arange(P - 1, -1, -1)
+    out = []
+    for ranks in itertools.product(range(p), repeat=P):
+        out.append(sum(int(codes_row[s, r]) * int(weights[s]) for s, r in enumerate(ranks)))
+    return np.array(out, dtype=np.int64)
+
+
+# ------------------------------------------------------------ 4. posting lists
+def build_lists(addr_row: np.ndarray, A: int, cap: int):
+    """Bounded causal posting lists of one (sequence, KV head).
+
+    Blocks are inserted in ascending block order; a block is stored if its
+    address's list holds fewer than cap blocks, otherwise it is an overflow
+    event.  Whether block i is stored depends only on blocks before it, so no
+    later block can change what an earlier query sees.  load counts every block
+    hashed to the address (the "assigned load", which may exceed capacity).
+    Returns lists [A, cap] (-1 padded, ascending), load [A], overflow, maxload.
+    """
+    lists = np.full((A, cap), -1, dtype=np.int64)
+    load = np.zeros(A, dtype=np.int64)
+    for i, a in enumerate(addr_row):
+        if load[a] < cap:
+            lists[a, load[a]] = i
+        load[a] += 1
+    overflow = int(np.maximum(load - cap, 0).sum())
+    return lists, load, overflow, int(load.max()) if A else 0
+
+
+# ------------------------------------------------------------------- 5. route
+@dataclass
+class RouteRow:
+    sel: np.ndarray          # [R+L]: remote ids ascending, -1 pads, then locals
+    slots: np.ndarray        # [p**P, cap] fixed candidate slots (-1 = empty)
+    cand: np.ndarray         # eligible candidate ids
+    scores: np.ndarray       # their float32 scores
+    margin: float            # score gap between rank R and R+1 (inf if none)
+
+
+def candidate_slots(lists: np.ndarray, probe_addrs: np.ndarray, j: int, L: int) -> np.ndarray:
+    """The fixed candidate slots of query block j: one row of cap slots per
+    probed address, holding the listed blocks that are remote-eligible
+    (i <= j - L); every other slot is -1.  Always p**P x cap."""
+    slots = lists[probe_addrs].copy()
+    slots[(slots < 0) | (slots > j - L)] = -1
+    return slots
+
+
+def route_row(qbar_j: np.ndarray, kbar_h: np.ndarray, probe_addrs: np.ndarray,
+              lists: np.ndarray, j: int, R: int, L: int) -> RouteRow:
+    """Route one query block: probe -> candidates -> rerank -> top R, plus the
+    L local blocks j-L+1..j (Article: "A query probes addresses, receives
+    candidates, reranks them, and selects a fixed number of remote blocks";
+    "The query also receives guaranteed local blocks").
+
+    Rerank score of candidate i is <qbar_j, kbar_i> over the full head
+    dimension, rounded to float32; top R by score, lower id on equal scores.
+    The chosen remote ids are stored in ascending order.
+    """
+    slots = candidate_slots(lists, probe_addrs, j, L)
+    cand = slots[slots >= 0]
+    scores = f32(f32(kbar_h[cand]) @ f32(qbar_j)) if cand.size else np.zeros(0)
+    order = np.lexsort((cand, -scores))
+    top = cand[order[:R]]
+    margin = np.inf
+    if cand.size > R and R > 0:
+        margin = float(scores[order[R - 1]] - scores[order[R]])
+    remote = np.full(R, -1, dtype=np.int64)
+    remote[: top.size] = np.sort(top)
+    local = np.arange(j - L + 1, j + 1, dtype=np.int64)
+    local[local < 0] = -1
+    return RouteRow(np.concatenate([remote, local]), slots, cand, scores, margin)
+
+
+# ------------------------------------------------------------------ 6. attend
+def selected_tokens(sel_row: np.ndarray, bs: int) -> np.ndarray:
+    blocks = np.sort(sel_row[sel_row >= 0])
+    return (blocks[:, None] * bs + np.arange(bs)[None, :]).ravel()
+
+
+def attend(qr, kr, v, sel, bs: int, scale: float, rows=None) -> np.ndarray:
+    """Exact causal softmax over the tokens of the selected blocks.
+
+    For token t of query block j, head hq: the keys are every token s of every
+    selected block with s <= t; weights softmax(scale * <q'_t, k'_s>) applied
+    to v_s (Report, Mixer: "Attention over that set is ordinary causal softmax.
+    No value summary replaces selected source values").  Query head hq reads KV
+    head hq // (Hq/Hkv).  rows: optional list of (b, hq, j) to compute; the
+    others stay NaN.  -> [B,S,Hq,D] float64.
+    """
+    B, S, Hq, D = qr.shape
+    g = Hq // kr.shape[2]
+    out = np.full((B, S, Hq, v.shape[3]), np.nan)
+    nb = S // bs
+    todo = rows if rows is not None else itertools.product(range(B), range(Hq), range(nb))
+    for b, hq, j in todo:
+        toks = selected_tokens(sel[b, hq, j], bs)
+        qpos = np.arange(j * bs, (j + 1) * bs)
+        Q = qr[b, qpos, hq]
+        Kt = kr[b, toks, hq // g]
+        Vt = v[b, toks, hq // g]
+        s = (Q @ Kt.T) * scale
+        s[toks[None, :] > qpos[:, None]] = -np.inf
+        s -= s.max(axis=1, keepdims=True)
+        w = np.exp(s)
+        out[b, qpos, hq] = (w @ Vt) / w.sum(axis=1, keepdims=True)
+    return out
+
+
+def selected_mask(sel_bh: np.ndarray, S: int, bs: int) -> np.ndarray:
+    """Dense boolean [S, S] mask of one (sequence, head): M[t, s] is true when
+    s's block is selected for t's block and s <= t."""
+    nb = S // bs
+    blk = np.zeros((nb, nb), dtype=bool)
+    for j in range(nb):
+        ids = sel_bh[j][sel_bh[j] >= 0]
+        blk[j, ids] = True
+    M = np.repeat(np.repeat(blk, bs, axis=0), bs, axis=1)
+    return M & np.tril(np.ones((S, S), dtype=bool))
+
+
+def attend_dense_mask(qr, kr, v, sel, bs: int, scale: float) -> np.ndarray:
+    """The same attention as a dense masked softmax over all S keys, built
+    independently of the gathered form (Report, Evidence: selected-mask
+    oracle)."""
+    B, S, Hq, D = qr.shape
+    g = Hq // kr.shape[2]
+    out = np.empty((B, S, Hq, v.shape[3]))
+    for b in range(B):
+        for hq in range(Hq):
+            M = selected_mask(sel[b, hq], S, bs)
+            s = (qr[b, :, hq] @ kr[b, :, hq // g].T) * scale
+            s = np.where(M, s, -np.inf)
+            s -= s.max(axis=1, keepdims=True)
+            w = np.exp(s)
+            out[b, :, hq] = (w @ v[b, :, hq // g]) / w.sum(axis=1, keepdims=True)
+    return out
+
+
+# ----------------------------------------------------------------- forward
+@dataclass
+class Params:
+    B: int
+    S: int
+    Hq: int
+    Hkv: int
+    D: int
+    block: int
+    P: int
+    K: int
+    cap: int
+    probes: int
+    R: int
+    L: int
+    rope_base: float = 10000.0
+    scale: float = 0.0
+
+    @property
+    def nb(self):
+        return self.S // self.block
+
+    @property
+    def A(self):
+        return self.K ** self.P
+
+    @property
+    def softmax_scale(self):
+        return self.scale if self.scale > 0 else 1.0 / np.sqrt(self.D)
+
+    @classmethod
+    def of(cls, w) -> "Params":
+        return cls(**{f: getattr(w, f) for f in cls.__dataclass_fields__})
+
+
+@dataclass
+class Result:
+    qr: np.ndarray
+    kr: np.ndarray
+    qbar: np.ndarray
+    kbar: np.ndarray
+    addr: np.ndarray
+    codes: np.ndarray
+    code_margin: np.ndarray
+    qcodes: np.ndarray
+    qcode_margin: np.ndarray
+    lists: np.ndarray
+    load: np.ndarray
+    overflow: np.ndarray
+    maxload: np.ndarray
+    sel: np.ndarray
+    sel_margin: np.ndarray
+    ncand: np.ndarray
+    out: np.ndarray | None = None
+    slots: dict = field(default_factory=dict)
+
+
+def build_index(kr, codebooks, p: Params):
+    """Index of every (sequence, KV head): summaries, addresses, lists."""
+    kbar = block_means(kr, p.block)
+    addr, codes, margin = assign_codes(kbar, codebooks)
+    B, H, nb = addr.shape
+    lists = np.empty((B, H, p.A, p.cap), dtype=np.int64)
+    load = np.empty((B, H, p.A), dtype=np.int64)
+    overflow = np.empty((B, H), dtype=np.int64)
+    maxload = np.empty((B, H), dtype=np.int64)
+    for b in range(B):
+        for h in range(H):
+            lists[b, h], load[b, h], overflow[b, h], maxload[b, h] = build_lists(addr[b, h], p.A, p.cap)
+    return kbar, addr, codes, margin, lists, load, overflow, maxload
+
+
+def route(qr, kbar, lists, codebooks, p: Params, keep_slots=False):
+    qbar = block_means(qr, p.block)
+    qcodes, qmargin = probe_codes(qbar, codebooks, p.probes)
+    B, Hq, nb = qbar.shape[:3]
+    g = Hq // kbar.shape[1]
+    sel = np.empty((B, Hq, nb, p.R + p.L), dtype=np.int64)
+    sel_margin = np.empty((B, Hq, nb))
+    ncand = np.empty((B, Hq, nb), dtype=np.int64)
+    slots = {}
+    for b in range(B):
+        for hq in range(Hq):
+            for j in range(nb):
+                pa = probe_addresses(qcodes[b, hq, j], p.K)
+                row = route_row(qbar[b, hq, j], kbar[b, hq // g], pa,
+                                lists[b, hq // g], j, p.R, p.L)
+                sel[b, hq, j] = row.sel
+                sel_margin[b, hq, j] = row.margin
+                ncand[b, hq, j] = row.cand.size
+                if keep_slots:
+                    slots[(b, hq, j)] = row.slots
+    return qbar, qcodes, qmargin, sel, sel_margin, ncand, slots
+
+
+def forward(q, k, v, codebooks, p: Params, *, attention=True, rows=None, keep_slots=False) -> Result:
+    """Index -> route -> attend for stored inputs q [B,S,Hq,D], k, v [B,S,Hkv,D]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    qr = rope(q, p.rope_base)
+    kr = rope(k, p.rope_base)
+    kbar, addr, codes, cmargin, lists, load, overflow, maxload = build_index(kr, codebooks, p)
+    qbar, qcodes, qmargin, sel, smargin, ncand, slots = route(qr, kbar, lists, codebooks, p, keep_slots)
+    out = attend(qr, kr, v, sel, p.block, p.softmax_scale, rows) if attention else None
+    return Result(qr, kr, qbar, kbar, addr, codes, cmargin, qcodes, qmargin, lists, load,
+                  overflow, maxload, sel, smargin, ncand, out, slots)
+
+
+def near_tie(margin, scale_ref) -> np.ndarray:
+    """True where a float32 decision margin is below 1e-6*max(1,|s|)."""
+    return np.asarray(margin) < TIE_REL * np.maximum(1.0, np.abs(scale_ref))
