@@ -1,0 +1,322 @@
+#!/usr/bin/env python
+"""Routed-attention forward throughput (index + route + attend) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+                    [--workload scaling32k]
+
+One step = one mdr_forward (rotary + summaries + codes, posting lists,
+probe/rerank/top-R, selected-set attention) over one sequence of the
+workload, inputs resident in HBM.  Each GPU (one process per GPU under
+torchrun) runs its own sequence: weak scaling, no collective on the data path.
+L2 is flushed (256 MiB write, outside the timed events) before every step.
+Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (oracle/mdr_oracle.py) as it stands on
+the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from workloads import SCALING_SWEEP, ALL, make_inputs  # noqa: E402
+
+METRIC = "routed-attention fwd tokens/s (index+route+attend) at 32K; % HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x20: "sync_boost", 0x40: "sw_thermal_slowdown", 0x80: "hw_thermal_slowdown",
+               0x100: "hw_power_brake_slowdown", 0x200: "display_clock"}
+
+
+def workload(name):
+    for w in list(ALL.values()) + SCALING_SWEEP:
+        if w.name == name:
+            return w
+    raise SystemExit(f"unknown workload {name}")
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons during the timed region."""
+
+    def __init__(self, dev):
+        self.dev, self.proc, self.path = dev, None, None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev),
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], [], set()
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+                bits = int(parts[3], 16)
+            except ValueError:
+                continue
+            for b, n in REASON_BITS.items():
+                if bits & b:
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons - {"gpu_idle"})}
+
+
+def oracle_group_seconds(w, inp, h):
+    """CPU oracle forward of one KV-head group: KV head h of sequence 0 and
+    its query heads, all query blocks.  Returns seconds."""
+    from oracle import mdr_oracle as O
+    g = w.Hq // w.Hkv
+    p = O.Params.of(w.with_(B=1, Hq=g, Hkv=1))
+    q = inp.q[:1, :, h * g:(h + 1) * g]
+    k, v = inp.k[:1, :, h:h + 1], inp.v[:1, :, h:h + 1]
+    t0 = time.perf_counter()
+    O.forward(q, k, v, inp.codebooks, p)
+    return time.perf_counter() - t0
+
+
+def oracle_sample(w, seed, max_seconds):
+    """Time whole KV-head groups until max_seconds; tokens/s of the full
+    workload (B sequences, all groups) at that speed."""
+    inp = make_inputs(w, seed)
+    secs = []
+    for h in range(w.Hkv):
+        secs.append(oracle_group_seconds(w, inp, h))
+        if sum(secs) >= max_seconds:
+            break
+    t_full = statistics.mean(secs) * w.Hkv * w.B
+    return w.B * w.S / t_full, sum(secs), len(secs)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    inp = make_inputs(w, 1000)
+    secs = []
+    for it in range(args.warmup + args.steps):
+        t = oracle_group_seconds(w, inp, it % w.Hkv)
+        if it >= args.warmup:
+            secs.append(t)
+    t_full = statistics.mean(secs) * w.Hkv * w.B
+    tps = w.B * w.S / t_full
+    g = w.Hq // w.Hkv
+    line = {"impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_full * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, args),
+            "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"each step: one KV-head group ({g} query heads, all {w.nb} query "
+                                       f"blocks) of one sequence; ms_per_step scaled by {w.Hkv * w.B} groups"},
+            "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, args):
+    return {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "block": w.block,
+            "P": w.P, "K": w.K, "cap": w.cap, "probes": w.probes, "R": w.R, "L": w.L, "keys": w.keys,
+            "l2": "flushed between steps (256 MiB write, outside the timed events)",
+            "parallelism": f"one sequence per GPU x {args.gpus}"}
+
+
+def run_mine(args, w):
+    import torch
+    from learned_product_hash_b200 import mdr
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = init_dist(world, "nccl")
+    dev = torch.device("cuda", local)
+    es = 2 if w.dtype == "bf16" else 4
+
+    inp = make_inputs(w, 1000 + rank)
+    conv = (lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16)) if w.dtype == "bf16" \
+        else torch.from_numpy
+    q_h, k_h, v_h = (conv(x) for x in (inp.q_store, inp.k_store, inp.v_store))
+    cb_h = torch.from_numpy(inp.codebooks)
+    q, k, v, cb = (t.to(dev) for t in (q_h, k_h, v_h, cb_h))
+    cfg = mdr.make_config(w)
+    idx = mdr.Index.empty(cfg, dev)
+    rt = mdr.RouteOut.empty(cfg, dev)
+    out = torch.empty_like(q)
+    ws = mdr.workspace(cfg, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(evs):
+        flush.zero_()
+        mdr.mdr_forward_profiled(cfg, q, k, v, cb, idx, rt, out, ws, evs)
+
+    for _ in range(args.warmup):
+        step([None] * 5)
+    torch.cuda.synchronize()
+    assert mdr.mdr_read_device_status(ws) == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for s in range(args.steps):
+            step(evs[s])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    assert mdr.mdr_read_device_status(ws) == 0
+    tot = [e[0].elapsed_time(e[4]) for e in evs]
+    ker = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+           for i, n in enumerate(("summarize", "lists", "route", "attend"))}
+    ms = statistics.mean(tot)
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    tokens = w.B * w.S * world
+    value = tokens / (ms_max / 1e3)
+
+    # Roofline of the attention kernel: q read + gathered K/V of valid
+    # selected blocks + out write, per (b, hq, j) route.
+    sel = rt.sel.cpu().numpy()
+    nsel = int((sel >= 0).sum())
+    routes = w.B * w.Hq * w.nb
+    attn_bytes = routes * 2 * w.block * w.D * es + nsel * w.block * 2 * w.D * es
+    peak, peak_kind = peaks()
+    achieved = attn_bytes / (ker["attend"] / 1e3) / 1e9
+    total_bytes = (w.Hq + w.Hkv) * w.S * w.D * es * w.B + attn_bytes
+
+    # End to end through the C ABI with host buffers.
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp = (x.pin_memory() for x in (q_h, k_h, v_h))
+        cbp = cb_h.pin_memory()
+        outp = torch.empty_like(qp).pin_memory()
+        selp = torch.empty(sel.shape, dtype=torch.int32).pin_memory()
+        ovp = torch.empty(w.B, w.Hkv, dtype=torch.int32).pin_memory()
+        mxp = torch.empty(w.B, w.Hkv, dtype=torch.int32).pin_memory()
+        dws = torch.empty(mdr.mdr_host_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+        nE = max(3, min(args.steps, 10))
+        times = []
+        for it in range(2 + nE):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            mdr.mdr_forward_host(cfg, qp, kp, vp, cbp, outp, selp, ovp, mxp, dws)
+            e1.record(stream)
+            e1.synchronize()
+            if it >= 2:
+                times.append(e0.elapsed_time(e1))
+        te = torch.tensor([statistics.mean(times)], device=dev, dtype=torch.float64)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        h2d = sum(x.numel() * x.element_size() for x in (qp, kp, vp, cbp))
+        d2h = sum(x.numel() * x.element_size() for x in (outp, selp, ovp, mxp))
+        e2e = {"value": tokens / (float(te.item()) / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": float(te.item())}
+        del dws
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        tps, secs, groups = oracle_sample(w, 1000, max_seconds=args.cpu_seconds)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{groups} of {w.Hkv} KV-head groups of one sequence (all {w.nb} query blocks), "
+                         f"{secs:.1f} s, scaled to the full forward"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+                "config": config_of(w, argparse.Namespace(gpus=world)),
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                             "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                             "kernel": "attend", "algorithmic_bytes_per_launch": attn_bytes},
+                "path_roofline_frac": total_bytes / (ms_max / 1e3) / 1e9 / peak,
+                "kernels_ms": ker, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": 4 * args.steps, "clocks": clk.summary(),
+                "overflow": int(idx.overflow.sum().item()), "selected_blocks": nsel}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--workload", default="scaling32k")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    w = workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_mine(args, w)
+
+
+if __name__ == "__main__":
+    main()

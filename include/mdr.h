@@ -1,0 +1,210 @@
+/*
+ * mdr.h -- C ABI of libmdr: learned product-hash routed attention (forward)
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The method (pages cited by title and section):
+ *   "Monodratic: a reproducible sparse attention mixer" (technical report
+ *   summary; "Report" below) and "Monodratic Claims Learned Routing Can Make
+ *   Sparse Causal Attention More Selective" ("Article" below).
+ *
+ *   After rotary position embedding, every source block of keys gets a
+ *   product address from P codebooks and is written into a bounded causal
+ *   posting list; every query block probes addresses, gathers the listed
+ *   earlier blocks as candidates, reranks them and keeps R remote blocks,
+ *   adds L local blocks, and runs ordinary causal softmax over the tokens of
+ *   the selected blocks (Report, "Mixer"; Article, "Monodratic Turns Sparse
+ *   Attention Into a Retrieval Decision").
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument named "device" points to GPU memory of the
+ *     current device; "host" pointers point to CPU memory (pinned memory
+ *     makes the copies asynchronous).  The caller owns every buffer; the
+ *     library allocates nothing and keeps no state between calls.
+ *   - Layouts are C-contiguous.  q is [B,S,Hq,D]; k and v are [B,S,Hkv,D];
+ *     out is [B,S,Hq,D]; all four have the element type cfg->dtype.
+ *     Query head hq reads KV head hq / (Hq/Hkv).
+ *   - codebooks are float32 [P,K,D/P]: P codebooks of K codewords, one per
+ *     contiguous subspace of D/P coordinates.  They are used as given (the
+ *     library does not renormalise them).
+ *   - "stream" is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Device work is enqueued on it and the call returns without
+ *     synchronising, except mdr_forward_host and mdr_read_device_status.
+ *   - Argument checks run on the host before anything is enqueued; a failed
+ *     check returns its status and enqueues nothing.  They touch no GPU, so
+ *     they also work on a machine without one.
+ *   - Kernels that wait on asynchronous copies or tensor-core work bound every
+ *     wait; a wait that runs out sets a nonzero code in the device status
+ *     word (the first 4 bytes of the workspace) and the kernel returns.  Read
+ *     it with mdr_read_device_status after the call.
+ */
+#ifndef MDR_H_
+#define MDR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MDR_ABI_VERSION 1
+
+typedef enum mdr_status {
+  MDR_OK = 0,
+  MDR_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, inconsistent shape */
+  MDR_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels implement */
+  MDR_ERR_WORKSPACE = 3,     /* workspace missing, too small or not 256-byte aligned */
+  MDR_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  MDR_ERR_DEVICE = 5         /* the device status word reports a failed check */
+} mdr_status;
+
+typedef enum mdr_dtype { MDR_F32 = 0, MDR_BF16 = 1 } mdr_dtype;
+
+/* Shapes and routing parameters of one call.
+ *   B, S, Hq, Hkv, D : batch, tokens, query heads, KV heads, head dimension.
+ *   block            : tokens per block (bs); S % block == 0, nb = S / block.
+ *   P, K             : P codebooks of K codewords; A = K^P addresses.
+ *   cap              : capacity of each posting list (blocks).
+ *   probes           : codewords probed per subspace (p); p^P addresses probed.
+ *   R, L             : remote blocks kept, local blocks added (L >= 1).
+ *   rope_base        : rotary base (10000 in the pages' tiny case).
+ *   scale            : softmax scale; 0 means 1/sqrt(D).
+ *   dtype            : mdr_dtype of q, k, v, out.
+ * Supported: D in {32,64,128}; block in {16,32,64,128}; 1 <= P <= 4 with
+ * D % P == 0 and (D/P) % 4 == 0; 1 <= K <= 128; A <= 16384; 1 <= cap <= 1024;
+ * 1 <= probes <= K with probes^P <= 64 and probes^P * cap <= 4096;
+ * 0 <= R <= 32; 1 <= L <= 32.  MDR_BF16 additionally needs block in {64,128}
+ * and D in {64,128} (the tensor-core attention tiles).                      */
+typedef struct mdr_config {
+  int32_t B, S, Hq, Hkv, D, block;
+  int32_t P, K, cap, probes, R, L;
+  float rope_base;
+  float scale;
+  int32_t dtype;
+} mdr_config;
+
+/* The index of every (sequence, KV head); all device pointers, all required.
+ *   kbar     float32 [B,Hkv,nb,D]  mean rotated key of each block.
+ *   addr     int32   [B,Hkv,nb]    product address of each block, in [0, A).
+ *   lists    int32   [B,Hkv,A,cap] posting lists: the first cap blocks (in
+ *                                  ascending block order) hashed to each
+ *                                  address, -1 padded.
+ *   load     int32   [B,Hkv,A]     blocks hashed to each address (uncapped:
+ *                                  the assigned load of Report, Capacity).
+ *   overflow int32   [B,Hkv]       blocks not stored: sum of max(0, load-cap).
+ *   maxload  int32   [B,Hkv]       largest load.                              */
+typedef struct mdr_index {
+  float* kbar;
+  int32_t* addr;
+  int32_t* lists;
+  int32_t* load;
+  int32_t* overflow;
+  int32_t* maxload;
+} mdr_index;
+
+/* Route outputs; device pointers.  sel is required, the others may be NULL.
+ *   sel    int32   [B,Hq,nb,R+L] selected blocks of each query block: the
+ *                                remote blocks in ascending order, -1 where
+ *                                fewer than R candidates exist, then the
+ *                                local blocks j-L+1..j (-1 where negative).
+ *   qbar   float32 [B,Hq,nb,D]   mean rotated query of each block.
+ *   qcodes int32   [B,Hq,nb,P,probes] probed codewords per subspace, best
+ *                                first.
+ *   ncand  int32   [B,Hq,nb]     eligible candidates found in the probed
+ *                                lists (at most probes^P * cap).            */
+typedef struct mdr_route_out {
+  int32_t* sel;
+  float* qbar;
+  int32_t* qcodes;
+  int32_t* ncand;
+} mdr_route_out;
+
+/* Library and ABI version; MDR_ABI_VERSION of the build. */
+int32_t mdr_abi_version(void);
+
+/* Static text for a status code. */
+const char* mdr_status_string(mdr_status s);
+
+/* Check a configuration (the rules listed at mdr_config). */
+mdr_status mdr_check_config(const mdr_config* cfg);
+
+/* Device workspace the device entry points need, in bytes (host only). */
+mdr_status mdr_workspace_bytes(const mdr_config* cfg, size_t* bytes);
+
+/* Index: rotate the keys, average each block, give each block a product
+ * address made of one codeword choice per subspace, and write the blocks
+ * into bounded causal posting lists, counting overflow (Article, "Monodratic
+ * Turns Sparse Attention Into a Retrieval Decision"; Report, sections Mixer
+ * and Capacity).  k: device [B,S,Hkv,D]; codebooks: device.                */
+mdr_status mdr_build_index(const mdr_config* cfg, const void* k,
+                           const float* codebooks, const mdr_index* idx,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Route: rotate the queries, average each block, probe the p best codewords
+ * per subspace, gather the listed blocks i <= j-L as candidates in fixed
+ * slots, rerank by <qbar_j, kbar_i> (float32), keep the R best (ties to the
+ * lower block id) and add the L local blocks (Article, "Monodratic Turns
+ * Sparse Attention Into a Retrieval Decision": probe, candidates, rerank, a
+ * fixed count of remote blocks, local blocks always added).
+ * q: device [B,S,Hq,D]; idx as filled by mdr_build_index (kbar, lists, load
+ * are read).                                                                 */
+mdr_status mdr_route(const mdr_config* cfg, const void* q,
+                     const float* codebooks, const mdr_index* idx,
+                     const mdr_route_out* rt, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* Attend: for token t of block j, causal softmax of scale*<q'_t, k'_s> over
+ * every token s <= t of the blocks in sel[j], applied to v_s; q', k' are the
+ * rotated queries and keys; exact softmax over the selected tokens, the
+ * values used as they are (Report, section Mixer).  sel: device int32 [B,Hq,nb,R+L]; any valid block id in
+ * [0, j] may appear, -1 entries are skipped, ids must not repeat within a
+ * row.  out: device [B,S,Hq,D].                                             */
+mdr_status mdr_attend(const mdr_config* cfg, const void* q, const void* k,
+                      const void* v, const int32_t* sel, void* out, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/* The whole forward, index -> route -> attend, with the rotation and the
+ * summaries of both sides computed once.                                    */
+mdr_status mdr_forward(const mdr_config* cfg, const void* q, const void* k,
+                       const void* v, const float* codebooks,
+                       const mdr_index* idx, const mdr_route_out* rt,
+                       void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* mdr_forward that also records CUDA events at the kernel boundaries, for
+ * timing each kernel on the stream it runs on.  events: host array of
+ * n_events cudaEvent_t (as void*), each NULL to skip; events[0] before the
+ * first kernel, events[1] after the summary kernel, events[2] after the
+ * list kernel, events[3] after the route kernel, events[4] after the
+ * attention kernel.  Same work and outputs as mdr_forward.                   */
+mdr_status mdr_forward_profiled(const mdr_config* cfg, const void* q,
+                                const void* k, const void* v,
+                                const float* codebooks, const mdr_index* idx,
+                                const mdr_route_out* rt, void* out, void* ws,
+                                size_t ws_bytes, void* stream,
+                                void* const* events, int32_t n_events);
+
+/* Device workspace mdr_forward_host needs, in bytes (host only).           */
+mdr_status mdr_host_workspace_bytes(const mdr_config* cfg, size_t* bytes);
+
+/* The forward from host buffers: copies q, k, v, codebooks to the device
+ * workspace, runs mdr_forward there, copies out, sel, overflow and maxload
+ * back, and synchronises the stream before returning.  q, k, v, codebooks,
+ * out: host; sel_host [B,Hq,nb,R+L], overflow_host and maxload_host [B,Hkv]:
+ * host int32 (each may be NULL to skip its copy).  dev_ws: device, at least
+ * mdr_host_workspace_bytes.                                                 */
+mdr_status mdr_forward_host(const mdr_config* cfg, const void* q_host,
+                            const void* k_host, const void* v_host,
+                            const float* codebooks_host, void* out_host,
+                            int32_t* sel_host, int32_t* overflow_host,
+                            int32_t* maxload_host, void* dev_ws,
+                            size_t dev_ws_bytes, void* stream);
+
+/* Synchronise the stream and copy the device status word (first 4 bytes of
+ * ws) to *code (0 = no device-side failure).  Returns MDR_ERR_DEVICE when the
+ * word is nonzero.                                                           */
+mdr_status mdr_read_device_status(const void* ws, int32_t* code, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MDR_H_ */

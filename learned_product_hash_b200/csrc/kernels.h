@@ -1,0 +1,63 @@
+// Internal launch interface of the libmdr kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mdr {
+
+// K1 + K2: rotate, summarise and code one or both sides.
+struct SummarizeArgs {
+  const void* x[2];        // side 0 = queries [B,S,Hq,D], side 1 = keys [B,S,Hkv,D]; null skips a side
+  void* xrot[2];           // rotated copies (same layout and type); null = not written
+  float* xbar[2];          // block means [B,H,nb,D] float32; null = not written
+  int H[2];                // Hq, Hkv
+  int32_t* qcodes;         // [B,Hq,nb,P,probes]; null = no query codes
+  int32_t* addr;           // [B,Hkv,nb]; null = no key addresses
+  const float* codebooks;  // [P,K,D/P]
+  int B, S, D, bs, nb, P, K, probes;
+  float inv_freq[64];      // omega_i, i < D/2
+};
+size_t summarize_smem_bytes(int bs, int D, int Hq, int Hkv);
+cudaError_t launch_summarize(const SummarizeArgs& a, bool bf16, cudaStream_t st);
+
+// K3: bounded causal posting lists of every (b, kv head).
+struct ListsArgs {
+  const int32_t* addr;     // [B,Hkv,nb]
+  int32_t* lists;          // [B,Hkv,A,cap]
+  int32_t* load;           // [B,Hkv,A]
+  int32_t* overflow;       // [B,Hkv]
+  int32_t* maxload;        // [B,Hkv]
+  int B, H, nb, A, cap;
+};
+cudaError_t launch_lists(const ListsArgs& a, cudaStream_t st);
+
+// K4: probe / rerank / top-R + locals, one warp per (b, hq, j).
+struct RouteArgs {
+  const float* qbar;       // [B,Hq,nb,D]
+  const int32_t* qcodes;   // [B,Hq,nb,P,probes]
+  const float* kbar;       // [B,Hkv,nb,D]
+  const int32_t* lists;    // [B,Hkv,A,cap]
+  const int32_t* load;     // [B,Hkv,A]
+  int32_t* sel;            // [B,Hq,nb,R+L]
+  int32_t* ncand;          // [B,Hq,nb] or null
+  int B, Hq, Hkv, nb, D, P, K, A, probes, cap, R, L;
+};
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
+
+// K5: selected-set causal attention over rotated q', k' and v.
+struct AttendArgs {
+  const void* q;           // rotated queries [B,S,Hq,D]
+  const void* k;           // rotated keys    [B,S,Hkv,D]
+  const void* v;           // values          [B,S,Hkv,D]
+  const int32_t* sel;      // [B,Hq,nb,R+L]
+  void* out;               // [B,S,Hq,D]
+  int32_t* status;         // device status word
+  int B, S, Hq, Hkv, D, bs, nb, nsel;
+  float scale;
+};
+cudaError_t launch_attend_simt(const AttendArgs& a, bool bf16, cudaStream_t st);
+cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t st);
+
+}  // namespace mdr

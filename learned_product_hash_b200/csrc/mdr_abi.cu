@@ -1,0 +1,360 @@
+// C ABI of libmdr: argument checks, workspace carving and kernel launches.
+// Declarations and the contract of every entry point are in include/mdr.h.
+
+#include <cmath>
+#include <cstring>
+
+#include "../../include/mdr.h"
+#include "kernels.h"
+
+namespace {
+
+using mdr::SummarizeArgs;
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+size_t esize(const mdr_config* c) { return c->dtype == MDR_BF16 ? 2 : 4; }
+
+int ipow(int b, int e) {
+  long long r = 1;
+  for (int i = 0; i < e; ++i) {
+    r *= b;
+    if (r > (1LL << 30)) return -1;
+  }
+  return static_cast<int>(r);
+}
+
+bool is_pow2_in(int x, std::initializer_list<int> allowed) {
+  for (int a : allowed)
+    if (x == a) return true;
+  return false;
+}
+
+mdr_status check(const mdr_config* c) {
+  if (!c) return MDR_ERR_INVALID_ARG;
+  if (c->B < 1 || c->S < 1 || c->Hq < 1 || c->Hkv < 1 || c->D < 1 || c->block < 1 || c->P < 1 ||
+      c->K < 1 || c->cap < 1 || c->probes < 1 || c->R < 0 || c->L < 1)
+    return MDR_ERR_INVALID_ARG;
+  if (c->S % c->block != 0 || c->Hq % c->Hkv != 0 || c->D % c->P != 0 || c->probes > c->K)
+    return MDR_ERR_INVALID_ARG;
+  if (!(c->rope_base > 1.0f) || !(c->scale >= 0.0f) || !std::isfinite(c->rope_base) ||
+      !std::isfinite(c->scale))
+    return MDR_ERR_INVALID_ARG;
+  if (c->dtype != MDR_F32 && c->dtype != MDR_BF16) return MDR_ERR_INVALID_ARG;
+  if (!is_pow2_in(c->D, {32, 64, 128}) || !is_pow2_in(c->block, {16, 32, 64, 128}))
+    return MDR_ERR_UNSUPPORTED;
+  if (c->P > 4 || (c->D / c->P) % 4 != 0 || c->K > 128 || c->cap > 1024 || c->R > 32 || c->L > 32)
+    return MDR_ERR_UNSUPPORTED;
+  const int A = ipow(c->K, c->P);
+  if (A < 0 || A > 16384) return MDR_ERR_UNSUPPORTED;
+  const int np = ipow(c->probes, c->P);
+  if (np < 0 || np > 64 || np * c->cap > 4096) return MDR_ERR_UNSUPPORTED;
+  if (c->dtype == MDR_BF16 && (!is_pow2_in(c->block, {64, 128}) || !is_pow2_in(c->D, {64, 128})))
+    return MDR_ERR_UNSUPPORTED;
+  const long long tokens = static_cast<long long>(c->B) * c->S;
+  if (tokens * (c->Hq + c->Hkv) * c->D > (1LL << 40)) return MDR_ERR_UNSUPPORTED;
+  return MDR_OK;
+}
+
+struct Layout {
+  size_t status, qrot, krot, qbar, qcodes, total;
+};
+
+Layout layout_of(const mdr_config* c) {
+  const size_t nb = c->S / c->block;
+  const size_t tok = static_cast<size_t>(c->B) * c->S;
+  Layout l{};
+  size_t o = 0;
+  l.status = o; o += align_up(16);
+  l.qrot = o;   o += align_up(tok * c->Hq * c->D * esize(c));
+  l.krot = o;   o += align_up(tok * c->Hkv * c->D * esize(c));
+  l.qbar = o;   o += align_up(static_cast<size_t>(c->B) * c->Hq * nb * c->D * sizeof(float));
+  l.qcodes = o; o += align_up(static_cast<size_t>(c->B) * c->Hq * nb * c->P * c->probes * sizeof(int32_t));
+  l.total = o;
+  return l;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+
+mdr_status check_ws(const mdr_config* c, void* ws, size_t ws_bytes) {
+  if (!ws) return MDR_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign != 0) return MDR_ERR_WORKSPACE;
+  if (ws_bytes < layout_of(c).total) return MDR_ERR_WORKSPACE;
+  return MDR_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+mdr_status check_index(const mdr_index* idx) {
+  if (!idx || !idx->kbar || !idx->addr || !idx->lists || !idx->load || !idx->overflow || !idx->maxload)
+    return MDR_ERR_INVALID_ARG;
+  return MDR_OK;
+}
+
+void fill_common(SummarizeArgs& a, const mdr_config* c, const float* codebooks) {
+  std::memset(&a, 0, sizeof(a));
+  a.H[0] = c->Hq;
+  a.H[1] = c->Hkv;
+  a.codebooks = codebooks;
+  a.B = c->B; a.S = c->S; a.D = c->D; a.bs = c->block; a.nb = c->S / c->block;
+  a.P = c->P; a.K = c->K; a.probes = c->probes;
+  // omega_i = base^(-2i/D) in double, rounded to float.
+  for (int i = 0; i < c->D / 2; ++i)
+    a.inv_freq[i] = static_cast<float>(std::pow(static_cast<double>(c->rope_base), -2.0 * i / c->D));
+}
+
+mdr_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MDR_OK : MDR_ERR_CUDA; }
+
+#define MDR_TRY(x)                       \
+  do {                                   \
+    mdr_status s_ = (x);                 \
+    if (s_ != MDR_OK) return s_;         \
+  } while (0)
+
+#define MDR_CUDA(x) MDR_TRY(cuda_status(x))
+
+mdr_status run_lists(const mdr_config* c, const mdr_index* idx, cudaStream_t st) {
+  mdr::ListsArgs la{};
+  la.addr = idx->addr; la.lists = idx->lists; la.load = idx->load;
+  la.overflow = idx->overflow; la.maxload = idx->maxload;
+  la.B = c->B; la.H = c->Hkv; la.nb = c->S / c->block; la.A = ipow(c->K, c->P); la.cap = c->cap;
+  return cuda_status(mdr::launch_lists(la, st));
+}
+
+mdr_status run_route(const mdr_config* c, const float* qbar, const int32_t* qcodes,
+                     const mdr_index* idx, int32_t* sel, int32_t* ncand, cudaStream_t st) {
+  mdr::RouteArgs ra{};
+  ra.qbar = qbar; ra.qcodes = qcodes; ra.kbar = idx->kbar; ra.lists = idx->lists; ra.load = idx->load;
+  ra.sel = sel; ra.ncand = ncand;
+  ra.B = c->B; ra.Hq = c->Hq; ra.Hkv = c->Hkv; ra.nb = c->S / c->block; ra.D = c->D;
+  ra.P = c->P; ra.K = c->K; ra.A = ipow(c->K, c->P); ra.probes = c->probes; ra.cap = c->cap;
+  ra.R = c->R; ra.L = c->L;
+  return cuda_status(mdr::launch_route(ra, st));
+}
+
+mdr_status run_attend(const mdr_config* c, const void* qrot, const void* krot, const void* v,
+                      const int32_t* sel, void* out, int32_t* status, cudaStream_t st) {
+  mdr::AttendArgs aa{};
+  aa.q = qrot; aa.k = krot; aa.v = v; aa.sel = sel; aa.out = out; aa.status = status;
+  aa.B = c->B; aa.S = c->S; aa.Hq = c->Hq; aa.Hkv = c->Hkv; aa.D = c->D; aa.bs = c->block;
+  aa.nb = c->S / c->block; aa.nsel = c->R + c->L;
+  aa.scale = c->scale > 0.f ? c->scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(c->D)));
+  return cuda_status(mdr::launch_attend_simt(aa, c->dtype == MDR_BF16, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t mdr_abi_version(void) { return MDR_ABI_VERSION; }
+
+const char* mdr_status_string(mdr_status s) {
+  switch (s) {
+    case MDR_OK: return "ok";
+    case MDR_ERR_INVALID_ARG: return "invalid argument";
+    case MDR_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MDR_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case MDR_ERR_CUDA: return "CUDA error";
+    case MDR_ERR_DEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+mdr_status mdr_check_config(const mdr_config* cfg) { return check(cfg); }
+
+mdr_status mdr_workspace_bytes(const mdr_config* cfg, size_t* bytes) {
+  MDR_TRY(check(cfg));
+  if (!bytes) return MDR_ERR_INVALID_ARG;
+  *bytes = layout_of(cfg).total;
+  return MDR_OK;
+}
+
+mdr_status mdr_build_index(const mdr_config* cfg, const void* k, const float* codebooks,
+                           const mdr_index* idx, void* ws, size_t ws_bytes, void* stream) {
+  MDR_TRY(check(cfg));
+  if (!k || !codebooks || !aligned16(k)) return MDR_ERR_INVALID_ARG;
+  MDR_TRY(check_index(idx));
+  MDR_TRY(check_ws(cfg, ws, ws_bytes));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout l = layout_of(cfg);
+  MDR_CUDA(cudaMemsetAsync(at<int32_t>(ws, l.status), 0, sizeof(int32_t), st));
+  SummarizeArgs a;
+  fill_common(a, cfg, codebooks);
+  a.x[1] = k; a.xbar[1] = idx->kbar; a.addr = idx->addr;
+  MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
+  return run_lists(cfg, idx, st);
+}
+
+mdr_status mdr_route(const mdr_config* cfg, const void* q, const float* codebooks,
+                     const mdr_index* idx, const mdr_route_out* rt, void* ws, size_t ws_bytes,
+                     void* stream) {
+  MDR_TRY(check(cfg));
+  if (!q || !codebooks || !rt || !rt->sel || !aligned16(q)) return MDR_ERR_INVALID_ARG;
+  MDR_TRY(check_index(idx));
+  MDR_TRY(check_ws(cfg, ws, ws_bytes));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout l = layout_of(cfg);
+  float* qbar = rt->qbar ? rt->qbar : at<float>(ws, l.qbar);
+  int32_t* qcodes = rt->qcodes ? rt->qcodes : at<int32_t>(ws, l.qcodes);
+  MDR_CUDA(cudaMemsetAsync(at<int32_t>(ws, l.status), 0, sizeof(int32_t), st));
+  SummarizeArgs a;
+  fill_common(a, cfg, codebooks);
+  a.x[0] = q; a.xbar[0] = qbar; a.qcodes = qcodes;
+  MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
+  return run_route(cfg, qbar, qcodes, idx, rt->sel, rt->ncand, st);
+}
+
+mdr_status mdr_attend(const mdr_config* cfg, const void* q, const void* k, const void* v,
+                      const int32_t* sel, void* out, void* ws, size_t ws_bytes, void* stream) {
+  MDR_TRY(check(cfg));
+  if (!q || !k || !v || !sel || !out) return MDR_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MDR_ERR_INVALID_ARG;
+  MDR_TRY(check_ws(cfg, ws, ws_bytes));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout l = layout_of(cfg);
+  int32_t* status = at<int32_t>(ws, l.status);
+  MDR_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+  SummarizeArgs a;
+  fill_common(a, cfg, nullptr);
+  a.x[0] = q; a.x[1] = k;
+  a.xrot[0] = at<void>(ws, l.qrot); a.xrot[1] = at<void>(ws, l.krot);
+  MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
+  return run_attend(cfg, at<void>(ws, l.qrot), at<void>(ws, l.krot), v, sel, out, status, st);
+}
+
+static mdr_status forward_impl(const mdr_config* cfg, const void* q, const void* k, const void* v,
+                               const float* codebooks, const mdr_index* idx, const mdr_route_out* rt,
+                               void* out, void* ws, size_t ws_bytes, void* stream,
+                               void* const* events, int32_t n_events) {
+  MDR_TRY(check(cfg));
+  if (!q || !k || !v || !codebooks || !out || !rt || !rt->sel) return MDR_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MDR_ERR_INVALID_ARG;
+  if (n_events < 0 || (n_events > 0 && !events)) return MDR_ERR_INVALID_ARG;
+  MDR_TRY(check_index(idx));
+  MDR_TRY(check_ws(cfg, ws, ws_bytes));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) -> mdr_status {
+    if (i < n_events && events[i])
+      return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st));
+    return MDR_OK;
+  };
+  const Layout l = layout_of(cfg);
+  int32_t* status = at<int32_t>(ws, l.status);
+  float* qbar = rt->qbar ? rt->qbar : at<float>(ws, l.qbar);
+  int32_t* qcodes = rt->qcodes ? rt->qcodes : at<int32_t>(ws, l.qcodes);
+  MDR_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+  SummarizeArgs a;
+  fill_common(a, cfg, codebooks);
+  a.x[0] = q; a.x[1] = k;
+  a.xrot[0] = at<void>(ws, l.qrot); a.xrot[1] = at<void>(ws, l.krot);
+  a.xbar[0] = qbar; a.xbar[1] = idx->kbar;
+  a.qcodes = qcodes; a.addr = idx->addr;
+  MDR_TRY(mark(0));
+  MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
+  MDR_TRY(mark(1));
+  MDR_TRY(run_lists(cfg, idx, st));
+  MDR_TRY(mark(2));
+  MDR_TRY(run_route(cfg, qbar, qcodes, idx, rt->sel, rt->ncand, st));
+  MDR_TRY(mark(3));
+  MDR_TRY(run_attend(cfg, at<void>(ws, l.qrot), at<void>(ws, l.krot), v, rt->sel, out, status, st));
+  return mark(4);
+}
+
+mdr_status mdr_forward(const mdr_config* cfg, const void* q, const void* k, const void* v,
+                       const float* codebooks, const mdr_index* idx, const mdr_route_out* rt,
+                       void* out, void* ws, size_t ws_bytes, void* stream) {
+  return forward_impl(cfg, q, k, v, codebooks, idx, rt, out, ws, ws_bytes, stream, nullptr, 0);
+}
+
+mdr_status mdr_forward_profiled(const mdr_config* cfg, const void* q, const void* k, const void* v,
+                                const float* codebooks, const mdr_index* idx, const mdr_route_out* rt,
+                                void* out, void* ws, size_t ws_bytes, void* stream,
+                                void* const* events, int32_t n_events) {
+  return forward_impl(cfg, q, k, v, codebooks, idx, rt, out, ws, ws_bytes, stream, events, n_events);
+}
+
+namespace {
+struct HostLayout {
+  size_t dev, q, k, v, cb, out, sel, kbar, addr, lists, load, ovf, maxl, total;
+};
+HostLayout host_layout_of(const mdr_config* c) {
+  HostLayout h{};
+  const size_t nb = c->S / c->block, tok = static_cast<size_t>(c->B) * c->S;
+  const size_t A = static_cast<size_t>(ipow(c->K, c->P));
+  size_t o = 0;
+  h.dev = o;   o += align_up(layout_of(c).total);
+  h.q = o;     o += align_up(tok * c->Hq * c->D * esize(c));
+  h.k = o;     o += align_up(tok * c->Hkv * c->D * esize(c));
+  h.v = o;     o += align_up(tok * c->Hkv * c->D * esize(c));
+  h.cb = o;    o += align_up(static_cast<size_t>(c->K) * c->D * sizeof(float));
+  h.out = o;   o += align_up(tok * c->Hq * c->D * esize(c));
+  h.sel = o;   o += align_up(static_cast<size_t>(c->B) * c->Hq * nb * (c->R + c->L) * sizeof(int32_t));
+  h.kbar = o;  o += align_up(static_cast<size_t>(c->B) * c->Hkv * nb * c->D * sizeof(float));
+  h.addr = o;  o += align_up(static_cast<size_t>(c->B) * c->Hkv * nb * sizeof(int32_t));
+  h.lists = o; o += align_up(static_cast<size_t>(c->B) * c->Hkv * A * c->cap * sizeof(int32_t));
+  h.load = o;  o += align_up(static_cast<size_t>(c->B) * c->Hkv * A * sizeof(int32_t));
+  h.ovf = o;   o += align_up(static_cast<size_t>(c->B) * c->Hkv * sizeof(int32_t));
+  h.maxl = o;  o += align_up(static_cast<size_t>(c->B) * c->Hkv * sizeof(int32_t));
+  h.total = o;
+  return h;
+}
+}  // namespace
+
+mdr_status mdr_host_workspace_bytes(const mdr_config* cfg, size_t* bytes) {
+  MDR_TRY(check(cfg));
+  if (!bytes) return MDR_ERR_INVALID_ARG;
+  *bytes = host_layout_of(cfg).total;
+  return MDR_OK;
+}
+
+mdr_status mdr_forward_host(const mdr_config* cfg, const void* q_host, const void* k_host,
+                            const void* v_host, const float* codebooks_host, void* out_host,
+                            int32_t* sel_host, int32_t* overflow_host, int32_t* maxload_host,
+                            void* dev_ws, size_t dev_ws_bytes, void* stream) {
+  MDR_TRY(check(cfg));
+  if (!q_host || !k_host || !v_host || !codebooks_host || !out_host) return MDR_ERR_INVALID_ARG;
+  const HostLayout h = host_layout_of(cfg);
+  if (!dev_ws || reinterpret_cast<uintptr_t>(dev_ws) % kAlign != 0 || dev_ws_bytes < h.total)
+    return MDR_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t nb = cfg->S / cfg->block, tok = static_cast<size_t>(cfg->B) * cfg->S;
+  const size_t qb = tok * cfg->Hq * cfg->D * esize(cfg), kb = tok * cfg->Hkv * cfg->D * esize(cfg);
+  MDR_CUDA(cudaMemcpyAsync(at<void>(dev_ws, h.q), q_host, qb, cudaMemcpyHostToDevice, st));
+  MDR_CUDA(cudaMemcpyAsync(at<void>(dev_ws, h.k), k_host, kb, cudaMemcpyHostToDevice, st));
+  MDR_CUDA(cudaMemcpyAsync(at<void>(dev_ws, h.v), v_host, kb, cudaMemcpyHostToDevice, st));
+  MDR_CUDA(cudaMemcpyAsync(at<void>(dev_ws, h.cb), codebooks_host,
+                           static_cast<size_t>(cfg->K) * cfg->D * sizeof(float), cudaMemcpyHostToDevice, st));
+  mdr_index idx{at<float>(dev_ws, h.kbar), at<int32_t>(dev_ws, h.addr), at<int32_t>(dev_ws, h.lists),
+                at<int32_t>(dev_ws, h.load), at<int32_t>(dev_ws, h.ovf), at<int32_t>(dev_ws, h.maxl)};
+  mdr_route_out rt{at<int32_t>(dev_ws, h.sel), nullptr, nullptr, nullptr};
+  MDR_TRY(mdr_forward(cfg, at<void>(dev_ws, h.q), at<void>(dev_ws, h.k), at<void>(dev_ws, h.v),
+                      at<float>(dev_ws, h.cb), &idx, &rt, at<void>(dev_ws, h.out),
+                      at<void>(dev_ws, h.dev), layout_of(cfg).total, stream));
+  MDR_CUDA(cudaMemcpyAsync(out_host, at<void>(dev_ws, h.out), qb, cudaMemcpyDeviceToHost, st));
+  if (sel_host)
+    MDR_CUDA(cudaMemcpyAsync(sel_host, rt.sel, static_cast<size_t>(cfg->B) * cfg->Hq * nb * (cfg->R + cfg->L) * sizeof(int32_t),
+                             cudaMemcpyDeviceToHost, st));
+  if (overflow_host)
+    MDR_CUDA(cudaMemcpyAsync(overflow_host, idx.overflow, static_cast<size_t>(cfg->B) * cfg->Hkv * sizeof(int32_t),
+                             cudaMemcpyDeviceToHost, st));
+  if (maxload_host)
+    MDR_CUDA(cudaMemcpyAsync(maxload_host, idx.maxload, static_cast<size_t>(cfg->B) * cfg->Hkv * sizeof(int32_t),
+                             cudaMemcpyDeviceToHost, st));
+  MDR_CUDA(cudaStreamSynchronize(st));
+  int32_t code = 0;
+  MDR_CUDA(cudaMemcpy(&code, at<int32_t>(dev_ws, h.dev), sizeof(int32_t), cudaMemcpyDeviceToHost));
+  return code == 0 ? MDR_OK : MDR_ERR_DEVICE;
+}
+
+mdr_status mdr_read_device_status(const void* ws, int32_t* code, void* stream) {
+  if (!ws || !code) return MDR_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MDR_CUDA(cudaStreamSynchronize(st));
+  MDR_CUDA(cudaMemcpy(code, ws, sizeof(int32_t), cudaMemcpyDeviceToHost));
+  return *code == 0 ? MDR_OK : MDR_ERR_DEVICE;
+}
+
+}  // extern "C"

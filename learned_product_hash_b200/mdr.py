@@ -1,0 +1,231 @@
+"""Thin ctypes binding of libmdr (include/mdr.h), same names as the C ABI.
+
+Argument marshalling only: every step of the forward runs in the CUDA kernels
+behind the C ABI.  PyTorch provides device memory and the current stream.
+The shared library must be built (``python -m learned_product_hash_b200.build``
+or ``__graft_entry__.build()``); without it every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmdr.so")
+
+MDR_OK, MDR_ERR_INVALID_ARG, MDR_ERR_UNSUPPORTED, MDR_ERR_WORKSPACE, MDR_ERR_CUDA, MDR_ERR_DEVICE = range(6)
+MDR_F32, MDR_BF16 = 0, 1
+
+EXPORTED = (
+    "mdr_abi_version", "mdr_status_string", "mdr_check_config", "mdr_workspace_bytes",
+    "mdr_build_index", "mdr_route", "mdr_attend", "mdr_forward", "mdr_host_workspace_bytes",
+    "mdr_forward_host", "mdr_read_device_status", "mdr_forward_profiled",
+)
+
+
+class MdrError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+class mdr_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "S", "Hq", "Hkv", "D", "block", "P", "K", "cap", "probes", "R", "L")] + \
+               [("rope_base", ctypes.c_float), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32)]
+
+
+class mdr_index(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("kbar", "addr", "lists", "load", "overflow", "maxload")]
+
+
+class mdr_route_out(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("sel", "qbar", "qcodes", "ncand")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmdr.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libmdr.so is not built ({LIB_PATH}); run "
+                              "`python -m learned_product_hash_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        cfgp = ctypes.POINTER(mdr_config)
+        idxp = ctypes.POINTER(mdr_index)
+        rtp = ctypes.POINTER(mdr_route_out)
+        sig = {
+            "mdr_abi_version": ([], ctypes.c_int32),
+            "mdr_status_string": ([i32], ctypes.c_char_p),
+            "mdr_check_config": ([cfgp], i32),
+            "mdr_workspace_bytes": ([cfgp, ctypes.POINTER(sz)], i32),
+            "mdr_build_index": ([cfgp, vp, vp, idxp, vp, sz, vp], i32),
+            "mdr_route": ([cfgp, vp, vp, idxp, rtp, vp, sz, vp], i32),
+            "mdr_attend": ([cfgp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "mdr_forward": ([cfgp, vp, vp, vp, vp, idxp, rtp, vp, vp, sz, vp], i32),
+            "mdr_host_workspace_bytes": ([cfgp, ctypes.POINTER(sz)], i32),
+            "mdr_forward_host": ([cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "mdr_read_device_status": ([vp, ctypes.POINTER(ctypes.c_int32), vp], i32),
+            "mdr_forward_profiled": ([cfgp, vp, vp, vp, vp, idxp, rtp, vp, vp, sz, vp,
+                                      ctypes.POINTER(vp), ctypes.c_int32], i32),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes, f.restype = args, res
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().mdr_status_string(int(s)).decode()
+
+
+def _ok(status: int, what: str):
+    if status != MDR_OK:
+        raise MdrError(status, what)
+
+
+def make_config(w) -> mdr_config:
+    """mdr_config from any object with the workload fields (B, S, Hq, ...)."""
+    dt = {"bf16": MDR_BF16, "f32": MDR_F32}[w.dtype] if isinstance(w.dtype, str) else int(w.dtype)
+    return mdr_config(w.B, w.S, w.Hq, w.Hkv, w.D, w.block, w.P, w.K, w.cap, w.probes, w.R, w.L,
+                      float(w.rope_base), float(w.scale), dt)
+
+
+def mdr_abi_version() -> int:
+    return lib().mdr_abi_version()
+
+
+def mdr_check_config(cfg: mdr_config) -> int:
+    return lib().mdr_check_config(ctypes.byref(cfg))
+
+
+def mdr_workspace_bytes(cfg: mdr_config) -> int:
+    n = ctypes.c_size_t(0)
+    _ok(lib().mdr_workspace_bytes(ctypes.byref(cfg), ctypes.byref(n)), "mdr_workspace_bytes")
+    return n.value
+
+
+def mdr_host_workspace_bytes(cfg: mdr_config) -> int:
+    n = ctypes.c_size_t(0)
+    _ok(lib().mdr_host_workspace_bytes(ctypes.byref(cfg), ctypes.byref(n)), "mdr_host_workspace_bytes")
+    return n.value
+
+
+# ------------------------------------------------------------ torch helpers
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+@dataclass
+class Index:
+    """Device buffers of mdr_index (torch tensors)."""
+    kbar: object
+    addr: object
+    lists: object
+    load: object
+    overflow: object
+    maxload: object
+
+    @classmethod
+    def empty(cls, cfg: mdr_config, device="cuda") -> "Index":
+        import torch
+        nb, A = cfg.S // cfg.block, cfg.K ** cfg.P
+        i32 = dict(dtype=torch.int32, device=device)
+        return cls(torch.empty(cfg.B, cfg.Hkv, nb, cfg.D, dtype=torch.float32, device=device),
+                   torch.empty(cfg.B, cfg.Hkv, nb, **i32),
+                   torch.empty(cfg.B, cfg.Hkv, A, cfg.cap, **i32),
+                   torch.empty(cfg.B, cfg.Hkv, A, **i32),
+                   torch.empty(cfg.B, cfg.Hkv, **i32),
+                   torch.empty(cfg.B, cfg.Hkv, **i32))
+
+    def c(self) -> mdr_index:
+        return mdr_index(*(_ptr(getattr(self, f)) for f in ("kbar", "addr", "lists", "load", "overflow", "maxload")))
+
+
+@dataclass
+class RouteOut:
+    sel: object
+    qbar: object = None
+    qcodes: object = None
+    ncand: object = None
+
+    @classmethod
+    def empty(cls, cfg: mdr_config, device="cuda", debug=False) -> "RouteOut":
+        import torch
+        nb = cfg.S // cfg.block
+        i32 = dict(dtype=torch.int32, device=device)
+        sel = torch.empty(cfg.B, cfg.Hq, nb, cfg.R + cfg.L, **i32)
+        if not debug:
+            return cls(sel)
+        return cls(sel, torch.empty(cfg.B, cfg.Hq, nb, cfg.D, dtype=torch.float32, device=device),
+                   torch.empty(cfg.B, cfg.Hq, nb, cfg.P, cfg.probes, **i32),
+                   torch.empty(cfg.B, cfg.Hq, nb, **i32))
+
+    def c(self) -> mdr_route_out:
+        return mdr_route_out(_ptr(self.sel), _ptr(self.qbar), _ptr(self.qcodes), _ptr(self.ncand))
+
+
+def workspace(cfg: mdr_config, device="cuda"):
+    import torch
+    return torch.empty(mdr_workspace_bytes(cfg), dtype=torch.uint8, device=device)
+
+
+def mdr_build_index(cfg, k, codebooks, idx: Index, ws, stream=None):
+    _ok(lib().mdr_build_index(ctypes.byref(cfg), _ptr(k), _ptr(codebooks), ctypes.byref(idx.c()),
+                              _ptr(ws), ws.numel(), _stream(stream)), "mdr_build_index")
+
+
+def mdr_route(cfg, q, codebooks, idx: Index, rt: RouteOut, ws, stream=None):
+    _ok(lib().mdr_route(ctypes.byref(cfg), _ptr(q), _ptr(codebooks), ctypes.byref(idx.c()),
+                        ctypes.byref(rt.c()), _ptr(ws), ws.numel(), _stream(stream)), "mdr_route")
+
+
+def mdr_attend(cfg, q, k, v, sel, out, ws, stream=None):
+    _ok(lib().mdr_attend(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(out),
+                         _ptr(ws), ws.numel(), _stream(stream)), "mdr_attend")
+
+
+def mdr_forward(cfg, q, k, v, codebooks, idx: Index, rt: RouteOut, out, ws, stream=None):
+    _ok(lib().mdr_forward(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(codebooks),
+                          ctypes.byref(idx.c()), ctypes.byref(rt.c()), _ptr(out), _ptr(ws),
+                          ws.numel(), _stream(stream)), "mdr_forward")
+
+
+def mdr_forward_profiled(cfg, q, k, v, codebooks, idx: Index, rt: RouteOut, out, ws, events, stream=None):
+    """events: list of torch.cuda.Event(enable_timing=True) (or None), recorded
+    before K1 and after K1, K3, K4, K5."""
+    for e in events:
+        if e is not None and not e.cuda_event:
+            e.record()          # torch creates the CUDA event on its first record
+    arr = (ctypes.c_void_p * len(events))(*[None if e is None else e.cuda_event for e in events])
+    _ok(lib().mdr_forward_profiled(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(codebooks),
+                                   ctypes.byref(idx.c()), ctypes.byref(rt.c()), _ptr(out), _ptr(ws),
+                                   ws.numel(), _stream(stream), arr, len(events)), "mdr_forward_profiled")
+
+
+def mdr_forward_host(cfg, q, k, v, codebooks, out, sel=None, overflow=None, maxload=None,
+                     dev_ws=None, stream=None):
+    """Host buffers (torch CPU tensors, ideally pinned) in and out."""
+    _ok(lib().mdr_forward_host(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(codebooks), _ptr(out),
+                               _ptr(sel), _ptr(overflow), _ptr(maxload), _ptr(dev_ws), dev_ws.numel(),
+                               _stream(stream)), "mdr_forward_host")
+
+
+def mdr_read_device_status(ws, stream=None) -> int:
+    code = ctypes.c_int32(0)
+    s = lib().mdr_read_device_status(_ptr(ws), ctypes.byref(code), _stream(stream))
+    if s not in (MDR_OK, MDR_ERR_DEVICE):
+        raise MdrError(s, "mdr_read_device_status")
+    return code.value

@@ -16,19 +16,17 @@ It is written to be read against the two pages that describe the method:
 The forward is index -> route -> attend:
   1. rotary embedding of queries and keys (Report, Mixer; Article);
   2. per-block summaries of the rotated queries and keys;
-  3. a product address per source block from P codebooks (Article: "each
-     product address combines decisions from multiple learned code
-     components"; Report, Capacity: "spherical codebook");
-  4. bounded causal posting lists, overflow counted (Report, Mixer: "writes
-     keys into bounded causal posting lists"; Report, Capacity and Evidence:
-     overflow, maximum assigned load);
+  3. a product address per source block: one codeword choice per subspace,
+     combined (Article; Report, Capacity, for the spherical codebooks);
+  4. bounded causal posting lists, overflow counted (Report, Mixer; Report,
+     Capacity and Evidence: overflow events, maximum assigned load);
   5. probe -> candidates in fixed slots -> rerank -> R remote blocks, plus L
      local blocks added separately (Article; Report, Mixer; Report,
-     Finite-range scaling: "fixed candidate-slot checks");
-  6. ordinary causal softmax over the tokens of the selected blocks, no value
-     summary (Report, Mixer; Article).
-And the independent dense selected-mask form of step 6 (Report, Evidence:
-"Selected-mask oracle error"; Article, "Why Learned Product-Hash Routing
+     Finite-range scaling, for the fixed candidate slots);
+  6. exact causal softmax over the tokens of the selected blocks, with their
+     own values (Report, Mixer; Article).
+And the independent dense selected-mask form of step 6 (Report, Evidence,
+the selected-mask oracle row; Article, "Why Learned Product-Hash Routing
 Matters Now").
 
 Precision.  Every value is computed in float64 from the stored inputs.  Two
@@ -76,7 +74,7 @@ def rope(x: np.ndarray, base: float) -> np.ndarray:
 
     Rotate-half pairing: coordinate i is paired with i + D/2 and the pair is
     rotated by the angle of position t and frequency i.  Applied to queries and
-    keys, never to values (Report, Mixer: "After rotary position embedding").
+    keys, never to values (Report, Mixer: routing follows the rotation).
     """
     B, S, H, D = x.shape
     th = rope_angles(S, D, base).astype(np.float64)
@@ -92,8 +90,8 @@ def block_means(xr: np.ndarray, bs: int) -> np.ndarray:
     """Mean of the rotated vectors over each block of bs tokens.
 
     [B,S,H,D] -> [B,H,nb,D].  Source blocks and query blocks are both
-    summarised this way (Article: "source blocks receive learned product
-    addresses"; the query of a block is its mean rotated query).
+    summarised this way (Article: addresses are given to source blocks; the
+    query of a block is its mean rotated query).
     """
     B, S, H, D = xr.shape
     nb = S // bs
@@ -201,9 +199,10 @@ def candidate_slots(lists: np.ndarray, probe_addrs: np.ndarray, j: int, L: int) 
 def route_row(qbar_j: np.ndarray, kbar_h: np.ndarray, probe_addrs: np.ndarray,
               lists: np.ndarray, j: int, R: int, L: int) -> RouteRow:
     """Route one query block: probe -> candidates -> rerank -> top R, plus the
-    L local blocks j-L+1..j (Article: "A query probes addresses, receives
-    candidates, reranks them, and selects a fixed number of remote blocks";
-    "The query also receives guaranteed local blocks").
+    L local blocks j-L+1..j (Article, section "Monodratic Turns Sparse
+    Attention Into a Retrieval Decision": the query probes addresses, gets
+    candidates, reranks them and keeps a fixed count of remote blocks; local
+    blocks are always added).
 
     Rerank score of candidate i is <qbar_j, kbar_i> over the full head
     dimension, rounded to float32; top R by score, lower id on equal scores.
@@ -235,8 +234,8 @@ def attend(qr, kr, v, sel, bs: int, scale: float, rows=None) -> np.ndarray:
 
     For token t of query block j, head hq: the keys are every token s of every
     selected block with s <= t; weights softmax(scale * <q'_t, k'_s>) applied
-    to v_s (Report, Mixer: "Attention over that set is ordinary causal softmax.
-    No value summary replaces selected source values").  Query head hq reads KV
+    to v_s (Report, Mixer: exact causal softmax over the selected set, with the
+    selected values, not a summary of them).  Query head hq reads KV
     head hq // (Hq/Hkv).  rows: optional list of (b, hq, j) to compute; the
     others stay NaN.  -> [B,S,Hq,D] float64.
     """

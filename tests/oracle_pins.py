@@ -238,8 +238,8 @@ def check_route_bruteforce_all_eligible():
 
 
 def check_route_causal_and_fixed_slots():
-    """No block is reachable from an earlier query block (Article: "A source
-    block must not become available to a query positioned before it"), the
+    """No block is reachable from an earlier query block (Article, section
+    "Monodratic Turns Sparse Attention Into a Retrieval Decision"), the
     locals are j-L+1..j, and every route has p**P x cap candidate slots
     (Report, Finite-range scaling: fixed candidate-slot checks)."""
     p = _p(S=256, block=16, K=4, P=2, cap=2, probes=2, R=3, L=2, D=16)

@@ -1,0 +1,106 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/mdr.h declares, and its host-side argument checks answer correctly
+before anything is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from learned_product_hash_b200 import mdr
+from workloads import ALL, TINY, SCALING_32K
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^\s*(?:mdr_status|int32_t|const char\*)\s+(mdr_\w+)\s*\(", src, re.M)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    L = mdr.lib()
+    declared = _declared()
+    assert len(declared) >= 11
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(declared) == set(mdr.EXPORTED) | (set(declared) - set(mdr.EXPORTED))
+    assert mdr.mdr_abi_version() == 1
+
+
+@pytest.mark.parametrize("name", sorted(ALL))
+def test_workload_configs_are_supported(name):
+    cfg = mdr.make_config(ALL[name])
+    assert mdr.mdr_check_config(cfg) == mdr.MDR_OK
+    assert mdr.mdr_workspace_bytes(cfg) > 0
+    assert mdr.mdr_host_workspace_bytes(cfg) > mdr.mdr_workspace_bytes(cfg)
+
+
+BAD = [
+    (dict(S=100), mdr.MDR_ERR_INVALID_ARG),             # S % block != 0
+    (dict(Hq=3, Hkv=2), mdr.MDR_ERR_INVALID_ARG),       # Hq % Hkv != 0
+    (dict(L=0), mdr.MDR_ERR_INVALID_ARG),               # own block must be local
+    (dict(probes=9), mdr.MDR_ERR_INVALID_ARG),          # probes > K
+    (dict(cap=0), mdr.MDR_ERR_INVALID_ARG),
+    (dict(R=-1), mdr.MDR_ERR_INVALID_ARG),
+    (dict(rope_base=1.0), mdr.MDR_ERR_INVALID_ARG),
+    (dict(dtype=7), mdr.MDR_ERR_INVALID_ARG),
+    (dict(D=48), mdr.MDR_ERR_UNSUPPORTED),
+    (dict(block=8, S=96), mdr.MDR_ERR_UNSUPPORTED),
+    (dict(K=200, probes=2), mdr.MDR_ERR_UNSUPPORTED),
+    (dict(R=33), mdr.MDR_ERR_UNSUPPORTED),
+    (dict(P=3, D=32), mdr.MDR_ERR_INVALID_ARG),         # D % P != 0
+]
+
+
+@pytest.mark.parametrize("change,expect", BAD)
+def test_bad_configs_rejected(change, expect):
+    cfg = mdr.make_config(TINY.with_(**change))
+    assert mdr.mdr_check_config(cfg) == expect
+
+
+def test_bf16_needs_tensor_core_tiles():
+    cfg = mdr.make_config(TINY.with_(dtype="bf16"))       # block 16, D 32
+    assert mdr.mdr_check_config(cfg) == mdr.MDR_ERR_UNSUPPORTED
+    assert mdr.mdr_check_config(mdr.make_config(SCALING_32K)) == mdr.MDR_OK
+
+
+def test_entry_points_check_arguments_before_any_gpu_work():
+    L = mdr.lib()
+    cfg = mdr.make_config(TINY)
+    n = mdr.mdr_workspace_bytes(cfg)
+    idx = mdr.mdr_index()
+    rt = mdr.mdr_route_out()
+    fake = ctypes.c_void_p(0x10000)            # never dereferenced: checks fail first
+    # null inputs
+    assert L.mdr_forward(ctypes.byref(cfg), None, fake, fake, fake, ctypes.byref(idx), ctypes.byref(rt),
+                         fake, fake, n, None) == mdr.MDR_ERR_INVALID_ARG
+    # missing index buffers
+    rt.sel = 0x10000
+    assert L.mdr_forward(ctypes.byref(cfg), fake, fake, fake, fake, ctypes.byref(idx), ctypes.byref(rt),
+                         fake, fake, n, None) == mdr.MDR_ERR_INVALID_ARG
+    idx = mdr.mdr_index(*([0x10000] * 6))
+    # workspace too small, then misaligned
+    assert L.mdr_forward(ctypes.byref(cfg), fake, fake, fake, fake, ctypes.byref(idx), ctypes.byref(rt),
+                         fake, fake, n - 1, None) == mdr.MDR_ERR_WORKSPACE
+    assert L.mdr_forward(ctypes.byref(cfg), fake, fake, fake, fake, ctypes.byref(idx), ctypes.byref(rt),
+                         fake, ctypes.c_void_p(0x10010), n, None) == mdr.MDR_ERR_WORKSPACE
+    # unsupported config is reported before pointers are looked at
+    bad = mdr.make_config(TINY.with_(D=48))
+    assert L.mdr_build_index(ctypes.byref(bad), None, None, None, None, 0, None) == mdr.MDR_ERR_UNSUPPORTED
+    assert L.mdr_attend(ctypes.byref(cfg), fake, None, fake, fake, fake, fake, n, None) == mdr.MDR_ERR_INVALID_ARG
+    assert L.mdr_route(ctypes.byref(cfg), fake, fake, ctypes.byref(idx), None, fake, n, None) == mdr.MDR_ERR_INVALID_ARG
+    # unaligned tensors
+    odd = ctypes.c_void_p(0x10004)
+    assert L.mdr_attend(ctypes.byref(cfg), odd, fake, fake, fake, fake, fake, n, None) == mdr.MDR_ERR_INVALID_ARG
+    assert L.mdr_read_device_status(None, None, None) == mdr.MDR_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    for s in range(6):
+        assert mdr.status_string(s)
+    assert mdr.status_string(99) == "unknown status"

@@ -1,0 +1,146 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle on
+seeded inputs of every workload, plus edge cases.  The bar is stated in
+tests/parity_util.py."""
+import numpy as np
+import pytest
+
+from oracle import mdr_oracle as O
+from tests import parity_util as U
+from workloads import ALL, AR, CAPACITY, LONG, SCALING_32K, TINY, make_inputs, scaling
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from learned_product_hash_b200 import mdr
+    mdr.lib()
+
+
+SMALL = [TINY, AR, CAPACITY, scaling(4096)]
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_forward_matches_oracle(w, seed):
+    inp = make_inputs(w, seed)
+    g = U.run_gpu(w, inp)
+    res = U.oracle_for(w, inp)
+    rep = U.compare(w, g, res, inp.codebooks)
+    assert rep["code_ties"] + rep["qcode_ties"] + rep["sel_ties"] <= 2, rep
+
+
+@pytest.mark.parametrize("w", [TINY, AR.with_(B=8), CAPACITY], ids=lambda w: w.name)
+def test_split_entry_points_equal_forward(w):
+    """mdr_build_index + mdr_route + mdr_attend give exactly what mdr_forward gives."""
+    inp = make_inputs(w, 3)
+    a = U.run_gpu(w, inp, "forward")
+    b = U.run_gpu(w, inp, "split")
+    for key in a:
+        assert np.array_equal(a[key], b[key]), key
+
+
+EDGE = {
+    # every block in one list: overflow nb - cap, ties everywhere resolved by index
+    "zeros_f32": (TINY, dict(zero=True)),
+    "zeros_bf16": (scaling(4096).with_(cap=16), dict(zero=True)),
+    # every eligible block admitted: the route is the exact top-R, the output dense causal
+    "dense_limit_bf16": (AR.with_(B=2, cap=6, K=4, probes=4, R=6), {}),
+    "dense_limit_f32": (TINY.with_(cap=6, K=2, probes=2, R=6), {}),
+    # local-only control
+    "local_only": (AR.with_(B=4, R=0), {}),
+    # ragged: 7 blocks, 3 query heads per KV head, block 128, D 64
+    "ragged_gqa": (CAPACITY.with_(S=7 * 128, block=128, Hq=6, Hkv=2, R=3, L=3, keys="gaussian"), {}),
+    # many locals, tiny capacity (heavy overflow), one probe
+    "overflow_heavy": (scaling(4096).with_(cap=1, probes=1, K=4, L=4), {}),
+    "fp32_d128": (TINY.with_(D=128, S=256, block=32, Hq=4, Hkv=2, K=16, cap=4, probes=3, R=3, L=2), {}),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_edge_cases(name):
+    w, kw = EDGE[name]
+    inp = make_inputs(w, 5, **kw)
+    g = U.run_gpu(w, inp)
+    res = U.oracle_for(w, inp)
+    rep = U.compare(w, g, res, inp.codebooks)
+    if kw.get("zero"):
+        assert (g["addr"] == 0).all()
+        assert (g["overflow"] == max(0, w.nb - w.cap)).all()
+    if name.startswith("dense_limit"):
+        assert (g["ncand"] == np.maximum(np.arange(w.nb) - w.L + 1, 0)[None, None, :]).all()
+
+
+def test_bad_selection_sets_device_status():
+    """mdr_attend checks every selected id against the block grid; an id that
+    points past the query block is skipped and reported in the status word."""
+    import torch
+    from learned_product_hash_b200 import mdr
+    w = TINY
+    inp = make_inputs(w, 0)
+    cfg = mdr.make_config(w)
+    q, k, v, _ = U.to_device(inp, w)
+    res = U.oracle_for(w, inp)
+    sel = torch.from_numpy(res.sel.astype(np.int32)).cuda()
+    sel[0, 0, 2, 0] = 5                                 # later than block 2
+    out = torch.empty_like(q)
+    ws = mdr.workspace(cfg)
+    mdr.mdr_attend(cfg, q, k, v, sel, out, ws)
+    assert mdr.mdr_read_device_status(ws) == 2
+    # the other query blocks are unaffected
+    rows = np.ones((1, w.S, 1), dtype=bool)
+    rows[0, 32:48] = False
+    U.check_out(w, out.cpu().numpy(), res.out, rows)
+
+
+def test_host_entry_point_matches_device():
+    import torch
+    from learned_product_hash_b200 import mdr
+    w = AR.with_(B=4)
+    inp = make_inputs(w, 7)
+    g = U.run_gpu(w, inp)
+    cfg = mdr.make_config(w)
+    pin = lambda x: torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).pin_memory()
+    q, k, v = pin(inp.q_store), pin(inp.k_store), pin(inp.v_store)
+    cb = torch.from_numpy(inp.codebooks).pin_memory()
+    out = torch.empty_like(q).pin_memory()
+    sel = torch.empty(g["sel"].shape, dtype=torch.int32).pin_memory()
+    ovf = torch.empty(g["overflow"].shape, dtype=torch.int32)
+    mx = torch.empty(g["maxload"].shape, dtype=torch.int32)
+    dws = torch.empty(mdr.mdr_host_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
+    mdr.mdr_forward_host(cfg, q, k, v, cb, out, sel, ovf, mx, dws)
+    assert np.array_equal(sel.numpy(), g["sel"])
+    assert np.array_equal(ovf.numpy(), g["overflow"]) and np.array_equal(mx.numpy(), g["maxload"])
+    got = out.view(torch.bfloat16).float().numpy()
+    assert np.array_equal(got, g["out"])
+
+
+def _sampled_rows(w, res, n=12, seed=0):
+    r = np.random.default_rng(seed)
+    rows = {(0, 0, 0), (0, w.Hq - 1, w.nb - 1)}
+    # heaviest routes and random ones
+    heavy = np.argsort(-res.ncand.ravel())[:4]
+    for f in heavy:
+        b, h, j = np.unravel_index(f, res.ncand.shape)
+        rows.add((int(b), int(h), int(j)))
+    while len(rows) < n:
+        rows.add((int(r.integers(w.B)), int(r.integers(w.Hq)), int(r.integers(w.nb))))
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("w", [SCALING_32K, LONG], ids=lambda w: w.name)
+def test_full_size_sampled(w):
+    """The benchmark's launch at full size: routing compared everywhere,
+    attention on sampled query blocks the oracle computes one by one."""
+    inp = make_inputs(w, 0)
+    g = U.run_gpu(w, inp)
+    p = O.Params.of(w)
+    res = O.forward(inp.q, inp.k, inp.v, inp.codebooks, p, attention=False)
+    rows = _sampled_rows(w, res)
+    res.out = O.attend(res.qr, res.kr, inp.v.astype(np.float64), res.sel, w.block, p.softmax_scale, rows)
+    rep = U.compare(w, g, res, inp.codebooks)
+    if w is LONG:
+        assert rep["overflow"] > 0, "the long workload must overflow its lists"
