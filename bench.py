@@ -59,6 +59,20 @@ def init_dist(world, backend):
     return dist
 
 
+def max_over_ranks(x: float, dist, world: int, device) -> float:
+    """The largest value over all ranks (every rank gets it)."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (ms_max / 1e3)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -227,13 +241,9 @@ def run_mine(args, w):
     tot = [e[0].elapsed_time(e[4]) for e in evs]
     ker = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
            for i, n in enumerate(("summarize", "lists", "route", "attend"))}
-    ms = statistics.mean(tot)
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(statistics.mean(tot), dist, world, dev)
     tokens = w.B * w.S * world
-    value = tokens / (ms_max / 1e3)
+    value = throughput(w.B * w.S, world, ms_max)
 
     # Roofline of the attention kernel: q read + gathered K/V of valid
     # selected blocks + out write, per (b, hq, j) route.
@@ -266,13 +276,11 @@ def run_mine(args, w):
             e1.synchronize()
             if it >= 2:
                 times.append(e0.elapsed_time(e1))
-        te = torch.tensor([statistics.mean(times)], device=dev, dtype=torch.float64)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        te_ms = max_over_ranks(statistics.mean(times), dist, world, dev)
         h2d = sum(x.numel() * x.element_size() for x in (qp, kp, vp, cbp))
         d2h = sum(x.numel() * x.element_size() for x in (outp, selp, ovp, mxp))
-        e2e = {"value": tokens / (float(te.item()) / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": float(te.item())}
+        e2e = {"value": throughput(w.B * w.S, world, te_ms), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": te_ms}
         del dws
 
     cpu = None

@@ -158,7 +158,10 @@ mdr_status mdr_route(const mdr_config* cfg, const void* q,
  * rotated queries and keys; exact softmax over the selected tokens, the
  * values used as they are (Report, section Mixer).  sel: device int32 [B,Hq,nb,R+L]; any valid block id in
  * [0, j] may appear, -1 entries are skipped, ids must not repeat within a
- * row.  out: device [B,S,Hq,D].                                             */
+ * row; an id outside [0, j] is skipped and sets status 2.  A query block
+ * left with no valid block gets a zero output.  out: device [B,S,Hq,D].
+ * bf16 runs on the tensor cores (tcgen05, TMEM accumulators, TMA loads);
+ * float32 runs on the CUDA cores in float32.                                             */
 mdr_status mdr_attend(const mdr_config* cfg, const void* q, const void* k,
                       const void* v, const int32_t* sel, void* out, void* ws,
                       size_t ws_bytes, void* stream);

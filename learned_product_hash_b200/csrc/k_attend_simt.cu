@@ -78,7 +78,7 @@ attend_simt_kernel(const AttendArgs a) {
         mx = mnew;
       }
     }
-    const float inv = 1.f / l;
+    const float inv = l > 0.f ? 1.f / l : 0.f;   // nothing selected: zero output
     const size_t ooff = ((static_cast<size_t>(b) * a.S + t) * a.Hq + hq) * a.D;
 #pragma unroll
     for (int m = 0; m < 4; ++m)

@@ -118,6 +118,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const int nblk = nblk_s;
   const int tok0 = b * a.S;                   // first token row of sequence b
 
+  if (nblk == 0) {                            // nothing selected: the output is zero
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+    for (int e = threadIdx.x; e < BS * D / 8; e += blockDim.x) {
+      const int rr = e / (D / 8), c8 = e % (D / 8);
+      *reinterpret_cast<uint4*>(out + ((static_cast<size_t>(tok0) + static_cast<size_t>(j) * BS + rr) * a.Hq + hq) * D +
+                                c8 * 8) = make_uint4(0, 0, 0, 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    if (warp == 0) tmem_dealloc(tmem, C::kCols);
+    return;
+  }
+
   const uint32_t idS = idesc_bf16_f32(BS, BS, 0, 0);
   const uint32_t idPV = idesc_bf16_f32(BS, D, 0, 1);
   int issued = 0;                             // K/V blocks whose TMA thread 0 issued
@@ -175,6 +189,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   for (int n = 0; n < nblk; ++n) {
     const int s = n % C::kStages;
     bool bad = !mbar_wait(BAR(kBarS), n & 1, kWaitNs);
+    __syncwarp();                               // tcgen05.ld is warp-collective
     tc_fence_after();
     float sv[BS];
 #pragma unroll
@@ -217,6 +232,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         *reinterpret_cast<uint4*>(prow + region * C::kRegion + chunk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
+    __syncwarp();
     if (__any_sync(0xffffffffu, rescale)) {
       float o[32];
 #pragma unroll
@@ -274,13 +290,17 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     tc_fence_after();
     mma_commit(BAR(kBarDone));
     if (aborted || t0_fail) {
-      // K/V loads issued but not consumed: n in [consumed, issued).
-      for (int n = 0; n < issued; ++n)
-        mbar_wait(BAR(kBarKV + n % C::kStages), (n / C::kStages) & 1, kWaitNs);
+      // The last load issued into each stage completes after the earlier ones.
+      for (int s = 0; s < C::kStages; ++s) {
+        int last = -1;
+        for (int n = s; n < issued; n += C::kStages) last = n;
+        if (last >= 0) mbar_wait(BAR(kBarKV + s), (last / C::kStages) & 1, kWaitNs);
+      }
       mbar_wait(BAR(kBarQ), 0, kWaitNs);
     }
   }
   const bool done = mbar_wait(BAR(kBarDone), 0, kWaitNs);
+  __syncwarp();
   if (!done && threadIdx.x == 0) fail();
   tc_fence_after();
   if (done && !aborted && !__syncthreads_or(abort_s)) {
@@ -308,6 +328,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   }
   tc_fence_before();
   __syncthreads();
+  __syncwarp();
   if (warp == 0) tmem_dealloc(tmem, C::kCols);
 }
 

@@ -142,7 +142,8 @@ mdr_status run_attend(const mdr_config* c, const void* qrot, const void* krot, c
   aa.B = c->B; aa.S = c->S; aa.Hq = c->Hq; aa.Hkv = c->Hkv; aa.D = c->D; aa.bs = c->block;
   aa.nb = c->S / c->block; aa.nsel = c->R + c->L;
   aa.scale = c->scale > 0.f ? c->scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(c->D)));
-  return cuda_status(mdr::launch_attend_simt(aa, c->dtype == MDR_BF16, st));
+  if (c->dtype == MDR_BF16) return cuda_status(mdr::launch_attend_tc(aa, st));
+  return cuda_status(mdr::launch_attend_simt(aa, false, st));
 }
 
 }  // namespace
