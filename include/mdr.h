@@ -202,6 +202,24 @@ mdr_status mdr_forward_host(const mdr_config* cfg, const void* q_host,
                             int32_t* maxload_host, void* dev_ws,
                             size_t dev_ws_bytes, void* stream);
 
+/* The route step without any workspace, for callers that can neither pass
+ * a workspace nor call cudaMalloc (a serving loop whose device memory is all
+ * reserved by its own pool, a plugin interface that hands an operator only
+ * its inputs and outputs).  The pages have no counterpart: this exists only
+ * for such callers.  Same inputs and outputs as mdr_route (sel required,
+ * ncand may be NULL; the query summaries and probe codes are not returned).
+ * Its scratch (query block means and probe codewords) lives in a 32 MiB
+ * array inside the library, held on every GPU that loads it until exit; it
+ * needs B*Hq*nb*(4*D + 4*P*probes) bytes (each part rounded up to 256) and
+ * larger calls return MDR_ERR_WORKSPACE before anything is enqueued.  The
+ * first call on each device looks up the array's device address with that
+ * device current; make it before any stream capture.  Calls share the array,
+ * so calls that overlap on the GPU race; nothing in it needs clearing
+ * between calls.  Allocates nothing.                                        */
+mdr_status mdr_route_noalloc(const mdr_config* cfg, const void* q,
+                             const float* codebooks, const mdr_index* idx,
+                             int32_t* sel, int32_t* ncand, void* stream);
+
 /* Synchronise the stream and copy the device status word (first 4 bytes of
  * ws) to *code (0 = no device-side failure).  Returns MDR_ERR_DEVICE when the
  * word is nonzero.                                                           */

@@ -20,7 +20,7 @@ MDR_F32, MDR_BF16 = 0, 1
 EXPORTED = (
     "mdr_abi_version", "mdr_status_string", "mdr_check_config", "mdr_workspace_bytes",
     "mdr_build_index", "mdr_route", "mdr_attend", "mdr_forward", "mdr_host_workspace_bytes",
-    "mdr_forward_host", "mdr_read_device_status", "mdr_forward_profiled",
+    "mdr_forward_host", "mdr_read_device_status", "mdr_forward_profiled", "mdr_route_noalloc",
 )
 
 
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "mdr_read_device_status": ([vp, ctypes.POINTER(ctypes.c_int32), vp], i32),
             "mdr_forward_profiled": ([cfgp, vp, vp, vp, vp, idxp, rtp, vp, vp, sz, vp,
                                       ctypes.POINTER(vp), ctypes.c_int32], i32),
+            "mdr_route_noalloc": ([cfgp, vp, vp, idxp, vp, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -229,3 +230,10 @@ def mdr_read_device_status(ws, stream=None) -> int:
     if s not in (MDR_OK, MDR_ERR_DEVICE):
         raise MdrError(s, "mdr_read_device_status")
     return code.value
+
+
+def mdr_route_noalloc(cfg, q, codebooks, idx: Index, sel, ncand=None, stream=None):
+    """Route with the library's built-in scratch instead of a workspace (for
+    callers that cannot allocate device memory); see include/mdr.h."""
+    _ok(lib().mdr_route_noalloc(ctypes.byref(cfg), _ptr(q), _ptr(codebooks), ctypes.byref(idx.c()),
+                                _ptr(sel), _ptr(ncand), _stream(stream)), "mdr_route_noalloc")
