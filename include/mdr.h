@@ -73,7 +73,7 @@ typedef enum mdr_dtype { MDR_F32 = 0, MDR_BF16 = 1 } mdr_dtype;
  * Supported: D in {32,64,128}; block in {16,32,64,128}; 1 <= P <= 4 with
  * D % P == 0 and (D/P) % 4 == 0; 1 <= K <= 128; A <= 16384; 1 <= cap <= 1024;
  * 1 <= probes <= K with probes^P <= 64 and probes^P * cap <= 4096;
- * 0 <= R <= 32; 1 <= L <= 32.  MDR_BF16 additionally needs block in {64,128}
+ * 0 <= R <= 32; 1 <= L <= 32; S/block <= 32768.  MDR_BF16 additionally needs block in {64,128}
  * and D in {64,128} (the tensor-core attention tiles).                      */
 typedef struct mdr_config {
   int32_t B, S, Hq, Hkv, D, block;

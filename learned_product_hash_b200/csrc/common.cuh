@@ -15,6 +15,7 @@ enum DeviceError : int32_t {
   kDevOk = 0,
   kDevWaitTimeout = 1,      // an mbarrier wait ran out of iterations
   kDevBadSelection = 2,     // a selected block id out of range
+  kDevMisaligned = 3,       // dynamic shared memory not 1024-byte aligned
 };
 
 // Element traits: 16-byte vectors of the storage type.
@@ -26,6 +27,10 @@ template <> struct Elem<float> {
     float4 v = __ldg(reinterpret_cast<const float4*>(p));
     out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
   }
+  __device__ static inline void unpack(const uint4& v, float* out) {
+    out[0] = __uint_as_float(v.x); out[1] = __uint_as_float(v.y);
+    out[2] = __uint_as_float(v.z); out[3] = __uint_as_float(v.w);
+  }
   __device__ static inline void store(float* p, const float* in) {
     *reinterpret_cast<float4*>(p) = make_float4(in[0], in[1], in[2], in[3]);
   }
@@ -36,6 +41,14 @@ template <> struct Elem<__nv_bfloat16> {
   static constexpr int kVec = 8;
   __device__ static inline void load(const __nv_bfloat16* p, float* out) {
     uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      out[2 * i] = __uint_as_float(w[i] << 16);
+      out[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+  __device__ static inline void unpack(const uint4& v, float* out) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {

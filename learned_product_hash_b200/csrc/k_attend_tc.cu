@@ -6,30 +6,38 @@
 // section Mixer: exact causal softmax over the selected set, with the
 // selected values themselves).
 //
-// One CTA (4 warps) per (b, hq, j).  Thread 0 drives the asynchronous units:
-// TMA brings the Q tile and, block by block, the K and V tiles of the
-// selected blocks into a two-stage ring of 128-byte-swizzled shared memory;
-// tcgen05.mma computes S = Q K^T (M = bs query rows, N = bs keys, K = D) into
-// tensor memory and O += P V (M = bs, N = D, K = bs keys) into a second TMEM
-// accumulator.  All 128 threads run the softmax: each owns one query row of
-// S (tcgen05.ld), applies the causal mask inside the query's own block,
-// keeps a running maximum and sum in float32, writes P = exp(S - max) as
-// bf16 into shared memory in the layout the next MMA reads, and rescales O
-// in TMEM only when the running maximum grows by more than 2^8 (exact:
-// the final division by the running sum uses the same maximum).
+// Persistent, warp-specialised kernel.  A CTA walks the (b, hq, j) tiles
+// blockIdx.x, blockIdx.x + gridDim.x, ...  (consecutive CTAs take
+// consecutive query blocks of one head, so that head's K/V stays in L2).
+//   warp 0        TMA producers: lane 0 loads the Q tile of each query block
+//                 into a Q ring and the K tile of every selected block into a
+//                 K ring, lane 1 the V tiles into a V ring (128-byte swizzle,
+//                 mbarrier expect-tx).  A K stage is refilled once the S MMA
+//                 that read it completed, a V stage once its PV completed.
+//   warp 1        MMA issuer (one lane): S = Q K^T (M = bs, N = bs, K = D)
+//                 into one of two TMEM S buffers, and O += P V (M = bs,
+//                 N = D, K = bs keys; V read MN-major from its TMA tile)
+//                 into the TMEM O accumulator.  S of block n+2 is issued as
+//                 soon as the softmax has consumed S of block n, so the
+//                 tensor core works on the next scores and the previous PV
+//                 while the softmax runs.
+//   warps 2..5    softmax: one query row per thread (tcgen05.ld), causal
+//                 mask inside the query's own block, running maximum and
+//                 sum in float32 (log2 units), P = exp(S - max) as bf16 into
+//                 one of two shared-memory P buffers in the K-major swizzled
+//                 layout the PV MMA reads; O is rescaled in TMEM only when the
+//                 running maximum grows by more than 2^8 (exact, since the
+//                 final division uses the same maximum); epilogue O / sum ->
+//                 bf16 -> global.
+// TMEM accumulators with M = 64 keep row r in lane (r % 16) + 32 (r / 16); with
+// M = 128 in lane r.  Warp w may only touch lanes 32 (w % 4) .. + 31.
 //
-// Tensor-memory layout of an accumulator with M = 64: row r sits in lane
-// (r % 16) + 32 * (r / 16); with M = 128 row r sits in lane r.  Warp w reads
-// lanes 32w..32w+31.
-//
-// Every mbarrier wait is bounded (2 s of wall time).  A wait that runs out
-// writes kDevWaitTimeout to the status word, the CTA stops issuing work,
-// waits (bounded) for what it already issued, frees its tensor memory and
-// exits.
+// Every wait is bounded (2 s of wall time) and also gives up when another
+// role has aborted; a wait that runs out writes status 1, every role stops
+// issuing, waits (bounded) for what it issued, and the CTA frees its tensor
+// memory and exits.
 
 #include <cuda.h>
-
-#include <climits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -40,279 +48,395 @@ namespace mdr {
 namespace {
 
 constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr int kThreads = 192;
 
 template <int BS, int D>
 struct TcCfg {
-  static constexpr int kStages = 2;
-  static constexpr int kTileBytes = BS * D * 2;     // one [BS x D] bf16 tile
+  static constexpr bool kBig = (BS == 128 && D == 128);
+  static constexpr int kQBuf = kBig ? 1 : 2;
+  static constexpr int kStages = (BS == 64 && D == 64) ? 4 : 2;
+  static constexpr int kPBuf = kBig ? 1 : 2;
+  static constexpr int kTile = BS * D * 2;          // one [BS x D] bf16 tile
   static constexpr int kPBytes = BS * BS * 2;
+  static constexpr int kRegion = BS * 128;          // one 64-column swizzled region of a tile
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kTileBytes;
-  static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffP = kOffV + kStages * kTileBytes;
-  static constexpr int kOffBar = kOffP + kPBytes;
-  static constexpr int kSmem = kOffBar + 128 + 1024;  // barriers + alignment slack
-  static constexpr int kColS = 0;
-  static constexpr int kColO = BS;
-  static constexpr int kCols = (BS + D) <= 128 ? 128 : 256;
-  static constexpr int kRegion = BS * 128;            // one 64-column swizzled region of a tile
-  static_assert(kTileBytes % 1024 == 0 && kPBytes % 1024 == 0, "1024-byte aligned tiles");
+  static constexpr int kOffK = kOffQ + kQBuf * kTile;
+  static constexpr int kOffV = kOffK + kStages * kTile;
+  static constexpr int kOffP = kOffV + kStages * kTile;
+  static constexpr int kOffBar = kOffP + kPBuf * kPBytes;
+  static constexpr int kOffMisc = kOffBar + 8 * 32;         // TMEM base address, abort flag
+  static constexpr int kSmem = kOffMisc + 16;
+  // M = 64 accumulators fill lanes 0-15 of each subpartition: two threads
+  // share a row (16x32bx2 loads), each taking 32 of every 64 columns.
+  static constexpr bool kHalf = (BS == 64);
+  static constexpr int kSCols = kHalf ? 32 : BS;            // S columns per thread
+  static constexpr int kColS = 0;                   // S buffers at columns 0 and BS
+  static constexpr int kColO = 2 * BS;
+  static constexpr int kCols = (2 * BS + D) <= 256 ? 256 : 512;
+  // barrier indices
+  static constexpr int bQFull = 0;
+  static constexpr int bQEmpty = bQFull + kQBuf;
+  static constexpr int bKFull = bQEmpty + kQBuf;
+  static constexpr int bKEmpty = bKFull + kStages;
+  static constexpr int bVFull = bKEmpty + kStages;
+  static constexpr int bVEmpty = bVFull + kStages;
+  static constexpr int bSFull = bVEmpty + kStages;   // 2
+  static constexpr int bPFull = bSFull + 2;          // kPBuf
+  static constexpr int bPVDone = bPFull + kPBuf;     // 2
+  static constexpr int bOFull = bPVDone + 2;
+  static constexpr int bOFree = bOFull + 1;
+  static constexpr int bFin = bOFree + 1;
+  static constexpr int kNumBars = bFin + 1;
+  static_assert(kNumBars <= 32, "barrier space");
+  static_assert(kTile % 1024 == 0 && kPBytes % 1024 == 0, "1024-byte aligned tiles");
 };
 
-enum Bar { kBarQ = 0, kBarKV = 1, kBarFree = 3, kBarS = 5, kBarDone = 6 };
+// Valid entries of a sel row are ids in [0, j]; everything else is skipped.
+__device__ __forceinline__ bool valid_id(int id, int j) { return id >= 0 && id <= j; }
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  using namespace tc;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kWaitNs) return false;
+  }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 
 }  // namespace
 
 template <int BS, int D>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kThreads, BS == 64 ? 2 : 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const AttendArgs a) {
   using C = TcCfg<BS, D>;
   using namespace tc;
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ uint32_t tmem_base_s;
-  __shared__ int blocks[kMaxSel];
-  __shared__ int nblk_s;
-  __shared__ int abort_s;
-
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* sm = smem_raw + (base - raw);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The swizzled tiles need 1024-byte alignment; the kernel declares no
+  // static shared memory, so the dynamic region starts the CTA's window.
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicExch(a.status, kDevMisaligned);
+    return;
+  }
+  uint8_t* sm = smem_raw;
+  uint32_t& tmem_base_s = *reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
+  int& abort_s = *reinterpret_cast<int*>(sm + C::kOffMisc + 4);
+  volatile int* abort_flag = &abort_s;
+  const uint32_t base = smem_u32(smem_raw);
   const uint32_t sQ = base + C::kOffQ, sK = base + C::kOffK, sV = base + C::kOffV, sP = base + C::kOffP;
   uint8_t* pP = sm + C::kOffP;
   const uint32_t bar0 = base + C::kOffBar;
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x;
-  const int j = tile % a.nb;
-  const int hq = (tile / a.nb) % a.Hq;
-  const int b = tile / (a.nb * a.Hq);
-  const int hkv = hq / (a.Hq / a.Hkv);
+  const int ntiles = a.B * a.Hq * a.nb;
+  const int g = a.Hq / a.Hkv;
 
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(smem_u32(&tmem_base_s), C::kCols);
     tmem_relinquish();
   }
-  if (threadIdx.x == 32) {
-    for (int i = 0; i < 7; ++i) mbar_init(BAR(i), 1);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kQBuf; ++i) { mbar_init(BAR(C::bQFull + i), 1); mbar_init(BAR(C::bQEmpty + i), 1); }
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(BAR(C::bKFull + i), 1);
+      mbar_init(BAR(C::bKEmpty + i), 1);
+      mbar_init(BAR(C::bVFull + i), 1);
+      mbar_init(BAR(C::bVEmpty + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) { mbar_init(BAR(C::bSFull + i), 1); mbar_init(BAR(C::bPVDone + i), 1); }
+    for (int i = 0; i < C::kPBuf; ++i) mbar_init(BAR(C::bPFull + i), 4);
+    mbar_init(BAR(C::bOFull), 1);
+    mbar_init(BAR(C::bOFree), 4);
+    mbar_init(BAR(C::bFin), 1);
     fence_mbar_init();
     abort_s = 0;
-  }
-  if (threadIdx.x == 64) {
-    const int32_t* row = a.sel + static_cast<size_t>(tile) * a.nsel;
-    int n = 0;
-    for (int e = 0; e < a.nsel; ++e) {
-      const int id = row[e];
-      if (id < 0) continue;
-      if (id > j || id >= a.nb) { atomicExch(a.status, kDevBadSelection); continue; }
-      blocks[n++] = id;
-    }
-    nblk_s = n;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
-  const uint32_t tS = tmem + C::kColS, tO = tmem + C::kColO;
-  const int nblk = nblk_s;
-  const int tok0 = b * a.S;                   // first token row of sequence b
 
-  if (nblk == 0) {                            // nothing selected: the output is zero
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
-    for (int e = threadIdx.x; e < BS * D / 8; e += blockDim.x) {
-      const int rr = e / (D / 8), c8 = e % (D / 8);
-      *reinterpret_cast<uint4*>(out + ((static_cast<size_t>(tok0) + static_cast<size_t>(j) * BS + rr) * a.Hq + hq) * D +
-                                c8 * 8) = make_uint4(0, 0, 0, 0);
-    }
-    tc_fence_before();
-    __syncthreads();
-    __syncwarp();
-    if (warp == 0) tmem_dealloc(tmem, C::kCols);
-    return;
-  }
-
-  const uint32_t idS = idesc_bf16_f32(BS, BS, 0, 0);
-  const uint32_t idPV = idesc_bf16_f32(BS, D, 0, 1);
-  int issued = 0;                             // K/V blocks whose TMA thread 0 issued
-
-  auto issue_kv = [&](int n, int s) {
-    const uint32_t bar = BAR(kBarKV + s);
-    mbar_expect_tx(bar, 2 * C::kTileBytes);
-    const int row = tok0 + blocks[n] * BS;
-#pragma unroll
-    for (int g = 0; g < D / 64; ++g) {
-      tma_load_3d(sK + s * C::kTileBytes + g * C::kRegion, &tmK, bar, g * 64, hkv, row);
-      tma_load_3d(sV + s * C::kTileBytes + g * C::kRegion, &tmV, bar, g * 64, hkv, row);
-    }
-  };
-  auto issue_s = [&](int s) {
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off = (kk / 4) * C::kRegion + (kk % 4) * 32;
-      mma_bf16(tS, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK + s * C::kTileBytes + off, 16, 1024),
-               idS, kk > 0);
-    }
-    mma_commit(BAR(kBarS));
-  };
   auto fail = [&]() {
     atomicExch(a.status, kDevWaitTimeout);
-    abort_s = 1;
+    *abort_flag = 1;
   };
 
-  bool t0_fail = false;
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&tmQ);
-    prefetch_tmap(&tmK);
-    prefetch_tmap(&tmV);
-    mbar_expect_tx(BAR(kBarQ), C::kTileBytes);
-#pragma unroll
-    for (int g = 0; g < D / 64; ++g) tma_load_3d(sQ + g * C::kRegion, &tmQ, BAR(kBarQ), g * 64, hq, tok0 + j * BS);
-    for (int n = 0; n < C::kStages && n < nblk; ++n) { issue_kv(n, n); ++issued; }
-    if (mbar_wait(BAR(kBarQ), 0, kWaitNs) && mbar_wait(BAR(kBarKV), 0, kWaitNs)) {
-      tc_fence_after();
-      issue_s(0);
-    } else {
-      t0_fail = true;
-      fail();
-      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(BAR(kBarS)) : "memory");
-    }
-  }
-
-  const bool has_row = (BS == 128) || (lane < 16);
-  const int r = (BS == 128) ? (warp * 32 + lane) : (warp * 16 + lane);
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-  const float sl2 = a.scale * 1.4426950408889634f;   // scores in log2 units
-  float m_used = -INFINITY, l_sum = 0.f;
-  bool aborted = false;
-
-  for (int n = 0; n < nblk; ++n) {
-    const int s = n % C::kStages;
-    bool bad = !mbar_wait(BAR(kBarS), n & 1, kWaitNs);
-    __syncwarp();                               // tcgen05.ld is warp-collective
-    tc_fence_after();
-    float sv[BS];
-#pragma unroll
-    for (int c = 0; c < BS / 32; ++c) tmem_ld32(tS + lane_base + c * 32, sv + c * 32);
-    tmem_ld_wait();
-    float alpha = 1.f;
-    bool rescale = false;
-    if (has_row) {
-      const bool diag = blocks[n] == j;
-      float mb = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BS; ++c) {
-        float x = sv[c] * sl2;
-        if (diag && c > r) x = -INFINITY;
-        sv[c] = x;
-        mb = fmaxf(mb, x);
+  if (warp == 0) {
+    // ----------------------------------------------------------- producers
+    // Lane 0 loads Q and K, lane 1 loads V: a K stage is refilled as soon as
+    // the S MMA that read it completes, independently of the later PV.
+    if (lane < 2) {
+      const bool is_k = lane == 0;
+      if (is_k) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+      } else {
+        prefetch_tmap(&tmV);
       }
-      if (mb > m_used + 8.f) {
-        alpha = exp2f(m_used - mb);
-        rescale = n > 0;
-        m_used = mb;
-        l_sum *= alpha;
-      }
-      uint8_t* prow = pP + r * 128;
-#pragma unroll
-      for (int q8 = 0; q8 < BS / 8; ++q8) {
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = exp2f(sv[q8 * 8 + e] - m_used);
-          l_sum += p[e];
+      const int bFull = is_k ? C::bKFull : C::bVFull, bEmpty = is_k ? C::bKEmpty : C::bVEmpty;
+      const uint32_t ring = is_k ? sK : sV;
+      const void* tm = is_k ? static_cast<const void*>(&tmK) : static_cast<const void*>(&tmV);
+      int itv = 0, gb = 0;                      // non-empty tiles, blocks issued
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int j = tile % a.nb, hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq);
+        const int32_t* row = a.sel + static_cast<size_t>(tile) * a.nsel;
+        int nblk = 0;
+        for (int e = 0; e < a.nsel; ++e) {
+          const int id = row[e];
+          if (valid_id(id, j)) ++nblk;
+          else if (is_k && id >= 0) atomicExch(a.status, kDevBadSelection);
         }
-        uint32_t w[4];
+        if (nblk == 0) continue;
+        const int tok0 = b * a.S;
+        if (is_k) {
+          const int qs = itv % C::kQBuf;
+          if (itv >= C::kQBuf && !wait_bar(BAR(C::bQEmpty + qs), ((itv / C::kQBuf) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(BAR(C::bQFull + qs), C::kTile);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          __nv_bfloat162 h = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
-          w[e] = *reinterpret_cast<uint32_t*>(&h);
+          for (int gg = 0; gg < D / 64; ++gg)
+            tma_load_3d(sQ + qs * C::kTile + gg * C::kRegion, &tmQ, BAR(C::bQFull + qs), gg * 64, hq,
+                        tok0 + j * BS);
         }
-        const int region = q8 / 8, chunk = (q8 % 8) ^ (r % 8);
-        *reinterpret_cast<uint4*>(prow + region * C::kRegion + chunk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        const int hkv = hq / g;
+        for (int e = 0; e < a.nsel && ok; ++e) {
+          const int id = row[e];
+          if (!valid_id(id, j)) continue;
+          const int st = gb % C::kStages;
+          if (gb >= C::kStages && !wait_bar(BAR(bEmpty + st), ((gb / C::kStages) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t bar = BAR(bFull + st);
+          mbar_expect_tx(bar, C::kTile);
+#pragma unroll
+          for (int gg = 0; gg < D / 64; ++gg)
+            tma_load_3d(ring + st * C::kTile + gg * C::kRegion, tm, bar, gg * 64, hkv, tok0 + id * BS);
+          ++gb;
+        }
+        ++itv;
+      }
+      if (!ok) {
+        fail();
+        // Loads already issued: the last one of each stage completes after the
+        // earlier ones of that stage.
+        for (int st = 0; st < C::kStages; ++st) {
+          int last = -1;
+          for (int n = st; n < gb; n += C::kStages) last = n;
+          if (last >= 0) mbar_wait(BAR(bFull + st), (last / C::kStages) & 1, kWaitNs);
+        }
       }
     }
-    __syncwarp();
-    if (__any_sync(0xffffffffu, rescale)) {
-      float o[32];
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16_f32(BS, BS, 0, 0);
+      const uint32_t idPV = idesc_bf16_f32(BS, D, 0, 1);
+      const uint32_t tO = tmem + C::kColO;
+      int itv = 0, g0 = 0;
+      bool ok = true;
+      auto issue_s = [&](int gblk, int qs) -> bool {
+        const int st = gblk % C::kStages;
+        if (!wait_bar(BAR(C::bKFull + st), (gblk / C::kStages) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t tS = tmem + C::kColS + (gblk & 1) * BS;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        tmem_ld32(tO + lane_base + c * 32, o);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] *= alpha;
-        tmem_st32(tO + lane_base + c * 32, o);
-      }
-      tmem_st_wait();
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    if (__syncthreads_or(bad || t0_fail || abort_s)) {
-      aborted = true;
-      if (bad && threadIdx.x == 0) fail();
-      break;
-    }
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      const uint32_t vbase = sV + s * C::kTileBytes;
-#pragma unroll
-      for (int kk = 0; kk < BS / 16; ++kk) {
-        const uint32_t poff = (kk / 4) * C::kRegion + (kk % 4) * 32;
-        mma_bf16(tO, smem_desc_sw128(sP + poff, 16, 1024), smem_desc_sw128(vbase + kk * 2048, C::kRegion, 1024),
-                 idPV, (n > 0 || kk > 0) ? 1u : 0u);
-      }
-      mma_commit(BAR(kBarFree + s));
-      if (n + 1 < nblk) {
-        const int s1 = (n + 1) % C::kStages;
-        if (mbar_wait(BAR(kBarKV + s1), ((n + 1) / C::kStages) & 1, kWaitNs)) {
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * C::kRegion + (kk % 4) * 32;
+          mma_bf16(tS, smem_desc_sw128(sQ + qs * C::kTile + off, 16, 1024),
+                   smem_desc_sw128(sK + st * C::kTile + off, 16, 1024), idS, kk > 0);
+        }
+        mma_commit(BAR(C::bSFull + (gblk & 1)));
+        mma_commit(BAR(C::bKEmpty + st));
+        return true;
+      };
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int j = tile % a.nb;
+        const int32_t* row = a.sel + static_cast<size_t>(tile) * a.nsel;
+        int nblk = 0;
+        for (int e = 0; e < a.nsel; ++e) nblk += valid_id(row[e], j);
+        if (nblk == 0) continue;
+        const int qs = itv % C::kQBuf;
+        if (!wait_bar(BAR(C::bQFull + qs), (itv / C::kQBuf) & 1, abort_flag)) { ok = false; break; }
+        for (int n = 0; n < 2 && n < nblk && ok; ++n) ok = issue_s(g0 + n, qs);
+        for (int n = 0; n < nblk && ok; ++n) {
+          const int gblk = g0 + n;
+          if (!wait_bar(BAR(C::bPFull + gblk % C::kPBuf), (gblk / C::kPBuf) & 1, abort_flag)) { ok = false; break; }
+          if (n == 0 && itv > 0 && !wait_bar(BAR(C::bOFree), (itv - 1) & 1, abort_flag)) { ok = false; break; }
+          if (!wait_bar(BAR(C::bVFull + gblk % C::kStages), (gblk / C::kStages) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          issue_s(s1);
-        } else {
-          t0_fail = true;
-          fail();
-          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(BAR(kBarS)) : "memory");
-        }
-      }
-      if (!t0_fail && n + C::kStages < nblk) {
-        if (mbar_wait(BAR(kBarFree + s), (n / C::kStages) & 1, kWaitNs)) {
-          issue_kv(n + C::kStages, s);
-          ++issued;
-        } else {
-          t0_fail = true;
-          fail();
-        }
-      }
-    }
-  }
-
-  // Drain: every MMA this CTA issued, and every TMA still in flight.
-  if (threadIdx.x == 0) {
-    tc_fence_after();
-    mma_commit(BAR(kBarDone));
-    if (aborted || t0_fail) {
-      // The last load issued into each stage completes after the earlier ones.
-      for (int s = 0; s < C::kStages; ++s) {
-        int last = -1;
-        for (int n = s; n < issued; n += C::kStages) last = n;
-        if (last >= 0) mbar_wait(BAR(kBarKV + s), (last / C::kStages) & 1, kWaitNs);
-      }
-      mbar_wait(BAR(kBarQ), 0, kWaitNs);
-    }
-  }
-  const bool done = mbar_wait(BAR(kBarDone), 0, kWaitNs);
-  __syncwarp();
-  if (!done && threadIdx.x == 0) fail();
-  tc_fence_after();
-  if (done && !aborted && !__syncthreads_or(abort_s)) {
-    const float inv = 1.f / l_sum;
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
-                         ((static_cast<size_t>(tok0) + static_cast<size_t>(j) * BS + r) * a.Hq + hq) * D;
+          const uint32_t pbase = sP + (gblk % C::kPBuf) * C::kPBytes;
+          const uint32_t vbase = sV + (gblk % C::kStages) * C::kTile;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      float o[32];
-      tmem_ld32(tO + lane_base + c * 32, o);
-      tmem_ld_wait();
-      if (has_row) {
+          for (int kk = 0; kk < BS / 16; ++kk) {
+            const uint32_t poff = (kk / 4) * C::kRegion + (kk % 4) * 32;
+            mma_bf16(tO, smem_desc_sw128(pbase + poff, 16, 1024), smem_desc_sw128(vbase + kk * 2048, C::kRegion, 1024),
+                     idPV, (n > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(BAR(C::bPVDone + (gblk & 1)));
+          mma_commit(BAR(C::bVEmpty + gblk % C::kStages));
+          if (n + 2 < nblk) ok = issue_s(gblk + 2, qs);
+        }
+        if (!ok) break;
+        mma_commit(BAR(C::bQEmpty + qs));
+        mma_commit(BAR(C::bOFull));
+        g0 += nblk;
+        ++itv;
+      }
+      if (!ok) fail();
+      // Everything this thread issued has completed once bFin fires.
+      mma_commit(BAR(C::bFin));
+      mbar_wait(BAR(C::bFin), 0, kWaitNs);
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    constexpr bool kHalf = C::kHalf;
+    constexpr int kSC = C::kSCols;
+    const int sp = warp & 3;                          // TMEM subpartition of this warp
+    const int hlf = kHalf ? (lane >> 4) : 0;          // M = 64: which 32 of each 64 columns
+    const int r = kHalf ? (sp * 16 + (lane & 15)) : (sp * 32 + lane);
+    const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
+    const uint32_t tO = tmem + C::kColO + lane_base;
+    const float sl2 = a.scale * 1.4426950408889634f;  // scores in log2 units
+    int itv = 0, g0 = 0;
+    bool ok = true;
+    // O chunk k of this thread: columns 64k + 32 hlf .. +31 (M = 64) or 32k .. +31.
+    auto o_ld = [&](int k, float* o) {
+      if constexpr (kHalf) tmem_ld16x2_32(tO + 64 * k, o);
+      else tmem_ld32(tO + 32 * k, o);
+    };
+    auto o_st = [&](int k, const float* o) {
+      if constexpr (kHalf) tmem_st16x2_32(tO + 64 * k, o);
+      else tmem_st32(tO + 32 * k, o);
+    };
+    constexpr int kOChunks = kHalf ? D / 64 : D / 32;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      const int j = tile % a.nb, hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq);
+      const int32_t* row = a.sel + static_cast<size_t>(tile) * a.nsel;
+      int nblk = 0, diag = -1;
+      for (int e = 0; e < a.nsel; ++e) {
+        const int id = row[e];
+        if (!valid_id(id, j)) continue;
+        if (id == j) diag = nblk;
+        ++nblk;
+      }
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
+                           ((static_cast<size_t>(b) * a.S + static_cast<size_t>(j) * BS + r) * a.Hq + hq) * D;
+      if (nblk == 0) {                                 // nothing selected: zero output
+        const int c_lo = kHalf ? hlf * (D / 16) : 0, c_hi = kHalf ? c_lo + D / 16 : D / 8;
+        for (int c = c_lo; c < c_hi; ++c) reinterpret_cast<uint4*>(out)[c] = make_uint4(0, 0, 0, 0);
+        continue;
+      }
+      float m_used = -INFINITY, l_sum = 0.f;
+      for (int n = 0; n < nblk; ++n) {
+        const int gblk = g0 + n;
+        if (!wait_bar(BAR(C::bSFull + (gblk & 1)), (gblk >> 1) & 1, abort_flag)) { ok = false; break; }
+        __syncwarp();
+        tc_fence_after();
+        float sv[kSC];
+        const uint32_t tS = tmem + C::kColS + (gblk & 1) * BS + lane_base;
+        if constexpr (kHalf) {
+          tmem_ld16x2_32(tS, sv);
+        } else {
+#pragma unroll
+          for (int c = 0; c < BS / 32; ++c) tmem_ld32(tS + c * 32, sv + c * 32);
+        }
+        tmem_ld_wait();
+        float mb = -INFINITY;
+        const bool is_diag = n == diag;
+        const int col0 = hlf * 32;
+#pragma unroll
+        for (int c = 0; c < kSC; ++c) {
+          float x = sv[c] * sl2;
+          if (is_diag && col0 + c > r) x = -INFINITY;
+          sv[c] = x;
+          mb = fmaxf(mb, x);
+        }
+        if constexpr (kHalf) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 16));
+        float alpha = 1.f;
+        bool rescale = false;
+        if (mb > m_used + 8.f) {
+          alpha = exp2f(m_used - mb);
+          rescale = n > 0;
+          m_used = mb;
+          l_sum *= alpha;
+        }
+        // O holds PV(n-1) once it completes; the P buffer is free once the PV
+        // that last read it completed.
+        const bool need_o = __any_sync(0xffffffffu, rescale);
+        if (need_o && !wait_bar(BAR(C::bPVDone + ((gblk - 1) & 1)), ((gblk - 1) >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (gblk >= C::kPBuf &&
+            !wait_bar(BAR(C::bPVDone + ((gblk - C::kPBuf) & 1)), ((gblk - C::kPBuf) >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        tc_fence_after();
+        if (need_o) {
+          float o[32];
+#pragma unroll
+          for (int k = 0; k < kOChunks; ++k) {
+            o_ld(k, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            o_st(k, o);
+          }
+          tmem_st_wait();
+        }
+        uint8_t* prow = pP + (gblk % C::kPBuf) * C::kPBytes + r * 128;
+#pragma unroll
+        for (int q = 0; q < kSC / 8; ++q) {
+          const int q8 = hlf * 4 + q;                  // 8-column chunk of the row
+          float p[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            p[e] = exp2f(sv[q * 8 + e] - m_used);
+            l_sum += p[e];
+          }
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
+            w[e] = *reinterpret_cast<uint32_t*>(&h);
+          }
+          const int region = q8 / 8, chunk = (q8 % 8) ^ (r % 8);
+          *reinterpret_cast<uint4*>(prow + region * C::kRegion + chunk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::bPFull + gblk % C::kPBuf));
+      }
+      if (!ok) break;
+      // Epilogue: wait for the last PV of this tile, then O / sum -> bf16.
+      if (!wait_bar(BAR(C::bOFull), itv & 1, abort_flag)) { ok = false; break; }
+      __syncwarp();
+      tc_fence_after();
+      float l_row = l_sum;
+      if constexpr (kHalf) l_row += __shfl_xor_sync(0xffffffffu, l_sum, 16);
+      const float inv = 1.f / l_row;
+#pragma unroll
+      for (int k = 0; k < kOChunks; ++k) {
+        float o[32];
+        o_ld(k, o);
+        tmem_ld_wait();
+        const int col = kHalf ? 64 * k + 32 * hlf : 32 * k;
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           uint32_t w[4];
@@ -321,15 +445,25 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             __nv_bfloat162 h = __floats2bfloat162_rn(o[q8 * 8 + 2 * e] * inv, o[q8 * 8 + 2 * e + 1] * inv);
             w[e] = *reinterpret_cast<uint32_t*>(&h);
           }
-          *reinterpret_cast<uint4*>(out + c * 32 + q8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(out + col + q8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::bOFree));
+      g0 += nblk;
+      ++itv;
     }
+    if (!ok) fail();
   }
+
   tc_fence_before();
   __syncthreads();
-  __syncwarp();
-  if (warp == 0) tmem_dealloc(tmem, C::kCols);
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, C::kCols);
+  }
 }
 
 namespace {
@@ -374,8 +508,17 @@ cudaError_t launch_tc(const AttendArgs& a, cudaStream_t st) {
   auto k = attend_tc_kernel<BS, D>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(a.B) * a.Hq * a.nb;
-  k<<<grid, 128, C::kSmem, st>>>(mq, mk, mv, a);
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, C::kSmem)) != cudaSuccess) return e;
+  // Tensor memory: at most 512 columns per SM.
+  per_sm = per_sm < 512 / C::kCols ? per_sm : 512 / C::kCols;
+  if (per_sm < 1) per_sm = 1;
+  const long long ntiles = static_cast<long long>(a.B) * a.Hq * a.nb;
+  const long long want = static_cast<long long>(sms) * per_sm;
+  const unsigned grid = static_cast<unsigned>(ntiles < want ? ntiles : want);
+  k<<<grid, kThreads, C::kSmem, st>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 

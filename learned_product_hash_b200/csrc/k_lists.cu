@@ -9,63 +9,65 @@
 // load).  Keeping the first cap blocks makes storage causal: whether block i
 // is stored depends only on blocks before it.
 //
-// This is a stable counting sort by (address, block id).  One warp walks the
-// blocks 32 at a time in order; lanes with equal addresses find each other
-// with __match_any_sync, the lowest of them adds the group's size to the
-// address's shared-memory counter (a warp-aggregated atomic) and every lane's
-// rank is that counter's old value plus its rank inside the group.  The other
-// warps meanwhile pad the lists with -1.
+// This is a stable counting sort by (address, block id) in shared memory:
+// the head's addresses are staged in shared memory once; the blocks are taken
+// in chunks of 256 in order; each thread counts the earlier blocks of its
+// chunk with the same address and adds the address's running count from the
+// earlier chunks; then the running counts are bumped, lanes of a warp with
+// equal addresses finding each other with __match_any_sync so that only the
+// lowest of them adds the group's size (a warp-aggregated atomic).  The
+// lists arrive padded with -1: the summary kernel of the key side, which runs
+// just before on the same stream, writes the padding.
 
 #include "common.cuh"
 #include "kernels.h"
 
 namespace mdr {
 
-__global__ void __launch_bounds__(1024)
+constexpr int kListThreads = 256;
+
+__global__ void __launch_bounds__(kListThreads)
 lists_kernel(const ListsArgs a) {
-  extern __shared__ int32_t cnt[];                 // [A]
+  extern __shared__ int32_t cnt[];                 // [A] running counts, then [nb] addresses
   __shared__ int32_t s_ovf, s_max;
   const int bh = blockIdx.x;
-  const size_t nlist = static_cast<size_t>(a.A) * a.cap;
-  int32_t* lists = a.lists + static_cast<size_t>(bh) * nlist;
+  int32_t* lists = a.lists + static_cast<size_t>(bh) * static_cast<size_t>(a.A) * a.cap;
   const int32_t* addr = a.addr + static_cast<size_t>(bh) * a.nb;
   const int tid = threadIdx.x, lane = tid & 31;
+  int32_t* saddr = cnt + a.A;
 
-  for (int x = tid; x < a.A; x += blockDim.x) cnt[x] = 0;
+  for (int x = tid; x < a.A; x += kListThreads) cnt[x] = 0;
+  for (int x = tid; x < a.nb; x += kListThreads) saddr[x] = addr[x];   // one coalesced read
   if (tid == 0) { s_ovf = 0; s_max = 0; }
-  if ((nlist & 3) == 0 && (reinterpret_cast<uintptr_t>(lists) & 15) == 0) {
-    int4* l4 = reinterpret_cast<int4*>(lists);
-    const int4 m1 = make_int4(-1, -1, -1, -1);
-    for (size_t x = tid; x < nlist / 4; x += blockDim.x) l4[x] = m1;
-  } else {
-    for (size_t x = tid; x < nlist; x += blockDim.x) lists[x] = -1;
-  }
   __syncthreads();
 
-  if (tid < 32) {
-    for (int base = 0; base < a.nb; base += 32) {
-      const int i = base + lane;
-      const bool valid = i < a.nb;
-      const unsigned vm = __ballot_sync(0xffffffffu, valid);
-      if (valid) {
-        const int ad = addr[i];
-        const unsigned peers = __match_any_sync(vm, ad);
-        const int leader = __ffs(peers) - 1;
-        const int inner = __popc(peers & ((1u << lane) - 1u));
-        int before = 0;
-        if (lane == leader) before = atomicAdd(&cnt[ad], __popc(peers));
-        before = __shfl_sync(peers, before, leader);
-        const int rank = before + inner;
-        if (rank < a.cap) lists[static_cast<size_t>(ad) * a.cap + rank] = i;
-      }
-      __syncwarp();
+  // Chunks of kListThreads blocks, in order.  Within a chunk, block i's rank
+  // among the chunk's earlier blocks of its address is counted directly;
+  // adding the address's count from earlier chunks gives rank(i).
+  for (int c0 = 0; c0 < a.nb; c0 += kListThreads) {
+    const int i = c0 + tid;
+    const bool valid = i < a.nb;
+    const int ad = valid ? saddr[i] : -1;
+    int rank = 0;
+    if (valid) {
+      for (int k = c0; k < i; ++k) rank += saddr[k] == ad;
+      rank += cnt[ad];
+      if (rank < a.cap) lists[static_cast<size_t>(ad) * a.cap + rank] = i;
     }
+    __syncthreads();                               // every rank read the old counts
+    // Count update: lanes of a warp with equal addresses add once, through
+    // their lowest lane (a warp-aggregated atomic).
+    const unsigned vm = __ballot_sync(0xffffffffu, valid);
+    if (valid) {
+      const unsigned peers = __match_any_sync(vm, ad);
+      if (lane == __ffs(peers) - 1) atomicAdd(&cnt[ad], __popc(peers));
+    }
+    __syncthreads();
   }
-  __syncthreads();
 
   int ovf = 0, mx = 0;
   int32_t* load = a.load + static_cast<size_t>(bh) * a.A;
-  for (int x = tid; x < a.A; x += blockDim.x) {
+  for (int x = tid; x < a.A; x += kListThreads) {
     const int c = cnt[x];
     load[x] = c;
     ovf += c > a.cap ? c - a.cap : 0;
@@ -82,11 +84,11 @@ lists_kernel(const ListsArgs a) {
 }
 
 cudaError_t launch_lists(const ListsArgs& a, cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(a.A) * sizeof(int32_t);
+  const size_t smem = static_cast<size_t>(a.A + a.nb) * sizeof(int32_t);
   cudaError_t e = cudaFuncSetAttribute(lists_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  lists_kernel<<<a.B * a.H, 1024, smem, st>>>(a);
+  lists_kernel<<<a.B * a.H, kListThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 

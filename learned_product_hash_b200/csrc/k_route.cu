@@ -3,12 +3,14 @@
 // One warp per route (sequence b, query head hq, query block j).  The probed
 // addresses are the product of the p best codewords of each subspace (first
 // subspace's rank slowest).  Each probed address owns cap candidate slots:
-// the stored blocks of its list that are remote-eligible, i <= j - L; lists
-// hold ascending ids, so those are a prefix and the walk stops at the first
-// later block.  Candidates are scored by <qbar_j, kbar_i> in float32 (lanes
-// split the head dimension, a butterfly sum combines them), the R best are
-// kept (higher score first, lower id on equal scores) and written in
-// ascending id order, -1 padded; then the local blocks j-L+1..j.
+// the stored blocks of its list that are remote-eligible, i <= j - L.  The
+// lanes look up all probes' list lengths at once, prefix-sum them into slot
+// offsets, and read the stored slots 32 at a time, so a route costs a few
+// dependent memory round trips, not one per probe.  Each lane scores whole
+// candidates by <qbar_j, kbar_i> in float32 (coordinates in order), in
+// batches of at most 224 merged into the running top R (higher score first,
+// lower id on equal scores); the R winners are written in ascending id
+// order, -1 padded; then the local blocks j-L+1..j.
 // Pages: "Monodratic Claims Learned Routing Can Make Sparse Causal Attention
 // More Selective", section "Monodratic Turns Sparse Attention Into a
 // Retrieval Decision" (probe, candidates, rerank, fixed number of remote
@@ -24,14 +26,26 @@ namespace mdr {
 
 constexpr int kRouteWarps = 4;
 
+// Candidates are scored and merged into the running top R in batches of at
+// most kBatch, so a warp's shared memory does not grow with probes^P * cap.
+constexpr int kBatch = 224;
+// Shared memory of one warp, in 4-byte words: the query summary (D <= 128),
+// probe addresses (64), slot offsets (65, padded to 68), candidate ids and
+// scores (kBatch + 32 each: a batch, then the running winners).
+constexpr int kRouteWarpWords = 128 + 64 + 68 + 2 * (kBatch + 32);
+
 __global__ void __launch_bounds__(kRouteWarps * 32)
 route_kernel(const RouteArgs a) {
   extern __shared__ int32_t rsmem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nprobe = [&] { int n = 1; for (int s = 0; s < a.P; ++s) n *= a.probes; return n; }();
-  const int cmax = nprobe * a.cap;
-  int32_t* cand = rsmem + warp * 2 * cmax;
-  float* score = reinterpret_cast<float*>(cand + cmax);
+  int nprobe = 1;
+  for (int s = 0; s < a.P; ++s) nprobe *= a.probes;
+  int32_t* wsm = rsmem + warp * kRouteWarpWords;
+  float* qs = reinterpret_cast<float*>(wsm);
+  int32_t* paddr = wsm + 128;
+  int32_t* offs = paddr + 64;
+  int32_t* cand = offs + 68;                       // [kBatch) batch, [kBatch, kBatch+R) winners
+  float* score = reinterpret_cast<float*>(cand + kBatch + 32);
 
   const long long route = static_cast<long long>(blockIdx.x) * kRouteWarps + warp;
   const long long nroutes = static_cast<long long>(a.B) * a.Hq * a.nb;
@@ -41,70 +55,116 @@ route_kernel(const RouteArgs a) {
   const int b = static_cast<int>(route / (static_cast<long long>(a.nb) * a.Hq));
   const int hkv = hq / (a.Hq / a.Hkv);
   const long long bh = static_cast<long long>(b) * a.Hkv + hkv;
-
-  // Query summary: lane holds coordinates lane + 32 m.
-  float qv[4];
-  const float* qb = a.qbar + route * a.D;
-  const int dm = a.D / 32;
-#pragma unroll
-  for (int m = 0; m < 4; ++m) qv[m] = m < dm ? qb[lane + 32 * m] : 0.f;
-
-  // Candidates in slot order.
-  const int32_t* qc = a.qcodes + route * a.P * a.probes;
   const int32_t* lists = a.lists + bh * a.A * a.cap;
-  int n = 0;
   const int last = j - a.L;                        // highest eligible block
-  for (int pr = 0; pr < nprobe; ++pr) {
-    int ad = 0, rem = pr, div = nprobe;
-    for (int s = 0; s < a.P; ++s) {
-      div /= a.probes;
-      const int rank = rem / div;
-      rem -= rank * div;
-      ad = ad * a.K + qc[s * a.probes + rank];
-    }
-    int cnt = a.load[bh * a.A + ad];
-    cnt = cnt < a.cap ? cnt : a.cap;
-    const int32_t* lst = lists + static_cast<long long>(ad) * a.cap;
-    for (int base = 0; base < cnt; base += 32) {
-      const int e = base + lane;
-      const int id = e < cnt ? lst[e] : INT_MAX;
-      const bool ok = id <= last;
-      const unsigned m = __ballot_sync(0xffffffffu, ok);
-      if (ok) cand[n + __popc(m & ((1u << lane) - 1u))] = id;
-      n += __popc(m);
-      if (__ballot_sync(0xffffffffu, e < cnt && !ok)) break;   // ascending ids: the rest are later
-    }
-  }
-  __syncwarp();
 
-  // Rerank.
-  const float* kb = a.kbar + bh * a.nb * a.D;
-  for (int c = 0; c < n; ++c) {
-    const float* kr = kb + static_cast<long long>(cand[c]) * a.D;
-    float acc = 0.f;
+  for (int d = lane; d < a.D; d += 32) qs[d] = a.qbar[route * a.D + d];
+
+  // Probed addresses and their stored counts, all probes at once: lane l
+  // owns probes l and l + 32 (first subspace's rank slowest).
+  const int32_t* qc = a.qcodes + route * a.P * a.probes;
+  int c0 = 0, c1 = 0;
 #pragma unroll
-    for (int m = 0; m < 4; ++m)
-      if (m < dm) acc = __fmaf_rn(qv[m], kr[lane + 32 * m], acc);
-    acc = warp_sum(acc);
-    if (lane == 0) score[c] = acc;
+  for (int h = 0; h < 2; ++h) {
+    const int pr = lane + 32 * h;
+    if (pr < nprobe) {
+      int ad = 0, rem = pr, div = nprobe;
+      for (int s = 0; s < a.P; ++s) {
+        div /= a.probes;
+        const int rank = rem / div;
+        rem -= rank * div;
+        ad = ad * a.K + qc[s * a.probes + rank];
+      }
+      paddr[pr] = ad;
+      const int cl = a.load[bh * a.A + ad];
+      if (h == 0) c0 = cl < a.cap ? cl : a.cap;
+      else c1 = cl < a.cap ? cl : a.cap;
+    }
   }
+  // Exclusive prefix sums of the counts give each probe's first slot.
+  int s0 = c0, s1 = c1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u0 = __shfl_up_sync(0xffffffffu, s0, o);
+    const int u1 = __shfl_up_sync(0xffffffffu, s1, o);
+    if (lane >= o) { s0 += u0; s1 += u1; }
+  }
+  const int t0 = __shfl_sync(0xffffffffu, s0, 31);
+  const int total = t0 + __shfl_sync(0xffffffffu, s1, 31);
+  if (lane < nprobe) offs[lane] = s0 - c0;
+  if (lane + 32 < nprobe) offs[lane + 32] = t0 + s1 - c1;
+  if (lane == 0) offs[nprobe] = total;
   __syncwarp();
 
-  // Top R: R rounds of a warp-wide best, removing the winner each time.
-  int mine = INT_MAX;                               // lane r keeps the r-th winner
-  for (int r = 0; r < a.R; ++r) {
-    float bs = -INFINITY;
-    int bi = INT_MAX, bc = -1;
-    for (int c = lane; c < n; c += 32) {
-      const int id = cand[c];
-      if (id >= 0 && better(score[c], id, bs, bi)) { bs = score[c]; bi = id; bc = c; }
+  // Read every stored slot of the probed lists, 32 per step, keep the
+  // remote-eligible blocks; every kBatch of them (and at the end) score the
+  // batch and merge it with the running winners.
+  const float* kb = a.kbar + bh * a.nb * a.D;
+  int nbuf = 0, n = 0, nwin = 0;
+  int mine = INT_MAX;                              // lane r: r-th winner id
+  for (int base = 0; base < total; base += 32) {
+    const int e = base + lane;
+    int id = INT_MAX;
+    if (e < total) {
+      int lo = 0, hi = nprobe - 1;                 // probe p with offs[p] <= e < offs[p+1]
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offs[mid] <= e) lo = mid; else hi = mid - 1;
+      }
+      id = lists[static_cast<long long>(paddr[lo]) * a.cap + (e - offs[lo])];
     }
-    float ws = bs;
-    int wi = bi;
-    warp_best(ws, wi);
-    if (wi == INT_MAX) break;
-    if (bi == wi && bc >= 0) cand[bc] = -1;
-    if (lane == r) mine = wi;
+    const bool ok = id <= last;
+    const unsigned m = __ballot_sync(0xffffffffu, ok);
+    if (ok) cand[nbuf + __popc(m & ((1u << lane) - 1u))] = id;
+    nbuf += __popc(m);
+    n += __popc(m);
+    if (nbuf <= kBatch - 32 && base + 32 < total) continue;
+    __syncwarp();
+    // Score the batch: each lane whole candidates, float32, coordinates in order.
+    for (int c = lane; c < nbuf; c += 32) {
+      const float4* kr = reinterpret_cast<const float4*>(kb + static_cast<long long>(cand[c]) * a.D);
+      const float4* q4 = reinterpret_cast<const float4*>(qs);
+      float acc = 0.f;
+      for (int d4 = 0; d4 < a.D / 4; ++d4) {
+        const float4 kv = __ldg(kr + d4);
+        const float4 qv = q4[d4];
+        acc = __fmaf_rn(qv.x, kv.x, acc);
+        acc = __fmaf_rn(qv.y, kv.y, acc);
+        acc = __fmaf_rn(qv.z, kv.z, acc);
+        acc = __fmaf_rn(qv.w, kv.w, acc);
+      }
+      score[c] = acc;
+    }
+    __syncwarp();
+    // Top R of the batch and the previous winners (higher score, lower id).
+    int newwin = 0;
+    float myscore = -INFINITY;
+    mine = INT_MAX;
+    for (int r = 0; r < a.R; ++r) {
+      float bs = -INFINITY;
+      int bi = INT_MAX, bc = -1;
+      for (int c = lane; c < nbuf; c += 32) {
+        const int cid = cand[c];
+        if (cid >= 0 && better(score[c], cid, bs, bi)) { bs = score[c]; bi = cid; bc = c; }
+      }
+      if (lane < nwin) {
+        const int c = kBatch + lane;
+        const int cid = cand[c];
+        if (cid >= 0 && better(score[c], cid, bs, bi)) { bs = score[c]; bi = cid; bc = c; }
+      }
+      float ws = bs;
+      int wi = bi;
+      warp_best(ws, wi);
+      if (wi == INT_MAX) break;
+      if (bi == wi && bc >= 0) cand[bc] = -1;
+      if (lane == r) { mine = wi; myscore = ws; }
+      ++newwin;
+      __syncwarp();
+    }
+    __syncwarp();
+    if (lane < newwin) { cand[kBatch + lane] = mine; score[kBatch + lane] = myscore; }
+    nwin = newwin;
+    nbuf = 0;
     __syncwarp();
   }
 
@@ -129,7 +189,7 @@ route_kernel(const RouteArgs a) {
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   int nprobe = 1;
   for (int s = 0; s < a.P; ++s) nprobe *= a.probes;
-  const size_t smem = static_cast<size_t>(kRouteWarps) * 2 * nprobe * a.cap * sizeof(int32_t);
+  const size_t smem = static_cast<size_t>(kRouteWarps) * kRouteWarpWords * sizeof(int32_t);
   cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;

@@ -4,7 +4,7 @@
 #include <cmath>
 #include <cstring>
 
-#include "../../include/mdr.h"
+#include "mdr.h"
 #include "kernels.h"
 
 namespace {
@@ -53,6 +53,7 @@ mdr_status check(const mdr_config* c) {
   if (np < 0 || np > 64 || np * c->cap > 4096) return MDR_ERR_UNSUPPORTED;
   if (c->dtype == MDR_BF16 && (!is_pow2_in(c->block, {64, 128}) || !is_pow2_in(c->D, {64, 128})))
     return MDR_ERR_UNSUPPORTED;
+  if (c->S / c->block > 32768) return MDR_ERR_UNSUPPORTED;
   const long long tokens = static_cast<long long>(c->B) * c->S;
   if (tokens * (c->Hq + c->Hkv) * c->D > (1LL << 40)) return MDR_ERR_UNSUPPORTED;
   return MDR_OK;
@@ -185,6 +186,8 @@ mdr_status mdr_build_index(const mdr_config* cfg, const void* k, const float* co
   SummarizeArgs a;
   fill_common(a, cfg, codebooks);
   a.x[1] = k; a.xbar[1] = idx->kbar; a.addr = idx->addr;
+  a.lists_fill = idx->lists;
+  a.lists_per_seq = static_cast<size_t>(cfg->Hkv) * ipow(cfg->K, cfg->P) * cfg->cap;
   MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
   return run_lists(cfg, idx, st);
 }
@@ -253,6 +256,8 @@ static mdr_status forward_impl(const mdr_config* cfg, const void* q, const void*
   a.xrot[0] = at<void>(ws, l.qrot); a.xrot[1] = at<void>(ws, l.krot);
   a.xbar[0] = qbar; a.xbar[1] = idx->kbar;
   a.qcodes = qcodes; a.addr = idx->addr;
+  a.lists_fill = idx->lists;
+  a.lists_per_seq = static_cast<size_t>(cfg->Hkv) * ipow(cfg->K, cfg->P) * cfg->cap;
   MDR_TRY(mark(0));
   MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
   MDR_TRY(mark(1));

@@ -23,7 +23,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/mdr.h"
+#include "mdr.h"
 #include "kernels.h"
 
 namespace {
