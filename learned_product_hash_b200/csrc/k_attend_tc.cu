@@ -9,34 +9,36 @@
 // Persistent, warp-specialised kernel, one CTA per SM.  A CTA walks the
 // (b, hq, j) tiles blockIdx.x, blockIdx.x + gridDim.x, ... (consecutive CTAs
 // take consecutive query blocks of one head, so that head's K/V stays in L2).
-//   warp 0        TMA producers: lane 0 loads the Q tile of each query block
-//                 into a Q ring and the K tile of every selected block into a
-//                 K ring, lane 1 the V tiles into a V ring (128-byte swizzle,
-//                 mbarrier expect-tx).  A K stage is refilled once the S MMA
-//                 that read it completed, a V stage once its PV completed.
-//   warp 1        MMA issuer (one lane).  The selected blocks of a tile are
-//                 taken in groups of 128 keys: two consecutive 64-token
-//                 blocks (their K tiles sit in adjacent stages of the K ring,
-//                 which is laid out so that they form one 128-row operand),
-//                 or one 128-token block.  S = Q K^T (M = bs, N = keys of
-//                 the group, K = D) goes into one of two TMEM S buffers; O +=
-//                 P V (M = bs, N = D, 16 keys per MMA, V read MN-major from
-//                 its TMA tile) into one of two TMEM O accumulators,
-//                 alternating by tile.  S of the next group is issued before
-//                 the PV of the current one, across tile boundaries.  (A
-//                 tcgen05.mma costs about 60 cycles however small it is, so
-//                 wider N per instruction is what keeps the tensor pipe busy.)
-//   warps 2..5    softmax: one query row per thread (two threads per row for
-//                 bs = 64, whose accumulator rows fill lanes 0-15 of each
+// The selected blocks of a tile are taken in groups of 128 keys: two
+// consecutive 64-token blocks, or one 128-token block.
+//   warp 0        reads each sel row once (warp-parallel, ballot compaction)
+//                 into a shared-memory ring of tile descriptors, then lane 0
+//                 loads the Q tile and each group's K tiles by TMA into a
+//                 ring of group slots (laid out so that a group's two K tiles
+//                 form one 128-row, 128-byte-swizzled operand).
+//   warp 10       loads each group's V tiles into a second ring of slots.
+//   warp 1        MMA issuer (one lane): S = Q K^T (M = bs, N = keys of the
+//                 group, K = D) into one of two TMEM S buffers, O += P V (M =
+//                 bs, N = D, 16 keys per MMA, V read MN-major from its TMA
+//                 tile) into one of two TMEM O accumulators, alternating by
+//                 tile.  S of the next group is issued before the PV of the
+//                 current one, across tile boundaries.  One full/empty
+//                 mbarrier pair per group slot keeps waits and commits at a
+//                 few per group (each costs tens of cycles; a tcgen05.mma
+//                 about 60 however small it is).
+//   warps 2..9    softmax, two warps per TMEM subpartition, each taking 64 of
+//                 a group's 128 columns: rows of the accumulator (two threads
+//                 per row for bs = 64, whose rows fill lanes 0-15 of each
 //                 subpartition: tcgen05.ld 16x32bx2), causal mask inside the
-//                 query's own block, running maximum and sum in float32
-//                 (log2 units, ex2.approx), P = exp(S - max) as bf16 into one
-//                 of two shared-memory P buffers in the K-major 128-byte
-//                 swizzled layout the PV MMA reads.  O is rescaled in TMEM only
-//                 when the running maximum grows by more than 2^8 (exact, since
-//                 the final division uses the same maximum).  A tile's epilogue
-//                 (O / sum -> bf16 -> global) runs after the next tile's first
-//                 P is handed over, overlapping tensor-core work.
+//                 query's own block, the row maximum exchanged between the two
+//                 warps through shared memory and a named barrier, running
+//                 maximum and sum in float32 (log2 units, ex2.approx), P =
+//                 exp(S - max) as bf16 into one of two shared-memory P buffers
+//                 in the K-major swizzled layout the PV MMA reads.  O is
+//                 rescaled in TMEM only when the running maximum grows by more
+//                 than 2^8 (exact: the final division uses the same maximum).
+//                 A tile's epilogue (O / sum -> bf16 -> global) runs after the
+//                 next tile's first P is handed over, overlapping MMA work.
 // Warp w may only touch TMEM lanes 32 (w % 4) .. + 31.
 //
 // Every wait is bounded (2 s of wall time) and also gives up when another
@@ -55,35 +57,38 @@ namespace mdr {
 namespace {
 
 constexpr uint64_t kWaitNs = 2000000000ull;
-constexpr int kThreads = 224;   // warp 0 K/Q producer, 1 MMA, 2-5 softmax, 6 V producer
-constexpr int kSlots = 6;       // tile descriptors in flight
-constexpr int kSlotInts = 68;   // tile, nblk, diag, 65 ids (nsel <= 64)
+constexpr int kThreads = 352;   // 11 warps
+constexpr int kSlots = 4;       // tile descriptors in flight
+constexpr int kSlotBytes = 144; // int32 tile; int16 nblk, diag; int16 ids[64]
 
 template <int BS, int D>
 struct TcCfg {
   static constexpr bool kPair = (BS == 64);         // a group is two 64-token blocks
-  static constexpr int kGroupKeys = 128;            // keys of a full group
+  static constexpr int kGroupKeys = 128;
   static constexpr bool kBig = (BS == 128 && D == 128);
   static constexpr int kQBuf = kBig ? 1 : 2;
-  static constexpr int kKStages = (BS == 64) ? (D == 64 ? 8 : 6) : (D == 64 ? 4 : 2);   // even
-  static constexpr int kVStages = (BS == 64) ? (D == 64 ? 8 : 4) : (D == 64 ? 4 : 2);
+  static constexpr int kKSlots = (BS == 64) ? (D == 64 ? 4 : 3) : (D == 64 ? 3 : 2);
+  static constexpr int kVSlots = (BS == 64) ? (D == 64 ? 4 : 2) : (D == 64 ? 3 : 2);
   static constexpr int kPBuf = kBig ? 1 : 2;
-  static constexpr int kTile = BS * D * 2;          // one [BS x D] bf16 tile
-  static constexpr int kRegion = BS * 128;          // 64 columns of one tile, 128B-swizzled
-  static constexpr int kKRegion = kKStages * kRegion;   // K ring: region-major
+  static constexpr int kTile = BS * D * 2;          // one [BS x D] bf16 block tile
+  static constexpr int kGroupBytes = kGroupKeys * D * 2;
+  static constexpr int kRegion = BS * 128;          // 64 columns of one block tile
+  static constexpr int kGRegion = kGroupKeys * 128; // 64 columns of one group slot
+  static constexpr int kKRing = kKSlots * kGRegion; // K ring: region-major
   static constexpr int kPBytes = BS * kGroupKeys * 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBuf * kTile;
-  static constexpr int kOffV = kOffK + kKStages * kTile;
-  static constexpr int kOffP = kOffV + kVStages * kTile;
+  static constexpr int kOffV = kOffK + kKSlots * kGroupBytes;
+  static constexpr int kOffP = kOffV + kVSlots * kGroupBytes;
   static constexpr int kOffBar = kOffP + kPBuf * kPBytes;
-  static constexpr int kOffInfo = kOffBar + 8 * 64;         // tile descriptors
-  static constexpr int kOffMisc = kOffInfo + kSlots * kSlotInts * 4;   // TMEM base, abort flag
+  static constexpr int kNumBarsMax = 48;
+  static constexpr int kOffInfo = kOffBar + 8 * kNumBarsMax;
+  static constexpr int kOffXch = kOffInfo + kSlots * kSlotBytes;       // [2][2][BS] row maxima
+  static constexpr int kOffXl = kOffXch + 2 * 2 * BS * 4;             // [2][BS] row sums
+  static constexpr int kOffMisc = kOffXl + 2 * BS * 4;                 // TMEM base, abort flag
   static constexpr int kSmem = kOffMisc + 16;
   static_assert(kSmem <= 232448, "shared memory per CTA");
-  static_assert(kKStages % 2 == 0, "pairs of K stages must not wrap");
-  // bs = 64: two threads share an accumulator row (16x32bx2 loads).
-  static constexpr bool kHalf = (BS == 64);
+  static constexpr bool kHalfRows = (BS == 64);     // two threads per accumulator row
   // TMEM: two S buffers of 128 columns, two O accumulators of D columns.
   static constexpr int kColS = 0;
   static constexpr int kColO = 2 * kGroupKeys;
@@ -92,29 +97,31 @@ struct TcCfg {
   static constexpr int bQFull = 0;
   static constexpr int bQEmpty = bQFull + kQBuf;
   static constexpr int bKFull = bQEmpty + kQBuf;
-  static constexpr int bKEmpty = bKFull + kKStages;
-  static constexpr int bVFull = bKEmpty + kKStages;
-  static constexpr int bVEmpty = bVFull + kVStages;
-  static constexpr int bSFull = bVEmpty + kVStages;  // 2
-  static constexpr int bPFull = bSFull + 2;          // kPBuf
+  static constexpr int bKEmpty = bKFull + kKSlots;
+  static constexpr int bVFull = bKEmpty + kKSlots;
+  static constexpr int bVEmpty = bVFull + kVSlots;
+  static constexpr int bSFull = bVEmpty + kVSlots;   // 2
+  static constexpr int bPFull = bSFull + 2;          // kPBuf (8 arrivals)
   static constexpr int bPVDone = bPFull + kPBuf;     // 2
   static constexpr int bOFull = bPVDone + 2;         // 2
-  static constexpr int bOFree = bOFull + 2;          // 2
-  static constexpr int bTFull = bOFree + 2;         // kSlots
-  static constexpr int bTEmpty = bTFull + kSlots;    // kSlots
-  static constexpr int bFin = bTEmpty + kSlots;
+  static constexpr int bOFree = bOFull + 2;          // 2 (8 arrivals)
+  static constexpr int bTFull = bOFree + 2;          // kSlots
+  static constexpr int bTEmpty = bTFull + kSlots;    // kSlots (10 arrivals)
+  static constexpr int bX = bTEmpty + kSlots;       // 4 (2 arrivals): row exchange per subpartition
+  static constexpr int bFin = bX + 4;
   static constexpr int kNumBars = bFin + 1;
-  static_assert(kNumBars <= 64, "barrier space");
-  static_assert(kTile % 1024 == 0 && kPBytes % 1024 == 0, "1024-byte aligned tiles");
+  static_assert(kNumBars <= kNumBarsMax, "barrier space");
+  static_assert(kTile % 1024 == 0 && kPBytes % 1024 == 0 && kGRegion % 1024 == 0, "1024-byte aligned tiles");
 };
 
 // Valid entries of a sel row are ids in [0, j]; everything else is skipped.
 __device__ __forceinline__ bool valid_id(int id, int j) { return id >= 0 && id <= j; }
 
-// Size of the group that starts at global block g of a tile ending at gend.
+// Size of the group that starts at block n (0-based, in the tile's list) of
+// a tile with nblk selected blocks: blocks 0-1, 2-3, ... pair up for bs = 64.
 template <bool kPair>
-__device__ __forceinline__ int group_size(int g, int gend) {
-  return (kPair && (g & 1) == 0 && g + 1 < gend) ? 2 : 1;
+__device__ __forceinline__ int group_size(int n, int nblk) {
+  return (kPair && (n & 1) == 0 && n + 1 < nblk) ? 2 : 1;
 }
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
@@ -142,6 +149,11 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 }  // namespace
 
 template <int BS, int D>
@@ -164,13 +176,19 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const uint32_t base = smem_u32(smem_raw);
   const uint32_t sQ = base + C::kOffQ, sK = base + C::kOffK, sV = base + C::kOffV, sP = base + C::kOffP;
   uint8_t* pP = sm + C::kOffP;
-  int32_t* info = reinterpret_cast<int32_t*>(sm + C::kOffInfo);   // [kSlots][kSlotInts]
+  uint8_t* info = sm + C::kOffInfo;
+  float* xch = reinterpret_cast<float*>(sm + C::kOffXch);   // [G & 1][half][row]
+  float* xl = reinterpret_cast<float*>(sm + C::kOffXl);     // [half][row]
   const uint32_t bar0 = base + C::kOffBar;
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  auto slot_tile = [&](int s) -> int& { return *reinterpret_cast<int*>(info + s * kSlotBytes); };
+  auto slot_s16 = [&](int s, int i) -> int16_t& { return *reinterpret_cast<int16_t*>(info + s * kSlotBytes + 4 + 2 * i); };
+  // slot_s16(s, 0) = nblk, (s, 1) = diag, (s, 2 + n) = id n
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = a.B * a.Hq * a.nb;
   const int g = a.Hq / a.Hkv;
+  const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
   if (warp == 1) {
     tmem_alloc(smem_u32(&tmem_base_s), C::kCols);
@@ -178,18 +196,19 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kQBuf; ++i) { mbar_init(BAR(C::bQFull + i), 1); mbar_init(BAR(C::bQEmpty + i), 1); }
-    for (int i = 0; i < C::kKStages; ++i) { mbar_init(BAR(C::bKFull + i), 1); mbar_init(BAR(C::bKEmpty + i), 1); }
-    for (int i = 0; i < C::kVStages; ++i) { mbar_init(BAR(C::bVFull + i), 1); mbar_init(BAR(C::bVEmpty + i), 1); }
+    for (int i = 0; i < C::kKSlots; ++i) { mbar_init(BAR(C::bKFull + i), 1); mbar_init(BAR(C::bKEmpty + i), 1); }
+    for (int i = 0; i < C::kVSlots; ++i) { mbar_init(BAR(C::bVFull + i), 1); mbar_init(BAR(C::bVEmpty + i), 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(BAR(C::bSFull + i), 1);
       mbar_init(BAR(C::bPVDone + i), 1);
       mbar_init(BAR(C::bOFull + i), 1);
-      mbar_init(BAR(C::bOFree + i), 4);
+      mbar_init(BAR(C::bOFree + i), 8);
     }
-    for (int i = 0; i < C::kPBuf; ++i) mbar_init(BAR(C::bPFull + i), 4);
+    for (int i = 0; i < C::kPBuf; ++i) mbar_init(BAR(C::bPFull + i), 8);
     // A tile descriptor is released by the V producer, the MMA lane and the
-    // four softmax warps.
-    for (int i = 0; i < kSlots; ++i) { mbar_init(BAR(C::bTFull + i), 1); mbar_init(BAR(C::bTEmpty + i), 6); }
+    // eight softmax warps.
+    for (int i = 0; i < kSlots; ++i) { mbar_init(BAR(C::bTFull + i), 1); mbar_init(BAR(C::bTEmpty + i), 10); }
+    for (int i = 0; i < 4; ++i) mbar_init(BAR(C::bX + i), 2);
     mbar_init(BAR(C::bFin), 1);
     fence_mbar_init();
     abort_s = 0;
@@ -206,19 +225,19 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   if (warp == 0) {
     // ------------------------------------------------ tile descriptors, Q, K
-    // The warp reads each sel row once (lane e: entries e and e + 32),
-    // compacts the valid ids with ballots into a shared-memory tile
-    // descriptor for the other roles, then lane 0 loads Q and the K tiles.
     if (lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
     }
-    int it = 0, itv = 0, gb = 0;               // tiles, non-empty tiles, blocks issued
+    int itv = 0, G = 0;                        // non-empty tiles, groups issued
+    int last_q[2] = {-1, -1};                  // last tile whose Q each buffer received
     bool ok = true;
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+    for (int it = 0; it < my_tiles && ok; ++it) {
+      const int tile = blockIdx.x + it * gridDim.x;
       const int j = tile % a.nb, hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq);
       const int slot = it % kSlots;
-      if (it >= kSlots && !wait_bar(BAR(C::bTEmpty + slot), ((it / kSlots) - 1) & 1, abort_flag)) {
+      if (it >= kSlots &&
+          !__all_sync(0xffffffffu, wait_bar(BAR(C::bTEmpty + slot), ((it / kSlots) - 1) & 1, abort_flag))) {
         ok = false;
         break;
       }
@@ -228,16 +247,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       if ((e0 >= 0 && !v0) || (e1 >= 0 && !v1)) atomicExch(a.status, kDevBadSelection);
       const unsigned m0 = __ballot_sync(0xffffffffu, v0), m1 = __ballot_sync(0xffffffffu, v1);
       const unsigned lt = (1u << lane) - 1u;
-      int32_t* slot_p = info + slot * kSlotInts;
-      if (v0) slot_p[3 + __popc(m0 & lt)] = e0;
-      if (v1) slot_p[3 + __popc(m0) + __popc(m1 & lt)] = e1;
+      if (v0) slot_s16(slot, 2 + __popc(m0 & lt)) = static_cast<int16_t>(e0);
+      if (v1) slot_s16(slot, 2 + __popc(m0) + __popc(m1 & lt)) = static_cast<int16_t>(e1);
       const int nblk = __popc(m0) + __popc(m1);
       const unsigned d0 = __ballot_sync(0xffffffffu, v0 && e0 == j), d1 = __ballot_sync(0xffffffffu, v1 && e1 == j);
       if (lane == 0) {
-        slot_p[0] = tile;
-        slot_p[1] = nblk;
-        slot_p[2] = d0 ? __popc(m0 & ((1u << (__ffs(d0) - 1)) - 1u))
-                       : d1 ? __popc(m0) + __popc(m1 & ((1u << (__ffs(d1) - 1)) - 1u)) : -1;
+        slot_tile(slot) = tile;
+        slot_s16(slot, 0) = static_cast<int16_t>(nblk);
+        slot_s16(slot, 1) = static_cast<int16_t>(
+            d0 ? __popc(m0 & ((1u << (__ffs(d0) - 1)) - 1u))
+               : d1 ? __popc(m0) + __popc(m1 & ((1u << (__ffs(d1) - 1)) - 1u)) : -1);
       }
       __threadfence_block();
       __syncwarp();
@@ -253,22 +272,26 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           for (int gg = 0; gg < D / 64; ++gg)
             tma_load_3d(sQ + qs * C::kTile + gg * C::kRegion, &tmQ, BAR(C::bQFull + qs), gg * 64, hq,
                         tok0 + j * BS);
+          last_q[qs] = itv;
         }
         const int hkv = hq / g;
-        for (int n = 0; n < nblk && ok; ++n) {
-          const int id = slot_p[3 + n];
-          const int st = gb % C::kKStages;
-          if (gb >= C::kKStages &&
-              !wait_bar(BAR(C::bKEmpty + st), ((gb / C::kKStages) - 1) & 1, abort_flag)) {
+        for (int n = 0; n < nblk && ok; ++G) {
+          const int ng = group_size<C::kPair>(n, nblk);
+          const int ks = G % C::kKSlots;
+          if (G >= C::kKSlots && !wait_bar(BAR(C::bKEmpty + ks), ((G / C::kKSlots) - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
-          const uint32_t bar = BAR(C::bKFull + st);
-          mbar_expect_tx(bar, C::kTile);
+          const uint32_t bar = BAR(C::bKFull + ks);
+          mbar_expect_tx(bar, ng * C::kTile);
+          for (int h = 0; h < ng; ++h) {
+            const int id = slot_s16(slot, 2 + n + h);
 #pragma unroll
-          for (int gg = 0; gg < D / 64; ++gg)   // region-major: region gg of every stage together
-            tma_load_3d(sK + gg * C::kKRegion + st * C::kRegion, &tmK, bar, gg * 64, hkv, tok0 + id * BS);
-          ++gb;
+            for (int gg = 0; gg < D / 64; ++gg)
+              tma_load_3d(sK + gg * C::kKRing + ks * C::kGRegion + h * C::kRegion, &tmK, bar, gg * 64, hkv,
+                          tok0 + id * BS);
+          }
+          n += ng;
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -276,47 +299,52 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
     if (!ok && lane == 0) {
       fail();
-      for (int st = 0; st < C::kKStages; ++st) {
+      for (int k = 0; k < C::kKSlots; ++k) {
         int last = -1;
-        for (int n = st; n < gb; n += C::kKStages) last = n;
-        if (last >= 0) mbar_wait(BAR(C::bKFull + st), (last / C::kKStages) & 1, kWaitNs);
+        for (int n = k; n < G; n += C::kKSlots) last = n;
+        if (last >= 0) mbar_wait(BAR(C::bKFull + k), (last / C::kKSlots) & 1, kWaitNs);
       }
+      for (int k = 0; k < C::kQBuf; ++k)
+        if (last_q[k] >= 0) mbar_wait(BAR(C::bQFull + k), (last_q[k] / C::kQBuf) & 1, kWaitNs);
     }
-  } else if (warp == 6) {
+  } else if (warp == 10) {
     // ------------------------------------------------------------ V loads
     if (lane == 0) {
       prefetch_tmap(&tmV);
-      int it = 0, gb = 0;
+      int G = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+      for (int it = 0; it < my_tiles && ok; ++it) {
+        const int tile = blockIdx.x + it * gridDim.x;
         const int slot = it % kSlots;
         if (!wait_bar(BAR(C::bTFull + slot), (it / kSlots) & 1, abort_flag)) { ok = false; break; }
-        const int32_t* slot_p = info + slot * kSlotInts;
-        const int nblk = slot_p[1];
+        const int nblk = slot_s16(slot, 0);
         const int hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq), hkv = hq / g, tok0 = b * a.S;
-        for (int n = 0; n < nblk && ok; ++n) {
-          const int id = slot_p[3 + n];
-          const int st = gb % C::kVStages;
-          if (gb >= C::kVStages &&
-              !wait_bar(BAR(C::bVEmpty + st), ((gb / C::kVStages) - 1) & 1, abort_flag)) {
+        for (int n = 0; n < nblk && ok; ++G) {
+          const int ng = group_size<C::kPair>(n, nblk);
+          const int vs = G % C::kVSlots;
+          if (G >= C::kVSlots && !wait_bar(BAR(C::bVEmpty + vs), ((G / C::kVSlots) - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
-          const uint32_t bar = BAR(C::bVFull + st);
-          mbar_expect_tx(bar, C::kTile);
+          const uint32_t bar = BAR(C::bVFull + vs);
+          mbar_expect_tx(bar, ng * C::kTile);
+          for (int h = 0; h < ng; ++h) {
+            const int id = slot_s16(slot, 2 + n + h);
 #pragma unroll
-          for (int gg = 0; gg < D / 64; ++gg)
-            tma_load_3d(sV + st * C::kTile + gg * C::kRegion, &tmV, bar, gg * 64, hkv, tok0 + id * BS);
-          ++gb;
+            for (int gg = 0; gg < D / 64; ++gg)
+              tma_load_3d(sV + vs * C::kGroupBytes + h * C::kTile + gg * C::kRegion, &tmV, bar, gg * 64, hkv,
+                          tok0 + id * BS);
+          }
+          n += ng;
         }
         if (ok) mbar_arrive(BAR(C::bTEmpty + slot));
       }
       if (!ok) {
         fail();
-        for (int st = 0; st < C::kVStages; ++st) {
+        for (int k = 0; k < C::kVSlots; ++k) {
           int last = -1;
-          for (int n = st; n < gb; n += C::kVStages) last = n;
-          if (last >= 0) mbar_wait(BAR(C::bVFull + st), (last / C::kVStages) & 1, kWaitNs);
+          for (int n = k; n < G; n += C::kVSlots) last = n;
+          if (last >= 0) mbar_wait(BAR(C::bVFull + k), (last / C::kVSlots) & 1, kWaitNs);
         }
       }
     }
@@ -324,21 +352,24 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t idS1 = idesc_bf16_f32(BS, BS, 0, 0);            // one block
-      constexpr uint32_t idS2 = idesc_bf16_f32(BS, 2 * BS, 0, 0);        // a pair (bs = 64)
+      constexpr uint32_t idS2 = idesc_bf16_f32(BS, C::kPair ? 2 * BS : BS, 0, 0);   // a pair
       constexpr uint32_t idPV = idesc_bf16_f32(BS, D, 0, 1);
       const uint64_t dQ0 = smem_desc_sw128(sQ, 16, 1024);
       const uint64_t dK0 = smem_desc_sw128(sK, 16, 1024);
       const uint64_t dP0 = smem_desc_sw128(sP, 16, 1024);
       const uint64_t dV0 = smem_desc_sw128(sV, C::kRegion, 1024);
-      constexpr uint32_t kTile16 = C::kTile / 16, kP16 = C::kPBytes / 16, kKReg16 = C::kKRegion / 16;
-      constexpr uint32_t kRegion16 = C::kRegion / 16;
-      // Tile queue: the PV cursor's tile and up to three after it, read from
-      // the shared-memory tile descriptors (empty tiles are released at once).
-      int q_nblk[4], q_g0[4], q_itv[4], q_slot[4];
+      // Tile queue: the PV cursor's tile and up to three after it.
+      int q_nblk[4], q_g0[4], q_itv[4];
       int nring = 0, head = 0;
       int next_it = 0, next_itv = 0, next_g0 = 0;
-      const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
       bool ok = true;
+      auto get = [&](const int* arr, int qi) {
+        int v = arr[0];
+#pragma unroll
+        for (int x = 1; x < 4; ++x)
+          if (x == qi) v = arr[x];
+        return v;
+      };
       // Append the next non-empty tile.  Only blocks when asked to: the
       // producer publishes a tile only after loading the previous tile's K,
       // which needs this lane's S MMAs.
@@ -349,62 +380,51 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           if (!block && !mbar_try_wait(BAR(C::bTFull + slot), par)) return;
           if (block && !wait_bar(BAR(C::bTFull + slot), par, abort_flag)) { ok = false; return; }
           ++next_it;
-          const int nblk = info[slot * kSlotInts + 1];
-          if (nblk == 0) { mbar_arrive(BAR(C::bTEmpty + slot)); continue; }
+          const int nblk = slot_s16(slot, 0);
+          mbar_arrive(BAR(C::bTEmpty + slot));   // nothing else is read from the slot
+          if (nblk == 0) continue;
           const int qi = (head + nring) & 3;
 #pragma unroll
           for (int x = 0; x < 4; ++x)
-            if (x == qi) { q_nblk[x] = nblk; q_g0[x] = next_g0; q_itv[x] = next_itv; q_slot[x] = slot; }
+            if (x == qi) { q_nblk[x] = nblk; q_g0[x] = next_g0; q_itv[x] = next_itv; }
           ++nring;
           next_g0 += nblk;
           ++next_itv;
           return;
         }
       };
-      auto get = [&](const int* arr, int qi) {
-        int v = arr[0];
-#pragma unroll
-        for (int x = 1; x < 4; ++x)
-          if (x == qi) v = arr[x];
-        return v;
-      };
       int s_t = 0, s_b = -1;                     // S cursor: queue offset from head, next block (global)
-      int Gs = 0, Gp = 0;                        // global group counters (S issued, PV issued)
+      int Gs = 0, Gp = 0;                        // groups whose S / PV were issued
       while (ok) {
         if (nring == 0) fetch(true);
         if (nring == 0) break;
-        const int c_nblk = get(q_nblk, head), c_g0 = get(q_g0, head), c_itv = get(q_itv, head);
-        const int c_end = c_g0 + c_nblk;
+        const int c_g0 = get(q_g0, head), c_end = c_g0 + get(q_nblk, head), c_itv = get(q_itv, head);
         const uint32_t tO = tmem + C::kColO + (c_itv & 1) * D;
         for (int gp = c_g0; gp < c_end && ok;) {
-          const int np = group_size<C::kPair>(gp, c_end);
-          // Issue S while at most one group ahead of this PV and at most one tile ahead.
+          const int np = group_size<C::kPair>(gp - c_g0, c_end - c_g0);
+          // Issue S while at most one group ahead of this PV and one tile ahead.
           if (s_t >= nring - 1) fetch(false);
           while (Gs <= Gp + 1 && s_t < nring && s_t <= 1) {
-            const int slot = (head + s_t) & 3;
-            const int t_g0 = get(q_g0, slot), t_end = t_g0 + get(q_nblk, slot), t_itv = get(q_itv, slot);
+            const int qi = (head + s_t) & 3;
+            const int t_g0 = get(q_g0, qi), t_end = t_g0 + get(q_nblk, qi), t_itv = get(q_itv, qi);
             if (s_b < 0) s_b = t_g0;
-            const int ns = group_size<C::kPair>(s_b, t_end);
-            const int qs = t_itv % C::kQBuf;
+            const int ns = group_size<C::kPair>(s_b - t_g0, t_end - t_g0);
+            const int qs = t_itv % C::kQBuf, ks = Gs % C::kKSlots;
             if (s_b == t_g0 && !wait_bar(BAR(C::bQFull + qs), (t_itv / C::kQBuf) & 1, abort_flag)) { ok = false; break; }
-            const int st = s_b % C::kKStages;
-            bool kready = wait_bar(BAR(C::bKFull + st), (s_b / C::kKStages) & 1, abort_flag);
-            if (kready && ns == 2) kready = wait_bar(BAR(C::bKFull + st + 1), ((s_b + 1) / C::kKStages) & 1, abort_flag);
-            if (!kready) { ok = false; break; }
+            if (!wait_bar(BAR(C::bKFull + ks), (Gs / C::kKSlots) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t tS = tmem + C::kColS + (Gs & 1) * C::kGroupKeys;
-            const uint64_t dq = dQ0 + qs * kTile16, dk = dK0 + st * kRegion16;
+            const uint64_t dq = dQ0 + qs * (C::kTile / 16), dk = dK0 + ks * (C::kGRegion / 16);
             const uint32_t idS = ns == 2 ? idS2 : idS1;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t qoff = ((kk / 4) * C::kRegion + (kk % 4) * 32) / 16;
-              const uint32_t koff = (kk / 4) * kKReg16 + (kk % 4) * 2;
+              const uint32_t koff = (kk / 4) * (C::kKRing / 16) + (kk % 4) * 2;
               if (kk == 0) mma_bf16_c<false>(tS, dq + qoff, dk + koff, idS);
               else mma_bf16_c<true>(tS, dq + qoff, dk + koff, idS);
             }
             mma_commit(BAR(C::bSFull + (Gs & 1)));
-            mma_commit(BAR(C::bKEmpty + st));
-            if (ns == 2) mma_commit(BAR(C::bKEmpty + st + 1));
+            mma_commit(BAR(C::bKEmpty + ks));
             ++Gs;
             s_b += ns;
             if (s_b == t_end) {                   // all S of that tile issued: its Q slot frees
@@ -416,37 +436,33 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           }
           if (!ok) break;
           // PV of group Gp (blocks gp .. gp + np - 1).
+          const int vs = Gp % C::kVSlots;
           if (!wait_bar(BAR(C::bPFull + Gp % C::kPBuf), (Gp / C::kPBuf) & 1, abort_flag)) { ok = false; break; }
           if (gp == c_g0 && c_itv >= 2 &&
               !wait_bar(BAR(C::bOFree + (c_itv & 1)), ((c_itv >> 1) - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
+          if (!wait_bar(BAR(C::bVFull + vs), (Gp / C::kVSlots) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t dp = dP0 + (Gp % C::kPBuf) * kP16;
-          for (int h = 0; h < np && ok; ++h) {
-            const int blk = gp + h, vs = blk % C::kVStages;
-            if (!wait_bar(BAR(C::bVFull + vs), (blk / C::kVStages) & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            const uint64_t dv = dV0 + vs * kTile16;
+          const uint64_t dp = dP0 + (Gp % C::kPBuf) * (C::kPBytes / 16);
+          for (int h = 0; h < np; ++h) {
+            const uint64_t dv = dV0 + vs * (C::kGroupBytes / 16) + h * (C::kTile / 16);
 #pragma unroll
             for (int kk = 0; kk < BS / 16; ++kk) {
-              // keys 16kk.. of this block: P region (h*BS + 16kk)/64, V rows 16kk..
-              const int key = h * BS + kk * 16;
+              const int key = h * BS + kk * 16;   // P region key / 64, V rows 16 kk ..
               const uint32_t poff = ((key / 64) * C::kRegion + ((key % 64) / 16) * 32) / 16;
               if (kk == 0 && h == 0 && gp == c_g0) mma_bf16_c<false>(tO, dp + poff, dv + kk * 128, idPV);
               else mma_bf16_c<true>(tO, dp + poff, dv + kk * 128, idPV);
             }
-            mma_commit(BAR(C::bVEmpty + vs));
           }
-          if (!ok) break;
           mma_commit(BAR(C::bPVDone + (Gp & 1)));
+          mma_commit(BAR(C::bVEmpty + vs));
           ++Gp;
           gp += np;
         }
         if (!ok) break;
         mma_commit(BAR(C::bOFull + (c_itv & 1)));
-        mbar_arrive(BAR(C::bTEmpty + get(q_slot, head)));
         head = (head + 1) & 3;
         --nring;
         --s_t;
@@ -458,50 +474,77 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------- softmax
-    constexpr bool kHalf = C::kHalf;
-    // Columns of a group held by this thread: bs = 64: 64 (32 of each block);
-    // bs = 128: 128.
-    constexpr int kSC = kHalf ? 64 : 128;
-    const int sp = warp & 3;                          // TMEM subpartition of this warp
-    const int hlf = kHalf ? (lane >> 4) : 0;          // bs = 64: which 32 of each 64 columns
-    const int r = kHalf ? (sp * 16 + (lane & 15)) : (sp * 32 + lane);
+    constexpr bool kHR = C::kHalfRows;
+    constexpr int kSC = kHR ? 32 : 64;                // S columns per thread per group
+    const int sp = warp & 3;                          // TMEM subpartition
+    const int half = (warp - 2) >> 2;                 // which 64 of a group's 128 columns
+    const int tsub = kHR ? (lane >> 4) : 0;           // bs = 64: which 32 of those 64
+    const int r = kHR ? (sp * 16 + (lane & 15)) : (sp * 32 + lane);
+    const bool writer = !kHR || tsub == 0;            // one lane per row publishes row values
     const uint32_t lane_base = static_cast<uint32_t>(sp * 32) << 16;
-    const float sl2 = a.scale * 1.4426950408889634f;  // scores in log2 units
-    constexpr int kOChunks = kHalf ? D / 64 : D / 32;
-    // O chunk k of this thread: columns 64k + 32 hlf .. +31 (bs = 64) or 32k .. +31.
-    auto o_ld = [&](uint32_t tO, int k, float* o) {
-      if constexpr (kHalf) tmem_ld16x2_32(tO + 64 * k, o);
-      else tmem_ld32(tO + 32 * k, o);
+    // Waits give the same answer in every lane (a lane may see the abort flag
+    // while another already saw the phase complete).
+    auto wwait = [&](int bar, uint32_t par) {
+      return __all_sync(0xffffffffu, wait_bar(BAR(bar), par, abort_flag));
     };
-    auto o_st = [&](uint32_t tO, int k, const float* o) {
-      if constexpr (kHalf) tmem_st16x2_32(tO + 64 * k, o);
-      else tmem_st32(tO + 32 * k, o);
+    // Row values pass between the two warps of a subpartition through shared
+    // memory; each exchange is one phase of that pair's mbarrier.
+    int xph = 0;
+    auto exchange = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::bX + sp));
+      const bool done = wwait(C::bX + sp, xph & 1);
+      ++xph;
+      return done;
+    };
+    const float sl2 = a.scale * 1.4426950408889634f;  // scores in log2 units
+    // This thread's O columns: kHR: (D/2) half + (D/4) tsub, D/4 of them (one
+    // 16x32bx2 load); otherwise (D/2) half + 32 i for i < D/64.
+    constexpr int kOParts = kHR ? 1 : D / 64;
+    constexpr int kOW = kHR ? D / 4 : 32;
+    auto o_col = [&](int i) { return (D / 2) * half + (kHR ? (D / 4) * tsub : 32 * i); };
+    auto o_ld = [&](uint32_t tO, int i, float* o) {
+      if constexpr (kHR) {
+        if constexpr (D == 128) tmem_ld16x2_32(tO + (D / 2) * half, o);
+        else tmem_ld16x2_16(tO + (D / 2) * half, o);
+      } else {
+        tmem_ld32(tO + (D / 2) * half + 32 * i, o);
+      }
+    };
+    auto o_st = [&](uint32_t tO, int i, const float* o) {
+      if constexpr (kHR) {
+        if constexpr (D == 128) tmem_st16x2_32(tO + (D / 2) * half, o);
+        else tmem_st16x2_16(tO + (D / 2) * half, o);
+      } else {
+        tmem_st32(tO + (D / 2) * half + 32 * i, o);
+      }
     };
     bool pend = false;
     int pend_itv = 0;
-    float pend_l = 1.f;
+    float pend_l = 0.f;
     __nv_bfloat16* pend_out = nullptr;
     auto epilogue = [&]() -> bool {
-      if (!wait_bar(BAR(C::bOFull + (pend_itv & 1)), (pend_itv >> 1) & 1, abort_flag)) return false;
-      __syncwarp();
+      if (!wwait(C::bOFull + (pend_itv & 1), (pend_itv >> 1) & 1)) return false;
+      // Row sum: the two threads of a row, then the partner warp.
+      float l = pend_l;
+      if constexpr (kHR) l += __shfl_xor_sync(0xffffffffu, l, 16);
+      if (writer) xl[half * BS + r] = l;
+      if (!exchange()) return false;
+      l += xl[(1 - half) * BS + r];
       tc_fence_after();
       const uint32_t tO = tmem + C::kColO + (pend_itv & 1) * D + lane_base;
-      const float inv = 1.f / pend_l;
+      const float inv = 1.f / l;
 #pragma unroll
-      for (int k = 0; k < kOChunks; ++k) {
-        float o[32];
-        o_ld(tO, k, o);
+      for (int i = 0; i < kOParts; ++i) {
+        float o[kOW];
+        o_ld(tO, i, o);
         tmem_ld_wait();
-        const int col = kHalf ? 64 * k + 32 * hlf : 32 * k;
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
+        for (int q8 = 0; q8 < kOW / 8; ++q8) {
           uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(o[q8 * 8 + 2 * e] * inv, o[q8 * 8 + 2 * e + 1] * inv);
-            w[e] = *reinterpret_cast<uint32_t*>(&h);
-          }
-          *reinterpret_cast<uint4*>(pend_out + col + q8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int e = 0; e < 4; ++e) w[e] = pack_bf16(o[q8 * 8 + 2 * e] * inv, o[q8 * 8 + 2 * e + 1] * inv);
+          *reinterpret_cast<uint4*>(pend_out + o_col(i) + q8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       tc_fence_before();
@@ -510,20 +553,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       pend = false;
       return true;
     };
-    int it = 0, itv = 0, g0 = 0, G = 0;
+    int itv = 0, g0 = 0, G = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
-      const int j = tile % a.nb, hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq);
+    for (int it = 0; it < my_tiles && ok; ++it) {
       const int slot = it % kSlots;
-      if (!wait_bar(BAR(C::bTFull + slot), (it / kSlots) & 1, abort_flag)) { ok = false; break; }
-      const int nblk = info[slot * kSlotInts + 1], diag = info[slot * kSlotInts + 2];
+      if (!wwait(C::bTFull + slot, (it / kSlots) & 1)) { ok = false; break; }
+      const int tile = slot_tile(slot), nblk = slot_s16(slot, 0), diag = slot_s16(slot, 1);
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::bTEmpty + slot));
+      const int j = tile % a.nb, hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq);
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
                            ((static_cast<size_t>(b) * a.S + static_cast<size_t>(j) * BS + r) * a.Hq + hq) * D;
       if (nblk == 0) {                                 // nothing selected: zero output
-        const int c_lo = kHalf ? hlf * (D / 16) : 0, c_hi = kHalf ? c_lo + D / 16 : D / 8;
-        for (int c = c_lo; c < c_hi; ++c) reinterpret_cast<uint4*>(out)[c] = make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < kOParts; ++i)
+          for (int q8 = 0; q8 < kOW / 8; ++q8) *reinterpret_cast<uint4*>(out + o_col(i) + q8 * 8) = make_uint4(0, 0, 0, 0);
         continue;
       }
       const uint32_t tO = tmem + C::kColO + (itv & 1) * D + lane_base;
@@ -531,35 +574,38 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       float m_used = -INFINITY, l_sum = 0.f;          // running max in log2 units
       bool first = true;
       for (int gb = g0; gb < gend; ++G) {
-        const int ng = group_size<C::kPair>(gb, gend);
-        const int n_in_tile = gb - g0;              // index of the group's first block in the tile
-        if (!wait_bar(BAR(C::bSFull + (G & 1)), (G >> 1) & 1, abort_flag)) { ok = false; break; }
-        __syncwarp();
+        const int n_in_tile = gb - g0;
+        const int ng = group_size<C::kPair>(n_in_tile, nblk);
+        const bool has = !C::kPair || half < ng;      // bs = 64: the second block of a pair
+        if (!wwait(C::bSFull + (G & 1), (G >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         float sv[kSC];
-        const uint32_t tS = tmem + C::kColS + (G & 1) * C::kGroupKeys + lane_base;
-        if constexpr (kHalf) {
-          tmem_ld16x2_32(tS, sv);                  // block 0 of the group
-          if (ng == 2) tmem_ld16x2_32(tS + 64, sv + 32);
-        } else {
+        float pmax = -INFINITY;
+        if (has) {
+          const uint32_t tS = tmem + C::kColS + (G & 1) * C::kGroupKeys + lane_base + 64 * half;
+          if constexpr (kHR) {
+            tmem_ld16x2_32(tS, sv);
+          } else {
+            tmem_ld32(tS, sv);
+            tmem_ld32(tS + 32, sv + 32);
+          }
+          tmem_ld_wait();
+          // Column c: block (kPair ? half : 0) of the group, key kb + c.
+          const int blk = C::kPair ? half : 0;
+          const int kb = kHR ? 32 * tsub : 64 * half;
+          if (n_in_tile + blk == diag) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sv + c * 32);
+            for (int c = 0; c < kSC; ++c)
+              if (kb + c > r) sv[c] = -INFINITY;
+          }
+#pragma unroll
+          for (int c = 0; c < kSC; ++c) pmax = fmaxf(pmax, sv[c]);
         }
-        tmem_ld_wait();
-        // Column c of sv: block c / 32 of the group, key 32 hlf + c % 32 (bs = 64);
-        // block 0, key c (bs = 128).
-        constexpr int kPerBlk = kHalf ? 32 : 128;
-        const int nvalid = kHalf ? 32 * ng : 128;
-#pragma unroll
-        for (int c = 0; c < kSC; ++c) {
-          const int blk = c / kPerBlk, key = (kHalf ? 32 * hlf : 0) + c % kPerBlk;
-          if (c >= nvalid || (n_in_tile + blk == diag && key > r)) sv[c] = -INFINITY;
-        }
-        float mraw = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < kSC; ++c) mraw = fmaxf(mraw, sv[c]);
-        if constexpr (kHalf) mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 16));
-        const float mb = mraw * sl2;
+        if constexpr (kHR) pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 16));
+        float* xg = xch + (G & 1) * 2 * BS;
+        if (writer) xg[half * BS + r] = pmax;
+        if (!exchange()) { ok = false; break; }
+        const float mb = fmaxf(pmax, xg[(1 - half) * BS + r]) * sl2;
         float alpha = 1.f;
         bool rescale = false;
         if (mb > m_used + 8.f) {
@@ -571,50 +617,45 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         // O holds PV(G-1) once it completes; the P buffer is free once the PV
         // that last read it completed.
         const bool need_o = __any_sync(0xffffffffu, rescale);
-        if (need_o && !wait_bar(BAR(C::bPVDone + ((G - 1) & 1)), ((G - 1) >> 1) & 1, abort_flag)) {
+        if (need_o && !wwait(C::bPVDone + ((G - 1) & 1), ((G - 1) >> 1) & 1)) {
           ok = false;
           break;
         }
         if (G >= C::kPBuf &&
-            !wait_bar(BAR(C::bPVDone + ((G - C::kPBuf) & 1)), ((G - C::kPBuf) >> 1) & 1, abort_flag)) {
+            !wwait(C::bPVDone + ((G - C::kPBuf) & 1), ((G - C::kPBuf) >> 1) & 1)) {
           ok = false;
           break;
         }
         __syncwarp();
         tc_fence_after();
         if (need_o) {
-          float o[32];
+          float o[kOW];
 #pragma unroll
-          for (int k = 0; k < kOChunks; ++k) {
-            o_ld(tO, k, o);
+          for (int i = 0; i < kOParts; ++i) {
+            o_ld(tO, i, o);
             tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            o_st(tO, k, o);
+            for (int e = 0; e < kOW; ++e) o[e] *= alpha;
+            o_st(tO, i, o);
           }
           tmem_st_wait();
         }
-        uint8_t* prow = pP + (G % C::kPBuf) * C::kPBytes + r * 128;
+        if (has) {
+          // P region `half` holds keys 64 half .. of the group; this thread's
+          // 8-key chunks start at chunk (kHR ? 4 tsub : 0).
+          uint8_t* prow = pP + (G % C::kPBuf) * C::kPBytes + half * C::kRegion + r * 128;
 #pragma unroll
-        for (int q = 0; q < kSC / 8; ++q) {
-          // 8 columns of sv -> group key kq .. kq+7
-          const int blk = (q * 8) / kPerBlk;
-          const int kq = blk * BS + (kHalf ? 32 * hlf : 0) + (q * 8) % kPerBlk;
-          if (kHalf && blk >= ng) break;
-          float p[8];
+          for (int q = 0; q < kSC / 8; ++q) {
+            float p[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            p[e] = ex2_approx(__fmaf_rn(sv[q * 8 + e], sl2, -m_used));
-            l_sum += p[e];
+            for (int e = 0; e < 8; ++e) {
+              p[e] = ex2_approx(__fmaf_rn(sv[q * 8 + e], sl2, -m_used));
+              l_sum += p[e];
+            }
+            const int chunk = ((kHR ? 4 * tsub : 0) + q) ^ (r % 8);
+            *reinterpret_cast<uint4*>(prow + chunk * 16) =
+                make_uint4(pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
           }
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
-            w[e] = *reinterpret_cast<uint32_t*>(&h);
-          }
-          const int region = kq / 64, chunk = ((kq % 64) / 8) ^ (r % 8);
-          *reinterpret_cast<uint4*>(prow + region * C::kRegion + chunk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -625,11 +666,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         gb += ng;
       }
       if (!ok) break;
-      float l_row = l_sum;
-      if constexpr (kHalf) l_row += __shfl_xor_sync(0xffffffffu, l_sum, 16);
       pend = true;
       pend_itv = itv;
-      pend_l = l_row;
+      pend_l = l_sum;
       pend_out = out;
       g0 = gend;
       ++itv;
