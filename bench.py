@@ -8,7 +8,9 @@ One step = one mdr_forward (rotary + summaries + codes, posting lists,
 probe/rerank/top-R, selected-set attention) over one sequence of the
 workload, inputs resident in HBM.  Each GPU (one process per GPU under
 torchrun) runs its own sequence: weak scaling, no collective on the data path.
-L2 is flushed (256 MiB write, outside the timed events) before every step.
+L2 is flushed before every step, outside the timed events: a 256 MiB write,
+then a read of the same buffer, so that no dirty lines of the flush are left
+to be written back inside the timed region.
 Rank 0 prints one JSON line.
 
 --impl reference times the CPU oracle (oracle/mdr_oracle.py) as it stands on
@@ -191,7 +193,7 @@ def run_reference(args, w):
 def config_of(w, args):
     return {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "block": w.block,
             "P": w.P, "K": w.K, "cap": w.cap, "probes": w.probes, "R": w.R, "L": w.L, "keys": w.keys,
-            "l2": "flushed between steps (256 MiB write, outside the timed events)",
+            "l2": "flushed between steps (256 MiB write + read back, outside the timed events)",
             "parallelism": f"one sequence per GPU x {args.gpus}"}
 
 
@@ -218,8 +220,12 @@ def run_mine(args, w):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(evs):
+    def flush_l2():
         flush.zero_()
+        flush.max()
+
+    def step(evs):
+        flush_l2()
         mdr.mdr_forward_profiled(cfg, q, k, v, cb, idx, rt, out, ws, evs)
 
     for _ in range(args.warmup):
@@ -268,7 +274,7 @@ def run_mine(args, w):
         nE = max(3, min(args.steps, 10))
         times = []
         for it in range(2 + nE):
-            flush.zero_()
+            flush_l2()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             mdr.mdr_forward_host(cfg, qp, kp, vp, cbp, outp, selp, ovp, mxp, dws)

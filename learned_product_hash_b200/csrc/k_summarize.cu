@@ -1,13 +1,9 @@
 // K1 + K2: rotary embedding, per-block summaries and product codes.
 //
-// One CTA per (token block j, sequence b, side): side 0 reads the block's bs
-// tokens of q (all Hq heads), side 1 those of k (all Hkv heads), once, with
-// 16-byte loads.  A warp takes one head at a time: lane (tg, c) rotates the
-// 16-byte chunk c of both halves of its group of tokens, optionally writes
-// the rotated values (the attention kernel reads them), and sums them in
-// token order in float32; a fixed butterfly over the token groups then gives
-// the block sum, scaled by 1/bs to the block mean.  The same warp then
-// assigns the codes of the mean it just produced:
+// For every token block j of sequence b and every head of each side (side 0:
+// queries, Hq heads; side 1: keys, Hkv heads) the kernel rotates the block's
+// bs tokens, optionally writes the rotated copy (the attention kernel reads
+// it), averages them into the block summary, and assigns the summary's codes:
 //   keys    : per subspace the codeword of largest <kbar_s, C[s,k]> (lowest
 //             index on equal scores) -> product address sum_s c_s K^(P-1-s);
 //   queries : per subspace the p codewords of largest score, best first.
@@ -19,194 +15,443 @@
 //
 // Rotary convention: coordinate i pairs with i + D/2; the pair at absolute
 // position t turns by the float32 angle fp32(t) * omega_i, with omega_i =
-// base^(-2i/D) rounded to float32 on the host; the block's (cos, sin) table
-// is computed once per CTA with sincosf.
+// base^(-2i/D) rounded to float32 on the host; cosine and sine by sincosf.
+//
+// Layout of the work.  The kernel is a persistent stream over units; a unit
+// is (b, j, side, head group), a head group being up to 256 / (D / 2 / V)
+// consecutive heads (V elements per 16 bytes), so that one thread owns one
+// (head, 16-byte chunk) of both halves of a head row.  Per unit the block's
+// rows of those heads arrive in chunks of up to 32 KB through a ring of
+// shared-memory stages, filled with bulk copies by one producer thread that
+// runs ahead across units.  The 256 consumer threads (eight warps: with the
+// producer warp at most three warps share a scheduler, which leaves room for
+// 168 registers a thread and four tokens in flight per thread)
+//   1. build the block's (cos, sin) table in shared memory, laid out so that
+//      the eight lanes reading one token's chunk table hit distinct banks;
+//   2. per chunk, rotate their (token, head, chunk) pieces, write them to the
+//      rotated copy with 16-byte stores, and add them to float32 running
+//      sums (token group tg takes tokens tg, tg + TG, ... in order);
+//   3. sum the token groups in order 0, 1, ... TG-1 and scale by 1/bs into
+//      the block mean (float32);
+//   4. one warp per head: codes of that mean.
+// The read traffic is one pass over q and k, the write traffic the rotated
+// copies plus the (small) summaries and codes.
+//
+// Every wait is bounded (2 s of wall time) and gives up once another thread
+// has given up; a wait that runs out writes status 1 (if a status word was
+// given), and the producer waits (bounded) for its copies in flight.
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace mdr {
 
-constexpr int kSumThreads = 256;
+namespace {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;      // 256
+constexpr int kSumThreads = kConsumers + 32;         // + the producer warp
+constexpr int kStageBytes = 32768;
+constexpr int kMaxStages = 6;
+constexpr int kMaxRowBytes = 16384;     // one token's row of a head group
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr int kSmemLimit = 232448;
+
+// Host-computed plan of a launch.
+struct SumPlan {
+  int esize, V, CH, half, log2_half;
+  int HG[2];          // heads per group
+  int ng[2];          // head groups per side (0: side skipped)
+  int NG;             // ng[0] + ng[1]
+  int nunits;         // B * nb * NG
+  int nst;            // ring stages
+  int off_tab, off_part, off_mean, off_freq, off_sc, off_ring, off_bar, smem;
+};
+
+__device__ __forceinline__ int pow2_floor(int x) { return 1 << (31 - __clz(x)); }
+
+}  // namespace
 
 template <typename T>
-__global__ void __launch_bounds__(kSumThreads, 4)
-summarize_kernel(const SummarizeArgs a) {
+__global__ void __launch_bounds__(kSumThreads, 1)
+summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
   using E = Elem<T>;
+  using namespace tc;
   constexpr int V = E::kVec;
-  extern __shared__ float4 smem_f4[];
-  const int j = blockIdx.x, b = blockIdx.y, side = blockIdx.z;
-  if (!a.x[side]) return;
-  const int bs = a.bs, D = a.D, half = D / 2;
-  const int CH = half / V;                           // 16-byte chunks per half row
-  const int TGW = 32 / CH;                           // token groups per warp
-  const int per = bs / TGW;                          // tokens per lane
-  const int H = a.H[side];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = kSumThreads / 32;
-  const int c = lane % CH, tg = lane / CH;
+  constexpr int esize = static_cast<int>(sizeof(T));
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int D = a.D, half = D / 2, CH = half / V, bs = a.bs;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t full0 = sbase + pl.off_bar, empty0 = full0 + 8 * kMaxStages, cbar = empty0 + 8 * kMaxStages;
+  int& abort_s = *reinterpret_cast<int*>(smem + pl.off_bar + 8 * (2 * kMaxStages + 1));
+  volatile int* abort_flag = &abort_s;
+  const int nst = pl.nst;
 
-  float2* tab = reinterpret_cast<float2*>(smem_f4);  // [bs][half] (cos, sin)
-  float* xbar_w = reinterpret_cast<float*>(tab + bs * half) + warp * D;   // this warp's summary
-
-  // The key side pads this block's share of the posting lists with -1
-  // (the list kernel, which runs next, only scatters).
-  if (side == 1 && a.lists_fill) {
-    const size_t share = (a.lists_per_seq + a.nb - 1) / a.nb;
-    const size_t lo = static_cast<size_t>(j) * share;
-    const size_t hi = lo + share < a.lists_per_seq ? lo + share : a.lists_per_seq;
-    int32_t* l = a.lists_fill + static_cast<size_t>(b) * a.lists_per_seq;
-    for (size_t e = lo + threadIdx.x; e < hi; e += kSumThreads) l[e] = -1;
-  }
-
-  // Rotation table of this block, computed once for every head.
-  for (int e = threadIdx.x; e < bs * half; e += kSumThreads) {
-    const int tt = e / half, i = e % half;
-    const float ang = __fmul_rn(static_cast<float>(j * bs + tt), a.inv_freq[i]);
-    float sn, cs;
-    sincosf(ang, &sn, &cs);
-    tab[e] = make_float2(cs, sn);
+  if (tid == 0) {
+    for (int s = 0; s < nst; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kConsumerWarps);
+    }
+    mbar_init(cbar, kConsumerWarps);
+    fence_mbar_init();
+    abort_s = 0;
   }
   __syncthreads();
 
-  const T* __restrict__ x = static_cast<const T*>(a.x[side]);
-  T* __restrict__ xo = static_cast<T*>(a.xrot[side]);
-  const size_t row = static_cast<size_t>(H) * D;     // elements per token
-  const int dsub = D / a.P;
-  const bool codes = side == 0 ? a.qcodes != nullptr : a.addr != nullptr;
+  auto fail = [&]() {
+    if (a.status) atomicExch(a.status, kDevWaitTimeout);
+    *abort_flag = 1;
+  };
 
-  for (int h = warp; h < H; h += nwarps) {
-    // Lane (tg, c) sums tokens tg*per .. tg*per+per-1 of chunk c, in order.
-    const size_t base = (static_cast<size_t>(b) * a.S + static_cast<size_t>(j) * bs + tg * per) * row +
-                        static_cast<size_t>(h) * D + static_cast<size_t>(c) * V;
+  // Unit u: (b, j) = u / NG, group sg = u % NG (query groups first).
+  struct Unit {
+    int b, j, side, h0, HGa, rowbytes, TPC, nch;
+  };
+  auto unit_of = [&](int u) {
+    Unit x;
+    const int bj = u / pl.NG;
+    const int sg = u - bj * pl.NG;
+    x.b = bj / a.nb;
+    x.j = bj - x.b * a.nb;
+    x.side = sg < pl.ng[0] ? 0 : 1;
+    const int hg = x.side ? sg - pl.ng[0] : sg;
+    const int H = a.H[x.side];
+    x.h0 = hg * pl.HG[x.side];
+    x.HGa = min(pl.HG[x.side], H - x.h0);
+    x.rowbytes = x.HGa * D * esize;
+    x.TPC = min(bs, pow2_floor(kStageBytes / x.rowbytes));
+    x.nch = bs / x.TPC;
+    return x;
+  };
+
+  // This CTA's units: a contiguous range, so that the query and key units of
+  // a block follow each other and share the block's rotation table.
+  const int u_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * pl.nunits / gridDim.x);
+  const int u_end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * pl.nunits / gridDim.x);
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;         // chunks issued
+      int st = 0;             // stage of the next chunk
+      uint32_t ph = 0;        // parity of the ring round it belongs to
+      bool ok = true;
+      for (int u = u_begin; u < u_end && ok; ++u) {
+        const Unit x = unit_of(u);
+        const int H = a.H[x.side];
+        const T* src = static_cast<const T*>(a.x[x.side]);
+        for (int ci = 0; ci < x.nch; ++ci) {
+          // A stage is refilled once the consumers released it in the last round.
+          if (issued >= nst && !mbar_wait_or_abort(empty0 + 8 * st, ph ^ 1u, abort_flag, kWaitNs)) {
+            ok = false;
+            break;
+          }
+          const uint32_t bar = full0 + 8 * st, dst = sbase + pl.off_ring + st * kStageBytes;
+          mbar_expect_tx(bar, static_cast<uint32_t>(x.TPC * x.rowbytes));
+          const size_t tok0 = static_cast<size_t>(x.b) * a.S + static_cast<size_t>(x.j) * bs + ci * x.TPC;
+          if (x.HGa == H) {           // the chunk's rows are contiguous
+            bulk_load(dst, src + tok0 * H * D, static_cast<uint32_t>(x.TPC * x.rowbytes), bar);
+          } else {
+            for (int t = 0; t < x.TPC; ++t)
+              bulk_load(dst + t * x.rowbytes, src + ((tok0 + t) * H + x.h0) * D, static_cast<uint32_t>(x.rowbytes),
+                        bar);
+          }
+          ++issued;
+          if (++st == nst) { st = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok) {
+        fail();
+        for (int s = 0; s < nst; ++s) {   // the last copy issued into each stage
+          int last = -1;
+          for (int n = issued - 1; n >= 0 && n >= issued - nst; --n)
+            if (n % nst == s) last = n;
+          if (last >= 0) mbar_wait(full0 + 8 * s, static_cast<uint32_t>(last / nst) & 1u, kWaitNs);
+        }
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  float4* tab4 = reinterpret_cast<float4*>(smem + pl.off_tab);   // [bs][V/2][CH]
+  float4* part4 = reinterpret_cast<float4*>(smem + pl.off_part); // [TG][2V/4][combos]
+  float* mean = reinterpret_cast<float*>(smem + pl.off_mean);    // [HGa][D]
+  float* freq = reinterpret_cast<float*>(smem + pl.off_freq);    // omega_i
+  float* scs = reinterpret_cast<float*>(smem + pl.off_sc) + warp * 128;   // this warp's codeword scores
+  int* best = reinterpret_cast<int*>(smem + pl.off_sc + kConsumerWarps * 128 * 4) + warp * 4;
+  int cph = 0;                 // consumer barrier phases completed
+  auto cwait = [&](uint32_t bar, uint32_t par) {
+    return __all_sync(0xffffffffu, mbar_wait_or_abort(bar, par, abort_flag, kWaitNs));
+  };
+  auto csync = [&]() -> bool {  // all consumer warps
+    __syncwarp();
+    if (lane == 0) mbar_arrive(cbar);
+    const bool r = cwait(cbar, cph & 1);
+    ++cph;
+    return r;
+  };
+  const int dsub = D / a.P;
+  const float inv_bs = 1.0f / static_cast<float>(bs);   // bs is a power of two
+  int st = 0;                  // stage of the next chunk
+  uint32_t ph = 0;             // parity of its ring round
+  bool ok = true;
+  for (int i = tid; i < half; i += kConsumers) freq[i] = a.inv_freq[i];
+  int tab_j = -1;              // block whose table is in shared memory
+  bool prev_codes = true;      // the previous unit ended with a barrier after its means
+  for (int u = u_begin; u < u_end && ok; ++u) {
+    const Unit x = unit_of(u);
+    const int H = a.H[x.side];
+    // The key side's first head group pads this block's share of the
+    // posting lists with -1 (the list kernel, which runs next, only scatters).
+    if (x.side == 1 && x.h0 == 0 && a.lists_fill) {
+      const size_t share = (a.lists_per_seq + a.nb - 1) / a.nb;
+      const size_t lo = static_cast<size_t>(x.j) * share;
+      const size_t hi = lo + share < a.lists_per_seq ? lo + share : a.lists_per_seq;
+      int32_t* l = a.lists_fill + static_cast<size_t>(x.b) * a.lists_per_seq;
+      for (size_t e = lo + tid; e < hi; e += kConsumers) l[e] = -1;
+    }
+    // 1. (cos, sin) of pair i at token t of the block: float4 (t, v2, c)
+    //    holds pairs c*V + 2*v2 and c*V + 2*v2 + 1.  Rebuilt only when the
+    //    block changes; every reader of the old table passed the barrier
+    //    after the previous unit's chunks.
+    const bool rebuild = x.j != tab_j;
+    if (rebuild) {
+      if (tab_j < 0 && !csync()) { ok = false; break; }   // freq visible to all
+#pragma unroll 4
+      for (int e = tid; e < bs * half; e += kConsumers) {
+        const int t = e >> pl.log2_half, i = e & (half - 1);
+        const float ang = __fmul_rn(static_cast<float>(x.j * bs + t), freq[i]);
+        float sn, cs;
+        sincosf(ang, &sn, &cs);
+        const int c = i / V, v = i % V;
+        float* dst = reinterpret_cast<float*>(tab4 + (t * (V / 2) + v / 2) * CH + c) + 2 * (v & 1);
+        dst[0] = cs;
+        dst[1] = sn;
+      }
+      tab_j = x.j;
+    }
+    // The table must be complete before use, and (without a barrier after
+    // the previous unit's means) the partial sums read before rewritten.
+    if ((rebuild || !prev_codes) && !csync()) { ok = false; break; }
+
+    // 2. rotate, store, accumulate.
+    const int combos = x.HGa * CH, TG = kConsumers / combos;
+    const int combo = tid % combos, tg = tid / combos;
+    const int hl = combo / CH, c = combo % CH;
+    const bool active = tg < TG;
+    T* __restrict__ xo = static_cast<T*>(a.xrot[x.side]);
     float s1[V], s2[V];
 #pragma unroll
     for (int v = 0; v < V; ++v) { s1[v] = 0.f; s2[v] = 0.f; }
-    constexpr int kAhead = 2;                        // per is a power of two >= 2
-    for (int t0 = 0; t0 < per; t0 += kAhead) {
-      uint4 r1[kAhead], r2[kAhead];
+    for (int ci = 0; ci < x.nch; ++ci) {
+      if (!cwait(full0 + 8 * st, ph)) { ok = false; break; }
+      const uint8_t* stage = smem + pl.off_ring + st * kStageBytes;
+      if (active) {
+#pragma unroll 4
+        for (int tl = tg; tl < x.TPC; tl += TG) {
+          const int t = ci * x.TPC + tl;
+          const uint8_t* row = stage + tl * x.rowbytes + hl * D * esize;
+          const uint4 r1 = *reinterpret_cast<const uint4*>(row + c * 16);
+          const uint4 r2 = *reinterpret_cast<const uint4*>(row + half * esize + c * 16);
+          float x1[V], x2[V], y1[V], y2[V];
+          E::unpack(r1, x1);
+          E::unpack(r2, x2);
+          const float4* tr = tab4 + t * (V / 2) * CH + c;
 #pragma unroll
-      for (int u = 0; u < kAhead; ++u) {
-        const size_t off = base + static_cast<size_t>(t0 + u) * row;
-        r1[u] = __ldg(reinterpret_cast<const uint4*>(x + off));
-        r2[u] = __ldg(reinterpret_cast<const uint4*>(x + off + half));
-      }
+          for (int v2 = 0; v2 < V / 2; ++v2) {
+            const float4 cs = tr[v2 * CH];          // (cos, sin) of two pairs
+            const int v = 2 * v2;
+            y1[v] = __fmaf_rn(x1[v], cs.x, -__fmul_rn(x2[v], cs.y));
+            y2[v] = __fmaf_rn(x2[v], cs.x, __fmul_rn(x1[v], cs.y));
+            y1[v + 1] = __fmaf_rn(x1[v + 1], cs.z, -__fmul_rn(x2[v + 1], cs.w));
+            y2[v + 1] = __fmaf_rn(x2[v + 1], cs.z, __fmul_rn(x1[v + 1], cs.w));
+          }
 #pragma unroll
-      for (int u = 0; u < kAhead; ++u) {
-        float x1[V], x2[V], y1[V], y2[V];
-        E::unpack(r1[u], x1);
-        E::unpack(r2[u], x2);
-        const float4* tr = reinterpret_cast<const float4*>(tab + (tg * per + t0 + u) * half + c * V);
-#pragma unroll
-        for (int v2 = 0; v2 < V / 2; ++v2) {
-          const float4 cs = tr[v2];                  // (cos, sin) of two pairs
-          const int v = 2 * v2;
-          y1[v] = __fsub_rn(__fmul_rn(x1[v], cs.x), __fmul_rn(x2[v], cs.y));
-          y2[v] = __fadd_rn(__fmul_rn(x2[v], cs.x), __fmul_rn(x1[v], cs.y));
-          y1[v + 1] = __fsub_rn(__fmul_rn(x1[v + 1], cs.z), __fmul_rn(x2[v + 1], cs.w));
-          y2[v + 1] = __fadd_rn(__fmul_rn(x2[v + 1], cs.z), __fmul_rn(x1[v + 1], cs.w));
-          s1[v] = __fadd_rn(s1[v], y1[v]);
-          s2[v] = __fadd_rn(s2[v], y2[v]);
-          s1[v + 1] = __fadd_rn(s1[v + 1], y1[v + 1]);
-          s2[v + 1] = __fadd_rn(s2[v + 1], y2[v + 1]);
+          for (int v = 0; v < V; ++v) {
+            s1[v] = __fadd_rn(s1[v], y1[v]);
+            s2[v] = __fadd_rn(s2[v], y2[v]);
+          }
+          if (xo) {
+            T* o = xo + ((static_cast<size_t>(x.b) * a.S + static_cast<size_t>(x.j) * bs + t) * H + x.h0 + hl) * D +
+                   c * V;
+            E::store(o, y1);
+            E::store(o + half, y2);
+          }
         }
-        if (xo) {
-          const size_t off = base + static_cast<size_t>(t0 + u) * row;
-          E::store(xo + off, y1);
-          E::store(xo + off + half, y2);
-        }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * st);
+      if (++st == nst) { st = 0; ph ^= 1u; }
     }
-    // Combine the token groups: a fixed butterfly over the tg lane bits.
-    for (int o = CH; o < 32; o <<= 1) {
+    if (!ok) break;
+    // Partial sums of this thread's token group: float4 e4 of its chunk
+    // pair (e4 < V/4: first half, otherwise second half).
+    constexpr int NE4 = 2 * V / 4;
+    if (active) {
 #pragma unroll
-      for (int v = 0; v < V; ++v) {
-        s1[v] = __fadd_rn(s1[v], __shfl_xor_sync(0xffffffffu, s1[v], o));
-        s2[v] = __fadd_rn(s2[v], __shfl_xor_sync(0xffffffffu, s2[v], o));
+      for (int e4 = 0; e4 < NE4; ++e4) {
+        const float* sp = e4 < V / 4 ? s1 + 4 * e4 : s2 + 4 * (e4 - V / 4);
+        part4[(tg * NE4 + e4) * combos + combo] = make_float4(sp[0], sp[1], sp[2], sp[3]);
       }
     }
-    const float inv = 1.0f / static_cast<float>(bs);  // bs is a power of two
-    if (tg == 0) {
-      float* g = a.xbar[side] ? a.xbar[side] + ((static_cast<size_t>(b) * H + h) * a.nb + j) * D + c * V : nullptr;
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        const float m1 = s1[v] * inv, m2 = s2[v] * inv;
-        xbar_w[c * V + v] = m1;
-        xbar_w[half + c * V + v] = m2;
-        if (g) { g[v] = m1; g[half + v] = m2; }
-      }
-    }
-    __syncwarp();
-    if (!codes) continue;
+    if (!csync()) { ok = false; break; }
 
-    // Codes of this head: lane scores codewords lane, lane+32, ... (K <= 128).
-    int addr = 0;
-    for (int sdx = 0; sdx < a.P; ++sdx) {
-      float sc[4];
-      int ki[4];
-      const float4* xs4 = reinterpret_cast<const float4*>(xbar_w + sdx * dsub);
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int k = lane + 32 * m;
-        ki[m] = 0x7fffffff;
-        sc[m] = -INFINITY;
-        if (k < a.K) {
-          const float4* cw = reinterpret_cast<const float4*>(a.codebooks + (static_cast<size_t>(sdx) * a.K + k) * dsub);
-          float acc = 0.f;
+    // 3. block means.
+    float* xbar = a.xbar[x.side];
+    for (int i = tid; i < combos * NE4; i += kConsumers) {
+      const int e4 = i / combos, cb = i % combos;
+      float4 sm = part4[e4 * combos + cb];
+      for (int g = 1; g < TG; ++g) {
+        const float4 p = part4[(g * NE4 + e4) * combos + cb];
+        sm.x = __fadd_rn(sm.x, p.x); sm.y = __fadd_rn(sm.y, p.y);
+        sm.z = __fadd_rn(sm.z, p.z); sm.w = __fadd_rn(sm.w, p.w);
+      }
+      sm.x *= inv_bs; sm.y *= inv_bs; sm.z *= inv_bs; sm.w *= inv_bs;
+      const int h = cb / CH, cc = cb % CH;
+      const int elem = e4 < V / 4 ? cc * V + 4 * e4 : half + cc * V + 4 * (e4 - V / 4);
+      *reinterpret_cast<float4*>(mean + h * D + elem) = sm;
+      if (xbar)
+        *reinterpret_cast<float4*>(xbar + ((static_cast<size_t>(x.b) * H + x.h0 + h) * a.nb + x.j) * D + elem) = sm;
+    }
+    const bool codes = x.side == 0 ? a.qcodes != nullptr : a.addr != nullptr;
+    prev_codes = codes;
+    if (!codes) continue;
+    if (!csync()) { ok = false; break; }
+
+    // 4. codes, one warp per head.  Lane scores codewords lane, lane + 32,
+    //    ... (four partial sums over the subspace, then added pairwise); the
+    //    rank of a codeword is the number of codewords with a higher score or
+    //    an equal score and a lower index, so ranks 0 .. need-1 are the
+    //    selected codewords in order (a NaN score counts as -inf).
+    const int need = x.side == 0 ? a.probes : 1;
+    for (int hh = warp; hh < x.HGa; hh += kConsumerWarps) {
+      const int h = x.h0 + hh;
+      for (int sdx = 0; sdx < a.P; ++sdx) {
+        const float4* xs4 = reinterpret_cast<const float4*>(mean + hh * D + sdx * dsub);
+        for (int k = lane; k < a.K; k += 32) {
+          const float4* cw =
+              reinterpret_cast<const float4*>(a.codebooks + (static_cast<size_t>(sdx) * a.K + k) * dsub);
+          float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll 4
           for (int d4 = 0; d4 < dsub / 4; ++d4) {
             const float4 xv = xs4[d4], cv = __ldg(cw + d4);
-            acc = __fmaf_rn(xv.x, cv.x, acc);
-            acc = __fmaf_rn(xv.y, cv.y, acc);
-            acc = __fmaf_rn(xv.z, cv.z, acc);
-            acc = __fmaf_rn(xv.w, cv.w, acc);
+            acc0 = __fmaf_rn(xv.x, cv.x, acc0);
+            acc1 = __fmaf_rn(xv.y, cv.y, acc1);
+            acc2 = __fmaf_rn(xv.z, cv.z, acc2);
+            acc3 = __fmaf_rn(xv.w, cv.w, acc3);
           }
-          sc[m] = acc;
-          ki[m] = k;
+          float sc = __fadd_rn(__fadd_rn(acc0, acc1), __fadd_rn(acc2, acc3));
+          if (!(sc == sc)) sc = -INFINITY;
+          scs[k] = sc;
         }
-      }
-      const int rounds = side == 0 ? a.probes : 1;
-      for (int rr = 0; rr < rounds; ++rr) {
-        float bsc = sc[0];
-        int bi = ki[0];
-#pragma unroll
-        for (int m = 1; m < 4; ++m)
-          if (better(sc[m], ki[m], bsc, bi)) { bsc = sc[m]; bi = ki[m]; }
-        warp_best(bsc, bi);
-        if (side == 0) {
-          if (lane == 0)
-            a.qcodes[((((static_cast<size_t>(b) * H + h) * a.nb + j) * a.P + sdx) * a.probes) + rr] = bi;
-#pragma unroll
-          for (int m = 0; m < 4; ++m)
-            if (ki[m] == bi) { sc[m] = -INFINITY; ki[m] = 0x7fffffff; }
-        } else {
-          addr = addr * a.K + bi;
+        __syncwarp();
+        for (int k = lane; k < a.K; k += 32) {
+          const float sc = scs[k];
+          int rank = 0;
+#pragma unroll 4
+          for (int k2 = 0; k2 < a.K; ++k2) {
+            const float s2v = scs[k2];
+            rank += (s2v > sc || (s2v == sc && k2 < k)) ? 1 : 0;
+          }
+          if (rank < need) {
+            if (x.side == 0)
+              a.qcodes[((((static_cast<size_t>(x.b) * H + h) * a.nb + x.j) * a.P + sdx) * a.probes) + rank] = k;
+            else
+              best[sdx] = k;
+          }
         }
+        __syncwarp();
       }
+      if (x.side == 1 && lane == 0) {
+        int addr = 0;
+        for (int sdx = 0; sdx < a.P; ++sdx) addr = addr * a.K + best[sdx];
+        a.addr[(static_cast<size_t>(x.b) * H + h) * a.nb + x.j] = addr;
+      }
+      __syncwarp();
     }
-    if (side == 1 && lane == 0) a.addr[(static_cast<size_t>(b) * H + h) * a.nb + j] = addr;
-    __syncwarp();
   }
+  if (!ok) fail();
 }
 
+namespace {
+
+bool make_plan(const SummarizeArgs& a, bool bf16, SumPlan& pl) {
+  pl.esize = bf16 ? 2 : 4;
+  pl.V = 16 / pl.esize;
+  pl.half = a.D / 2;
+  pl.log2_half = 0;
+  while ((1 << pl.log2_half) < pl.half) ++pl.log2_half;
+  if ((1 << pl.log2_half) != pl.half) return false;
+  pl.CH = pl.half / pl.V;
+  if (pl.CH < 1 || pl.half % pl.V != 0) return false;
+  const int max_heads = kConsumers / pl.CH;
+  // Partial sums: TG * combos <= 256 threads, 2V floats each.
+  const size_t part = static_cast<size_t>(kConsumers) * 2 * pl.V * sizeof(float);
+  size_t mean = 0;
+  for (int s = 0; s < 2; ++s) {
+    if (!a.x[s]) { pl.HG[s] = 1; pl.ng[s] = 0; continue; }
+    pl.HG[s] = a.H[s] < max_heads ? a.H[s] : max_heads;
+    pl.ng[s] = (a.H[s] + pl.HG[s] - 1) / pl.HG[s];
+    const int rowbytes = pl.HG[s] * a.D * pl.esize;
+    if (rowbytes > kMaxRowBytes || rowbytes % 16 != 0) return false;
+    mean = std::max(mean, static_cast<size_t>(pl.HG[s]) * a.D * sizeof(float));
+  }
+  pl.NG = pl.ng[0] + pl.ng[1];
+  const long long nunits = static_cast<long long>(a.B) * a.nb * pl.NG;
+  if (nunits > 0x7fffffffLL) return false;
+  pl.nunits = static_cast<int>(nunits);
+  const size_t tab = static_cast<size_t>(a.bs) * pl.half * 2 * sizeof(float);
+  auto up = [](size_t x) { return (x + 127) / 128 * 128; };
+  pl.off_tab = 0;
+  pl.off_part = static_cast<int>(up(tab));
+  pl.off_mean = pl.off_part + static_cast<int>(up(part));
+  pl.off_freq = pl.off_mean + static_cast<int>(up(mean));
+  pl.off_sc = pl.off_freq + static_cast<int>(up(pl.half * sizeof(float)));
+  // codeword scores (K <= 128) and key codes (P <= 4) of each consumer warp
+  pl.off_ring = pl.off_sc + static_cast<int>(up(kConsumerWarps * (128 + 4) * sizeof(float)));
+  const int bar_bytes = 8 * (2 * kMaxStages + 1) + 16;
+  const int room = kSmemLimit - pl.off_ring - bar_bytes;
+  pl.nst = std::min(kMaxStages, room / kStageBytes);
+  if (pl.nst < 2) return false;
+  pl.off_bar = pl.off_ring + pl.nst * kStageBytes;
+  pl.smem = pl.off_bar + bar_bytes;
+  return true;
+}
+
+}  // namespace
+
 size_t summarize_smem_bytes(int bs, int D, int Hq, int Hkv) {
-  (void)Hq;
-  (void)Hkv;
-  return static_cast<size_t>(bs) * (D / 2) * sizeof(float2) + static_cast<size_t>(kSumThreads / 32) * D * sizeof(float);
+  SummarizeArgs a{};
+  a.bs = bs; a.D = D; a.H[0] = Hq; a.H[1] = Hkv; a.B = 1; a.nb = 1;
+  int dummy = 0;
+  a.x[0] = &dummy; a.x[1] = &dummy;
+  SumPlan pl{};
+  return make_plan(a, true, pl) ? static_cast<size_t>(pl.smem) : 0;
 }
 
 cudaError_t launch_summarize(const SummarizeArgs& a, bool bf16, cudaStream_t st) {
-  const dim3 grid(a.nb, a.B, 2);
-  const size_t smem = summarize_smem_bytes(a.bs, a.D, a.H[0], a.H[1]);
+  SumPlan pl{};
+  if (!make_plan(a, bf16, pl)) return cudaErrorInvalidValue;
+  if (pl.nunits == 0) return cudaSuccess;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int grid = pl.nunits < sms ? pl.nunits : sms;
   if (bf16) {
     auto k = summarize_kernel<__nv_bfloat16>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    k<<<grid, kSumThreads, smem, st>>>(a);
+    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem)) != cudaSuccess) return e;
+    k<<<static_cast<unsigned>(grid), kSumThreads, pl.smem, st>>>(a, pl);
   } else {
     auto k = summarize_kernel<float>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    k<<<grid, kSumThreads, smem, st>>>(a);
+    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem)) != cudaSuccess) return e;
+    k<<<static_cast<unsigned>(grid), kSumThreads, pl.smem, st>>>(a, pl);
   }
   return cudaGetLastError();
 }

@@ -20,6 +20,7 @@ struct SummarizeArgs {
   float inv_freq[64];      // omega_i, i < D/2
   int32_t* lists_fill;     // posting lists [B, Hkv*A*cap] padded with -1 by the key side; null = skip
   size_t lists_per_seq;    // Hkv*A*cap
+  int32_t* status;         // device status word (a wait that ran out writes 1); null = none
 };
 size_t summarize_smem_bytes(int bs, int D, int Hq, int Hkv);
 cudaError_t launch_summarize(const SummarizeArgs& a, bool bf16, cudaStream_t st);

@@ -188,6 +188,7 @@ mdr_status mdr_build_index(const mdr_config* cfg, const void* k, const float* co
   a.x[1] = k; a.xbar[1] = idx->kbar; a.addr = idx->addr;
   a.lists_fill = idx->lists;
   a.lists_per_seq = static_cast<size_t>(cfg->Hkv) * ipow(cfg->K, cfg->P) * cfg->cap;
+  a.status = at<int32_t>(ws, l.status);
   MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
   return run_lists(cfg, idx, st);
 }
@@ -207,6 +208,7 @@ mdr_status mdr_route(const mdr_config* cfg, const void* q, const float* codebook
   SummarizeArgs a;
   fill_common(a, cfg, codebooks);
   a.x[0] = q; a.xbar[0] = qbar; a.qcodes = qcodes;
+  a.status = at<int32_t>(ws, l.status);
   MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
   return run_route(cfg, qbar, qcodes, idx, rt->sel, rt->ncand, st);
 }
@@ -225,6 +227,7 @@ mdr_status mdr_attend(const mdr_config* cfg, const void* q, const void* k, const
   fill_common(a, cfg, nullptr);
   a.x[0] = q; a.x[1] = k;
   a.xrot[0] = at<void>(ws, l.qrot); a.xrot[1] = at<void>(ws, l.krot);
+  a.status = status;
   MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
   return run_attend(cfg, at<void>(ws, l.qrot), at<void>(ws, l.krot), v, sel, out, status, st);
 }
@@ -258,6 +261,7 @@ static mdr_status forward_impl(const mdr_config* cfg, const void* q, const void*
   a.qcodes = qcodes; a.addr = idx->addr;
   a.lists_fill = idx->lists;
   a.lists_per_seq = static_cast<size_t>(cfg->Hkv) * ipow(cfg->K, cfg->P) * cfg->cap;
+  a.status = status;
   MDR_TRY(mark(0));
   MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
   MDR_TRY(mark(1));

@@ -57,6 +57,12 @@ EDGE = {
     # many locals, tiny capacity (heavy overflow), one probe
     "overflow_heavy": (scaling(4096).with_(cap=1, probes=1, K=4, L=4), {}),
     "fp32_d128": (TINY.with_(D=128, S=256, block=32, Hq=4, Hkv=2, K=16, cap=4, probes=3, R=3, L=2), {}),
+    # more heads than one summary pass takes at once (32 for f32 D=128, 64 for
+    # bf16 D=128): head groups with a ragged last group, strided row copies
+    "many_heads_f32": (TINY.with_(D=128, S=128, block=32, Hq=40, Hkv=40, K=16, cap=4, probes=3, R=2, L=1), {}),
+    "many_heads_bf16": (AR.with_(B=1, S=256, Hq=72, Hkv=72, D=128, keys="gaussian"), {}),
+    # odd head count: token groups that do not tile the 512 summary threads
+    "three_heads_bf16": (AR.with_(B=2, S=512, Hq=3, Hkv=3, D=128, block=128, keys="gaussian"), {}),
 }
 
 
