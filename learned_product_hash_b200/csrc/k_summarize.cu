@@ -54,7 +54,6 @@ namespace {
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;      // 256
 constexpr int kSumThreads = kConsumers + 32;         // + the producer warp
-constexpr int kStageBytes = 32768;
 constexpr int kMaxStages = 6;
 constexpr int kMaxRowBytes = 16384;     // one token's row of a head group
 constexpr uint64_t kWaitNs = 2000000000ull;
@@ -68,7 +67,8 @@ struct SumPlan {
   int NG;             // ng[0] + ng[1]
   int nunits;         // B * nb * NG
   int nst;            // ring stages
-  int off_tab, off_part, off_mean, off_freq, off_sc, off_ring, off_bar, smem;
+  int stage_bytes;    // 32 KB, or 16 KB when shared memory is short
+  int off_tab, off_part, off_mean, off_freq, off_sc, off_cb, off_ring, off_bar, smem;
 };
 
 __device__ __forceinline__ int pow2_floor(int x) { return 1 << (31 - __clz(x)); }
@@ -124,7 +124,7 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
     x.h0 = hg * pl.HG[x.side];
     x.HGa = min(pl.HG[x.side], H - x.h0);
     x.rowbytes = x.HGa * D * esize;
-    x.TPC = min(bs, pow2_floor(kStageBytes / x.rowbytes));
+    x.TPC = min(bs, pow2_floor(pl.stage_bytes / x.rowbytes));
     x.nch = bs / x.TPC;
     return x;
   };
@@ -151,7 +151,7 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
             ok = false;
             break;
           }
-          const uint32_t bar = full0 + 8 * st, dst = sbase + pl.off_ring + st * kStageBytes;
+          const uint32_t bar = full0 + 8 * st, dst = sbase + pl.off_ring + st * pl.stage_bytes;
           mbar_expect_tx(bar, static_cast<uint32_t>(x.TPC * x.rowbytes));
           const size_t tok0 = static_cast<size_t>(x.b) * a.S + static_cast<size_t>(x.j) * bs + ci * x.TPC;
           if (x.HGa == H) {           // the chunk's rows are contiguous
@@ -202,6 +202,17 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
   uint32_t ph = 0;             // parity of its ring round
   bool ok = true;
   for (int i = tid; i < half; i += kConsumers) freq[i] = a.inv_freq[i];
+  // The codebooks, read by every code assignment of this CTA, transposed to
+  // [subspace][dimension][codeword] so that the lanes of a warp (one
+  // codeword each) read consecutive words.
+  float* cbt = reinterpret_cast<float*>(smem + pl.off_cb);
+  if (a.qcodes || a.addr) {
+    const int dsub0 = D / a.P;
+    for (int i = tid; i < a.K * D; i += kConsumers) {
+      const int sdx = i / (a.K * dsub0), r = i % (a.K * dsub0), k = r / dsub0, d = r % dsub0;
+      cbt[(sdx * dsub0 + d) * a.K + k] = __ldg(a.codebooks + i);
+    }
+  }
   int tab_j = -1;              // block whose table is in shared memory
   bool prev_codes = true;      // the previous unit ended with a barrier after its means
   for (int u = u_begin; u < u_end && ok; ++u) {
@@ -222,7 +233,7 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
     //    after the previous unit's chunks.
     const bool rebuild = x.j != tab_j;
     if (rebuild) {
-      if (tab_j < 0 && !csync()) { ok = false; break; }   // freq visible to all
+      if (tab_j < 0 && !csync()) { ok = false; break; }   // freq, codebooks visible to all
 #pragma unroll 4
       for (int e = tid; e < bs * half; e += kConsumers) {
         const int t = e >> pl.log2_half, i = e & (half - 1);
@@ -251,7 +262,7 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
     for (int v = 0; v < V; ++v) { s1[v] = 0.f; s2[v] = 0.f; }
     for (int ci = 0; ci < x.nch; ++ci) {
       if (!cwait(full0 + 8 * st, ph)) { ok = false; break; }
-      const uint8_t* stage = smem + pl.off_ring + st * kStageBytes;
+      const uint8_t* stage = smem + pl.off_ring + st * pl.stage_bytes;
       if (active) {
 #pragma unroll 4
         for (int tl = tg; tl < x.TPC; tl += TG) {
@@ -325,30 +336,30 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
     if (!csync()) { ok = false; break; }
 
     // 4. codes, one warp per head.  Lane scores codewords lane, lane + 32,
-    //    ... (four partial sums over the subspace, then added pairwise); the
-    //    rank of a codeword is the number of codewords with a higher score or
-    //    an equal score and a lower index, so ranks 0 .. need-1 are the
-    //    selected codewords in order (a NaN score counts as -inf).
+    //    ... over the subspace with four partial sums (dimensions d mod 4),
+    //    added pairwise at the end.  The rank of a codeword is the number of
+    //    codewords with a higher score or an equal score and a lower index,
+    //    so ranks 0 .. need-1 are the selected codewords in order (a NaN
+    //    score counts as -inf).
     const int need = x.side == 0 ? a.probes : 1;
     for (int hh = warp; hh < x.HGa; hh += kConsumerWarps) {
       const int h = x.h0 + hh;
       for (int sdx = 0; sdx < a.P; ++sdx) {
         const float4* xs4 = reinterpret_cast<const float4*>(mean + hh * D + sdx * dsub);
+        const float* cw = cbt + sdx * dsub * a.K;
         for (int k = lane; k < a.K; k += 32) {
-          const float4* cw =
-              reinterpret_cast<const float4*>(a.codebooks + (static_cast<size_t>(sdx) * a.K + k) * dsub);
           float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
 #pragma unroll 4
           for (int d4 = 0; d4 < dsub / 4; ++d4) {
-            const float4 xv = xs4[d4], cv = __ldg(cw + d4);
-            acc0 = __fmaf_rn(xv.x, cv.x, acc0);
-            acc1 = __fmaf_rn(xv.y, cv.y, acc1);
-            acc2 = __fmaf_rn(xv.z, cv.z, acc2);
-            acc3 = __fmaf_rn(xv.w, cv.w, acc3);
+            const float4 xv = xs4[d4];
+            const float* c4 = cw + 4 * d4 * a.K + k;
+            acc0 = __fmaf_rn(xv.x, c4[0], acc0);
+            acc1 = __fmaf_rn(xv.y, c4[a.K], acc1);
+            acc2 = __fmaf_rn(xv.z, c4[2 * a.K], acc2);
+            acc3 = __fmaf_rn(xv.w, c4[3 * a.K], acc3);
           }
-          float sc = __fadd_rn(__fadd_rn(acc0, acc1), __fadd_rn(acc2, acc3));
-          if (!(sc == sc)) sc = -INFINITY;
-          scs[k] = sc;
+          const float sc = __fadd_rn(__fadd_rn(acc0, acc1), __fadd_rn(acc2, acc3));
+          scs[k] = sc == sc ? sc : -INFINITY;
         }
         __syncwarp();
         for (int k = lane; k < a.K; k += 32) {
@@ -414,12 +425,15 @@ bool make_plan(const SummarizeArgs& a, bool bf16, SumPlan& pl) {
   pl.off_freq = pl.off_mean + static_cast<int>(up(mean));
   pl.off_sc = pl.off_freq + static_cast<int>(up(pl.half * sizeof(float)));
   // codeword scores (K <= 128) and key codes (P <= 4) of each consumer warp
-  pl.off_ring = pl.off_sc + static_cast<int>(up(kConsumerWarps * (128 + 4) * sizeof(float)));
+  pl.off_cb = pl.off_sc + static_cast<int>(up(kConsumerWarps * (128 + 4) * sizeof(float)));
+  const bool codes = a.qcodes || a.addr;
+  pl.off_ring = pl.off_cb + static_cast<int>(up(codes ? static_cast<size_t>(a.K) * a.D * sizeof(float) : 0));
   const int bar_bytes = 8 * (2 * kMaxStages + 1) + 16;
   const int room = kSmemLimit - pl.off_ring - bar_bytes;
-  pl.nst = std::min(kMaxStages, room / kStageBytes);
+  pl.stage_bytes = room >= 4 * 32768 ? 32768 : 16384;
+  pl.nst = std::min(kMaxStages, room / pl.stage_bytes);
   if (pl.nst < 2) return false;
-  pl.off_bar = pl.off_ring + pl.nst * kStageBytes;
+  pl.off_bar = pl.off_ring + pl.nst * pl.stage_bytes;
   pl.smem = pl.off_bar + bar_bytes;
   return true;
 }
