@@ -267,7 +267,11 @@ def run_mine(args, w):
         step([None] * 5)
     torch.cuda.synchronize()
     assert mdr.mdr_read_device_status(ws) == 0
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # Timed steps: events before the first and after the last kernel only
+    # (an event between two kernels would hold the next one back until the
+    # previous has drained, undoing the overlap of their launches).
+    evs = [[torch.cuda.Event(enable_timing=True), None, None, None, torch.cuda.Event(enable_timing=True)]
+           for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -280,7 +284,12 @@ def run_mine(args, w):
     torch.cuda.synchronize()
     assert mdr.mdr_read_device_status(ws) == 0
     tot = [e[0].elapsed_time(e[4]) for e in evs]
-    ker = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+    # Per-kernel breakdown: separate steps with an event at every kernel boundary.
+    kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(min(args.steps, 20))]
+    for e in kevs:
+        step(e)
+    torch.cuda.synchronize()
+    ker = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in kevs)
            for i, n in enumerate(("summarize", "lists", "route", "attend"))}
     ms_max = max_over_ranks(statistics.mean(tot), dist, world, dev)
     tokens = w.B * w.S * world

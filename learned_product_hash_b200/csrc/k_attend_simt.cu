@@ -23,6 +23,7 @@ __global__ void __launch_bounds__(128)
 attend_simt_kernel(const AttendArgs a) {
   __shared__ int32_t blocks[kMaxSel];
   __shared__ int nblk;
+  grid_dependency_wait();
   const int tile = blockIdx.x;
   const int j = tile % a.nb;
   const int hq = (tile / a.nb) % a.Hq;
@@ -91,8 +92,9 @@ attend_simt_kernel(const AttendArgs a) {
 
 cudaError_t launch_attend_simt(const AttendArgs& a, bool bf16, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(a.B) * a.Hq * a.nb;
-  if (bf16) attend_simt_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(a);
-  else attend_simt_kernel<float><<<grid, 128, 0, st>>>(a);
+  const cudaError_t e = bf16 ? launch_pdl(attend_simt_kernel<__nv_bfloat16>, dim3(grid), dim3(128), 0, st, a)
+                             : launch_pdl(attend_simt_kernel<float>, dim3(grid), dim3(128), 0, st, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -213,6 +213,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
+  grid_dependency_wait();          // q', k' and sel come from earlier kernels
 
   auto fail = [&]() {
     atomicExch(a.status, kDevWaitTimeout);
@@ -734,7 +735,8 @@ cudaError_t launch_tc(const AttendArgs& a, cudaStream_t st) {
   const long long ntiles = static_cast<long long>(a.B) * a.Hq * a.nb;
   const long long want = static_cast<long long>(sms) * per_sm;
   const unsigned grid = static_cast<unsigned>(ntiles < want ? ntiles : want);
-  k<<<grid, kThreads, C::kSmem, st>>>(mq, mk, mv, a);
+  e = launch_pdl(k, dim3(grid), dim3(kThreads), C::kSmem, st, mq, mk, mv, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

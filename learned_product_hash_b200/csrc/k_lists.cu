@@ -30,6 +30,7 @@ __global__ void __launch_bounds__(kListThreads)
 lists_kernel(const ListsArgs a) {
   extern __shared__ int32_t cnt[];                 // [A] running counts, then [nb] addresses
   __shared__ int32_t s_ovf, s_max;
+  grid_dependency_wait();
   const int bh = blockIdx.x;
   int32_t* lists = a.lists + static_cast<size_t>(bh) * static_cast<size_t>(a.A) * a.cap;
   const int32_t* addr = a.addr + static_cast<size_t>(bh) * a.nb;
@@ -88,7 +89,8 @@ cudaError_t launch_lists(const ListsArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(lists_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  lists_kernel<<<a.B * a.H, kListThreads, smem, st>>>(a);
+  e = launch_pdl(lists_kernel, dim3(a.B * a.H), dim3(kListThreads), smem, st, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

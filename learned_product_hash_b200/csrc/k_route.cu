@@ -37,6 +37,7 @@ constexpr int kRouteWarpWords = 128 + 64 + 68 + 2 * (kBatch + 32);
 __global__ void __launch_bounds__(kRouteWarps * 32)
 route_kernel(const RouteArgs a) {
   extern __shared__ int32_t rsmem[];
+  grid_dependency_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int nprobe = 1;
   for (int s = 0; s < a.P; ++s) nprobe *= a.probes;
@@ -195,7 +196,8 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const long long nroutes = static_cast<long long>(a.B) * a.Hq * a.nb;
   const unsigned grid = static_cast<unsigned>((nroutes + kRouteWarps - 1) / kRouteWarps);
-  route_kernel<<<grid, kRouteWarps * 32, smem, st>>>(a);
+  e = launch_pdl(route_kernel, dim3(grid), dim3(kRouteWarps * 32), smem, st, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

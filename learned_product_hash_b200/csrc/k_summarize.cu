@@ -102,6 +102,7 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
     abort_s = 0;
   }
   __syncthreads();
+  grid_dependency_wait();
 
   auto fail = [&]() {
     if (a.status) atomicExch(a.status, kDevWaitTimeout);
@@ -461,11 +462,11 @@ cudaError_t launch_summarize(const SummarizeArgs& a, bool bf16, cudaStream_t st)
   if (bf16) {
     auto k = summarize_kernel<__nv_bfloat16>;
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem)) != cudaSuccess) return e;
-    k<<<static_cast<unsigned>(grid), kSumThreads, pl.smem, st>>>(a, pl);
+    if ((e = launch_pdl(k, dim3(grid), dim3(kSumThreads), pl.smem, st, a, pl)) != cudaSuccess) return e;
   } else {
     auto k = summarize_kernel<float>;
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem)) != cudaSuccess) return e;
-    k<<<static_cast<unsigned>(grid), kSumThreads, pl.smem, st>>>(a, pl);
+    if ((e = launch_pdl(k, dim3(grid), dim3(kSumThreads), pl.smem, st, a, pl)) != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
