@@ -10,14 +10,14 @@
 // is stored depends only on blocks before it.
 //
 // This is a stable counting sort by (address, block id) in shared memory:
-// the head's addresses are staged in shared memory once; the blocks are taken
-// in chunks of 256 in order; each thread counts the earlier blocks of its
-// chunk with the same address and adds the address's running count from the
-// earlier chunks; then the running counts are bumped, lanes of a warp with
-// equal addresses finding each other with __match_any_sync so that only the
-// lowest of them adds the group's size (a warp-aggregated atomic).  The
-// lists arrive padded with -1: the summary kernel of the key side, which runs
-// just before on the same stream, writes the padding.
+// all threads zero the per-address counts and stage the head's addresses;
+// then one warp walks the blocks in order, 32 at a time: lanes with equal
+// addresses find each other with __match_any_sync, a block's rank is the
+// address's count so far plus the number of its peers in lower lanes, and the
+// lowest peer adds the group's size to the count.  The walk is sequential in
+// steps of 32, not in blocks, and needs no block-wide barrier.  The lists
+// arrive padded with -1: the summary kernel of the key side, which runs just
+// before on the same stream, writes the padding.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -42,29 +42,27 @@ lists_kernel(const ListsArgs a) {
   if (tid == 0) { s_ovf = 0; s_max = 0; }
   __syncthreads();
 
-  // Chunks of kListThreads blocks, in order.  Within a chunk, block i's rank
-  // among the chunk's earlier blocks of its address is counted directly;
-  // adding the address's count from earlier chunks gives rank(i).
-  for (int c0 = 0; c0 < a.nb; c0 += kListThreads) {
-    const int i = c0 + tid;
-    const bool valid = i < a.nb;
-    const int ad = valid ? saddr[i] : -1;
-    int rank = 0;
-    if (valid) {
-      for (int k = c0; k < i; ++k) rank += saddr[k] == ad;
-      rank += cnt[ad];
-      if (rank < a.cap) lists[static_cast<size_t>(ad) * a.cap + rank] = i;
+  if (tid < 32) {
+    const unsigned lower = (1u << lane) - 1u;
+    int ad_next = lane < a.nb ? saddr[lane] : -1;
+    for (int c0 = 0; c0 < a.nb; c0 += 32) {
+      const int i = c0 + lane;
+      const int ad = ad_next;
+      ad_next = i + 32 < a.nb ? saddr[i + 32] : -1;
+      const bool valid = i < a.nb;
+      const unsigned vm = __ballot_sync(0xffffffffu, valid);
+      if (valid) {
+        const unsigned peers = __match_any_sync(vm, ad);
+        const int base = cnt[ad];
+        const int rank = base + __popc(peers & lower);
+        if (rank < a.cap) lists[static_cast<size_t>(ad) * a.cap + rank] = i;
+        __syncwarp(vm);                            // every peer read the old count
+        if ((peers & lower) == 0) cnt[ad] = base + __popc(peers);
+      }
+      __syncwarp();
     }
-    __syncthreads();                               // every rank read the old counts
-    // Count update: lanes of a warp with equal addresses add once, through
-    // their lowest lane (a warp-aggregated atomic).
-    const unsigned vm = __ballot_sync(0xffffffffu, valid);
-    if (valid) {
-      const unsigned peers = __match_any_sync(vm, ad);
-      if (lane == __ffs(peers) - 1) atomicAdd(&cnt[ad], __popc(peers));
-    }
-    __syncthreads();
   }
+  __syncthreads();
 
   int ovf = 0, mx = 0;
   int32_t* load = a.load + static_cast<size_t>(bh) * a.A;

@@ -6,11 +6,15 @@
 // the stored blocks of its list that are remote-eligible, i <= j - L.  The
 // lanes look up all probes' list lengths at once, prefix-sum them into slot
 // offsets, and read the stored slots 32 at a time, so a route costs a few
-// dependent memory round trips, not one per probe.  Each lane scores whole
-// candidates by <qbar_j, kbar_i> in float32 (coordinates in order), in
-// batches of at most 224 merged into the running top R (higher score first,
-// lower id on equal scores); the R winners are written in ascending id
-// order, -1 padded; then the local blocks j-L+1..j.
+// dependent memory round trips, not one per probe.  Candidates are scored by
+// <qbar_j, kbar_i> in float32: the D/4 lanes of a lane group read a
+// candidate's row together (one coalesced 16-byte read each, several
+// candidates in flight) and add their four-term partial sums with a fixed
+// butterfly.  Batches of at most 224 candidates are merged into the running
+// top R (higher score first, lower id on equal scores): by rank counting
+// when the batch and the winners are at most 64, else by R rounds of warp
+// arg-max.  The R winners are written in ascending id order, -1 padded; then
+// the local blocks j-L+1..j.
 // Pages: "Monodratic Claims Learned Routing Can Make Sparse Causal Attention
 // More Selective", section "Monodratic Turns Sparse Attention Into a
 // Retrieval Decision" (probe, candidates, rerank, fixed number of remote
@@ -121,26 +125,66 @@ route_kernel(const RouteArgs a) {
     n += __popc(m);
     if (nbuf <= kBatch - 32 && base + 32 < total) continue;
     __syncwarp();
-    // Score the batch: each lane whole candidates, float32, coordinates in order.
-    for (int c = lane; c < nbuf; c += 32) {
-      const float4* kr = reinterpret_cast<const float4*>(kb + static_cast<long long>(cand[c]) * a.D);
-      const float4* q4 = reinterpret_cast<const float4*>(qs);
-      float acc = 0.f;
-      for (int d4 = 0; d4 < a.D / 4; ++d4) {
-        const float4 kv = __ldg(kr + d4);
-        const float4 qv = q4[d4];
-        acc = __fmaf_rn(qv.x, kv.x, acc);
-        acc = __fmaf_rn(qv.y, kv.y, acc);
-        acc = __fmaf_rn(qv.z, kv.z, acc);
-        acc = __fmaf_rn(qv.w, kv.w, acc);
+    // Score the batch: lane group g (F4 = D/4 lanes) takes candidates g,
+    // g + 32/F4, ...; lane pos holds coordinates 4 pos .. 4 pos + 3.
+    {
+      const int F4 = a.D / 4, cpi = 32 / F4, grp = lane / F4, pos = lane % F4;
+      const float4 qv = reinterpret_cast<const float4*>(qs)[pos];
+      for (int c0 = 0; c0 < nbuf; c0 += 4 * cpi) {
+        float pr[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + u * cpi + grp;
+          pr[u] = 0.f;
+          if (c < nbuf) {
+            const float4 kv = __ldg(reinterpret_cast<const float4*>(kb + static_cast<long long>(cand[c]) * a.D) + pos);
+            pr[u] = __fmaf_rn(qv.w, kv.w, __fmaf_rn(qv.z, kv.z, __fmaf_rn(qv.y, kv.y, __fmul_rn(qv.x, kv.x))));
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          for (int o = F4 / 2; o > 0; o >>= 1) pr[u] = __fadd_rn(pr[u], __shfl_xor_sync(0xffffffffu, pr[u], o));
+          const int c = c0 + u * cpi + grp;
+          if (pos == 0 && c < nbuf) score[c] = pr[u];
+        }
       }
-      score[c] = acc;
     }
     __syncwarp();
     // Top R of the batch and the previous winners (higher score, lower id).
     int newwin = 0;
     float myscore = -INFINITY;
     mine = INT_MAX;
+    if (nbuf + nwin <= 64) {
+      // Rank of entry e (batch entries, then the winners) among all of them.
+      const int T = nbuf + nwin;
+      int rk[2], eid[2];
+      float esc[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int e = lane + 32 * h;
+        rk[h] = INT_MAX;
+        eid[h] = INT_MAX;
+        esc[h] = -INFINITY;
+        if (e < T) {
+          const int ce = e < nbuf ? e : kBatch + (e - nbuf);
+          eid[h] = cand[ce];
+          esc[h] = score[ce];
+          int r = 0;
+          for (int f = 0; f < T; ++f) {
+            const int cf = f < nbuf ? f : kBatch + (f - nbuf);
+            r += better(score[cf], cand[cf], esc[h], eid[h]) ? 1 : 0;
+          }
+          rk[h] = r;
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        if (rk[h] < a.R) { cand[kBatch + rk[h]] = eid[h]; score[kBatch + rk[h]] = esc[h]; }
+      __syncwarp();
+      newwin = T < a.R ? T : a.R;
+      if (lane < newwin) { mine = cand[kBatch + lane]; myscore = score[kBatch + lane]; }
+    } else {
     for (int r = 0; r < a.R; ++r) {
       float bs = -INFINITY;
       int bi = INT_MAX, bc = -1;
@@ -161,6 +205,7 @@ route_kernel(const RouteArgs a) {
       if (lane == r) { mine = wi; myscore = ws; }
       ++newwin;
       __syncwarp();
+    }
     }
     __syncwarp();
     if (lane < newwin) { cand[kBatch + lane] = mine; score[kBatch + lane] = myscore; }
