@@ -1,17 +1,12 @@
-// K1 + K2: rotary embedding, per-block summaries and product codes.
+// K1: rotary embedding and per-block summaries.
 //
 // For every token block j of sequence b and every head of each side (side 0:
 // queries, Hq heads; side 1: keys, Hkv heads) the kernel rotates the block's
 // bs tokens, optionally writes the rotated copy (the attention kernel reads
-// it), averages them into the block summary, and assigns the summary's codes:
-//   keys    : per subspace the codeword of largest <kbar_s, C[s,k]> (lowest
-//             index on equal scores) -> product address sum_s c_s K^(P-1-s);
-//   queries : per subspace the p codewords of largest score, best first.
-// Pages: "Monodratic: a reproducible sparse attention mixer", section Mixer
-// (routing acts on rotated keys and queries), and "Monodratic Claims Learned
-// Routing Can Make Sparse Causal Attention More Selective", section
-// "Monodratic Turns Sparse Attention Into a Retrieval Decision" (an address
-// is a combination of several code choices).
+// it) and averages them into the block summary ("Monodratic: a reproducible
+// sparse attention mixer", section Mixer: routing acts on rotated keys and
+// queries, summarised per block).  The codes of the summaries are K2
+// (k_codes.cu), launched right after by launch_summarize.
 //
 // Rotary convention: coordinate i pairs with i + D/2; the pair at absolute
 // position t turns by the float32 angle fp32(t) * omega_i, with omega_i =
@@ -20,8 +15,10 @@
 // Layout of the work.  The kernel is a persistent stream over units; a unit
 // is (b, j, side, head group), a head group being up to 256 / (D / 2 / V)
 // consecutive heads (V elements per 16 bytes), so that one thread owns one
-// (head, 16-byte chunk) of both halves of a head row.  Per unit the block's
-// rows of those heads arrive in chunks of up to 32 KB through a ring of
+// (head, 16-byte chunk) of both halves of a head row.  Each CTA takes a
+// contiguous range of units, so that the query and key units of a block
+// follow each other and share its rotation table.  Per unit the block's rows
+// of those heads arrive in chunks of up to 32 KB through a ring of
 // shared-memory stages, filled with bulk copies by one producer thread that
 // runs ahead across units.  The 256 consumer threads (eight warps: with the
 // producer warp at most three warps share a scheduler, which leaves room for
@@ -32,10 +29,9 @@
 //      rotated copy with 16-byte stores, and add them to float32 running
 //      sums (token group tg takes tokens tg, tg + TG, ... in order);
 //   3. sum the token groups in order 0, 1, ... TG-1 and scale by 1/bs into
-//      the block mean (float32);
-//   4. one warp per head: codes of that mean.
+//      the block mean (float32), written to the summaries.
 // The read traffic is one pass over q and k, the write traffic the rotated
-// copies plus the (small) summaries and codes.
+// copies plus the (small) summaries.
 //
 // Every wait is bounded (2 s of wall time) and gives up once another thread
 // has given up; a wait that runs out writes status 1 (if a status word was
@@ -68,7 +64,7 @@ struct SumPlan {
   int nunits;         // B * nb * NG
   int nst;            // ring stages
   int stage_bytes;    // 32 KB, or 16 KB when shared memory is short
-  int off_tab, off_part, off_mean, off_freq, off_sc, off_cb, off_ring, off_bar, smem;
+  int off_tab, off_part, off_freq, off_ring, off_bar, smem;
 };
 
 __device__ __forceinline__ int pow2_floor(int x) { return 1 << (31 - __clz(x)); }
@@ -181,11 +177,8 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
 
   // -------------------------------------------------------------- consumers
   float4* tab4 = reinterpret_cast<float4*>(smem + pl.off_tab);   // [bs][V/2][CH]
-  float4* part4 = reinterpret_cast<float4*>(smem + pl.off_part); // [TG][2V/4][combos]
-  float* mean = reinterpret_cast<float*>(smem + pl.off_mean);    // [HGa][D]
+  float4* part0 = reinterpret_cast<float4*>(smem + pl.off_part); // 2 x [TG][2V/4][combos]
   float* freq = reinterpret_cast<float*>(smem + pl.off_freq);    // omega_i
-  float* scs = reinterpret_cast<float*>(smem + pl.off_sc) + warp * 128;   // this warp's codeword scores
-  int* best = reinterpret_cast<int*>(smem + pl.off_sc + kConsumerWarps * 128 * 4) + warp * 4;
   int cph = 0;                 // consumer barrier phases completed
   auto cwait = [&](uint32_t bar, uint32_t par) {
     return __all_sync(0xffffffffu, mbar_wait_or_abort(bar, par, abort_flag, kWaitNs));
@@ -197,25 +190,12 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
     ++cph;
     return r;
   };
-  const int dsub = D / a.P;
   const float inv_bs = 1.0f / static_cast<float>(bs);   // bs is a power of two
   int st = 0;                  // stage of the next chunk
   uint32_t ph = 0;             // parity of its ring round
   bool ok = true;
   for (int i = tid; i < half; i += kConsumers) freq[i] = a.inv_freq[i];
-  // The codebooks, read by every code assignment of this CTA, transposed to
-  // [subspace][dimension][codeword] so that the lanes of a warp (one
-  // codeword each) read consecutive words.
-  float* cbt = reinterpret_cast<float*>(smem + pl.off_cb);
-  if (a.qcodes || a.addr) {
-    const int dsub0 = D / a.P;
-    for (int i = tid; i < a.K * D; i += kConsumers) {
-      const int sdx = i / (a.K * dsub0), r = i % (a.K * dsub0), k = r / dsub0, d = r % dsub0;
-      cbt[(sdx * dsub0 + d) * a.K + k] = __ldg(a.codebooks + i);
-    }
-  }
   int tab_j = -1;              // block whose table is in shared memory
-  bool prev_codes = true;      // the previous unit ended with a barrier after its means
   for (int u = u_begin; u < u_end && ok; ++u) {
     const Unit x = unit_of(u);
     const int H = a.H[x.side];
@@ -232,9 +212,8 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
     //    holds pairs c*V + 2*v2 and c*V + 2*v2 + 1.  Rebuilt only when the
     //    block changes; every reader of the old table passed the barrier
     //    after the previous unit's chunks.
-    const bool rebuild = x.j != tab_j;
-    if (rebuild) {
-      if (tab_j < 0 && !csync()) { ok = false; break; }   // freq, codebooks visible to all
+    if (x.j != tab_j) {
+      if (tab_j < 0 && !csync()) { ok = false; break; }   // omega visible to all
 #pragma unroll 4
       for (int e = tid; e < bs * half; e += kConsumers) {
         const int t = e >> pl.log2_half, i = e & (half - 1);
@@ -247,10 +226,8 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
         dst[1] = sn;
       }
       tab_j = x.j;
+      if (!csync()) { ok = false; break; }
     }
-    // The table must be complete before use, and (without a barrier after
-    // the previous unit's means) the partial sums read before rewritten.
-    if ((rebuild || !prev_codes) && !csync()) { ok = false; break; }
 
     // 2. rotate, store, accumulate.
     const int combos = x.HGa * CH, TG = kConsumers / combos;
@@ -302,9 +279,12 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
       if (++st == nst) { st = 0; ph ^= 1u; }
     }
     if (!ok) break;
-    // Partial sums of this thread's token group: float4 e4 of its chunk
-    // pair (e4 < V/4: first half, otherwise second half).
+    // Partial sums of this thread's token group into buffer u & 1: float4 e4
+    // of its chunk pair (e4 < V/4: first half, otherwise second half).  That
+    // buffer was last read two units ago, before the barrier that follows
+    // the previous unit's partial sums.
     constexpr int NE4 = 2 * V / 4;
+    float4* part4 = part0 + (u & 1) * (kConsumers * NE4);
     if (active) {
 #pragma unroll
       for (int e4 = 0; e4 < NE4; ++e4) {
@@ -316,76 +296,20 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
 
     // 3. block means.
     float* xbar = a.xbar[x.side];
-    for (int i = tid; i < combos * NE4; i += kConsumers) {
-      const int e4 = i / combos, cb = i % combos;
-      float4 sm = part4[e4 * combos + cb];
-      for (int g = 1; g < TG; ++g) {
-        const float4 p = part4[(g * NE4 + e4) * combos + cb];
-        sm.x = __fadd_rn(sm.x, p.x); sm.y = __fadd_rn(sm.y, p.y);
-        sm.z = __fadd_rn(sm.z, p.z); sm.w = __fadd_rn(sm.w, p.w);
-      }
-      sm.x *= inv_bs; sm.y *= inv_bs; sm.z *= inv_bs; sm.w *= inv_bs;
-      const int h = cb / CH, cc = cb % CH;
-      const int elem = e4 < V / 4 ? cc * V + 4 * e4 : half + cc * V + 4 * (e4 - V / 4);
-      *reinterpret_cast<float4*>(mean + h * D + elem) = sm;
-      if (xbar)
+    if (xbar) {
+      for (int i = tid; i < combos * NE4; i += kConsumers) {
+        const int e4 = i / combos, cb = i % combos;
+        float4 sm = part4[e4 * combos + cb];
+        for (int g = 1; g < TG; ++g) {
+          const float4 p = part4[(g * NE4 + e4) * combos + cb];
+          sm.x = __fadd_rn(sm.x, p.x); sm.y = __fadd_rn(sm.y, p.y);
+          sm.z = __fadd_rn(sm.z, p.z); sm.w = __fadd_rn(sm.w, p.w);
+        }
+        sm.x *= inv_bs; sm.y *= inv_bs; sm.z *= inv_bs; sm.w *= inv_bs;
+        const int h = cb / CH, cc = cb % CH;
+        const int elem = e4 < V / 4 ? cc * V + 4 * e4 : half + cc * V + 4 * (e4 - V / 4);
         *reinterpret_cast<float4*>(xbar + ((static_cast<size_t>(x.b) * H + x.h0 + h) * a.nb + x.j) * D + elem) = sm;
-    }
-    const bool codes = x.side == 0 ? a.qcodes != nullptr : a.addr != nullptr;
-    prev_codes = codes;
-    if (!codes) continue;
-    if (!csync()) { ok = false; break; }
-
-    // 4. codes, one warp per head.  Lane scores codewords lane, lane + 32,
-    //    ... over the subspace with four partial sums (dimensions d mod 4),
-    //    added pairwise at the end.  The rank of a codeword is the number of
-    //    codewords with a higher score or an equal score and a lower index,
-    //    so ranks 0 .. need-1 are the selected codewords in order (a NaN
-    //    score counts as -inf).
-    const int need = x.side == 0 ? a.probes : 1;
-    for (int hh = warp; hh < x.HGa; hh += kConsumerWarps) {
-      const int h = x.h0 + hh;
-      for (int sdx = 0; sdx < a.P; ++sdx) {
-        const float4* xs4 = reinterpret_cast<const float4*>(mean + hh * D + sdx * dsub);
-        const float* cw = cbt + sdx * dsub * a.K;
-        for (int k = lane; k < a.K; k += 32) {
-          float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll 4
-          for (int d4 = 0; d4 < dsub / 4; ++d4) {
-            const float4 xv = xs4[d4];
-            const float* c4 = cw + 4 * d4 * a.K + k;
-            acc0 = __fmaf_rn(xv.x, c4[0], acc0);
-            acc1 = __fmaf_rn(xv.y, c4[a.K], acc1);
-            acc2 = __fmaf_rn(xv.z, c4[2 * a.K], acc2);
-            acc3 = __fmaf_rn(xv.w, c4[3 * a.K], acc3);
-          }
-          const float sc = __fadd_rn(__fadd_rn(acc0, acc1), __fadd_rn(acc2, acc3));
-          scs[k] = sc == sc ? sc : -INFINITY;
-        }
-        __syncwarp();
-        for (int k = lane; k < a.K; k += 32) {
-          const float sc = scs[k];
-          int rank = 0;
-#pragma unroll 4
-          for (int k2 = 0; k2 < a.K; ++k2) {
-            const float s2v = scs[k2];
-            rank += (s2v > sc || (s2v == sc && k2 < k)) ? 1 : 0;
-          }
-          if (rank < need) {
-            if (x.side == 0)
-              a.qcodes[((((static_cast<size_t>(x.b) * H + h) * a.nb + x.j) * a.P + sdx) * a.probes) + rank] = k;
-            else
-              best[sdx] = k;
-          }
-        }
-        __syncwarp();
       }
-      if (x.side == 1 && lane == 0) {
-        int addr = 0;
-        for (int sdx = 0; sdx < a.P; ++sdx) addr = addr * a.K + best[sdx];
-        a.addr[(static_cast<size_t>(x.b) * H + h) * a.nb + x.j] = addr;
-      }
-      __syncwarp();
     }
   }
   if (!ok) fail();
@@ -403,32 +327,24 @@ bool make_plan(const SummarizeArgs& a, bool bf16, SumPlan& pl) {
   pl.CH = pl.half / pl.V;
   if (pl.CH < 1 || pl.half % pl.V != 0) return false;
   const int max_heads = kConsumers / pl.CH;
-  // Partial sums: TG * combos <= 256 threads, 2V floats each.
-  const size_t part = static_cast<size_t>(kConsumers) * 2 * pl.V * sizeof(float);
-  size_t mean = 0;
   for (int s = 0; s < 2; ++s) {
     if (!a.x[s]) { pl.HG[s] = 1; pl.ng[s] = 0; continue; }
     pl.HG[s] = a.H[s] < max_heads ? a.H[s] : max_heads;
     pl.ng[s] = (a.H[s] + pl.HG[s] - 1) / pl.HG[s];
     const int rowbytes = pl.HG[s] * a.D * pl.esize;
     if (rowbytes > kMaxRowBytes || rowbytes % 16 != 0) return false;
-    mean = std::max(mean, static_cast<size_t>(pl.HG[s]) * a.D * sizeof(float));
   }
   pl.NG = pl.ng[0] + pl.ng[1];
   const long long nunits = static_cast<long long>(a.B) * a.nb * pl.NG;
   if (nunits > 0x7fffffffLL) return false;
   pl.nunits = static_cast<int>(nunits);
-  const size_t tab = static_cast<size_t>(a.bs) * pl.half * 2 * sizeof(float);
   auto up = [](size_t x) { return (x + 127) / 128 * 128; };
+  // Partial sums: two buffers of TG * combos <= 256 threads, 2V floats each.
+  const size_t part = static_cast<size_t>(kConsumers) * 2 * pl.V * sizeof(float);
   pl.off_tab = 0;
-  pl.off_part = static_cast<int>(up(tab));
-  pl.off_mean = pl.off_part + static_cast<int>(up(part));
-  pl.off_freq = pl.off_mean + static_cast<int>(up(mean));
-  pl.off_sc = pl.off_freq + static_cast<int>(up(pl.half * sizeof(float)));
-  // codeword scores (K <= 128) and key codes (P <= 4) of each consumer warp
-  pl.off_cb = pl.off_sc + static_cast<int>(up(kConsumerWarps * (128 + 4) * sizeof(float)));
-  const bool codes = a.qcodes || a.addr;
-  pl.off_ring = pl.off_cb + static_cast<int>(up(codes ? static_cast<size_t>(a.K) * a.D * sizeof(float) : 0));
+  pl.off_part = static_cast<int>(up(static_cast<size_t>(a.bs) * pl.half * 2 * sizeof(float)));
+  pl.off_freq = pl.off_part + static_cast<int>(2 * up(part));
+  pl.off_ring = pl.off_freq + static_cast<int>(up(pl.half * sizeof(float)));
   const int bar_bytes = 8 * (2 * kMaxStages + 1) + 16;
   const int room = kSmemLimit - pl.off_ring - bar_bytes;
   pl.stage_bytes = room >= 4 * 32768 ? 32768 : 16384;
@@ -468,7 +384,16 @@ cudaError_t launch_summarize(const SummarizeArgs& a, bool bf16, cudaStream_t st)
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem)) != cudaSuccess) return e;
     if ((e = launch_pdl(k, dim3(grid), dim3(kSumThreads), pl.smem, st, a, pl)) != cudaSuccess) return e;
   }
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // K2 on the summaries just written.
+  CodesArgs c{};
+  c.xbar[0] = a.qcodes ? a.xbar[0] : nullptr;
+  c.xbar[1] = a.addr ? a.xbar[1] : nullptr;
+  if (!c.xbar[0] && !c.xbar[1]) return cudaSuccess;
+  c.H[0] = a.H[0]; c.H[1] = a.H[1];
+  c.qcodes = a.qcodes; c.addr = a.addr; c.codebooks = a.codebooks;
+  c.B = a.B; c.nb = a.nb; c.D = a.D; c.P = a.P; c.K = a.K; c.probes = a.probes;
+  return launch_codes(c, st);
 }
 
 }  // namespace mdr

@@ -23,7 +23,19 @@ struct SummarizeArgs {
   int32_t* status;         // device status word (a wait that ran out writes 1); null = none
 };
 size_t summarize_smem_bytes(int bs, int D, int Hq, int Hkv);
+// Launches K1 (rotation, summaries) and, when qcodes or addr is given, K2.
 cudaError_t launch_summarize(const SummarizeArgs& a, bool bf16, cudaStream_t st);
+
+// K2: codes of the block summaries (queries: top-p per subspace; keys: address).
+struct CodesArgs {
+  const float* xbar[2];    // summaries [B,H,nb,D] per side; null skips a side
+  int H[2];                // Hq, Hkv
+  int32_t* qcodes;         // [B,Hq,nb,P,probes] (side 0)
+  int32_t* addr;           // [B,Hkv,nb] (side 1)
+  const float* codebooks;  // [P,K,D/P]
+  int B, nb, D, P, K, probes;
+};
+cudaError_t launch_codes(const CodesArgs& a, cudaStream_t st);
 
 // K3: bounded causal posting lists of every (b, kv head).
 struct ListsArgs {
