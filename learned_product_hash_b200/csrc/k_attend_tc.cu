@@ -723,12 +723,11 @@ cudaError_t launch_tc(const AttendArgs& a, cudaStream_t st) {
       !make_map(&mv, a.v, rows, a.Hkv, D, BS))
     return cudaErrorInvalidValue;
   auto k = attend_tc_kernel<BS, D>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(k), C::kSmem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0, per_sm = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, C::kSmem)) != cudaSuccess) return e;
+  const int sms = cached_sm_count();
+  int per_sm = cached_occupancy(reinterpret_cast<const void*>(k), kThreads, C::kSmem);
+  if (sms <= 0) return cudaErrorUnknown;
   // Tensor memory: at most 512 columns per SM.
   per_sm = per_sm < 512 / C::kCols ? per_sm : 512 / C::kCols;
   if (per_sm < 1) per_sm = 1;

@@ -11,13 +11,12 @@
 //
 // One warp per summary row (side, b, h, j), 16 warps per CTA, about two CTAs
 // per SM so that the rows' memory latency overlaps.  Each CTA first copies the
-// codebooks into shared memory transposed to [subspace][dimension][codeword],
-// so that the lanes of a warp -- one codeword each -- read consecutive words.
-// A lane scores its codewords over the subspace with four float32 partial
-// sums (dimensions d mod 4) added pairwise at the end; the rank of a codeword
-// is the number of codewords with a higher score or an equal score and a
-// lower index, so ranks 0 .. need-1 are the selected codewords in order (a
-// NaN score counts as -inf).
+// codebooks into shared memory, one row per codeword padded to dsub + 4
+// words, so that the 16-byte reads of 32 lanes -- one codeword each -- spread
+// over all banks.  A lane scores its codewords over the subspace with four
+// float32 partial sums (dimensions d mod 4) added pairwise at the end; the
+// selected codewords are then taken by rounds of warp arg-max (higher score,
+// lower index on equal scores; a NaN score counts as -inf), best first.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -33,18 +32,15 @@ constexpr int kMaxK = 128;
 
 __global__ void __launch_bounds__(kCodeWarps * 32)
 codes_kernel(const __grid_constant__ CodesArgs a) {
-  extern __shared__ float csm[];
+  extern __shared__ float4 csm4[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int D = a.D, dsub = D / a.P;
-  float* cbt = csm;                                           // [P][dsub][K]
-  float* wsm = csm + a.K * D + warp * (D + kMaxK + 4);        // this warp: mean [D], scores [K], best [4]
-  float* xs = wsm;
-  float* scs = wsm + D;
-  int* best = reinterpret_cast<int*>(wsm + D + kMaxK);
+  const int D = a.D, dsub = D / a.P, RS = dsub + 4;           // codebook row stride (floats)
+  float* cbs = reinterpret_cast<float*>(csm4);                // [P][K][dsub + 4]
+  float* xs = cbs + a.P * a.K * RS + warp * D;                // this warp's summary row
 
   for (int i = threadIdx.x; i < a.K * D; i += kCodeWarps * 32) {
-    const int sdx = i / (a.K * dsub), r = i % (a.K * dsub), k = r / dsub, d = r % dsub;
-    cbt[(sdx * dsub + d) * a.K + k] = __ldg(a.codebooks + i);
+    const int row = i / dsub, d = i - row * dsub;              // row = sdx * K + k
+    cbs[row * RS + d] = __ldg(a.codebooks + i);
   }
   __syncthreads();
   grid_dependency_wait();          // the summaries come from the previous kernel
@@ -60,46 +56,50 @@ codes_kernel(const __grid_constant__ CodesArgs a) {
       reinterpret_cast<float4*>(xs)[d4] = __ldg(reinterpret_cast<const float4*>(xb) + d4);
     __syncwarp();
     const int need = side == 0 ? a.probes : 1;
+    int addr = 0;
     for (int sdx = 0; sdx < a.P; ++sdx) {
       const float4* xs4 = reinterpret_cast<const float4*>(xs + sdx * dsub);
-      const float* cw = cbt + sdx * dsub * a.K;
-      for (int k = lane; k < a.K; k += 32) {
-        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+      float sc[kMaxK / 32];
+      int ki[kMaxK / 32];
+#pragma unroll
+      for (int m = 0; m < kMaxK / 32; ++m) {
+        const int k = lane + 32 * m;
+        sc[m] = -INFINITY;
+        ki[m] = 0x7fffffff;
+        if (k < a.K) {
+          const float4* cw = reinterpret_cast<const float4*>(cbs + (sdx * a.K + k) * RS);
+          float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
 #pragma unroll 4
-        for (int d4 = 0; d4 < dsub / 4; ++d4) {
-          const float4 xv = xs4[d4];
-          const float* c4 = cw + 4 * d4 * a.K + k;
-          acc0 = __fmaf_rn(xv.x, c4[0], acc0);
-          acc1 = __fmaf_rn(xv.y, c4[a.K], acc1);
-          acc2 = __fmaf_rn(xv.z, c4[2 * a.K], acc2);
-          acc3 = __fmaf_rn(xv.w, c4[3 * a.K], acc3);
-        }
-        const float sc = __fadd_rn(__fadd_rn(acc0, acc1), __fadd_rn(acc2, acc3));
-        scs[k] = sc == sc ? sc : -INFINITY;
-      }
-      __syncwarp();
-      for (int k = lane; k < a.K; k += 32) {
-        const float sc = scs[k];
-        int rank = 0;
-#pragma unroll 4
-        for (int k2 = 0; k2 < a.K; ++k2) {
-          const float s2 = scs[k2];
-          rank += (s2 > sc || (s2 == sc && k2 < k)) ? 1 : 0;
-        }
-        if (rank < need) {
-          if (side == 0)
-            a.qcodes[(rr * a.P + sdx) * a.probes + rank] = k;
-          else
-            best[sdx] = k;
+          for (int d4 = 0; d4 < dsub / 4; ++d4) {
+            const float4 xv = xs4[d4], cv = cw[d4];
+            acc0 = __fmaf_rn(xv.x, cv.x, acc0);
+            acc1 = __fmaf_rn(xv.y, cv.y, acc1);
+            acc2 = __fmaf_rn(xv.z, cv.z, acc2);
+            acc3 = __fmaf_rn(xv.w, cv.w, acc3);
+          }
+          const float v = __fadd_rn(__fadd_rn(acc0, acc1), __fadd_rn(acc2, acc3));
+          sc[m] = v == v ? v : -INFINITY;
+          ki[m] = k;
         }
       }
-      __syncwarp();
+      for (int rnd = 0; rnd < need; ++rnd) {
+        float bsc = sc[0];
+        int bi = ki[0];
+#pragma unroll
+        for (int m = 1; m < kMaxK / 32; ++m)
+          if (better(sc[m], ki[m], bsc, bi)) { bsc = sc[m]; bi = ki[m]; }
+        warp_best(bsc, bi);
+        if (side == 0) {
+          if (lane == 0) a.qcodes[(rr * a.P + sdx) * a.probes + rnd] = bi;
+#pragma unroll
+          for (int m = 0; m < kMaxK / 32; ++m)
+            if (ki[m] == bi) { sc[m] = -INFINITY; ki[m] = 0x7fffffff; }
+        } else {
+          addr = addr * a.K + bi;
+        }
+      }
     }
-    if (side == 1 && lane == 0) {
-      int addr = 0;
-      for (int sdx = 0; sdx < a.P; ++sdx) addr = addr * a.K + best[sdx];
-      a.addr[rr] = addr;
-    }
+    if (side == 1 && lane == 0) a.addr[rr] = addr;
     __syncwarp();
   }
 }
@@ -109,17 +109,13 @@ cudaError_t launch_codes(const CodesArgs& a, cudaStream_t st) {
                          (a.xbar[1] ? static_cast<long long>(a.B) * a.H[1] * a.nb : 0);
   if (rows == 0) return cudaSuccess;
   if (a.K > kMaxK || a.P > 4) return cudaErrorInvalidValue;
-  const size_t smem = (static_cast<size_t>(a.K) * a.D + static_cast<size_t>(kCodeWarps) * (a.D + kMaxK + 4)) *
-                      sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(codes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  const size_t smem =
+      (static_cast<size_t>(a.P) * a.K * (a.D / a.P + 4) + static_cast<size_t>(kCodeWarps) * a.D) * sizeof(float);
+  cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(codes_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0, per_sm = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, codes_kernel, kCodeWarps * 32, smem)) !=
-      cudaSuccess)
-    return e;
+  const int sms = cached_sm_count();
+  int per_sm = cached_occupancy(reinterpret_cast<const void*>(codes_kernel), kCodeWarps * 32, smem);
+  if (sms <= 0) return cudaErrorUnknown;
   if (per_sm < 1) per_sm = 1;
   const long long need = (rows + kCodeWarps - 1) / kCodeWarps;
   const long long cap = static_cast<long long>(sms) * (per_sm < 2 ? per_sm : 2);

@@ -84,8 +84,7 @@ lists_kernel(const ListsArgs a) {
 
 cudaError_t launch_lists(const ListsArgs& a, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(a.A + a.nb) * sizeof(int32_t);
-  cudaError_t e = cudaFuncSetAttribute(lists_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(lists_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   e = launch_pdl(lists_kernel, dim3(a.B * a.H), dim3(kListThreads), smem, st, a);
   if (e != cudaSuccess) return e;

@@ -236,8 +236,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   int nprobe = 1;
   for (int s = 0; s < a.P; ++s) nprobe *= a.probes;
   const size_t smem = static_cast<size_t>(kRouteWarps) * kRouteWarpWords * sizeof(int32_t);
-  cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(route_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const long long nroutes = static_cast<long long>(a.B) * a.Hq * a.nb;
   const unsigned grid = static_cast<unsigned>((nroutes + kRouteWarps - 1) / kRouteWarps);

@@ -370,18 +370,17 @@ cudaError_t launch_summarize(const SummarizeArgs& a, bool bf16, cudaStream_t st)
   SumPlan pl{};
   if (!make_plan(a, bf16, pl)) return cudaErrorInvalidValue;
   if (pl.nunits == 0) return cudaSuccess;
-  int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  const int sms = cached_sm_count();
+  if (sms <= 0) return cudaErrorUnknown;
   const int grid = pl.nunits < sms ? pl.nunits : sms;
   if (bf16) {
     auto k = summarize_kernel<__nv_bfloat16>;
-    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem)) != cudaSuccess) return e;
+    if ((e = cached_allow_smem(reinterpret_cast<const void*>(k), pl.smem)) != cudaSuccess) return e;
     if ((e = launch_pdl(k, dim3(grid), dim3(kSumThreads), pl.smem, st, a, pl)) != cudaSuccess) return e;
   } else {
     auto k = summarize_kernel<float>;
-    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem)) != cudaSuccess) return e;
+    if ((e = cached_allow_smem(reinterpret_cast<const void*>(k), pl.smem)) != cudaSuccess) return e;
     if ((e = launch_pdl(k, dim3(grid), dim3(kSumThreads), pl.smem, st, a, pl)) != cudaSuccess) return e;
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -7,6 +7,11 @@
 
 namespace mdr {
 
+// Launch facts cached per device (launch_cache.cu).
+int cached_sm_count();                                        // 0 on error
+cudaError_t cached_allow_smem(const void* fn, int bytes);     // dynamic shared memory the kernel may use
+int cached_occupancy(const void* fn, int threads, size_t smem);   // blocks per SM, 0 on error
+
 // K1 + K2: rotate, summarise and code one or both sides.
 struct SummarizeArgs {
   const void* x[2];        // side 0 = queries [B,S,Hq,D], side 1 = keys [B,S,Hkv,D]; null skips a side
