@@ -14,9 +14,12 @@
 // codebooks into shared memory, one row per codeword padded to dsub + 4
 // words, so that the 16-byte reads of 32 lanes -- one codeword each -- spread
 // over all banks.  A lane scores its codewords over the subspace with four
-// float32 partial sums (dimensions d mod 4) added pairwise at the end; the
-// selected codewords are then taken by rounds of warp arg-max (higher score,
-// lower index on equal scores; a NaN score counts as -inf), best first.
+// float32 partial sums (dimensions d mod 4) added pairwise at the end (the
+// kernel is instantiated per dsub so that the loop unrolls completely).  The
+// selected codewords are taken by rounds of warp arg-max, best first: the
+// highest score by one warp max-reduction of an order-preserving integer
+// image of the score, then the lowest index among the lanes holding it (a NaN
+// score counts as -inf).
 
 #include "common.cuh"
 #include "kernels.h"
@@ -28,19 +31,27 @@ namespace {
 constexpr int kCodeWarps = 16;
 constexpr int kMaxK = 128;
 
+// Order-preserving map of a float32 (not NaN) to uint32.
+__device__ __forceinline__ uint32_t ordered_bits(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 }  // namespace
 
+template <int F4>   // dsub / 4
 __global__ void __launch_bounds__(kCodeWarps * 32)
 codes_kernel(const __grid_constant__ CodesArgs a) {
   extern __shared__ float4 csm4[];
+  constexpr int dsub = 4 * F4, RS = dsub + 4;                 // codebook row stride (floats)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int D = a.D, dsub = D / a.P, RS = dsub + 4;           // codebook row stride (floats)
+  const int D = a.D;
   float* cbs = reinterpret_cast<float*>(csm4);                // [P][K][dsub + 4]
   float* xs = cbs + a.P * a.K * RS + warp * D;                // this warp's summary row
 
-  for (int i = threadIdx.x; i < a.K * D; i += kCodeWarps * 32) {
-    const int row = i / dsub, d = i - row * dsub;              // row = sdx * K + k
-    cbs[row * RS + d] = __ldg(a.codebooks + i);
+  for (int i4 = threadIdx.x; i4 < a.K * D / 4; i4 += kCodeWarps * 32) {
+    const int i = 4 * i4, row = i / dsub, d = i - row * dsub;  // row = sdx * K + k
+    *reinterpret_cast<float4*>(cbs + row * RS + d) = __ldg(reinterpret_cast<const float4*>(a.codebooks) + i4);
   }
   __syncthreads();
   grid_dependency_wait();          // the summaries come from the previous kernel
@@ -59,18 +70,16 @@ codes_kernel(const __grid_constant__ CodesArgs a) {
     int addr = 0;
     for (int sdx = 0; sdx < a.P; ++sdx) {
       const float4* xs4 = reinterpret_cast<const float4*>(xs + sdx * dsub);
-      float sc[kMaxK / 32];
-      int ki[kMaxK / 32];
+      uint32_t key[kMaxK / 32];        // ordered score; 0 = no codeword (no float maps to 0)
 #pragma unroll
       for (int m = 0; m < kMaxK / 32; ++m) {
         const int k = lane + 32 * m;
-        sc[m] = -INFINITY;
-        ki[m] = 0x7fffffff;
+        key[m] = 0;
         if (k < a.K) {
           const float4* cw = reinterpret_cast<const float4*>(cbs + (sdx * a.K + k) * RS);
           float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll 4
-          for (int d4 = 0; d4 < dsub / 4; ++d4) {
+#pragma unroll
+          for (int d4 = 0; d4 < F4; ++d4) {
             const float4 xv = xs4[d4], cv = cw[d4];
             acc0 = __fmaf_rn(xv.x, cv.x, acc0);
             acc1 = __fmaf_rn(xv.y, cv.y, acc1);
@@ -78,22 +87,24 @@ codes_kernel(const __grid_constant__ CodesArgs a) {
             acc3 = __fmaf_rn(xv.w, cv.w, acc3);
           }
           const float v = __fadd_rn(__fadd_rn(acc0, acc1), __fadd_rn(acc2, acc3));
-          sc[m] = v == v ? v : -INFINITY;
-          ki[m] = k;
+          key[m] = ordered_bits(v == v ? v : -INFINITY);
         }
       }
       for (int rnd = 0; rnd < need; ++rnd) {
-        float bsc = sc[0];
-        int bi = ki[0];
+        // This lane's best: highest key, lowest index (m ascending).
+        uint32_t lk = key[0];
+        int lm = 0;
 #pragma unroll
         for (int m = 1; m < kMaxK / 32; ++m)
-          if (better(sc[m], ki[m], bsc, bi)) { bsc = sc[m]; bi = ki[m]; }
-        warp_best(bsc, bi);
+          if (key[m] > lk) { lk = key[m]; lm = m; }
+        const uint32_t top = __reduce_max_sync(0xffffffffu, lk);
+        const int bi = static_cast<int>(
+            __reduce_min_sync(0xffffffffu, lk == top ? static_cast<uint32_t>(lane + 32 * lm) : 0xffffffffu));
         if (side == 0) {
           if (lane == 0) a.qcodes[(rr * a.P + sdx) * a.probes + rnd] = bi;
 #pragma unroll
           for (int m = 0; m < kMaxK / 32; ++m)
-            if (ki[m] == bi) { sc[m] = -INFINITY; ki[m] = 0x7fffffff; }
+            if (lane + 32 * m == bi) key[m] = 0;
         } else {
           addr = addr * a.K + bi;
         }
@@ -111,16 +122,25 @@ cudaError_t launch_codes(const CodesArgs& a, cudaStream_t st) {
   if (a.K > kMaxK || a.P > 4) return cudaErrorInvalidValue;
   const size_t smem =
       (static_cast<size_t>(a.P) * a.K * (a.D / a.P + 4) + static_cast<size_t>(kCodeWarps) * a.D) * sizeof(float);
-  cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(codes_kernel), static_cast<int>(smem));
+  void (*k)(CodesArgs) = nullptr;
+  switch (a.D / a.P / 4) {
+    case 2: k = codes_kernel<2>; break;
+    case 4: k = codes_kernel<4>; break;
+    case 8: k = codes_kernel<8>; break;
+    case 16: k = codes_kernel<16>; break;
+    case 32: k = codes_kernel<32>; break;
+    default: return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(k), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int sms = cached_sm_count();
-  int per_sm = cached_occupancy(reinterpret_cast<const void*>(codes_kernel), kCodeWarps * 32, smem);
+  int per_sm = cached_occupancy(reinterpret_cast<const void*>(k), kCodeWarps * 32, smem);
   if (sms <= 0) return cudaErrorUnknown;
   if (per_sm < 1) per_sm = 1;
   const long long need = (rows + kCodeWarps - 1) / kCodeWarps;
   const long long cap = static_cast<long long>(sms) * (per_sm < 2 ? per_sm : 2);
   const unsigned grid = static_cast<unsigned>(need < cap ? need : cap);
-  e = launch_pdl(codes_kernel, dim3(grid), dim3(kCodeWarps * 32), smem, st, a);
+  e = launch_pdl(k, dim3(grid), dim3(kCodeWarps * 32), smem, st, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
