@@ -130,10 +130,10 @@ route_kernel(const RouteArgs a) {
     {
       const int F4 = a.D / 4, cpi = 32 / F4, grp = lane / F4, pos = lane % F4;
       const float4 qv = reinterpret_cast<const float4*>(qs)[pos];
-      for (int c0 = 0; c0 < nbuf; c0 += 4 * cpi) {
-        float pr[4];
+      for (int c0 = 0; c0 < nbuf; c0 += 8 * cpi) {
+        float pr[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
           const int c = c0 + u * cpi + grp;
           pr[u] = 0.f;
           if (c < nbuf) {
@@ -141,9 +141,17 @@ route_kernel(const RouteArgs a) {
             pr[u] = __fmaf_rn(qv.w, kv.w, __fmaf_rn(qv.z, kv.z, __fmaf_rn(qv.y, kv.y, __fmul_rn(qv.x, kv.x))));
           }
         }
+        // Fixed butterfly over the F4 lanes of a group (F4 in {8, 16, 32});
+        // the levels are unrolled so the eight sums proceed side by side.
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          for (int o = F4 / 2; o > 0; o >>= 1) pr[u] = __fadd_rn(pr[u], __shfl_xor_sync(0xffffffffu, pr[u], o));
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float t = __shfl_xor_sync(0xffffffffu, pr[u], o);
+            if (o < F4) pr[u] = __fadd_rn(pr[u], t);
+          }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
           const int c = c0 + u * cpi + grp;
           if (pos == 0 && c < nbuf) score[c] = pr[u];
         }
@@ -170,6 +178,7 @@ route_kernel(const RouteArgs a) {
           eid[h] = cand[ce];
           esc[h] = score[ce];
           int r = 0;
+#pragma unroll 4
           for (int f = 0; f < T; ++f) {
             const int cf = f < nbuf ? f : kBatch + (f - nbuf);
             r += better(score[cf], cand[cf], esc[h], eid[h]) ? 1 : 0;
