@@ -29,6 +29,8 @@ import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
+# libmdr kernels one forward launches: summaries, codes, posting lists, route, attention.
+KERNELS_PER_FORWARD = 5
 sys.path.insert(0, ROOT)
 
 import numpy as np  # noqa: E402
@@ -97,7 +99,7 @@ class ClockSampler:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev),
                  "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
-                 "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                 "--format=csv,noheader,nounits", "-lms", "20", "-f", self.path],
                 stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -351,7 +353,7 @@ def run_mine(args, w):
                              "kernel": "attend", "algorithmic_bytes_per_launch": attn_bytes},
                 "path_roofline_frac": total_bytes / (ms_max / 1e3) / 1e9 / peak,
                 "kernels_ms": ker, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": 4 * args.steps, "clocks": clk.summary(),
+                "gpu_launches": KERNELS_PER_FORWARD * args.steps, "clocks": clk.summary(),
                 "overflow": int(idx.overflow.sum().item()), "selected_blocks": nsel}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -362,7 +364,7 @@ def run_mine(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--workload", default="scaling32k")
