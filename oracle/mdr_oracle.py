@@ -400,3 +400,123 @@ def forward(q, k, v, codebooks, p: Params, *, attention=True, rows=None, keep_sl
 def near_tie(margin, scale_ref) -> np.ndarray:
     """True where a float32 decision margin is below 1e-6*max(1,|s|)."""
     return np.asarray(margin) < TIE_REL * np.maximum(1.0, np.abs(scale_ref))
+
+
+# ------------------------------------------------------------------ 7. decode
+# Decoding one token at a time with an incremental index.  The pages ask that
+# a deployed decoder update its routing structures as tokens arrive and keep
+# causality ("Monodratic Claims Learned Routing Can Make Sparse Causal
+# Attention More Selective", the section on what a deployed decoder must do;
+# the bounded lists make the update O(1)).  Readings (listed with the others
+# in the design notes):
+#   * a block enters the index when its last token arrives: its summary is
+#     the mean of its rotated keys, its address is assigned as in the batch
+#     build, and it is appended to its list if the list holds fewer than cap
+#     blocks -- exactly the batch build run one block at a time, so a decoder
+#     and a prefill of the same prefix hold the same index;
+#   * the new token t is routed by its own rotated query (a block of one
+#     token), with eligibility i <= j - L and local blocks j-L+1..j taken
+#     from its block j = t // bs; the current block is partly filled and the
+#     causal mask keeps s <= t.
+
+
+def rope_at(x: np.ndarray, t: int, base: float) -> np.ndarray:
+    """Rotary embedding of vectors x [..., D] at the single position t (the
+    same float32 angles as rope())."""
+    D = x.shape[-1]
+    th = (np.float32(t) * rope_inv_freq(D, base)).astype(np.float32).astype(np.float64)
+    c, s = np.cos(th), np.sin(th)
+    x1, x2 = x[..., : D // 2], x[..., D // 2:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+@dataclass
+class DecodeState:
+    """Rotated keys and values seen so far and, per (sequence, KV head), the
+    summaries, addresses and bounded lists of the completed blocks."""
+    kr: np.ndarray          # [B, Smax, Hkv, D] rotated keys (positions < t)
+    v: np.ndarray           # [B, Smax, Hkv, D]
+    kbar: np.ndarray        # [B, Hkv, nbmax, D]
+    addr: np.ndarray        # [B, Hkv, nbmax] (-1 until the block completes)
+    lists: np.ndarray       # [B, Hkv, A, cap]
+    load: np.ndarray        # [B, Hkv, A]
+    t: int = 0              # tokens seen
+
+    @property
+    def overflow(self):
+        cap = self.lists.shape[-1]
+        return np.maximum(self.load - cap, 0).sum(axis=-1)
+
+    @property
+    def maxload(self):
+        return self.load.max(axis=-1)
+
+
+def decode_init(p: Params, B: int) -> DecodeState:
+    """Empty state for sequences of up to p.S tokens."""
+    return DecodeState(np.zeros((B, p.S, p.Hkv, p.D)), np.zeros((B, p.S, p.Hkv, p.D)),
+                       np.zeros((B, p.Hkv, p.nb, p.D)), np.full((B, p.Hkv, p.nb), -1, dtype=np.int64),
+                       np.full((B, p.Hkv, p.A, p.cap), -1, dtype=np.int64),
+                       np.zeros((B, p.Hkv, p.A), dtype=np.int64))
+
+
+def append_block(st: DecodeState, codebooks: np.ndarray, p: Params, j: int):
+    """Block j has all its tokens: summarise it, give it an address and append
+    it to its list if that list holds fewer than cap blocks (load counts it in
+    any case)."""
+    toks = st.kr[:, j * p.block:(j + 1) * p.block]                 # [B, bs, Hkv, D]
+    st.kbar[:, :, j] = toks.mean(axis=1)
+    addr, _, _ = assign_codes(st.kbar[:, :, j], codebooks)          # [B, Hkv]
+    st.addr[:, :, j] = addr
+    B, H = addr.shape
+    for b in range(B):
+        for h in range(H):
+            a = addr[b, h]
+            if st.load[b, h, a] < p.cap:
+                st.lists[b, h, a, st.load[b, h, a]] = j
+            st.load[b, h, a] += 1
+
+
+@dataclass
+class DecodeOut:
+    out: np.ndarray          # [B, Hq, D] attention output of token t
+    sel: np.ndarray          # [B, Hq, R+L]
+    sel_margin: np.ndarray   # [B, Hq] top-R margin (float32 scores)
+    qcodes: np.ndarray       # [B, Hq, P, p]
+    qcode_margin: np.ndarray  # [B, Hq, P]
+    ncand: np.ndarray        # [B, Hq]
+
+
+def decode_step(st: DecodeState, q_t, k_t, v_t, codebooks, p: Params) -> DecodeOut:
+    """Token t = st.t of every sequence: store its rotated key and value,
+    complete a block if t is its last token, then route the token by its
+    rotated query and attend over the selected tokens s <= t.
+    q_t [B, Hq, D], k_t and v_t [B, Hkv, D] (stored inputs)."""
+    t = st.t
+    q_t, k_t, v_t = (np.asarray(x, dtype=np.float64) for x in (q_t, k_t, v_t))
+    st.kr[:, t] = rope_at(k_t, t, p.rope_base)
+    st.v[:, t] = v_t
+    if (t + 1) % p.block == 0:
+        append_block(st, codebooks, p, t // p.block)
+    qr = rope_at(q_t, t, p.rope_base)                                # [B, Hq, D]
+    qcodes, qmargin = probe_codes(qr, codebooks, p.probes)
+    B, Hq, D = qr.shape
+    g = Hq // p.Hkv
+    j = t // p.block
+    sel = np.empty((B, Hq, p.R + p.L), dtype=np.int64)
+    smargin = np.empty((B, Hq))
+    ncand = np.empty((B, Hq), dtype=np.int64)
+    out = np.empty((B, Hq, v_t.shape[-1]))
+    for b in range(B):
+        for hq in range(Hq):
+            h = hq // g
+            row = route_row(qr[b, hq], st.kbar[b, h], probe_addresses(qcodes[b, hq], p.K),
+                            st.lists[b, h], j, p.R, p.L)
+            sel[b, hq], smargin[b, hq], ncand[b, hq] = row.sel, row.margin, row.cand.size
+            toks = selected_tokens(row.sel, p.block)
+            toks = toks[toks <= t]
+            s = (st.kr[b, toks, h] @ qr[b, hq]) * p.softmax_scale
+            w = np.exp(s - s.max())
+            out[b, hq] = (w @ st.v[b, toks, h]) / w.sum()
+    st.t = t + 1
+    return DecodeOut(out, sel, smargin, qcodes, qmargin, ncand)
