@@ -220,6 +220,66 @@ mdr_status mdr_route_noalloc(const mdr_config* cfg, const void* q,
                              const float* codebooks, const mdr_index* idx,
                              int32_t* sel, int32_t* ncand, void* stream);
 
+/* ------------------------------------------------------------- decoding
+ * One token at a time with an incremental index.  The pages leave decoding
+ * open and ask that a deployed decoder update its routing structures as
+ * tokens arrive while keeping causality (Article, on what a deployed decoder
+ * must do; bounded lists keep each update O(1)).  Here a block enters the
+ * index when its last token arrives -- summary, address and list append as
+ * in mdr_build_index, so a decoder and a prefill of the same prefix hold the
+ * same lists -- and the new token t of block j = t / block is routed by its
+ * own rotated query (a block of one token): candidates i <= j-L from the
+ * probed lists, top R by <q'_t, kbar_i>, locals j-L+1..j, then causal
+ * softmax over the selected tokens s <= t.
+ *
+ * Decode state: everything a decoder keeps between tokens; device memory,
+ * caller-owned, sized by cfg (S = capacity in tokens, nb = S / block).
+ *   krot  cfg->dtype [B,S,Hkv,D]  rotated keys of the tokens seen so far.
+ *   v     cfg->dtype [B,S,Hkv,D]  their values.
+ *   ksum  float32    [B,Hkv,D]    float32 sum of the rotated keys of the
+ *                                 current, incomplete block (its summary is
+ *                                 taken from these, not from the rounded
+ *                                 cache).
+ *   idx   mdr_index of the completed blocks (kbar and addr rows of blocks
+ *         not yet complete are undefined).                                */
+typedef struct mdr_decode_state {
+  void* krot;
+  void* v;
+  float* ksum;
+  mdr_index idx;
+} mdr_decode_state;
+
+/* Device workspace mdr_decode_prefill and mdr_decode_step need, in bytes
+ * (host only); the first 4 bytes are the device status word.              */
+mdr_status mdr_decode_workspace_bytes(const mdr_config* cfg, size_t* bytes);
+
+/* Empty state (no token seen): lists -1, load, overflow, maxload and ksum 0. */
+mdr_status mdr_decode_reset(const mdr_config* cfg, const mdr_decode_state* st,
+                            void* stream);
+
+/* State after the first S0 tokens (0 <= S0 <= cfg->S, S0 % block == 0):
+ * rotates their keys into st->krot, copies their values into st->v and
+ * builds the index of their S0/block blocks with the prefill kernels; the
+ * rest of the state is reset.  k, v: device [B,S0,Hkv,D]; codebooks: device. */
+mdr_status mdr_decode_prefill(const mdr_config* cfg, int32_t S0, const void* k,
+                              const void* v, const float* codebooks,
+                              const mdr_decode_state* st, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* One token at position t (0 <= t < cfg->S) of every sequence; the state
+ * must hold tokens 0..t-1 (from mdr_decode_prefill and earlier steps; the
+ * library cannot check this).  Stores the token's rotated key and value,
+ * completes block t/block when t is its last token, routes the token and
+ * writes its attention output.  q_t: device [B,Hq,D]; k_t, v_t: device
+ * [B,Hkv,D]; out_t: device [B,Hq,D] (all cfg->dtype); sel_t: device int32
+ * [B,Hq,R+L] (remote ids ascending, -1 pads, then the locals; required);
+ * ncand_t: device int32 [B,Hq] eligible candidates found (may be NULL).     */
+mdr_status mdr_decode_step(const mdr_config* cfg, int32_t t, const void* q_t,
+                           const void* k_t, const void* v_t,
+                           const float* codebooks, const mdr_decode_state* st,
+                           void* out_t, int32_t* sel_t, int32_t* ncand_t,
+                           void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronise the stream and copy the device status word (first 4 bytes of
  * ws) to *code (0 = no device-side failure).  Returns MDR_ERR_DEVICE when the
  * word is nonzero.                                                           */

@@ -80,4 +80,29 @@ struct AttendArgs {
 cudaError_t launch_attend_simt(const AttendArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t st);
 
+// K6: one decode step (token t of every sequence) on a caller-owned state.
+struct DecodeArgs {
+  int t;                   // position of the new token
+  const void* q_t;         // [B,Hq,D]
+  const void* k_t;         // [B,Hkv,D]
+  const void* v_t;         // [B,Hkv,D]
+  void* krot;              // state: rotated keys [B,S,Hkv,D]
+  void* v;                 // state: values [B,S,Hkv,D]
+  float* ksum;             // state: float32 sum of the current block's rotated keys [B,Hkv,D]
+  float* kbar;             // state index [B,Hkv,nb,D]
+  int32_t* addr;           // [B,Hkv,nb]
+  int32_t* lists;          // [B,Hkv,A,cap]
+  int32_t* load;           // [B,Hkv,A]
+  int32_t* overflow;       // [B,Hkv]
+  int32_t* maxload;        // [B,Hkv]
+  const float* codebooks;  // [P,K,D/P]
+  void* out_t;             // [B,Hq,D]
+  int32_t* sel_t;          // [B,Hq,R+L]
+  int32_t* ncand_t;        // [B,Hq] or null
+  int B, S, Hq, Hkv, D, bs, nb, P, K, A, cap, probes, R, L;
+  float scale;
+  float inv_freq[64];      // omega_i, i < D/2
+};
+cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t st);
+
 }  // namespace mdr

@@ -77,6 +77,25 @@ Layout layout_of(const mdr_config* c) {
   return l;
 }
 
+// Decode workspace: the status word, then (for mdr_decode_prefill) the
+// rotated keys, summaries and addresses of the prefix at the prefix's own
+// strides before they are copied into the state's rows.
+struct DecodeLayout {
+  size_t status, krot, kbar, addr, total;
+};
+
+DecodeLayout decode_layout_of(const mdr_config* c) {
+  const size_t nb = c->S / c->block;
+  DecodeLayout l{};
+  size_t o = 0;
+  l.status = o; o += align_up(16);
+  l.krot = o;   o += align_up(static_cast<size_t>(c->B) * c->S * c->Hkv * c->D * esize(c));
+  l.kbar = o;   o += align_up(static_cast<size_t>(c->B) * c->Hkv * nb * c->D * sizeof(float));
+  l.addr = o;   o += align_up(static_cast<size_t>(c->B) * c->Hkv * nb * sizeof(int32_t));
+  l.total = o;
+  return l;
+}
+
 template <typename T>
 T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
 
@@ -365,6 +384,121 @@ mdr_status mdr_read_device_status(const void* ws, int32_t* code, void* stream) {
   MDR_CUDA(cudaStreamSynchronize(st));
   MDR_CUDA(cudaMemcpy(code, ws, sizeof(int32_t), cudaMemcpyDeviceToHost));
   return *code == 0 ? MDR_OK : MDR_ERR_DEVICE;
+}
+
+
+// ------------------------------------------------------------------ decoding
+static mdr_status check_decode_state(const mdr_decode_state* st) {
+  if (!st || !st->krot || !st->v || !st->ksum) return MDR_ERR_INVALID_ARG;
+  if (!aligned16(st->krot) || !aligned16(st->v) || !aligned16(st->ksum) || !aligned16(st->idx.kbar))
+    return MDR_ERR_INVALID_ARG;
+  return check_index(&st->idx);
+}
+
+static mdr_status check_decode_ws(const mdr_config* c, void* ws, size_t ws_bytes) {
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % kAlign != 0) return MDR_ERR_WORKSPACE;
+  if (ws_bytes < decode_layout_of(c).total) return MDR_ERR_WORKSPACE;
+  return MDR_OK;
+}
+
+mdr_status mdr_decode_workspace_bytes(const mdr_config* cfg, size_t* bytes) {
+  MDR_TRY(check(cfg));
+  if (!bytes) return MDR_ERR_INVALID_ARG;
+  *bytes = decode_layout_of(cfg).total;
+  return MDR_OK;
+}
+
+mdr_status mdr_decode_reset(const mdr_config* cfg, const mdr_decode_state* st, void* stream) {
+  MDR_TRY(check(cfg));
+  MDR_TRY(check_decode_state(st));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bh = static_cast<size_t>(cfg->B) * cfg->Hkv, A = static_cast<size_t>(ipow(cfg->K, cfg->P));
+  const size_t nb = cfg->S / cfg->block;
+  MDR_CUDA(cudaMemsetAsync(st->idx.lists, 0xff, bh * A * cfg->cap * sizeof(int32_t), s));
+  MDR_CUDA(cudaMemsetAsync(st->idx.addr, 0xff, bh * nb * sizeof(int32_t), s));
+  MDR_CUDA(cudaMemsetAsync(st->idx.load, 0, bh * A * sizeof(int32_t), s));
+  MDR_CUDA(cudaMemsetAsync(st->idx.overflow, 0, bh * sizeof(int32_t), s));
+  MDR_CUDA(cudaMemsetAsync(st->idx.maxload, 0, bh * sizeof(int32_t), s));
+  MDR_CUDA(cudaMemsetAsync(st->ksum, 0, bh * cfg->D * sizeof(float), s));
+  return MDR_OK;
+}
+
+mdr_status mdr_decode_prefill(const mdr_config* cfg, int32_t S0, const void* k, const void* v,
+                              const float* codebooks, const mdr_decode_state* st, void* ws,
+                              size_t ws_bytes, void* stream) {
+  MDR_TRY(check(cfg));
+  MDR_TRY(check_decode_state(st));
+  if (S0 < 0 || S0 > cfg->S || S0 % cfg->block != 0) return MDR_ERR_INVALID_ARG;
+  if (S0 > 0 && (!k || !v || !codebooks || !aligned16(k) || !aligned16(v))) return MDR_ERR_INVALID_ARG;
+  MDR_TRY(check_decode_ws(cfg, ws, ws_bytes));
+  MDR_TRY(mdr_decode_reset(cfg, st, stream));
+  if (S0 == 0) return MDR_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const DecodeLayout l = decode_layout_of(cfg);
+  int32_t* status = at<int32_t>(ws, l.status);
+  MDR_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+  mdr_config c0 = *cfg;
+  c0.S = S0;
+  const size_t nb = cfg->S / cfg->block, nb0 = S0 / cfg->block, e = esize(cfg);
+  const size_t rows_k = static_cast<size_t>(cfg->Hkv) * cfg->D * e;          // bytes of one token's keys
+  // The prefix's rows land in place when the strides agree; else in the
+  // workspace, then copied.
+  const bool k_in_place = cfg->B == 1 || S0 == cfg->S;
+  const bool kbar_in_place = static_cast<size_t>(cfg->B) * cfg->Hkv == 1 || nb0 == nb;
+  void* krot0 = k_in_place ? st->krot : at<void>(ws, l.krot);
+  float* kbar0 = kbar_in_place ? st->idx.kbar : at<float>(ws, l.kbar);
+  int32_t* addr0 = kbar_in_place ? st->idx.addr : at<int32_t>(ws, l.addr);
+  SummarizeArgs a;
+  fill_common(a, &c0, codebooks);
+  a.x[1] = k; a.xrot[1] = krot0; a.xbar[1] = kbar0; a.addr = addr0;
+  a.lists_fill = st->idx.lists;
+  a.lists_per_seq = static_cast<size_t>(cfg->Hkv) * ipow(cfg->K, cfg->P) * cfg->cap;
+  a.status = status;
+  MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, s));
+  mdr_index idx0 = st->idx;
+  idx0.kbar = kbar0;
+  idx0.addr = addr0;
+  MDR_TRY(run_lists(&c0, &idx0, s));
+  if (!k_in_place)
+    MDR_CUDA(cudaMemcpy2DAsync(st->krot, cfg->S * rows_k, krot0, S0 * rows_k, S0 * rows_k, cfg->B,
+                               cudaMemcpyDeviceToDevice, s));
+  MDR_CUDA(cudaMemcpy2DAsync(st->v, cfg->S * rows_k, v, S0 * rows_k, S0 * rows_k, cfg->B,
+                             cudaMemcpyDeviceToDevice, s));
+  if (!kbar_in_place) {
+    const size_t bh = static_cast<size_t>(cfg->B) * cfg->Hkv;
+    MDR_CUDA(cudaMemcpy2DAsync(st->idx.kbar, nb * cfg->D * sizeof(float), kbar0, nb0 * cfg->D * sizeof(float),
+                               nb0 * cfg->D * sizeof(float), bh, cudaMemcpyDeviceToDevice, s));
+    MDR_CUDA(cudaMemcpy2DAsync(st->idx.addr, nb * sizeof(int32_t), addr0, nb0 * sizeof(int32_t),
+                               nb0 * sizeof(int32_t), bh, cudaMemcpyDeviceToDevice, s));
+  }
+  return MDR_OK;
+}
+
+mdr_status mdr_decode_step(const mdr_config* cfg, int32_t t, const void* q_t, const void* k_t,
+                           const void* v_t, const float* codebooks, const mdr_decode_state* st,
+                           void* out_t, int32_t* sel_t, int32_t* ncand_t, void* ws, size_t ws_bytes,
+                           void* stream) {
+  MDR_TRY(check(cfg));
+  MDR_TRY(check_decode_state(st));
+  if (t < 0 || t >= cfg->S) return MDR_ERR_INVALID_ARG;
+  if (!q_t || !k_t || !v_t || !codebooks || !out_t || !sel_t || !aligned16(codebooks)) return MDR_ERR_INVALID_ARG;
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % kAlign != 0 || ws_bytes < 16) return MDR_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MDR_CUDA(cudaMemsetAsync(ws, 0, sizeof(int32_t), s));
+  mdr::DecodeArgs d;
+  std::memset(&d, 0, sizeof(d));
+  d.t = t; d.q_t = q_t; d.k_t = k_t; d.v_t = v_t;
+  d.krot = st->krot; d.v = st->v; d.ksum = st->ksum;
+  d.kbar = st->idx.kbar; d.addr = st->idx.addr; d.lists = st->idx.lists; d.load = st->idx.load;
+  d.overflow = st->idx.overflow; d.maxload = st->idx.maxload;
+  d.codebooks = codebooks; d.out_t = out_t; d.sel_t = sel_t; d.ncand_t = ncand_t;
+  d.B = cfg->B; d.S = cfg->S; d.Hq = cfg->Hq; d.Hkv = cfg->Hkv; d.D = cfg->D; d.bs = cfg->block;
+  d.nb = cfg->S / cfg->block; d.P = cfg->P; d.K = cfg->K; d.A = ipow(cfg->K, cfg->P); d.cap = cfg->cap;
+  d.probes = cfg->probes; d.R = cfg->R; d.L = cfg->L;
+  d.scale = cfg->scale > 0.f ? cfg->scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(cfg->D)));
+  for (int i = 0; i < cfg->D / 2; ++i)
+    d.inv_freq[i] = static_cast<float>(std::pow(static_cast<double>(cfg->rope_base), -2.0 * i / cfg->D));
+  return cuda_status(mdr::launch_decode(d, cfg->dtype == MDR_BF16, s));
 }
 
 }  // extern "C"

@@ -21,6 +21,7 @@ EXPORTED = (
     "mdr_abi_version", "mdr_status_string", "mdr_check_config", "mdr_workspace_bytes",
     "mdr_build_index", "mdr_route", "mdr_attend", "mdr_forward", "mdr_host_workspace_bytes",
     "mdr_forward_host", "mdr_read_device_status", "mdr_forward_profiled", "mdr_route_noalloc",
+    "mdr_decode_workspace_bytes", "mdr_decode_reset", "mdr_decode_prefill", "mdr_decode_step",
 )
 
 
@@ -42,6 +43,10 @@ class mdr_index(ctypes.Structure):
 
 class mdr_route_out(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("sel", "qbar", "qcodes", "ncand")]
+
+
+class mdr_decode_state(ctypes.Structure):
+    _fields_ = [("krot", ctypes.c_void_p), ("v", ctypes.c_void_p), ("ksum", ctypes.c_void_p), ("idx", mdr_index)]
 
 
 _lib = None
@@ -74,6 +79,12 @@ def lib() -> ctypes.CDLL:
             "mdr_forward_profiled": ([cfgp, vp, vp, vp, vp, idxp, rtp, vp, vp, sz, vp,
                                       ctypes.POINTER(vp), ctypes.c_int32], i32),
             "mdr_route_noalloc": ([cfgp, vp, vp, idxp, vp, vp, vp], i32),
+            "mdr_decode_workspace_bytes": ([cfgp, ctypes.POINTER(sz)], i32),
+            "mdr_decode_reset": ([cfgp, ctypes.POINTER(mdr_decode_state), vp], i32),
+            "mdr_decode_prefill": ([cfgp, ctypes.c_int32, vp, vp, vp, ctypes.POINTER(mdr_decode_state),
+                                    vp, sz, vp], i32),
+            "mdr_decode_step": ([cfgp, ctypes.c_int32, vp, vp, vp, vp, ctypes.POINTER(mdr_decode_state),
+                                 vp, vp, vp, vp, sz, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -237,3 +248,54 @@ def mdr_route_noalloc(cfg, q, codebooks, idx: Index, sel, ncand=None, stream=Non
     callers that cannot allocate device memory); see include/mdr.h."""
     _ok(lib().mdr_route_noalloc(ctypes.byref(cfg), _ptr(q), _ptr(codebooks), ctypes.byref(idx.c()),
                                 _ptr(sel), _ptr(ncand), _stream(stream)), "mdr_route_noalloc")
+
+
+# ------------------------------------------------------------------ decoding
+def mdr_decode_workspace_bytes(cfg: mdr_config) -> int:
+    n = ctypes.c_size_t(0)
+    _ok(lib().mdr_decode_workspace_bytes(ctypes.byref(cfg), ctypes.byref(n)), "mdr_decode_workspace_bytes")
+    return n.value
+
+
+@dataclass
+class DecodeState:
+    """Device buffers of mdr_decode_state (torch tensors); cfg.S is the
+    capacity in tokens."""
+    krot: object
+    v: object
+    ksum: object
+    idx: Index
+
+    @classmethod
+    def empty(cls, cfg: mdr_config, device="cuda") -> "DecodeState":
+        import torch
+        dt = torch.bfloat16 if cfg.dtype == MDR_BF16 else torch.float32
+        return cls(torch.empty(cfg.B, cfg.S, cfg.Hkv, cfg.D, dtype=dt, device=device),
+                   torch.empty(cfg.B, cfg.S, cfg.Hkv, cfg.D, dtype=dt, device=device),
+                   torch.empty(cfg.B, cfg.Hkv, cfg.D, dtype=torch.float32, device=device),
+                   Index.empty(cfg, device))
+
+    def c(self) -> mdr_decode_state:
+        return mdr_decode_state(_ptr(self.krot), _ptr(self.v), _ptr(self.ksum), self.idx.c())
+
+
+def decode_workspace(cfg: mdr_config, device="cuda"):
+    import torch
+    return torch.empty(mdr_decode_workspace_bytes(cfg), dtype=torch.uint8, device=device)
+
+
+def mdr_decode_reset(cfg, st: DecodeState, stream=None):
+    _ok(lib().mdr_decode_reset(ctypes.byref(cfg), ctypes.byref(st.c()), _stream(stream)), "mdr_decode_reset")
+
+
+def mdr_decode_prefill(cfg, S0: int, k, v, codebooks, st: DecodeState, ws, stream=None):
+    _ok(lib().mdr_decode_prefill(ctypes.byref(cfg), int(S0), _ptr(k), _ptr(v), _ptr(codebooks),
+                                 ctypes.byref(st.c()), _ptr(ws), ws.numel(), _stream(stream)),
+        "mdr_decode_prefill")
+
+
+def mdr_decode_step(cfg, t: int, q_t, k_t, v_t, codebooks, st: DecodeState, out_t, sel_t, ws,
+                    ncand_t=None, stream=None):
+    _ok(lib().mdr_decode_step(ctypes.byref(cfg), int(t), _ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(codebooks),
+                              ctypes.byref(st.c()), _ptr(out_t), _ptr(sel_t), _ptr(ncand_t), _ptr(ws),
+                              ws.numel(), _stream(stream)), "mdr_decode_step")

@@ -485,6 +485,8 @@ class DecodeOut:
     qcodes: np.ndarray       # [B, Hq, P, p]
     qcode_margin: np.ndarray  # [B, Hq, P]
     ncand: np.ndarray        # [B, Hq]
+    qcode_scale: np.ndarray  # [B, Hq, P] largest |codeword score| (reference for near ties)
+    sel_scale: np.ndarray    # [B, Hq] largest |candidate score| (reference for near ties)
 
 
 def decode_step(st: DecodeState, q_t, k_t, v_t, codebooks, p: Params) -> DecodeOut:
@@ -500,12 +502,14 @@ def decode_step(st: DecodeState, q_t, k_t, v_t, codebooks, p: Params) -> DecodeO
         append_block(st, codebooks, p, t // p.block)
     qr = rope_at(q_t, t, p.rope_base)                                # [B, Hq, D]
     qcodes, qmargin = probe_codes(qr, codebooks, p.probes)
+    qscale = np.abs(codeword_scores(qr, codebooks)).max(axis=-1)
     B, Hq, D = qr.shape
     g = Hq // p.Hkv
     j = t // p.block
     sel = np.empty((B, Hq, p.R + p.L), dtype=np.int64)
     smargin = np.empty((B, Hq))
     ncand = np.empty((B, Hq), dtype=np.int64)
+    sscale = np.zeros((B, Hq))
     out = np.empty((B, Hq, v_t.shape[-1]))
     for b in range(B):
         for hq in range(Hq):
@@ -513,10 +517,11 @@ def decode_step(st: DecodeState, q_t, k_t, v_t, codebooks, p: Params) -> DecodeO
             row = route_row(qr[b, hq], st.kbar[b, h], probe_addresses(qcodes[b, hq], p.K),
                             st.lists[b, h], j, p.R, p.L)
             sel[b, hq], smargin[b, hq], ncand[b, hq] = row.sel, row.margin, row.cand.size
+            sscale[b, hq] = np.abs(row.scores).max() if row.scores.size else 0.0
             toks = selected_tokens(row.sel, p.block)
             toks = toks[toks <= t]
             s = (st.kr[b, toks, h] @ qr[b, hq]) * p.softmax_scale
             w = np.exp(s - s.max())
             out[b, hq] = (w @ st.v[b, toks, h]) / w.sum()
     st.t = t + 1
-    return DecodeOut(out, sel, smargin, qcodes, qmargin, ncand)
+    return DecodeOut(out, sel, smargin, qcodes, qmargin, ncand, qscale, sscale)

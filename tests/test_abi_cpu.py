@@ -104,3 +104,29 @@ def test_status_strings():
     for s in range(6):
         assert mdr.status_string(s)
     assert mdr.status_string(99) == "unknown status"
+
+
+def test_decode_entry_points_check_arguments_before_any_gpu_work():
+    L = mdr.lib()
+    cfg = mdr.make_config(TINY)
+    assert mdr.mdr_decode_workspace_bytes(cfg) > 0
+    fake = ctypes.c_void_p(0x10000)            # 16-byte aligned, never dereferenced: checks fail first
+    st = mdr.mdr_decode_state(fake, fake, fake, mdr.mdr_index(fake, fake, fake, fake, fake, fake))
+    n = mdr.mdr_decode_workspace_bytes(cfg)
+    step = lambda t, **kw: L.mdr_decode_step(
+        ctypes.byref(kw.get("cfg", cfg)), t, fake, fake, fake, fake, ctypes.byref(kw.get("st", st)),
+        fake, kw.get("sel", fake), None, kw.get("ws", ctypes.c_void_p(0x100000)), kw.get("n", n), None)
+    assert step(-1) == mdr.MDR_ERR_INVALID_ARG                       # before the first position
+    assert step(TINY.S) == mdr.MDR_ERR_INVALID_ARG                   # past the capacity
+    assert step(0, sel=None) == mdr.MDR_ERR_INVALID_ARG              # sel is required
+    assert step(0, ws=None) == mdr.MDR_ERR_WORKSPACE
+    assert step(0, ws=ctypes.c_void_p(0x100010)) == mdr.MDR_ERR_WORKSPACE   # not 256-byte aligned
+    nost = mdr.mdr_decode_state(None, fake, fake, mdr.mdr_index(fake, fake, fake, fake, fake, fake))
+    assert step(0, st=nost) == mdr.MDR_ERR_INVALID_ARG               # state without a key cache
+    bad = mdr.make_config(TINY.with_(S=100))
+    assert step(0, cfg=bad) == mdr.MDR_ERR_INVALID_ARG
+    pre = lambda S0, nbytes=n: L.mdr_decode_prefill(ctypes.byref(cfg), S0, fake, fake, fake, ctypes.byref(st),
+                                                    ctypes.c_void_p(0x100000), nbytes, None)
+    assert pre(TINY.block + 1) == mdr.MDR_ERR_INVALID_ARG             # not a whole number of blocks
+    assert pre(TINY.S + TINY.block) == mdr.MDR_ERR_INVALID_ARG        # past the capacity
+    assert pre(TINY.block, nbytes=n - 1) == mdr.MDR_ERR_WORKSPACE
