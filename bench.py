@@ -307,6 +307,53 @@ def run_mine(args, w):
     achieved = attn_bytes / (ker["attend"] / 1e3) / 1e9
     total_bytes = (w.Hq + w.Hkv) * w.S * w.D * es * w.B + attn_bytes
 
+    # Decoding: the state of the first nb-1 blocks (prefill), then one token
+    # per sequence at a time through the last block, timed with CUDA events
+    # over consecutive steps (no block completes inside the timed steps).
+    decode = None
+    if not args.no_decode:
+        dst = mdr.DecodeState.empty(cfg, dev)
+        dws = mdr.decode_workspace(cfg, dev)
+        S0 = w.S - w.block
+        mdr.mdr_decode_prefill(cfg, S0, k[:, :S0].contiguous(), v[:, :S0].contiguous(), cb, dst, dws)
+        n_dec = min(60, w.block - 1)
+        toks = [(q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous()) for t in range(S0, S0 + n_dec)]
+        out_t = torch.empty(w.B, w.Hq, w.D, dtype=q.dtype, device=dev)
+        sel_t = torch.empty(w.B, w.Hq, w.R + w.L, dtype=torch.int32, device=dev)
+        for i in range(3):
+            mdr.mdr_decode_step(cfg, S0 + i, *toks[i], cb, dst, out_t, sel_t, dws)
+        torch.cuda.synchronize()
+        # The C entry point with its arguments marshalled once, so that the
+        # host stays ahead of the GPU and the events time the device work.
+        import ctypes
+        fn = mdr.lib().mdr_decode_step
+        cfg_r, st_r = ctypes.byref(cfg), ctypes.byref(dst.c())
+        sp = stream.cuda_stream
+        calls = [(cfg_r, S0 + i, qq.data_ptr(), kk.data_ptr(), vv.data_ptr(), cb.data_ptr(), st_r,
+                  out_t.data_ptr(), sel_t.data_ptr(), None, dws.data_ptr(), dws.numel(), sp)
+                 for i, (qq, kk, vv) in enumerate(toks)]
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for c_args in calls:
+            if fn(*c_args) != mdr.MDR_OK:
+                raise RuntimeError("mdr_decode_step failed")
+        d1.record(stream)
+        d1.synchronize()
+        assert mdr.mdr_read_device_status(dws) == 0
+        d_ms = d0.elapsed_time(d1) / n_dec
+        t_last = S0 + n_dec - 1
+        sl = sel_t.cpu().numpy()
+        ntok = int(sum(min(w.block, t_last + 1 - int(blk) * w.block) for blk in sl.ravel() if blk >= 0))
+        d_bytes = ntok * 2 * w.D * es + 2 * w.B * w.Hq * w.D * es     # gathered K, V + q, out
+        d_ms_max = max_over_ranks(d_ms, dist, world, dev)
+        decode = {"metric": "decode step latency (one token per sequence: key append, route, attend) at 32K",
+                  "value": d_ms_max * 1e3, "unit": "us/step", "tokens_per_s": w.B * world / (d_ms_max / 1e3),
+                  "batch_per_gpu": w.B, "steps": n_dec, "position": f"tokens {S0}..{t_last} ({S0 // w.block} blocks indexed)",
+                  "l2": "not flushed between steps", "gpu_launches": 2 * n_dec,
+                  "roofline": {"bound": "hbm", "achieved": d_bytes / (d_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                               "frac": d_bytes / (d_ms / 1e3) / 1e9 / peak, "algorithmic_bytes_per_step": d_bytes}}
+        del dst, dws
+
     # End to end through the C ABI with host buffers.
     e2e = None
     if not args.no_e2e:
@@ -352,7 +399,7 @@ def run_mine(args, w):
                              "peak_kind": peak_kind,
                              "kernel": "attend", "algorithmic_bytes_per_launch": attn_bytes},
                 "path_roofline_frac": total_bytes / (ms_max / 1e3) / 1e9 / peak,
-                "kernels_ms": ker, "cpu_baseline": cpu, "e2e": e2e,
+                "kernels_ms": ker, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
                 "gpu_launches": KERNELS_PER_FORWARD * args.steps, "clocks": clk.summary(),
                 "overflow": int(idx.overflow.sum().item()), "selected_blocks": nsel}
         print(json.dumps(line), flush=True)
@@ -369,6 +416,7 @@ def main():
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--workload", default="scaling32k")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()

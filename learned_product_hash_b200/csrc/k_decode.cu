@@ -11,7 +11,7 @@
 // same lists); the new token is routed by its own rotated query (a block of
 // one token) and attends causally over the selected tokens.
 //
-// Two kernels, chained by programmatic dependent launch:
+// Three kernels, chained by programmatic dependent launch:
 //   decode_keys_kernel    one CTA per (b, KV head): rotate k_t into the key
 //                         cache, copy v_t, add the rotated key (float32) to
 //                         the running sum of the block; when t completes its
@@ -20,17 +20,20 @@
 //                         address, and the O(1) list append (stored when the
 //                         list holds fewer than cap blocks; load, overflow
 //                         and maximum load updated).
-//   decode_attend_kernel  one CTA per (b, query head), eight warps: rotate
+//   decode_route_kernel   one CTA per (b, query head), eight warps: rotate
 //                         q_t; probe codes of each subspace (top p, best
 //                         first); route (warp 0): all probes' list lengths at
 //                         once, slots read 32 at a time and filtered to
-//                         i <= j - L, candidates scored <q'_t, kbar_i> in
-//                         float32, top R by rounds of warp arg-max (higher
-//                         score, lower id), remote ids ascending, then the
-//                         locals; attention: the selected tokens s <= t are
-//                         split over the eight warps, each with a float32
-//                         online softmax (lanes hold D/32 coordinates of the
-//                         key and value rows it reads), merged at the end.
+//                         i <= j - L; candidates scored <q'_t, kbar_i> in
+//                         float32 by all warps; top R by rounds of warp
+//                         arg-max (higher score, lower id), remote ids
+//                         ascending, then the locals.
+//   decode_partial_kernel one CTA per (b, query head, selected block): the
+//                         block's tokens s <= t with a float32 online softmax
+//                         (split-K over the selected blocks, so that a
+//                         single token's gathers run on many SMs at once);
+//                         the last CTA of a (b, query head) merges the blocks'
+//                         (max, sum, output) in slot order into the output.
 
 #include <climits>
 
@@ -60,6 +63,31 @@ template <typename T> __device__ __forceinline__ T st_f(float x);
 template <> __device__ __forceinline__ float st_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 st_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// vpl (1, 2 or 4) consecutive elements at p (aligned to vpl elements) as floats.
+__device__ __forceinline__ void ld_vec(const float* p, int vpl, float* o) {
+  if (vpl == 4) {
+    const float4 f = *reinterpret_cast<const float4*>(p);
+    o[0] = f.x; o[1] = f.y; o[2] = f.z; o[3] = f.w;
+  } else if (vpl == 2) {
+    const float2 f = *reinterpret_cast<const float2*>(p);
+    o[0] = f.x; o[1] = f.y;
+  } else {
+    o[0] = *p;
+  }
+}
+__device__ __forceinline__ void ld_vec(const __nv_bfloat16* p, int vpl, float* o) {
+  if (vpl == 4) {
+    const uint2 r = *reinterpret_cast<const uint2*>(p);
+    o[0] = __uint_as_float(r.x << 16); o[1] = __uint_as_float(r.x & 0xffff0000u);
+    o[2] = __uint_as_float(r.y << 16); o[3] = __uint_as_float(r.y & 0xffff0000u);
+  } else if (vpl == 2) {
+    const uint32_t r = *reinterpret_cast<const uint32_t*>(p);
+    o[0] = __uint_as_float(r << 16); o[1] = __uint_as_float(r & 0xffff0000u);
+  } else {
+    o[0] = __bfloat162float(*p);
+  }
+}
+
 // Score of codeword k of subspace sdx against xs (dsub floats, shared
 // memory): four float32 partial sums over d mod 4, added pairwise.
 __device__ __forceinline__ float codeword_score(const float* xs, const float* codebooks, int sdx, int k, int K,
@@ -67,12 +95,20 @@ __device__ __forceinline__ float codeword_score(const float* xs, const float* co
   const float4* cw = reinterpret_cast<const float4*>(codebooks + (static_cast<size_t>(sdx) * K + k) * dsub);
   const float4* x4 = reinterpret_cast<const float4*>(xs);
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  for (int d4 = 0; d4 < dsub / 4; ++d4) {
-    const float4 xv = x4[d4], cv = __ldg(cw + d4);
-    a0 = __fmaf_rn(xv.x, cv.x, a0);
-    a1 = __fmaf_rn(xv.y, cv.y, a1);
-    a2 = __fmaf_rn(xv.z, cv.z, a2);
-    a3 = __fmaf_rn(xv.w, cv.w, a3);
+  for (int c0 = 0; c0 < dsub / 4; c0 += 8) {      // eight row loads in flight (dsub/4 is a power of two)
+    float4 cv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (c0 + u < dsub / 4) cv[u] = __ldg(cw + c0 + u);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (c0 + u < dsub / 4) {
+        const float4 xv = x4[c0 + u];
+        a0 = __fmaf_rn(xv.x, cv[u].x, a0);
+        a1 = __fmaf_rn(xv.y, cv[u].y, a1);
+        a2 = __fmaf_rn(xv.z, cv[u].z, a2);
+        a3 = __fmaf_rn(xv.w, cv[u].w, a3);
+      }
   }
   const float v = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
   return v == v ? v : -INFINITY;
@@ -155,32 +191,26 @@ decode_keys_kernel(const __grid_constant__ DecodeArgs a) {
   }
 }
 
-// Shared memory of decode_attend_kernel, in 4-byte words.
+// Shared memory of decode_route_kernel, in 4-byte words.
 constexpr int kDecQ = 0;                          // rotated query [D <= 128]
 constexpr int kDecCode = kDecQ + 128;             // probe codes [P * probes <= 64]
 constexpr int kDecPAddr = kDecCode + 64;          // probed addresses [<= 64]
 constexpr int kDecOffs = kDecPAddr + 64;          // slot offsets [<= 65]
-constexpr int kDecSel = kDecOffs + 68;            // selected blocks [<= 64]
-constexpr int kDecTBase = kDecSel + 64;           // first token of each selected block [<= 65]
-constexpr int kDecCand = kDecTBase + 68;          // candidate ids [kMaxCand]
+constexpr int kDecCand = kDecOffs + 68;          // candidate ids [kMaxCand]
 constexpr int kDecKey = kDecCand + kMaxCand;      // candidate score keys [kMaxCand]
-constexpr int kDecPart = kDecKey + kMaxCand;      // per warp: max, sum, partial output [D]
-constexpr int kDecWords = kDecPart + kAttWarps * (2 + 128);
+constexpr int kDecWords = kDecKey + kMaxCand;
 
 template <typename T>
 __global__ void __launch_bounds__(kAttWarps * 32)
-decode_attend_kernel(const __grid_constant__ DecodeArgs a) {
+decode_route_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(16) float dsm[];
   float* qs = dsm + kDecQ;
   int* pcode = reinterpret_cast<int*>(dsm + kDecCode);
   int* paddr = reinterpret_cast<int*>(dsm + kDecPAddr);
   int* offs = reinterpret_cast<int*>(dsm + kDecOffs);
-  int* sblk = reinterpret_cast<int*>(dsm + kDecSel);
-  int* tbase = reinterpret_cast<int*>(dsm + kDecTBase);
   int* cand = reinterpret_cast<int*>(dsm + kDecCand);
   uint32_t* ckey = reinterpret_cast<uint32_t*>(dsm + kDecKey);
-  float* part = dsm + kDecPart;
-  __shared__ int s_nsel;
+  __shared__ int s_ncand;
   grid_dependency_wait();            // the key kernel of this step wrote token t
   const int b = blockIdx.x / a.Hq, hq = blockIdx.x % a.Hq, h = hq / (a.Hq / a.Hkv);
   const size_t bh = static_cast<size_t>(b) * a.Hkv + h, bq = static_cast<size_t>(b) * a.Hq + hq;
@@ -278,23 +308,58 @@ decode_attend_kernel(const __grid_constant__ DecodeArgs a) {
       if (ok) cand[n + __popc(m & ((1u << lane) - 1u))] = id;
       n += __popc(m);
     }
-    __syncwarp();
+    if (lane == 0) s_ncand = n;
+  }
+  __syncthreads();
+
+  // Candidate scores <q'_t, kbar_i>, float32, by all warps: warp w takes
+  // candidates w, w + 8, ..., four rows in flight; a lane holds D/32
+  // coordinates (in order), the lanes' partial sums meet in a fixed butterfly.
+  {
+    const int n = s_ncand, vpl = D / 32;
     const float* kb = a.kbar + bh * a.nb * D;
-    const float4* q4 = reinterpret_cast<const float4*>(qs);
-    for (int ci = lane; ci < n; ci += 32) {
-      const float4* kr = reinterpret_cast<const float4*>(kb + static_cast<size_t>(cand[ci]) * D);
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-      for (int d4 = 0; d4 < D / 4; ++d4) {
-        const float4 kv = __ldg(kr + d4), qv = q4[d4];
-        a0 = __fmaf_rn(qv.x, kv.x, a0);
-        a1 = __fmaf_rn(qv.y, kv.y, a1);
-        a2 = __fmaf_rn(qv.z, kv.z, a2);
-        a3 = __fmaf_rn(qv.w, kv.w, a3);
+    float qv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) qv[e] = e < vpl ? qs[lane * vpl + e] : 0.f;
+    for (int c0 = warp; c0 < n; c0 += 4 * kAttWarps) {
+      float sc[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int ci = c0 + x * kAttWarps;
+        float kv[4] = {0.f, 0.f, 0.f, 0.f};
+        if (ci < n) {
+          const float* kr = kb + static_cast<size_t>(cand[ci]) * D + lane * vpl;
+          if (vpl == 4) {
+            const float4 f = __ldg(reinterpret_cast<const float4*>(kr));
+            kv[0] = f.x; kv[1] = f.y; kv[2] = f.z; kv[3] = f.w;
+          } else if (vpl == 2) {
+            const float2 f = __ldg(reinterpret_cast<const float2*>(kr));
+            kv[0] = f.x; kv[1] = f.y;
+          } else {
+            kv[0] = __ldg(kr);
+          }
+        }
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc = __fmaf_rn(qv[e], kv[e], acc);
+        sc[x] = acc;
       }
-      const float v = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
-      ckey[ci] = dec_ordered(v == v ? v : -INFINITY);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) sc[x] = __fadd_rn(sc[x], __shfl_xor_sync(0xffffffffu, sc[x], off));
+      if (lane == 0)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const int ci = c0 + x * kAttWarps;
+          if (ci < n) ckey[ci] = dec_ordered(sc[x] == sc[x] ? sc[x] : -INFINITY);
+        }
     }
-    __syncwarp();
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    const int n = s_ncand;
     int mine = INT_MAX;                           // lane r: the r-th winner
     for (int r = 0; r < a.R; ++r) {
       uint32_t lk = 0u;
@@ -326,103 +391,120 @@ decode_attend_kernel(const __grid_constant__ DecodeArgs a) {
       srow[a.R + lane] = id >= 0 ? id : -1;
     }
     if (a.ncand_t && lane == 0) a.ncand_t[bq] = n;
-    // The selected blocks for the attention: valid remote ones, then locals.
-    const bool vr = lane < a.R && mine != INT_MAX;
-    const unsigned mr = __ballot_sync(0xffffffffu, vr);
-    if (vr) sblk[__popc(mr & ((1u << lane) - 1u))] = mine;
-    const int lid = j - a.L + 1 + lane;
-    const bool vl = lane < a.L && lid >= 0;
-    const unsigned ml = __ballot_sync(0xffffffffu, vl);
-    if (vl) sblk[__popc(mr) + __popc(ml & ((1u << lane) - 1u))] = lid;
-    if (lane == 0) {
-      const int ns = __popc(mr) + __popc(ml);
-      int tb = 0;
-      for (int i = 0; i < ns; ++i) {
-        tbase[i] = tb;
-        const int first = sblk[i] * a.bs;
-        tb += min(a.bs, t + 1 - first);
-      }
-      tbase[ns] = tb;
-      s_nsel = ns;
-    }
   }
-  __syncthreads();
+  // The rotated query, for the attention kernel of this step.
+  for (int i = tid; i < D; i += kAttWarps * 32) a.qrot_t[bq * D + i] = qs[i];
+}
 
-  // 4. attention over the selected tokens s <= t, split over the warps.
-  const int nsel = s_nsel, ntok = tbase[nsel];
-  const int vpl = D / 32;                         // coordinates per lane
-  float qv[4], o[4];
+// Attention of token t over one selected block: CTA (b*Hq + hq, slot) takes
+// block sel[slot] (tokens s <= t), four warps with a float32 online softmax
+// each (lanes hold D/32 coordinates of the rows they read, eight tokens in
+// flight), merged into the block's (max, sum, output); the last CTA of a
+// (b, hq) to finish merges all blocks, in slot order, into the output.
+template <typename T>
+__global__ void __launch_bounds__(128)
+decode_partial_kernel(const __grid_constant__ DecodeArgs a) {
+  __shared__ float wm[4], wl[4];
+  __shared__ float wo[4][128];
+  __shared__ int s_last;
+  grid_dependency_wait();            // sel and the rotated query of this step
+  const int bq = blockIdx.x, slot = blockIdx.y, nsl = a.R + a.L;
+  const int b = bq / a.Hq, hq = bq % a.Hq, h = hq / (a.Hq / a.Hkv);
+  const int t = a.t, D = a.D, vpl = D / 32;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int blk = a.sel_t[static_cast<size_t>(bq) * nsl + slot];
+  float m = -INFINITY, l = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+  if (blk >= 0) {
+    const int first = blk * a.bs, ntok = min(a.bs, t + 1 - first);
+    float qv[4];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    qv[e] = e < vpl ? qs[lane * vpl + e] * a.scale : 0.f;
-    o[e] = 0.f;
-  }
-  float m = -INFINITY, l = 0.f;
-  const int per = (ntok + kAttWarps - 1) / kAttWarps;
-  const int u0 = warp * per, u1 = min(ntok, u0 + per);
-  int bi = 0;
-  for (int u = u0; u < u1; u += 4) {
-    float sc[4], vv[4][4];
+    for (int e = 0; e < 4; ++e) qv[e] = e < vpl ? a.qrot_t[static_cast<size_t>(bq) * D + lane * vpl + e] * a.scale : 0.f;
+    const int per = (ntok + 3) / 4, u0 = warp * per, u1 = min(ntok, u0 + per);
+    constexpr int kTok = 8;
+    for (int u = u0; u < u1; u += kTok) {
+      float sc[kTok], vv[kTok][4], kv[kTok][4];
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      sc[x] = 0.f;
+      for (int x = 0; x < kTok; ++x) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) vv[x][e] = 0.f;
-      const int uu = u + x;
-      if (uu < u1) {
-        while (tbase[bi + 1] <= uu) ++bi;
-        const int s = sblk[bi] * a.bs + (uu - tbase[bi]);
-        const size_t off = ((static_cast<size_t>(b) * a.S + s) * a.Hkv + h) * D + lane * vpl;
-        const T* kr = static_cast<const T*>(a.krot) + off;
-        const T* vr2 = static_cast<const T*>(a.v) + off;
+        for (int e = 0; e < 4; ++e) { vv[x][e] = 0.f; kv[x][e] = 0.f; }
+        if (u + x < u1) {
+          const size_t off = ((static_cast<size_t>(b) * a.S + first + u + x) * a.Hkv + h) * D + lane * vpl;
+          ld_vec(static_cast<const T*>(a.krot) + off, vpl, kv[x]);
+          ld_vec(static_cast<const T*>(a.v) + off, vpl, vv[x]);
+        }
+      }
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (e < vpl) {
-            sc[x] = __fmaf_rn(qv[e], ld_f(kr + e), sc[x]);
-            vv[x][e] = ld_f(vr2 + e);
-          }
+      for (int x = 0; x < kTok; ++x) {
+        sc[x] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[x] = __fmaf_rn(qv[e], kv[x][e], sc[x]);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int x = 0; x < kTok; ++x) sc[x] = __fadd_rn(sc[x], __shfl_xor_sync(0xffffffffu, sc[x], off));
+#pragma unroll
+      for (int x = 0; x < kTok; ++x) {
+        if (u + x >= u1) break;
+        if (sc[x] > m) {
+          const float alpha = expf(m - sc[x]);
+          l *= alpha;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[e] *= alpha;
+          m = sc[x];
+        }
+        const float p = expf(sc[x] - m);
+        l += p;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] = __fmaf_rn(p, vv[x][e], o[e]);
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-      for (int x = 0; x < 4; ++x) sc[x] = __fadd_rn(sc[x], __shfl_xor_sync(0xffffffffu, sc[x], off));
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      if (u + x >= u1) break;
-      if (sc[x] > m) {
-        const float alpha = expf(m - sc[x]);
-        l *= alpha;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[e] *= alpha;
-        m = sc[x];
-      }
-      const float p = expf(sc[x] - m);
-      l += p;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] = __fmaf_rn(p, vv[x][e], o[e]);
-    }
   }
-  float* pw = part + warp * (2 + 128);
-  if (lane == 0) { pw[0] = m; pw[1] = l; }
+  if (lane == 0) { wm[warp] = m; wl[warp] = l; }
 #pragma unroll
   for (int e = 0; e < 4; ++e)
-    if (e < vpl) pw[2 + lane * vpl + e] = o[e];
+    if (e < vpl) wo[warp][lane * vpl + e] = o[e];
   __syncthreads();
-  T* out = static_cast<T*>(a.out_t) + bq * D;
-  for (int i = tid; i < D; i += kAttWarps * 32) {
-    float M = -INFINITY;
-    for (int w = 0; w < kAttWarps; ++w) M = fmaxf(M, part[w * (2 + 128)]);
+  // This block's (max, sum, output) over its four warps.
+  float* pp = a.part + (static_cast<size_t>(bq) * nsl + slot) * (2 + D);
+  float M = -INFINITY;
+  for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w]);
+  for (int i = tid; i < D; i += 128) {
+    float num = 0.f;
+    for (int w = 0; w < 4; ++w)
+      if (wm[w] != -INFINITY) num = __fmaf_rn(expf(wm[w] - M), wo[w][i], num);
+    pp[2 + i] = num;
+  }
+  if (tid == 0) {
+    float den = 0.f;
+    for (int w = 0; w < 4; ++w)
+      if (wm[w] != -INFINITY) den = __fmaf_rn(expf(wm[w] - M), wl[w], den);
+    pp[0] = M;
+    pp[1] = den;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(a.done + bq, 1) == nsl - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // Last block of this (b, hq): merge the blocks in slot order.
+  const float* pb = a.part + static_cast<size_t>(bq) * nsl * (2 + D);
+  float MM = -INFINITY;
+  for (int s = 0; s < nsl; ++s) MM = fmaxf(MM, __ldcg(pb + s * (2 + D)));
+  T* out = static_cast<T*>(a.out_t) + static_cast<size_t>(bq) * D;
+  for (int i = tid; i < D; i += 128) {
     float num = 0.f, den = 0.f;
-    for (int w = 0; w < kAttWarps; ++w) {
-      const float mw = part[w * (2 + 128)];
-      if (mw == -INFINITY) continue;
-      const float f = expf(mw - M);
-      num = __fmaf_rn(f, part[w * (2 + 128) + 2 + i], num);
-      den = __fmaf_rn(f, part[w * (2 + 128) + 1], den);
+    for (int s = 0; s < nsl; ++s) {
+      const float ms = __ldcg(pb + s * (2 + D));
+      if (ms == -INFINITY) continue;
+      const float f = expf(ms - MM);
+      num = __fmaf_rn(f, __ldcg(pb + s * (2 + D) + 2 + i), num);
+      den = __fmaf_rn(f, __ldcg(pb + s * (2 + D) + 1), den);
     }
     out[i] = st_f<T>(num / den);
   }
+  if (tid == 0) a.done[bq] = 0;
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t st) {
@@ -431,9 +513,11 @@ cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t st) {
                        : launch_pdl(decode_keys_kernel<float>, dim3(a.B * a.Hkv), dim3(kKeyThreads), 0, st, a);
   if (e != cudaSuccess) return e;
   const size_t smem = static_cast<size_t>(kDecWords) * sizeof(float);
-  void (*k)(DecodeArgs) = bf16 ? decode_attend_kernel<__nv_bfloat16> : decode_attend_kernel<float>;
+  void (*k)(DecodeArgs) = bf16 ? decode_route_kernel<__nv_bfloat16> : decode_route_kernel<float>;
   if ((e = cached_allow_smem(reinterpret_cast<const void*>(k), static_cast<int>(smem))) != cudaSuccess) return e;
   if ((e = launch_pdl(k, dim3(a.B * a.Hq), dim3(kAttWarps * 32), smem, st, a)) != cudaSuccess) return e;
+  void (*kp)(DecodeArgs) = bf16 ? decode_partial_kernel<__nv_bfloat16> : decode_partial_kernel<float>;
+  if ((e = launch_pdl(kp, dim3(a.B * a.Hq, a.R + a.L), dim3(128), 0, st, a)) != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -99,6 +99,9 @@ struct DecodeArgs {
   void* out_t;             // [B,Hq,D]
   int32_t* sel_t;          // [B,Hq,R+L]
   int32_t* ncand_t;        // [B,Hq] or null
+  float* qrot_t;           // scratch: rotated queries [B,Hq,D]
+  float* part;             // scratch: per selected block max, sum, output [B,Hq,R+L,2+D]
+  int32_t* done;           // scratch: blocks finished per (b, hq) [B,Hq], zero at the start of a step
   int B, S, Hq, Hkv, D, bs, nb, P, K, A, cap, probes, R, L;
   float scale;
   float inv_freq[64];      // omega_i, i < D/2

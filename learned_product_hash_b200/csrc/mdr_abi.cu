@@ -77,18 +77,25 @@ Layout layout_of(const mdr_config* c) {
   return l;
 }
 
-// Decode workspace: the status word, then (for mdr_decode_prefill) the
-// rotated keys, summaries and addresses of the prefix at the prefix's own
-// strides before they are copied into the state's rows.
+// Decode workspace: the status word and the per-(b, hq) counters of
+// finished blocks (zeroed together at the start of every step), the step's
+// rotated queries and per-block partial results, then (for
+// mdr_decode_prefill) the rotated keys, summaries and addresses of the prefix
+// at the prefix's own strides before they are copied into the state's rows.
 struct DecodeLayout {
-  size_t status, krot, kbar, addr, total;
+  size_t status, done, head, qrot, part, krot, kbar, addr, total;
 };
 
 DecodeLayout decode_layout_of(const mdr_config* c) {
-  const size_t nb = c->S / c->block;
+  const size_t nb = c->S / c->block, bq = static_cast<size_t>(c->B) * c->Hq;
   DecodeLayout l{};
   size_t o = 0;
-  l.status = o; o += align_up(16);
+  l.status = o;
+  l.done = 16;
+  l.head = 16 + bq * sizeof(int32_t);                 // bytes zeroed per step
+  o += align_up(l.head);
+  l.qrot = o;   o += align_up(bq * c->D * sizeof(float));
+  l.part = o;   o += align_up(bq * (c->R + c->L) * (2 + c->D) * sizeof(float));
   l.krot = o;   o += align_up(static_cast<size_t>(c->B) * c->S * c->Hkv * c->D * esize(c));
   l.kbar = o;   o += align_up(static_cast<size_t>(c->B) * c->Hkv * nb * c->D * sizeof(float));
   l.addr = o;   o += align_up(static_cast<size_t>(c->B) * c->Hkv * nb * sizeof(int32_t));
@@ -482,9 +489,10 @@ mdr_status mdr_decode_step(const mdr_config* cfg, int32_t t, const void* q_t, co
   MDR_TRY(check_decode_state(st));
   if (t < 0 || t >= cfg->S) return MDR_ERR_INVALID_ARG;
   if (!q_t || !k_t || !v_t || !codebooks || !out_t || !sel_t || !aligned16(codebooks)) return MDR_ERR_INVALID_ARG;
-  if (!ws || reinterpret_cast<uintptr_t>(ws) % kAlign != 0 || ws_bytes < 16) return MDR_ERR_WORKSPACE;
+  MDR_TRY(check_decode_ws(cfg, ws, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  MDR_CUDA(cudaMemsetAsync(ws, 0, sizeof(int32_t), s));
+  const DecodeLayout l = decode_layout_of(cfg);
+  MDR_CUDA(cudaMemsetAsync(ws, 0, l.head, s));
   mdr::DecodeArgs d;
   std::memset(&d, 0, sizeof(d));
   d.t = t; d.q_t = q_t; d.k_t = k_t; d.v_t = v_t;
@@ -492,6 +500,7 @@ mdr_status mdr_decode_step(const mdr_config* cfg, int32_t t, const void* q_t, co
   d.kbar = st->idx.kbar; d.addr = st->idx.addr; d.lists = st->idx.lists; d.load = st->idx.load;
   d.overflow = st->idx.overflow; d.maxload = st->idx.maxload;
   d.codebooks = codebooks; d.out_t = out_t; d.sel_t = sel_t; d.ncand_t = ncand_t;
+  d.qrot_t = at<float>(ws, l.qrot); d.part = at<float>(ws, l.part); d.done = at<int32_t>(ws, l.done);
   d.B = cfg->B; d.S = cfg->S; d.Hq = cfg->Hq; d.Hkv = cfg->Hkv; d.D = cfg->D; d.bs = cfg->block;
   d.nb = cfg->S / cfg->block; d.P = cfg->P; d.K = cfg->K; d.A = ipow(cfg->K, cfg->P); d.cap = cfg->cap;
   d.probes = cfg->probes; d.R = cfg->R; d.L = cfg->L;
