@@ -197,7 +197,7 @@ def candidate_slots(lists: np.ndarray, probe_addrs: np.ndarray, j: int, L: int) 
 
 
 def route_row(qbar_j: np.ndarray, kbar_h: np.ndarray, probe_addrs: np.ndarray,
-              lists: np.ndarray, j: int, R: int, L: int) -> RouteRow:
+              lists: np.ndarray, j: int, R: int, L: int, force: int = -1) -> RouteRow:
     """Route one query block: probe -> candidates -> rerank -> top R, plus the
     L local blocks j-L+1..j (Article, section "Monodratic Turns Sparse
     Attention Into a Retrieval Decision": the query probes addresses, gets
@@ -207,15 +207,29 @@ def route_row(qbar_j: np.ndarray, kbar_h: np.ndarray, probe_addrs: np.ndarray,
     Rerank score of candidate i is <qbar_j, kbar_i> over the full head
     dimension, rounded to float32; top R by score, lower id on equal scores.
     The chosen remote ids are stored in ascending order.
+
+    ``force`` is the forced-target diagnostic (Article, "Why Learned
+    Product-Hash Routing Matters Now": the labelled target block is put into
+    the selected set under the same attention budget).  Reading: when
+    0 <= force <= j - L and R > 0, the remote set is the forced block plus
+    the R - 1 best other candidates, so the target takes the place of the
+    weakest choice when routing missed it and changes nothing when routing
+    found it; any other value (no target, a local block, a later block)
+    leaves the route as it is.
     """
     slots = candidate_slots(lists, probe_addrs, j, L)
     cand = slots[slots >= 0]
-    scores = f32(f32(kbar_h[cand]) @ f32(qbar_j)) if cand.size else np.zeros(0)
-    order = np.lexsort((cand, -scores))
-    top = cand[order[:R]]
+    forced = 0 <= force <= j - L and R > 0
+    pool = cand[cand != force] if forced else cand
+    keep = R - 1 if forced else R
+    scores = f32(f32(kbar_h[pool]) @ f32(qbar_j)) if pool.size else np.zeros(0)
+    order = np.lexsort((pool, -scores))
+    top = pool[order[:keep]]
+    if forced:
+        top = np.concatenate([top, [force]])
     margin = np.inf
-    if cand.size > R and R > 0:
-        margin = float(scores[order[R - 1]] - scores[order[R]])
+    if pool.size > keep and keep > 0:
+        margin = float(scores[order[keep - 1]] - scores[order[keep]])
     remote = np.full(R, -1, dtype=np.int64)
     remote[: top.size] = np.sort(top)
     local = np.arange(j - L + 1, j + 1, dtype=np.int64)
@@ -360,7 +374,9 @@ def build_index(kr, codebooks, p: Params):
     return kbar, addr, codes, margin, lists, load, overflow, maxload
 
 
-def route(qr, kbar, lists, codebooks, p: Params, keep_slots=False):
+def route(qr, kbar, lists, codebooks, p: Params, keep_slots=False, force=None):
+    """Route every query block; ``force`` [B,Hq,nb] (or None) holds a forced
+    target block per route, -1 for none (see route_row)."""
     qbar = block_means(qr, p.block)
     qcodes, qmargin = probe_codes(qbar, codebooks, p.probes)
     B, Hq, nb = qbar.shape[:3]
@@ -374,7 +390,8 @@ def route(qr, kbar, lists, codebooks, p: Params, keep_slots=False):
             for j in range(nb):
                 pa = probe_addresses(qcodes[b, hq, j], p.K)
                 row = route_row(qbar[b, hq, j], kbar[b, hq // g], pa,
-                                lists[b, hq // g], j, p.R, p.L)
+                                lists[b, hq // g], j, p.R, p.L,
+                                -1 if force is None else int(force[b, hq, j]))
                 sel[b, hq, j] = row.sel
                 sel_margin[b, hq, j] = row.margin
                 ncand[b, hq, j] = row.cand.size
@@ -383,18 +400,37 @@ def route(qr, kbar, lists, codebooks, p: Params, keep_slots=False):
     return qbar, qcodes, qmargin, sel, sel_margin, ncand, slots
 
 
-def forward(q, k, v, codebooks, p: Params, *, attention=True, rows=None, keep_slots=False) -> Result:
-    """Index -> route -> attend for stored inputs q [B,S,Hq,D], k, v [B,S,Hkv,D]."""
+def forward(q, k, v, codebooks, p: Params, *, attention=True, rows=None, keep_slots=False,
+            force=None) -> Result:
+    """Index -> route -> attend for stored inputs q [B,S,Hq,D], k, v [B,S,Hkv,D];
+    ``force`` as in route."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     qr = rope(q, p.rope_base)
     kr = rope(k, p.rope_base)
     kbar, addr, codes, cmargin, lists, load, overflow, maxload = build_index(kr, codebooks, p)
-    qbar, qcodes, qmargin, sel, smargin, ncand, slots = route(qr, kbar, lists, codebooks, p, keep_slots)
+    qbar, qcodes, qmargin, sel, smargin, ncand, slots = route(qr, kbar, lists, codebooks, p, keep_slots, force)
     out = attend(qr, kr, v, sel, p.block, p.softmax_scale, rows) if attention else None
     return Result(qr, kr, qbar, kbar, addr, codes, cmargin, qcodes, qmargin, lists, load,
                   overflow, maxload, sel, smargin, ncand, out, slots)
+
+
+def target_hits(sel: np.ndarray, target: np.ndarray):
+    """Target-block hit diagnostic (Report, Evidence: the target-block hit
+    rate).  For every route with a target (target[b,hq,j] >= 0), whether that
+    block is in the route's selected set (remote or local part); routes with
+    no target (-1) are not counted.  Returns (hit [B,Hq,nb]: 1 hit, 0 miss,
+    -1 no target; number of routes with a target; number of hits)."""
+    B, Hq, nb = target.shape
+    hit = np.full((B, Hq, nb), -1, dtype=np.int64)
+    for b in range(B):
+        for hq in range(Hq):
+            for j in range(nb):
+                t = int(target[b, hq, j])
+                if t >= 0:
+                    hit[b, hq, j] = 1 if t in set(int(x) for x in sel[b, hq, j]) else 0
+    return hit, int((hit >= 0).sum()), int((hit == 1).sum())
 
 
 def near_tie(margin, scale_ref) -> np.ndarray:

@@ -69,7 +69,7 @@ def _slots_off_by_one(lists, probe_addrs, j, L):
     return slots
 
 
-def _route_row_lowest_scores(qbar_j, kbar_h, probe_addrs, lists, j, R, L):
+def _route_row_lowest_scores(qbar_j, kbar_h, probe_addrs, lists, j, R, L, force=-1):
     slots = O.candidate_slots(lists, probe_addrs, j, L)
     cand = slots[slots >= 0]
     scores = O.f32(O.f32(kbar_h[cand]) @ O.f32(qbar_j)) if cand.size else np.zeros(0)
@@ -127,6 +127,4 @@ def test_mutation_is_caught(name, monkeypatch):
             check()
         except AssertionError:
             caught.append(check.__name__)
-        except Exception:  # a mutation may also break shapes: that is caught too
-            caught.append(check.__name__ + "(error)")
     assert caught, f"no pin catches the mutation {name}"
