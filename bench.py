@@ -23,9 +23,7 @@ import datetime
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -39,9 +37,6 @@ from workloads import SCALING_SWEEP, ALL, make_inputs  # noqa: E402
 
 METRIC = "routed-attention fwd tokens/s (index+route+attend) at 32K; % HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
-REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
-               0x20: "sync_boost", 0x40: "sw_thermal_slowdown", 0x80: "hw_thermal_slowdown",
-               0x100: "hw_power_brake_slowdown", 0x200: "display_clock"}
 
 
 def workload(name):
@@ -87,50 +82,72 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons during the timed region."""
+    """SM clock, power and clock-event reasons of this process's GPU during
+    the timed region, read through NVML by a thread every ~2 ms (the timed
+    region is tens of milliseconds, too short for nvidia-smi's own loop).
+    The GPU is matched by PCI domain/bus/device, so a remapped
+    CUDA_VISIBLE_DEVICES does not matter; reason names come from NVML's own
+    bit constants.  Reads only."""
+
+    NAMES = {"GpuIdle": "gpu_idle", "ApplicationsClocksSetting": "applications_clocks",
+             "SwPowerCap": "sw_power_cap", "HwSlowdown": "hw_slowdown", "SyncBoost": "sync_boost",
+             "SwThermalSlowdown": "sw_thermal_slowdown", "HwThermalSlowdown": "hw_thermal_slowdown",
+             "HwPowerBrakeSlowdown": "hw_power_brake_slowdown", "DisplayClockSetting": "display_clock"}
 
     def __init__(self, dev):
-        self.dev, self.proc, self.path = dev, None, None
+        self.dev, self.samples, self.err, self.thread = dev, [], None, None
 
     def __enter__(self):
+        import threading
+        import torch
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev),
-                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
-                 "--format=csv,noheader,nounits", "-lms", "20", "-f", self.path],
-                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            pr = torch.cuda.get_device_properties(self.dev)
+            want = (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+            self.h = None
+            for i in range(nv.nvmlDeviceGetCount()):
+                h = nv.nvmlDeviceGetHandleByIndex(i)
+                pci = nv.nvmlDeviceGetPciInfo(h)
+                if (pci.domain, pci.bus, pci.device) == want:
+                    self.h = h
+            if self.h is None:
+                raise RuntimeError(f"no NVML device at PCI {want}")
+            self.nv = nv
+            self.bits = {getattr(nv, "nvmlClocksEventReason" + k): v for k, v in self.NAMES.items()}
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.stop, first = threading.Event(), threading.Event()
+
+            def run():
+                while not self.stop.is_set():
+                    self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                         nv.nvmlDeviceGetCurrentClocksEventReasons(self.h),
+                                         nv.nvmlDeviceGetPowerUsage(self.h)))
+                    first.set()
+                    self.stop.wait(0.002)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            first.wait(timeout=5)          # sampling has begun before the timed steps are issued
+        except Exception as e:             # no NVML: the line says why instead of carrying clocks
+            self.err = repr(e)
         return self
 
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            self.proc.wait(timeout=10)
+        if self.thread:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            self.nv.nvmlShutdown()
 
     def summary(self):
-        if not self.path or not os.path.exists(self.path):
-            return None
-        sm, mx, reasons = [], [], set()
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 4:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-                bits = int(parts[3], 16)
-            except ValueError:
-                continue
-            for b, n in REASON_BITS.items():
-                if bits & b:
-                    reasons.add(n)
-        os.unlink(self.path)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+        if not self.samples:
+            return {"error": self.err or "no samples"}
+        reasons = set()
+        for _, bits, _ in self.samples:
+            reasons |= {n for b, n in self.bits.items() if bits & b}
+        return {"sm_mhz": statistics.median(x[0] for x in self.samples), "sm_max_mhz": self.max_mhz,
+                "power_w": statistics.median(x[2] for x in self.samples) / 1e3,
+                "samples": len(self.samples), "source": "NVML, every 2 ms",
                 "reasons": sorted(reasons - {"gpu_idle"})}
 
 
@@ -349,10 +366,41 @@ def run_mine(args, w):
         decode = {"metric": "decode step latency (one token per sequence: key append, route, attend) at 32K",
                   "value": d_ms_max * 1e3, "unit": "us/step", "tokens_per_s": w.B * world / (d_ms_max / 1e3),
                   "batch_per_gpu": w.B, "steps": n_dec, "position": f"tokens {S0}..{t_last} ({S0 // w.block} blocks indexed)",
-                  "l2": "not flushed between steps", "gpu_launches": 2 * n_dec,
+                  "l2": "not flushed between steps", "gpu_launches": 3 * n_dec,
                   "roofline": {"bound": "hbm", "achieved": d_bytes / (d_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
                                "frac": d_bytes / (d_ms / 1e3) / 1e9 / peak, "algorithmic_bytes_per_step": d_bytes}}
         del dst, dws
+
+    # Controls on the planted-block workload (untimed): how often the route
+    # selects each sequence's planted block for its last query block, with
+    # the random unit codebooks (the untrained router), with the planted
+    # block forced in, and with no remote blocks at all (R = 0).
+    controls = None
+    if not args.no_controls:
+        wa = workload("ar")
+        ia = make_inputs(wa, 2000 + rank)
+        conv_a = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        qa, ka = conv_a(ia.q_store), conv_a(ia.k_store)
+        cba = torch.from_numpy(ia.codebooks).to(dev)
+        tg = np.full((wa.B, wa.Hq, wa.nb), -1, dtype=np.int32)
+        tg[:, :, wa.nb - 1] = ia.planted[:, None]
+        tg = torch.from_numpy(tg).to(dev)
+        counts = torch.empty(2, dtype=torch.int32, device=dev)
+        rates = {}
+        for name, wc, forced in (("route", wa, False), ("forced", wa, True), ("local_only", wa.with_(R=0), False)):
+            ca = mdr.make_config(wc)
+            ixa, rta, wsa = mdr.Index.empty(ca, dev), mdr.RouteOut.empty(ca, dev), mdr.workspace(ca, dev)
+            mdr.mdr_build_index(ca, ka, cba, ixa, wsa)
+            if forced:
+                mdr.mdr_route_forced(ca, qa, cba, ixa, tg, rta, wsa)
+            else:
+                mdr.mdr_route(ca, qa, cba, ixa, rta, wsa)
+            mdr.mdr_target_hits(ca, rta.sel, tg, counts)
+            n_t, n_h = (int(x) for x in counts.cpu())
+            rates[name] = n_h / n_t
+        controls = {"workload": f"{wa.name}: B={wa.B}, H={wa.Hq}, S={wa.S}, block {wa.block}, R={wa.R}, L={wa.L}, "
+                                "one planted block per sequence, random unit codebooks",
+                    "routes_with_target": n_t, "target_hit_rate": rates}
 
     # End to end through the C ABI with host buffers.
     e2e = None
@@ -400,6 +448,7 @@ def run_mine(args, w):
                              "kernel": "attend", "algorithmic_bytes_per_launch": attn_bytes},
                 "path_roofline_frac": total_bytes / (ms_max / 1e3) / 1e9 / peak,
                 "kernels_ms": ker, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
+                "controls": controls,
                 "gpu_launches": KERNELS_PER_FORWARD * args.steps, "clocks": clk.summary(),
                 "overflow": int(idx.overflow.sum().item()), "selected_blocks": nsel}
         print(json.dumps(line), flush=True)
@@ -417,6 +466,7 @@ def main():
     ap.add_argument("--workload", default="scaling32k")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-controls", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()

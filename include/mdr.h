@@ -220,6 +220,39 @@ mdr_status mdr_route_noalloc(const mdr_config* cfg, const void* q,
                              const float* codebooks, const mdr_index* idx,
                              int32_t* sel, int32_t* ncand, void* stream);
 
+/* ------------------------------------------------ controls and diagnostics
+ * The controls the pages run beside the learned route (Report, section
+ * Learned sparse route; Article, "Why Learned Product-Hash Routing Matters
+ * Now"): the local-only control is any call with R = 0; the untrained-router
+ * control is any call with random unit codebooks; the forced-target run and
+ * the target-block hit rate (Report, section Evidence) are these two calls. */
+
+/* mdr_route with a forced target block per route: the labelled target is put
+ * into the selected set under the same budget of R remote blocks.  force:
+ * device int32 [B,Hq,nb] (required).  Where 0 <= force[b,hq,j] <= j-L and
+ * R > 0, the remote part of sel[b,hq,j] is the forced block plus the R-1
+ * best other candidates (so the target replaces the weakest choice when the
+ * route missed it and changes nothing when it found it), in ascending order
+ * like every sel row; any other value (-1 for no target, a local block, a
+ * later block) leaves the route as mdr_route computes it.  ncand counts the
+ * eligible candidates the probes found, as in mdr_route.  Other arguments
+ * and outputs as mdr_route.                                                 */
+mdr_status mdr_route_forced(const mdr_config* cfg, const void* q,
+                            const float* codebooks, const mdr_index* idx,
+                            const int32_t* force, const mdr_route_out* rt,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Target-block hits: for every route (b, hq, j) with target[b,hq,j] >= 0,
+ * whether that block id appears anywhere in sel[b,hq,j] (remote or local
+ * part).  sel: device int32 [B,Hq,nb,R+L] as written by a route call;
+ * target: device int32 [B,Hq,nb], -1 = no target; hit: device int32
+ * [B,Hq,nb] or NULL: 1 hit, 0 miss, -1 no target; counts: device int32 [2],
+ * written (not accumulated): counts[0] = routes with a target, counts[1] =
+ * hits.  The hit rate is counts[1] / counts[0].  Needs no workspace.        */
+mdr_status mdr_target_hits(const mdr_config* cfg, const int32_t* sel,
+                           const int32_t* target, int32_t* hit,
+                           int32_t* counts, void* stream);
+
 /* ------------------------------------------------------------- decoding
  * One token at a time with an incremental index.  The pages leave decoding
  * open and ask that a deployed decoder update its routing structures as

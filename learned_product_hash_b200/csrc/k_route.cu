@@ -15,6 +15,15 @@
 // when the batch and the winners are at most 64, else by R rounds of warp
 // arg-max.  The R winners are written in ascending id order, -1 padded; then
 // the local blocks j-L+1..j.
+//
+// Forced-target diagnostic ("Why Learned Product-Hash Routing Matters Now":
+// the labelled target block is put into the selected set under the same
+// attention budget): a forced id f with 0 <= f <= j - L seeds the running
+// winners with score +inf, and f is left out of the probed candidates, so
+// the R winners are f and the R - 1 best others -- f replaces the weakest
+// choice when routing missed it and changes nothing when routing found it.
+// Any other forced value leaves the route unchanged; ncand still counts the
+// eligible candidates the probes found.
 // Pages: "Monodratic Claims Learned Routing Can Make Sparse Causal Attention
 // More Selective", section "Monodratic Turns Sparse Attention Into a
 // Retrieval Decision" (probe, candidates, rerank, fixed number of remote
@@ -38,6 +47,7 @@ constexpr int kBatch = 224;
 // scores (kBatch + 32 each: a batch, then the running winners).
 constexpr int kRouteWarpWords = 128 + 64 + 68 + 2 * (kBatch + 32);
 
+template <bool kForced>
 __global__ void __launch_bounds__(kRouteWarps * 32)
 route_kernel(const RouteArgs a) {
   extern __shared__ int32_t rsmem[];
@@ -64,6 +74,8 @@ route_kernel(const RouteArgs a) {
   const int last = j - a.L;                        // highest eligible block
 
   for (int d = lane; d < a.D; d += 32) qs[d] = a.qbar[route * a.D + d];
+  int forced = kForced ? a.force[route] : -1;
+  if (forced < 0 || forced > last || a.R <= 0) forced = INT_MIN;   // not a remote-eligible block
 
   // Probed addresses and their stored counts, all probes at once: lane l
   // owns probes l and l + 32 (first subspace's rank slowest).
@@ -107,6 +119,15 @@ route_kernel(const RouteArgs a) {
   const float* kb = a.kbar + bh * a.nb * a.D;
   int nbuf = 0, n = 0, nwin = 0;
   int mine = INT_MAX;                              // lane r: r-th winner id
+  if (kForced && forced != INT_MIN) {              // the forced block is winner 0 from the start
+    if (lane == 0) {
+      cand[kBatch] = forced;
+      score[kBatch] = INFINITY;
+      mine = forced;
+    }
+    nwin = 1;
+    __syncwarp();
+  }
   for (int base = 0; base < total; base += 32) {
     const int e = base + lane;
     int id = INT_MAX;
@@ -118,11 +139,12 @@ route_kernel(const RouteArgs a) {
       }
       id = lists[static_cast<long long>(paddr[lo]) * a.cap + (e - offs[lo])];
     }
-    const bool ok = id <= last;
+    const bool elig = id <= last;
+    const bool ok = elig && (!kForced || id != forced);
     const unsigned m = __ballot_sync(0xffffffffu, ok);
     if (ok) cand[nbuf + __popc(m & ((1u << lane) - 1u))] = id;
     nbuf += __popc(m);
-    n += __popc(m);
+    n += __popc(__ballot_sync(0xffffffffu, elig));
     if (nbuf <= kBatch - 32 && base + 32 < total) continue;
     __syncwarp();
     // Score the batch: lane group g (F4 = D/4 lanes) takes candidates g,
@@ -245,11 +267,12 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   int nprobe = 1;
   for (int s = 0; s < a.P; ++s) nprobe *= a.probes;
   const size_t smem = static_cast<size_t>(kRouteWarps) * kRouteWarpWords * sizeof(int32_t);
-  cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(route_kernel), static_cast<int>(smem));
+  const auto kern = a.force ? route_kernel<true> : route_kernel<false>;
+  cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const long long nroutes = static_cast<long long>(a.B) * a.Hq * a.nb;
   const unsigned grid = static_cast<unsigned>((nroutes + kRouteWarps - 1) / kRouteWarps);
-  e = launch_pdl(route_kernel, dim3(grid), dim3(kRouteWarps * 32), smem, st, a);
+  e = launch_pdl(kern, dim3(grid), dim3(kRouteWarps * 32), smem, st, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -62,9 +62,21 @@ struct RouteArgs {
   const int32_t* load;     // [B,Hkv,A]
   int32_t* sel;            // [B,Hq,nb,R+L]
   int32_t* ncand;          // [B,Hq,nb] or null
+  const int32_t* force;    // [B,Hq,nb] forced target block per route (-1 none) or null
   int B, Hq, Hkv, nb, D, P, K, A, probes, cap, R, L;
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
+
+// Target-block hit diagnostic: per route whether its target is selected.
+struct HitsArgs {
+  const int32_t* sel;      // [B,Hq,nb,nsel]
+  const int32_t* target;   // [B,Hq,nb], -1 = no target
+  int32_t* hit;            // [B,Hq,nb]: 1 hit, 0 miss, -1 no target; or null
+  int32_t* counts;         // [2]: routes with a target, hits
+  long long nroutes;
+  int nsel;
+};
+cudaError_t launch_hits(const HitsArgs& a, cudaStream_t st);
 
 // K5: selected-set causal attention over rotated q', k' and v.
 struct AttendArgs {

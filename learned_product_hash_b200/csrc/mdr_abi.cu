@@ -152,10 +152,11 @@ mdr_status run_lists(const mdr_config* c, const mdr_index* idx, cudaStream_t st)
 }
 
 mdr_status run_route(const mdr_config* c, const float* qbar, const int32_t* qcodes,
-                     const mdr_index* idx, int32_t* sel, int32_t* ncand, cudaStream_t st) {
+                     const mdr_index* idx, int32_t* sel, int32_t* ncand, cudaStream_t st,
+                     const int32_t* force = nullptr) {
   mdr::RouteArgs ra{};
   ra.qbar = qbar; ra.qcodes = qcodes; ra.kbar = idx->kbar; ra.lists = idx->lists; ra.load = idx->load;
-  ra.sel = sel; ra.ncand = ncand;
+  ra.sel = sel; ra.ncand = ncand; ra.force = force;
   ra.B = c->B; ra.Hq = c->Hq; ra.Hkv = c->Hkv; ra.nb = c->S / c->block; ra.D = c->D;
   ra.P = c->P; ra.K = c->K; ra.A = ipow(c->K, c->P); ra.probes = c->probes; ra.cap = c->cap;
   ra.R = c->R; ra.L = c->L;
@@ -219,9 +220,9 @@ mdr_status mdr_build_index(const mdr_config* cfg, const void* k, const float* co
   return run_lists(cfg, idx, st);
 }
 
-mdr_status mdr_route(const mdr_config* cfg, const void* q, const float* codebooks,
-                     const mdr_index* idx, const mdr_route_out* rt, void* ws, size_t ws_bytes,
-                     void* stream) {
+static mdr_status route_impl(const mdr_config* cfg, const void* q, const float* codebooks,
+                             const mdr_index* idx, const int32_t* force, const mdr_route_out* rt,
+                             void* ws, size_t ws_bytes, void* stream) {
   MDR_TRY(check(cfg));
   if (!q || !codebooks || !rt || !rt->sel || !aligned16(q)) return MDR_ERR_INVALID_ARG;
   MDR_TRY(check_index(idx));
@@ -236,7 +237,31 @@ mdr_status mdr_route(const mdr_config* cfg, const void* q, const float* codebook
   a.x[0] = q; a.xbar[0] = qbar; a.qcodes = qcodes;
   a.status = at<int32_t>(ws, l.status);
   MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
-  return run_route(cfg, qbar, qcodes, idx, rt->sel, rt->ncand, st);
+  return run_route(cfg, qbar, qcodes, idx, rt->sel, rt->ncand, st, force);
+}
+
+mdr_status mdr_route(const mdr_config* cfg, const void* q, const float* codebooks,
+                     const mdr_index* idx, const mdr_route_out* rt, void* ws, size_t ws_bytes,
+                     void* stream) {
+  return route_impl(cfg, q, codebooks, idx, nullptr, rt, ws, ws_bytes, stream);
+}
+
+mdr_status mdr_route_forced(const mdr_config* cfg, const void* q, const float* codebooks,
+                            const mdr_index* idx, const int32_t* force, const mdr_route_out* rt,
+                            void* ws, size_t ws_bytes, void* stream) {
+  if (!force) return MDR_ERR_INVALID_ARG;
+  return route_impl(cfg, q, codebooks, idx, force, rt, ws, ws_bytes, stream);
+}
+
+mdr_status mdr_target_hits(const mdr_config* cfg, const int32_t* sel, const int32_t* target,
+                           int32_t* hit, int32_t* counts, void* stream) {
+  MDR_TRY(check(cfg));
+  if (!sel || !target || !counts) return MDR_ERR_INVALID_ARG;
+  mdr::HitsArgs ha{};
+  ha.sel = sel; ha.target = target; ha.hit = hit; ha.counts = counts;
+  ha.nroutes = static_cast<long long>(cfg->B) * cfg->Hq * (cfg->S / cfg->block);
+  ha.nsel = cfg->R + cfg->L;
+  return cuda_status(mdr::launch_hits(ha, static_cast<cudaStream_t>(stream)));
 }
 
 mdr_status mdr_attend(const mdr_config* cfg, const void* q, const void* k, const void* v,

@@ -22,6 +22,7 @@ EXPORTED = (
     "mdr_build_index", "mdr_route", "mdr_attend", "mdr_forward", "mdr_host_workspace_bytes",
     "mdr_forward_host", "mdr_read_device_status", "mdr_forward_profiled", "mdr_route_noalloc",
     "mdr_decode_workspace_bytes", "mdr_decode_reset", "mdr_decode_prefill", "mdr_decode_step",
+    "mdr_route_forced", "mdr_target_hits",
 )
 
 
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
             "mdr_forward_profiled": ([cfgp, vp, vp, vp, vp, idxp, rtp, vp, vp, sz, vp,
                                       ctypes.POINTER(vp), ctypes.c_int32], i32),
             "mdr_route_noalloc": ([cfgp, vp, vp, idxp, vp, vp, vp], i32),
+            "mdr_route_forced": ([cfgp, vp, vp, idxp, vp, rtp, vp, sz, vp], i32),
+            "mdr_target_hits": ([cfgp, vp, vp, vp, vp, vp], i32),
             "mdr_decode_workspace_bytes": ([cfgp, ctypes.POINTER(sz)], i32),
             "mdr_decode_reset": ([cfgp, ctypes.POINTER(mdr_decode_state), vp], i32),
             "mdr_decode_prefill": ([cfgp, ctypes.c_int32, vp, vp, vp, ctypes.POINTER(mdr_decode_state),
@@ -248,6 +251,22 @@ def mdr_route_noalloc(cfg, q, codebooks, idx: Index, sel, ncand=None, stream=Non
     callers that cannot allocate device memory); see include/mdr.h."""
     _ok(lib().mdr_route_noalloc(ctypes.byref(cfg), _ptr(q), _ptr(codebooks), ctypes.byref(idx.c()),
                                 _ptr(sel), _ptr(ncand), _stream(stream)), "mdr_route_noalloc")
+
+
+# ------------------------------------------------- controls and diagnostics
+def mdr_route_forced(cfg, q, codebooks, idx: Index, force, rt: RouteOut, ws, stream=None):
+    """mdr_route with a forced target block per route (int32 [B,Hq,nb], -1
+    none); see include/mdr.h."""
+    _ok(lib().mdr_route_forced(ctypes.byref(cfg), _ptr(q), _ptr(codebooks), ctypes.byref(idx.c()),
+                               _ptr(force), ctypes.byref(rt.c()), _ptr(ws), ws.numel(), _stream(stream)),
+        "mdr_route_forced")
+
+
+def mdr_target_hits(cfg, sel, target, counts, hit=None, stream=None):
+    """Per-route target hits (hit, optional) and counts[0] = routes with a
+    target, counts[1] = hits (device int32 [2]); see include/mdr.h."""
+    _ok(lib().mdr_target_hits(ctypes.byref(cfg), _ptr(sel), _ptr(target), _ptr(hit), _ptr(counts),
+                              _stream(stream)), "mdr_target_hits")
 
 
 # ------------------------------------------------------------------ decoding

@@ -40,7 +40,10 @@ def out_to_numpy(out, w):
     return out.float().cpu().numpy()
 
 
-def run_gpu(w, inp, entry="forward"):
+def run_gpu(w, inp, entry="forward", force=None):
+    """entry "forward" = mdr_forward; "split" = mdr_build_index + mdr_route +
+    mdr_attend; "forced" = the split path with mdr_route_forced and the
+    forced ids ``force`` [B,Hq,nb]."""
     import torch
     from learned_product_hash_b200 import mdr
     cfg = mdr.make_config(w)
@@ -53,7 +56,11 @@ def run_gpu(w, inp, entry="forward"):
         mdr.mdr_forward(cfg, q, k, v, cb, idx, rt, out, ws)
     else:
         mdr.mdr_build_index(cfg, k, cb, idx, ws)
-        mdr.mdr_route(cfg, q, cb, idx, rt, ws)
+        if entry == "forced":
+            f = torch.from_numpy(np.ascontiguousarray(force, dtype=np.int32)).cuda()
+            mdr.mdr_route_forced(cfg, q, cb, idx, f, rt, ws)
+        else:
+            mdr.mdr_route(cfg, q, cb, idx, rt, ws)
         mdr.mdr_attend(cfg, q, k, v, rt.sel, out, ws)
     status = mdr.mdr_read_device_status(ws)
     torch.cuda.synchronize()
@@ -151,5 +158,20 @@ def compare(w, g, res, codebooks):
     return rep
 
 
-def oracle_for(w, inp, rows=None):
-    return O.forward(inp.q, inp.k, inp.v, inp.codebooks, O.Params.of(w), rows=rows)
+def sampled_rows(w, res, n=12, seed=0):
+    """Query blocks (b, hq, j) whose attention the oracle computes at full
+    size: the first and last, the four with the most candidates, and random
+    ones."""
+    r = np.random.default_rng(seed)
+    rows = {(0, 0, 0), (0, w.Hq - 1, w.nb - 1)}
+    heavy = np.argsort(-res.ncand.ravel())[:4]
+    for f in heavy:
+        b, h, j = np.unravel_index(f, res.ncand.shape)
+        rows.add((int(b), int(h), int(j)))
+    while len(rows) < n:
+        rows.add((int(r.integers(w.B)), int(r.integers(w.Hq)), int(r.integers(w.nb))))
+    return sorted(rows)
+
+
+def oracle_for(w, inp, rows=None, force=None):
+    return O.forward(inp.q, inp.k, inp.v, inp.codebooks, O.Params.of(w), rows=rows, force=force)

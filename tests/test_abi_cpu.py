@@ -130,3 +130,23 @@ def test_decode_entry_points_check_arguments_before_any_gpu_work():
     assert pre(TINY.block + 1) == mdr.MDR_ERR_INVALID_ARG             # not a whole number of blocks
     assert pre(TINY.S + TINY.block) == mdr.MDR_ERR_INVALID_ARG        # past the capacity
     assert pre(TINY.block, nbytes=n - 1) == mdr.MDR_ERR_WORKSPACE
+
+
+def test_control_entry_points_check_arguments_before_any_gpu_work():
+    L = mdr.lib()
+    cfg = mdr.make_config(TINY)
+    fake = ctypes.c_void_p(0x10000)            # never dereferenced: the checks fail first
+    idx = mdr.mdr_index(fake, fake, fake, fake, fake, fake)
+    rt = mdr.mdr_route_out(fake, None, None, None)
+    ws, n = ctypes.c_void_p(0x100000), 1 << 30
+    forced = lambda force, **kw: L.mdr_route_forced(
+        ctypes.byref(kw.get("cfg", cfg)), fake, fake, ctypes.byref(idx), force, ctypes.byref(kw.get("rt", rt)),
+        kw.get("ws", ws), n, None)
+    assert forced(None) == mdr.MDR_ERR_INVALID_ARG                      # the forced ids are required
+    assert forced(fake, rt=mdr.mdr_route_out(None, None, None, None)) == mdr.MDR_ERR_INVALID_ARG
+    assert forced(fake, ws=None) == mdr.MDR_ERR_WORKSPACE
+    assert forced(fake, cfg=mdr.make_config(TINY.with_(S=100))) == mdr.MDR_ERR_INVALID_ARG
+    hits = lambda sel, target, counts: L.mdr_target_hits(ctypes.byref(cfg), sel, target, None, counts, None)
+    assert hits(None, fake, fake) == mdr.MDR_ERR_INVALID_ARG
+    assert hits(fake, None, fake) == mdr.MDR_ERR_INVALID_ARG
+    assert hits(fake, fake, None) == mdr.MDR_ERR_INVALID_ARG

@@ -1,0 +1,60 @@
+"""Host logic of bench.py that needs no GPU: the clock sampler against a fake
+NVML (device matched by PCI address, reasons named from NVML's bits)."""
+import os
+import sys
+import time
+import types
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _fake_nvml(reason_bits):
+    nv = types.ModuleType("pynvml")
+    nv.NVML_CLOCK_SM = 1
+    for k, b in dict(GpuIdle=0x1, ApplicationsClocksSetting=0x2, SwPowerCap=0x4, HwSlowdown=0x8,
+                     SyncBoost=0x10, SwThermalSlowdown=0x20, HwThermalSlowdown=0x40,
+                     HwPowerBrakeSlowdown=0x80, DisplayClockSetting=0x100).items():
+        setattr(nv, "nvmlClocksEventReason" + k, b)
+    pcis = [types.SimpleNamespace(domain=0, bus=0x18, device=0), types.SimpleNamespace(domain=0, bus=0x2a, device=0)]
+    calls = {"shutdown": 0}
+    nv.nvmlInit = lambda: None
+    nv.nvmlShutdown = lambda: calls.__setitem__("shutdown", calls["shutdown"] + 1)
+    nv.nvmlDeviceGetCount = lambda: len(pcis)
+    nv.nvmlDeviceGetHandleByIndex = lambda i: i
+    nv.nvmlDeviceGetPciInfo = lambda h: pcis[h]
+    nv.nvmlDeviceGetMaxClockInfo = lambda h, c: 1965
+    nv.nvmlDeviceGetClockInfo = lambda h, c: 1965 if h == 1 else 300      # only the matched GPU is busy
+    nv.nvmlDeviceGetCurrentClocksEventReasons = lambda h: reason_bits if h == 1 else 0x1
+    nv.nvmlDeviceGetPowerUsage = lambda h: 700_000
+    return nv, calls
+
+
+@pytest.mark.parametrize("bits,want", [(0x0, []), (0x1, []), (0x4, ["sw_power_cap"]),
+                                       (0x10, ["sync_boost"]), (0x20, ["sw_thermal_slowdown"]),
+                                       (0x48, ["hw_slowdown", "hw_thermal_slowdown"])])
+def test_clock_sampler_matches_by_pci_and_names_reasons(monkeypatch, bits, want):
+    import bench
+    nv, calls = _fake_nvml(bits)
+    monkeypatch.setitem(sys.modules, "pynvml", nv)
+    props = types.SimpleNamespace(pci_domain_id=0, pci_bus_id=0x2a, pci_device_id=0)
+    monkeypatch.setattr(torch.cuda, "get_device_properties", lambda d: props)
+    with bench.ClockSampler(0) as clk:
+        time.sleep(0.02)
+    s = clk.summary()
+    assert s["samples"] >= 2
+    assert s["sm_mhz"] == 1965 and s["sm_max_mhz"] == 1965 and s["power_w"] == 700.0
+    assert s["reasons"] == want
+    assert calls["shutdown"] == 1
+
+
+def test_clock_sampler_without_nvml_reports_why(monkeypatch):
+    import bench
+    monkeypatch.setitem(sys.modules, "pynvml", None)         # import fails
+    with bench.ClockSampler(0) as clk:
+        pass
+    s = clk.summary()
+    assert "error" in s and "sm_mhz" not in s

@@ -124,19 +124,6 @@ def test_host_entry_point_matches_device():
     assert np.array_equal(got, g["out"])
 
 
-def _sampled_rows(w, res, n=12, seed=0):
-    r = np.random.default_rng(seed)
-    rows = {(0, 0, 0), (0, w.Hq - 1, w.nb - 1)}
-    # heaviest routes and random ones
-    heavy = np.argsort(-res.ncand.ravel())[:4]
-    for f in heavy:
-        b, h, j = np.unravel_index(f, res.ncand.shape)
-        rows.add((int(b), int(h), int(j)))
-    while len(rows) < n:
-        rows.add((int(r.integers(w.B)), int(r.integers(w.Hq)), int(r.integers(w.nb))))
-    return sorted(rows)
-
-
 @pytest.mark.parametrize("w", [SCALING_32K, LONG], ids=lambda w: w.name)
 def test_full_size_sampled(w):
     """The benchmark's launch at full size: routing compared everywhere,
@@ -145,7 +132,7 @@ def test_full_size_sampled(w):
     g = U.run_gpu(w, inp)
     p = O.Params.of(w)
     res = O.forward(inp.q, inp.k, inp.v, inp.codebooks, p, attention=False)
-    rows = _sampled_rows(w, res)
+    rows = U.sampled_rows(w, res)
     res.out = O.attend(res.qr, res.kr, inp.v.astype(np.float64), res.sel, w.block, p.softmax_scale, rows)
     rep = U.compare(w, g, res, inp.codebooks)
     if w is LONG:
