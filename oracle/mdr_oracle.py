@@ -561,3 +561,77 @@ def decode_step(st: DecodeState, q_t, k_t, v_t, codebooks, p: Params) -> DecodeO
             out[b, hq] = (w @ st.v[b, toks, h]) / w.sum()
     st.t = t + 1
     return DecodeOut(out, sel, smargin, qcodes, qmargin, ncand, qscale, sscale)
+
+
+# ------------------------------------------------------ 8. codebook calibration
+# Spherical codebook calibration ("Monodratic: a reproducible sparse attention
+# mixer", section Capacity and Figure 3: codebooks calibrated on a training
+# split remove the held-out overflow and lower the maximum assigned load).
+# The pages name the method and not its steps; the plainest reading is
+# spherical k-means run per subspace on the routing records (post-RoPE block
+# summaries, flattened), starting from the given codebooks:
+#   * assign: record x goes to the codeword k maximising <x_s, C[s,k]> --
+#     exactly the code assignment of section 3 (float32 scores, lower index
+#     on equal scores; the argmax does not depend on |x_s|);
+#   * update: C[s,k] becomes the normalised sum of the unit vectors
+#     x_s/|x_s| of its members (records with x_s = 0 have no direction and
+#     are left out); a codeword with no member, or whose members sum to zero,
+#     keeps its value.
+@dataclass
+class CalibStep:
+    codebooks: np.ndarray    # [P,K,dsub] float64, unit rows
+    assign: np.ndarray       # [N,P] codeword of each record per subspace
+    margin: np.ndarray       # [N,P] float32 gap between the best and second-best score
+    counts: np.ndarray       # [P,K] members with a direction (x_s != 0)
+
+
+def calibration_step(records: np.ndarray, codebooks: np.ndarray) -> CalibStep:
+    """One round of spherical k-means in every subspace.  records: [N,D]
+    (the values the calibration reads, float32 on the GPU); codebooks:
+    [P,K,D/P]."""
+    X = np.asarray(records, dtype=np.float64)
+    C = np.asarray(codebooks, dtype=np.float64)
+    P, K, dsub = C.shape
+    N = X.shape[0]
+    _, assign, margin = assign_codes(X.reshape(1, 1, N, P * dsub), C)
+    assign, margin = assign[0, 0], margin[0, 0]
+    new = C.copy()
+    counts = np.zeros((P, K), dtype=np.int64)
+    for s in range(P):
+        Xs = X[:, s * dsub:(s + 1) * dsub]
+        norm = np.linalg.norm(Xs, axis=1)
+        for k in range(K):
+            members = (assign[:, s] == k) & (norm > 0)
+            counts[s, k] = members.sum()
+            if counts[s, k] == 0:
+                continue
+            total = (Xs[members] / norm[members, None]).sum(axis=0)
+            tn = np.linalg.norm(total)
+            if tn > 0:
+                new[s, k] = total / tn
+    return CalibStep(new, assign, margin, counts)
+
+
+def calibrate(records: np.ndarray, codebooks: np.ndarray, iters: int) -> np.ndarray:
+    """iters rounds of calibration_step, each starting from the previous
+    round's codebooks rounded to float32 (the storage type of codebooks)."""
+    C = np.asarray(codebooks, dtype=np.float32)
+    for _ in range(iters):
+        C = calibration_step(records, C).codebooks.astype(np.float32)
+    return C
+
+
+def spherical_objective(records: np.ndarray, codebooks: np.ndarray) -> float:
+    """Sum over records and subspaces of the cosine between x_s and its best
+    codeword (records with x_s = 0 contribute nothing) -- the quantity
+    spherical k-means does not decrease."""
+    X = np.asarray(records, dtype=np.float64)
+    C = np.asarray(codebooks, dtype=np.float64)
+    P, K, dsub = C.shape
+    tot = 0.0
+    for s in range(P):
+        Xs = X[:, s * dsub:(s + 1) * dsub]
+        n = np.linalg.norm(Xs, axis=1)
+        ok = n > 0
+        tot += float((Xs[ok] / n[ok, None] @ C[s].T).max(axis=1).sum())
+    return tot

@@ -31,6 +31,10 @@ the storage type with round-to-nearest-even):
 
 Codebooks: P sets of K unit vectors of dimension D/P (Gaussian, normalised),
 the seeded untrained-router control.
+
+Calibration records (make_records): rows = one of n_centres unit centres
+times a log-normal length, plus sigma*N(0, I); optional zero rows and exact
+copies of a row (edge cases of the calibration).
 """
 from __future__ import annotations
 
@@ -168,3 +172,23 @@ def make_inputs(w: Workload, seed: int, *, keys: str | None = None,
     vv, vs_ = _store(v, w.dtype)
     return Inputs(q=qv, k=kv, v=vv, codebooks=make_codebooks(w, seed),
                   q_store=qs_, k_store=ks_, v_store=vs_, planted=planted)
+
+
+def make_records(N: int, D: int, n_centres: int, sigma: float, seed: int, *,
+                 zero_rows: int = 0, repeat_rows: int = 0) -> np.ndarray:
+    """Float32 records [N, D] for codebook calibration: each row is one of
+    n_centres unit centres (Gaussian, normalised; drawn uniformly per row)
+    scaled by a log-normal length, plus sigma*N(0, I).  zero_rows rows (at
+    seeded positions) are set to 0; repeat_rows rows are copies of row 0."""
+    r = rng_for(seed, "records", str(N), str(D), str(n_centres))
+    c = r.standard_normal((n_centres, D))
+    c /= np.linalg.norm(c, axis=1, keepdims=True)
+    which = r.integers(0, n_centres, size=N)
+    length = np.exp(0.5 * r.standard_normal(N))
+    x = c[which] * length[:, None] + sigma * r.standard_normal((N, D))
+    x = x.astype(np.float32)
+    if zero_rows:
+        x[r.choice(N, size=zero_rows, replace=False)] = 0.0
+    if repeat_rows:
+        x[r.choice(np.arange(1, N), size=repeat_rows, replace=False)] = x[0]
+    return x
