@@ -33,7 +33,7 @@ sys.path.insert(0, ROOT)
 
 import numpy as np  # noqa: E402
 
-from workloads import SCALING_SWEEP, ALL, make_inputs  # noqa: E402
+from workloads import SCALING_SWEEP, ALL, make_codebooks, make_inputs, make_keys  # noqa: E402
 
 METRIC = "routed-attention fwd tokens/s (index+route+attend) at 32K; % HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
@@ -402,6 +402,46 @@ def run_mine(args, w):
                                 "one planted block per sequence, random unit codebooks",
                     "routes_with_target": n_t, "target_hit_rate": rates}
 
+    # Codebook calibration on the long workload (the Report's Figure 3
+    # analogue): the key summaries of one training sequence, computed by
+    # mdr_build_index, calibrate the random codebooks for 20 rounds (timed);
+    # then a held-out sequence is indexed with the codebooks before and after.
+    calibration = None
+    if not args.no_calibration:
+        wl = workload("long")
+        cl = mdr.make_config(wl)
+        cb0 = torch.from_numpy(make_codebooks(wl, 3000 + rank)).to(dev)
+        ixl, wsl = mdr.Index.empty(cl, dev), mdr.workspace(cl, dev)
+        conv_b = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        mdr.mdr_build_index(cl, conv_b(make_keys(wl, 3001 + rank)[1]), cb0, ixl, wsl)
+        rec = ixl.kbar.clone()                                   # [1, Hkv, nb, D] = [N, D]
+        N = rec.numel() // wl.D
+        cws = mdr.calibrate_workspace(N, wl.D, wl.P, wl.K, dev)
+        cb1 = torch.empty_like(cb0)
+        rounds = 20
+        mdr.mdr_calibrate_codebooks(rec, cb0, cb1, 2, cws)       # warm-up
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        mdr.mdr_calibrate_codebooks(rec, cb0, cb1, rounds, cws)
+        c1.record(stream)
+        c1.synchronize()
+        c_ms = c0.elapsed_time(c1) / rounds
+        kh = conv_b(make_keys(wl, 3002 + rank)[1])
+        held = {}
+        for name, cbx in (("before", cb0), ("after", cb1)):
+            mdr.mdr_build_index(cl, kh, cbx, ixl, wsl)
+            held[name] = {"overflow": int(ixl.overflow.sum().item()), "max_load": int(ixl.maxload.max().item())}
+        c_bytes = 2 * N * wl.D * 4 + 2 * N * wl.P * 4           # records read by assign and update, assignment
+        peak_c, _ = peaks()
+        calibration = {"workload": f"{wl.name}: key summaries of one training sequence ({N} records of {wl.D}), "
+                                   f"P={wl.P}, K={wl.K}, {rounds} rounds from random unit codebooks",
+                       "us_per_round": c_ms * 1e3, "launches_per_round": 3,
+                       "roofline": {"bound": "hbm", "achieved": c_bytes / (c_ms / 1e3) / 1e9, "peak": peak_c,
+                                    "unit": "GB/s", "frac": c_bytes / (c_ms / 1e3) / 1e9 / peak_c,
+                                    "algorithmic_bytes_per_round": c_bytes},
+                       "held_out": held, "capacity": wl.cap}
+        del ixl, wsl, cws, rec
+
     # End to end through the C ABI with host buffers.
     e2e = None
     if not args.no_e2e:
@@ -448,7 +488,7 @@ def run_mine(args, w):
                              "kernel": "attend", "algorithmic_bytes_per_launch": attn_bytes},
                 "path_roofline_frac": total_bytes / (ms_max / 1e3) / 1e9 / peak,
                 "kernels_ms": ker, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
-                "controls": controls,
+                "controls": controls, "calibration": calibration,
                 "gpu_launches": KERNELS_PER_FORWARD * args.steps, "clocks": clk.summary(),
                 "overflow": int(idx.overflow.sum().item()), "selected_blocks": nsel}
         print(json.dumps(line), flush=True)
@@ -467,6 +507,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-controls", action="store_true")
+    ap.add_argument("--no-calibration", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()

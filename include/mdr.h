@@ -318,6 +318,42 @@ mdr_status mdr_decode_step(const mdr_config* cfg, int32_t t, const void* q_t,
  * word is nonzero.                                                           */
 mdr_status mdr_read_device_status(const void* ws, int32_t* code, void* stream);
 
+/* ------------------------------------------------- codebook calibration
+ * Spherical codebook calibration (Report, section Capacity and Figure 3:
+ * codebooks calibrated on a training split remove held-out overflow and
+ * lower the maximum assigned load).  The pages give the method's name, not
+ * its steps; this is spherical k-means per subspace, started from the
+ * given codebooks.  Each round:
+ *   assign  record x goes to the codeword of largest <x_s, C[s,k]> in each
+ *           subspace s (float32, lower index on equal scores: the address
+ *           code of mdr_build_index);
+ *   update  C[s,k] = the normalised sum of x_s/|x_s| over its members;
+ *           records whose x_s has no nonzero coordinate are not members; a
+ *           codeword with no member or a zero sum keeps its value.
+ * Sums run in a fixed order (float32), so a call is deterministic.
+ *
+ * records: device float32 [N,D], 16-byte aligned -- e.g. the block
+ *   summaries of a training split (mdr_index.kbar and mdr_route_out.qbar are
+ *   such arrays, [B,H,nb,D] = [N,D] with N = B*H*nb).
+ * codebooks_in, codebooks_out: device float32 [P,K,D/P], 16-byte aligned;
+ *   equal (in place) or disjoint.
+ * rounds: >= 0; 0 copies codebooks_in to codebooks_out.
+ * counts: device int32 [P,K] or NULL: members of each codeword in the last
+ *   round.  assign: device int32 [N,P] or NULL: each record's codeword in
+ *   the last round (the assignment to the codebooks that round started
+ *   from).
+ * ws: device, 256-byte aligned, at least mdr_calibrate_workspace_bytes.
+ * Supported: D in {32,64,128}, 1 <= P <= 4, D/P a multiple of 4 and >= 8,
+ * 1 <= K <= 128, 1 <= N <= 2^31/P (else MDR_ERR_UNSUPPORTED or
+ * MDR_ERR_INVALID_ARG, checked on the host before anything is enqueued).  */
+mdr_status mdr_calibrate_workspace_bytes(int64_t N, int32_t D, int32_t P, int32_t K,
+                                         size_t* bytes);
+mdr_status mdr_calibrate_codebooks(const float* records, int64_t N, int32_t D,
+                                   int32_t P, int32_t K, const float* codebooks_in,
+                                   float* codebooks_out, int32_t rounds,
+                                   int32_t* counts, int32_t* assign, void* ws,
+                                   size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

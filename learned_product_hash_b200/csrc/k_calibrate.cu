@@ -1,0 +1,174 @@
+// Codebook calibration: one round of spherical k-means per subspace
+// ("Monodratic: a reproducible sparse attention mixer", section Capacity and
+// Figure 3: codebooks calibrated on a training split).  The assignment step
+// is the codes kernel with one probe (the codeword of largest score, lower
+// index on equal scores); these two kernels do the update:
+//
+//   calib_partial_kernel   grid (chunks, P): each warp walks a contiguous run
+//                          of the chunk's records in order, turns the record's
+//                          sub-vector x_s into x_s/|x_s| (scaled by its
+//                          largest |coordinate| first, so no square
+//                          overflows or underflows) and adds it to its own
+//                          shared-memory row of the assigned codeword; a
+//                          sub-vector with no nonzero coordinate is skipped.
+//                          The warps' rows are added in warp order and
+//                          stored per chunk.
+//   calib_finalize_kernel  one warp per (subspace, codeword): adds the
+//                          chunks' sums in chunk order and normalises; a
+//                          codeword with no member, or a zero sum, keeps
+//                          the value the round started from.
+//
+// Every sum has a fixed order, so a round is deterministic.  Records are
+// read once per round by each kernel pair (N * D * 4 bytes, plus the
+// assignment); the per-chunk sums are P * chunks * K * dsub * 4 bytes, with
+// chunks chosen so that this stays below the records' size where possible.
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mdr {
+
+namespace {
+
+constexpr int kCalibMaxWarps = 8;
+constexpr size_t kCalibSmemBudget = 192 * 1024;
+
+}  // namespace
+
+void calib_plan(long long N, int D, int P, int K, int* chunk, int* nchunk, int* warps) {
+  const int dsub = D / P;
+  const size_t per_warp = (static_cast<size_t>(K) * dsub + K) * sizeof(float);
+  int w = static_cast<int>(kCalibSmemBudget / per_warp);
+  w = w < 1 ? 1 : (w > kCalibMaxWarps ? kCalibMaxWarps : w);
+  // About two CTAs per SM over all subspaces, at least 64 records per warp,
+  // and no more chunks than keep the per-chunk sums below the records.
+  const long long target_ctas = 296;
+  long long per = (N * P + target_ctas - 1) / target_ctas;
+  if (per < 64LL * w) per = 64LL * w;
+  const long long max_chunks = (N * D) / (static_cast<long long>(K) * D) + 1;   // N / K + 1
+  long long n = (N + per - 1) / per;
+  if (n > max_chunks) { n = max_chunks; per = (N + n - 1) / n; }
+  *chunk = static_cast<int>(per);
+  *nchunk = static_cast<int>((N + per - 1) / per);
+  *warps = w;
+}
+
+__global__ void calib_partial_kernel(const CalibArgs a) {
+  extern __shared__ float cal_smem[];
+  const int dsub = a.D / a.P;
+  const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* acc = cal_smem + static_cast<size_t>(warp) * a.K * dsub;
+  int* cnt = reinterpret_cast<int*>(cal_smem + static_cast<size_t>(nw) * a.K * dsub) + warp * a.K;
+  for (int i = lane; i < a.K * dsub; i += 32) acc[i] = 0.f;
+  for (int i = lane; i < a.K; i += 32) cnt[i] = 0;
+  __syncwarp();
+  grid_dependency_wait();                          // the assignment comes from the codes kernel
+
+  const int s = blockIdx.y;
+  const long long r0 = static_cast<long long>(blockIdx.x) * a.chunk;
+  const long long r1 = r0 + a.chunk < a.N ? r0 + a.chunk : a.N;
+  const long long per = (r1 - r0 + nw - 1) / nw;
+  const long long w0 = r0 + warp * per;
+  const long long w1 = w0 + per < r1 ? w0 + per : r1;
+  const int nj = (dsub + 31) / 32;                 // coordinates per lane (dsub <= 128)
+  const float* rec = a.records + s * dsub;
+  constexpr int U = 4;                             // records in flight per warp
+  for (long long r = w0; r < w1; r += U) {
+    float x[U][4];
+    int code[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long ru = r + u;
+      code[u] = ru < w1 ? a.assign[ru * a.P + s] : -1;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = lane + 32 * j;
+        x[u][j] = (ru < w1 && j < nj && c < dsub) ? rec[ru * a.D + c] : 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (code[u] < 0) break;
+      float m = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) m = fmaxf(m, fabsf(x[u][j]));
+      const float mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
+      if (mx == 0.f) continue;                     // no direction: not a member
+      float y[4], ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { y[j] = __fdiv_rn(x[u][j], mx); ss = __fmaf_rn(y[j], y[j], ss); }
+      const float n = __fsqrt_rn(warp_sum(ss));
+      float* row = acc + code[u] * dsub;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = lane + 32 * j;
+        if (j < nj && c < dsub) row[c] += __fdiv_rn(y[j], n);
+      }
+      if (lane == 0) cnt[code[u]] += 1;
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  const long long base = (static_cast<long long>(s) * a.nchunk + blockIdx.x) * a.K;
+  for (int i = threadIdx.x; i < a.K * dsub; i += blockDim.x) {
+    float v = 0.f;
+    for (int w = 0; w < nw; ++w) v += cal_smem[static_cast<size_t>(w) * a.K * dsub + i];
+    a.part[base * dsub + i] = v;
+  }
+  const int* cnts = reinterpret_cast<const int*>(cal_smem + static_cast<size_t>(nw) * a.K * dsub);
+  for (int k = threadIdx.x; k < a.K; k += blockDim.x) {
+    int c = 0;
+    for (int w = 0; w < nw; ++w) c += cnts[w * a.K + k];
+    a.pcount[base + k] = c;
+  }
+}
+
+__global__ void __launch_bounds__(128) calib_finalize_kernel(const CalibArgs a) {
+  grid_dependency_wait();                          // the sums come from the partial kernel
+  const int dsub = a.D / a.P;
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (gw >= a.P * a.K) return;
+  const int s = gw / a.K, k = gw % a.K;
+  float v[4] = {0.f, 0.f, 0.f, 0.f}, old[4];
+  int cnt = 0;
+  for (int c = 0; c < a.nchunk; ++c) {
+    const long long row = (static_cast<long long>(s) * a.nchunk + c) * a.K + k;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int d = lane + 32 * j;
+      if (d < dsub) v[j] += a.part[row * dsub + d];
+    }
+    cnt += a.pcount[row];
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int d = lane + 32 * j;
+    old[j] = d < dsub ? a.cb_old[(static_cast<long long>(s) * a.K + k) * dsub + d] : 0.f;
+    ss = __fmaf_rn(v[j], v[j], ss);
+  }
+  ss = warp_sum(ss);
+  const bool keep = cnt == 0 || ss == 0.f;
+  const float n = keep ? 1.f : __fsqrt_rn(ss);
+  __syncwarp();                                    // every lane has read its old value
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int d = lane + 32 * j;
+    if (d < dsub) a.cb_new[(static_cast<long long>(s) * a.K + k) * dsub + d] = keep ? old[j] : __fdiv_rn(v[j], n);
+  }
+  if (a.counts && lane == 0) a.counts[s * a.K + k] = cnt;
+}
+
+cudaError_t launch_calibrate_round(const CalibArgs& a, cudaStream_t st) {
+  const int dsub = a.D / a.P;
+  const size_t smem = static_cast<size_t>(a.warps) * (static_cast<size_t>(a.K) * dsub + a.K) * sizeof(float);
+  cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(calib_partial_kernel), static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(calib_partial_kernel, dim3(a.nchunk, a.P), dim3(a.warps * 32), smem, st, a);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(calib_finalize_kernel, dim3((a.P * a.K + 3) / 4), dim3(128), 0, st, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace mdr

@@ -49,12 +49,15 @@ codes_kernel(const __grid_constant__ CodesArgs a) {
   float* cbs = reinterpret_cast<float*>(csm4);                // [P][K][dsub + 4]
   float* xs = cbs + a.P * a.K * RS + warp * D;                // this warp's summary row
 
+  // The codebooks are staged before waiting on the previous kernel (they are
+  // an input of the forward), unless the previous kernel writes them.
+  if (a.codebooks_written_before) grid_dependency_wait();
   for (int i4 = threadIdx.x; i4 < a.K * D / 4; i4 += kCodeWarps * 32) {
     const int i = 4 * i4, row = i / dsub, d = i - row * dsub;  // row = sdx * K + k
-    *reinterpret_cast<float4*>(cbs + row * RS + d) = __ldg(reinterpret_cast<const float4*>(a.codebooks) + i4);
+    *reinterpret_cast<float4*>(cbs + row * RS + d) = reinterpret_cast<const float4*>(a.codebooks)[i4];
   }
   __syncthreads();
-  grid_dependency_wait();          // the summaries come from the previous kernel
+  if (!a.codebooks_written_before) grid_dependency_wait();   // the summaries come from the previous kernel
 
   const long long rows0 = a.xbar[0] ? static_cast<long long>(a.B) * a.H[0] * a.nb : 0;
   const long long rows1 = a.xbar[1] ? static_cast<long long>(a.B) * a.H[1] * a.nb : 0;

@@ -39,8 +39,27 @@ struct CodesArgs {
   int32_t* addr;           // [B,Hkv,nb] (side 1)
   const float* codebooks;  // [P,K,D/P]
   int B, nb, D, P, K, probes;
+  bool codebooks_written_before;   // the previous kernel on the stream writes the codebooks
 };
 cudaError_t launch_codes(const CodesArgs& a, cudaStream_t st);
+
+// Codebook calibration, one round of spherical k-means per subspace after
+// the codes kernel has assigned every record (probes = 1).
+struct CalibArgs {
+  const float* records;    // [N,D]
+  const int32_t* assign;   // [N,P]
+  const float* cb_old;     // [P,K,dsub] codebooks the round started from
+  float* cb_new;           // [P,K,dsub]; may equal cb_old
+  float* part;             // scratch [P,nchunk,K,dsub]
+  int32_t* pcount;         // scratch [P,nchunk,K]
+  int32_t* counts;         // [P,K] members per codeword, or null
+  long long N;
+  int D, P, K, chunk, nchunk, warps;
+};
+// Chunking of N records for the partial sums (records per CTA, CTAs per
+// subspace, warps per CTA) and the scratch it needs.
+void calib_plan(long long N, int D, int P, int K, int* chunk, int* nchunk, int* warps);
+cudaError_t launch_calibrate_round(const CalibArgs& a, cudaStream_t st);
 
 // K3: bounded causal posting lists of every (b, kv head).
 struct ListsArgs {

@@ -535,4 +535,74 @@ mdr_status mdr_decode_step(const mdr_config* cfg, int32_t t, const void* q_t, co
   return cuda_status(mdr::launch_decode(d, cfg->dtype == MDR_BF16, s));
 }
 
+// ------------------------------------------------------ codebook calibration
+struct CalibLayout {
+  size_t assign, part, pcount, total;
+  int chunk, nchunk, warps;
+};
+
+static mdr_status check_calib(int64_t N, int32_t D, int32_t P, int32_t K) {
+  if (N < 1 || P < 1 || K < 1) return MDR_ERR_INVALID_ARG;
+  if (D != 32 && D != 64 && D != 128) return MDR_ERR_UNSUPPORTED;
+  if (P > 4 || D % P != 0 || (D / P) % 4 != 0 || D / P < 8 || K > 128) return MDR_ERR_UNSUPPORTED;
+  if (N > INT32_MAX / P) return MDR_ERR_UNSUPPORTED;
+  return MDR_OK;
+}
+
+static CalibLayout calib_layout_of(int64_t N, int32_t D, int32_t P, int32_t K) {
+  CalibLayout l{};
+  mdr::calib_plan(N, D, P, K, &l.chunk, &l.nchunk, &l.warps);
+  size_t o = 0;
+  l.assign = o; o += align_up(static_cast<size_t>(N) * P * sizeof(int32_t));
+  l.part = o;   o += align_up(static_cast<size_t>(P) * l.nchunk * K * (D / P) * sizeof(float));
+  l.pcount = o; o += align_up(static_cast<size_t>(P) * l.nchunk * K * sizeof(int32_t));
+  l.total = o;
+  return l;
+}
+
+mdr_status mdr_calibrate_workspace_bytes(int64_t N, int32_t D, int32_t P, int32_t K, size_t* bytes) {
+  MDR_TRY(check_calib(N, D, P, K));
+  if (!bytes) return MDR_ERR_INVALID_ARG;
+  *bytes = calib_layout_of(N, D, P, K).total;
+  return MDR_OK;
+}
+
+mdr_status mdr_calibrate_codebooks(const float* records, int64_t N, int32_t D, int32_t P, int32_t K,
+                                   const float* codebooks_in, float* codebooks_out, int32_t rounds,
+                                   int32_t* counts, int32_t* assign, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  MDR_TRY(check_calib(N, D, P, K));
+  if (!records || !codebooks_in || !codebooks_out || rounds < 0) return MDR_ERR_INVALID_ARG;
+  if (!aligned16(records) || !aligned16(codebooks_in) || !aligned16(codebooks_out)) return MDR_ERR_INVALID_ARG;
+  const size_t cb_bytes = static_cast<size_t>(K) * D * sizeof(float);
+  const char* ci = reinterpret_cast<const char*>(codebooks_in);
+  const char* co = reinterpret_cast<const char*>(codebooks_out);
+  if (ci != co && ci < co + cb_bytes && co < ci + cb_bytes) return MDR_ERR_INVALID_ARG;   // partial overlap
+  const CalibLayout l = calib_layout_of(N, D, P, K);
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % kAlign != 0 || ws_bytes < l.total) return MDR_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (rounds == 0) {
+    if (ci != co) MDR_CUDA(cudaMemcpyAsync(codebooks_out, codebooks_in, cb_bytes, cudaMemcpyDeviceToDevice, st));
+    return MDR_OK;
+  }
+  int32_t* asg = assign ? assign : at<int32_t>(ws, l.assign);
+  mdr::CodesArgs ca{};
+  ca.xbar[0] = records; ca.H[0] = 1; ca.qcodes = asg;
+  ca.B = 1; ca.nb = static_cast<int>(N); ca.D = D; ca.P = P; ca.K = K; ca.probes = 1;
+  mdr::CalibArgs a{};
+  a.records = records; a.assign = asg; a.cb_new = codebooks_out;
+  a.part = at<float>(ws, l.part); a.pcount = at<int32_t>(ws, l.pcount);
+  a.N = N; a.D = D; a.P = P; a.K = K; a.chunk = l.chunk; a.nchunk = l.nchunk; a.warps = l.warps;
+  for (int r = 0; r < rounds; ++r) {
+    const float* cur = r == 0 ? codebooks_in : codebooks_out;
+    ca.codebooks = cur;
+    ca.codebooks_written_before = r > 0;
+    MDR_CUDA(mdr::launch_codes(ca, st));
+    a.cb_old = cur;
+    a.counts = r == rounds - 1 ? counts : nullptr;
+    MDR_CUDA(mdr::launch_calibrate_round(a, st));
+  }
+  return MDR_OK;
+}
+
 }  // extern "C"

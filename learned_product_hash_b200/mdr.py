@@ -22,7 +22,7 @@ EXPORTED = (
     "mdr_build_index", "mdr_route", "mdr_attend", "mdr_forward", "mdr_host_workspace_bytes",
     "mdr_forward_host", "mdr_read_device_status", "mdr_forward_profiled", "mdr_route_noalloc",
     "mdr_decode_workspace_bytes", "mdr_decode_reset", "mdr_decode_prefill", "mdr_decode_step",
-    "mdr_route_forced", "mdr_target_hits",
+    "mdr_route_forced", "mdr_target_hits", "mdr_calibrate_workspace_bytes", "mdr_calibrate_codebooks",
 )
 
 
@@ -82,6 +82,10 @@ def lib() -> ctypes.CDLL:
             "mdr_route_noalloc": ([cfgp, vp, vp, idxp, vp, vp, vp], i32),
             "mdr_route_forced": ([cfgp, vp, vp, idxp, vp, rtp, vp, sz, vp], i32),
             "mdr_target_hits": ([cfgp, vp, vp, vp, vp, vp], i32),
+            "mdr_calibrate_workspace_bytes": ([ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                               ctypes.POINTER(sz)], i32),
+            "mdr_calibrate_codebooks": ([vp, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                         vp, vp, ctypes.c_int32, vp, vp, vp, sz, vp], i32),
             "mdr_decode_workspace_bytes": ([cfgp, ctypes.POINTER(sz)], i32),
             "mdr_decode_reset": ([cfgp, ctypes.POINTER(mdr_decode_state), vp], i32),
             "mdr_decode_prefill": ([cfgp, ctypes.c_int32, vp, vp, vp, ctypes.POINTER(mdr_decode_state),
@@ -267,6 +271,31 @@ def mdr_target_hits(cfg, sel, target, counts, hit=None, stream=None):
     target, counts[1] = hits (device int32 [2]); see include/mdr.h."""
     _ok(lib().mdr_target_hits(ctypes.byref(cfg), _ptr(sel), _ptr(target), _ptr(hit), _ptr(counts),
                               _stream(stream)), "mdr_target_hits")
+
+
+# ------------------------------------------------------ codebook calibration
+def mdr_calibrate_workspace_bytes(N: int, D: int, P: int, K: int) -> int:
+    n = ctypes.c_size_t(0)
+    _ok(lib().mdr_calibrate_workspace_bytes(N, D, P, K, ctypes.byref(n)), "mdr_calibrate_workspace_bytes")
+    return n.value
+
+
+def calibrate_workspace(N: int, D: int, P: int, K: int, device=None):
+    import torch
+    return torch.empty(mdr_calibrate_workspace_bytes(N, D, P, K), dtype=torch.uint8,
+                       device=device or torch.device("cuda"))
+
+
+def mdr_calibrate_codebooks(records, codebooks_in, codebooks_out, rounds, ws, counts=None, assign=None,
+                            stream=None):
+    """records: float32 [N, D] (or any contiguous [..., D]); codebooks
+    float32 [P, K, D/P]; see include/mdr.h."""
+    D = records.shape[-1]
+    N = records.numel() // D
+    P, K = codebooks_in.shape[0], codebooks_in.shape[1]
+    _ok(lib().mdr_calibrate_codebooks(_ptr(records), N, D, P, K, _ptr(codebooks_in), _ptr(codebooks_out),
+                                      int(rounds), _ptr(counts), _ptr(assign), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "mdr_calibrate_codebooks")
 
 
 # ------------------------------------------------------------------ decoding

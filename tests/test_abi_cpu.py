@@ -150,3 +150,25 @@ def test_control_entry_points_check_arguments_before_any_gpu_work():
     assert hits(None, fake, fake) == mdr.MDR_ERR_INVALID_ARG
     assert hits(fake, None, fake) == mdr.MDR_ERR_INVALID_ARG
     assert hits(fake, fake, None) == mdr.MDR_ERR_INVALID_ARG
+
+
+def test_calibration_entry_points_check_arguments_before_any_gpu_work():
+    L = mdr.lib()
+    n = ctypes.c_size_t(0)
+    assert L.mdr_calibrate_workspace_bytes(8192, 128, 2, 64, ctypes.byref(n)) == mdr.MDR_OK and n.value > 0
+    assert L.mdr_calibrate_workspace_bytes(0, 128, 2, 64, ctypes.byref(n)) == mdr.MDR_ERR_INVALID_ARG
+    assert L.mdr_calibrate_workspace_bytes(10, 96, 2, 64, ctypes.byref(n)) == mdr.MDR_ERR_UNSUPPORTED
+    assert L.mdr_calibrate_workspace_bytes(10, 128, 2, 129, ctypes.byref(n)) == mdr.MDR_ERR_UNSUPPORTED
+    assert L.mdr_calibrate_workspace_bytes(10, 32, 8, 4, ctypes.byref(n)) == mdr.MDR_ERR_UNSUPPORTED   # P > 4
+    assert L.mdr_calibrate_workspace_bytes(10, 32, 4, 4, ctypes.byref(n)) == mdr.MDR_OK                  # dsub 8
+    fake = ctypes.c_void_p(0x10000)
+    ws, nbytes = ctypes.c_void_p(0x100000), 1 << 30
+    call = lambda rec=fake, cin=fake, cout=fake, rounds=1, ws=ws: L.mdr_calibrate_codebooks(
+        rec, 100, 64, 2, 16, cin, cout, rounds, None, None, ws, nbytes, None)
+    assert call(rec=None) == mdr.MDR_ERR_INVALID_ARG
+    assert call(rec=ctypes.c_void_p(0x10004)) == mdr.MDR_ERR_INVALID_ARG          # not 16-byte aligned
+    assert call(cout=None) == mdr.MDR_ERR_INVALID_ARG
+    assert call(rounds=-1) == mdr.MDR_ERR_INVALID_ARG
+    assert call(cout=ctypes.c_void_p(0x10010)) == mdr.MDR_ERR_INVALID_ARG         # overlaps the input codebooks
+    assert call(ws=None) == mdr.MDR_ERR_WORKSPACE
+    assert call(ws=ctypes.c_void_p(0x100010)) == mdr.MDR_ERR_WORKSPACE            # not 256-byte aligned

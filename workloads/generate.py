@@ -149,22 +149,7 @@ def make_inputs(w: Workload, seed: int, *, keys: str | None = None,
                         qb = q[b, (nb - 1) * bs:nb * bs, hq]
                         qb[:, coords] += ALPHA_PLANTED * u[None, :]
         elif keys == "clusters":
-            r = rng_for(seed, w.name, "k")
-            coords = slow_pair_coords(D, w.cluster_pairs)
-            C = w.n_clusters
-            centres = _unit(r, (Hkv, C, coords.size))
-            if w.zipf_s > 0:
-                pr = np.arange(1, C + 1, dtype=np.float64) ** (-w.zipf_s)
-                pr /= pr.sum()
-            else:
-                pr = np.full(C, 1.0 / C)
-            k = w.sigma * _normal(r, (B, S, Hkv, D))
-            member = r.choice(C, size=(B, Hkv, nb), p=pr)
-            for b in range(B):
-                for h in range(Hkv):
-                    cen = centres[h, member[b, h]]            # [nb, m]
-                    kh = k[b, :, h]                           # view [S, D]
-                    kh[:, coords] += np.repeat(cen, bs, axis=0)
+            k = _cluster_keys(w, seed)
         else:
             raise ValueError(keys)
     qv, qs_ = _store(q, w.dtype)
@@ -172,6 +157,41 @@ def make_inputs(w: Workload, seed: int, *, keys: str | None = None,
     vv, vs_ = _store(v, w.dtype)
     return Inputs(q=qv, k=kv, v=vv, codebooks=make_codebooks(w, seed),
                   q_store=qs_, k_store=ks_, v_store=vs_, planted=planted)
+
+
+def _cluster_keys(w: Workload, seed: int) -> np.ndarray:
+    B, S, Hkv, D, bs = w.B, w.S, w.Hkv, w.D, w.block
+    nb = S // bs
+    r = rng_for(seed, w.name, "k")
+    coords = slow_pair_coords(D, w.cluster_pairs)
+    C = w.n_clusters
+    centres = _unit(r, (Hkv, C, coords.size))
+    if w.zipf_s > 0:
+        pr = np.arange(1, C + 1, dtype=np.float64) ** (-w.zipf_s)
+        pr /= pr.sum()
+    else:
+        pr = np.full(C, 1.0 / C)
+    k = w.sigma * _normal(r, (B, S, Hkv, D))
+    member = r.choice(C, size=(B, Hkv, nb), p=pr)
+    for b in range(B):
+        for h in range(Hkv):
+            cen = centres[h, member[b, h]]            # [nb, m]
+            kh = k[b, :, h]                           # view [S, D]
+            kh[:, coords] += np.repeat(cen, bs, axis=0)
+    return k
+
+
+def make_keys(w: Workload, seed: int):
+    """The keys make_inputs(w, seed) would give (gaussian or clusters
+    recipe), without drawing q and v: (k as stored, widened to float32;
+    k in its storage type).  Used where only the index is built."""
+    if w.keys == "gaussian":
+        k = _normal(rng_for(seed, w.name, "k"), (w.B, w.S, w.Hkv, w.D))
+    elif w.keys == "clusters":
+        k = _cluster_keys(w, seed)
+    else:
+        raise ValueError(f"keys-only generation does not cover the {w.keys} recipe")
+    return _store(k, w.dtype)
 
 
 def make_records(N: int, D: int, n_centres: int, sigma: float, seed: int, *,
