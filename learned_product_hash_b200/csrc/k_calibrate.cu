@@ -5,12 +5,15 @@
 // index on equal scores); these two kernels do the update:
 //
 //   calib_partial_kernel   grid (chunks, P): each warp walks a contiguous run
-//                          of the chunk's records in order, turns the record's
-//                          sub-vector x_s into x_s/|x_s| (scaled by its
-//                          largest |coordinate| first, so no square
-//                          overflows or underflows) and adds it to its own
-//                          shared-memory row of the assigned codeword; a
-//                          sub-vector with no nonzero coordinate is skipped.
+//                          of the chunk's records in order, eight at a time:
+//                          turns each record's sub-vector x_s into x_s/|x_s|
+//                          (scaled first by the power of two that brings its
+//                          largest |coordinate| into [0.5, 1), which is
+//                          exact, then multiplied by the correctly rounded
+//                          1/sqrt of its sum of squares) and adds it to its
+//                          own shared-memory row of the assigned codeword, in
+//                          record order; a sub-vector with no nonzero
+//                          coordinate is skipped.
 //                          The warps' rows are added in warp order and
 //                          stored per chunk.
 //   calib_finalize_kernel  one warp per (subspace, codeword): adds the
@@ -40,12 +43,13 @@ void calib_plan(long long N, int D, int P, int K, int* chunk, int* nchunk, int* 
   const size_t per_warp = (static_cast<size_t>(K) * dsub + K) * sizeof(float);
   int w = static_cast<int>(kCalibSmemBudget / per_warp);
   w = w < 1 ? 1 : (w > kCalibMaxWarps ? kCalibMaxWarps : w);
-  // About two CTAs per SM over all subspaces, at least 64 records per warp,
-  // and no more chunks than keep the per-chunk sums below the records.
+  // About two CTAs per SM over all subspaces, at least 16 records per warp,
+  // and no more chunks than keep the per-chunk sums (K * dsub floats each)
+  // about the size of the records (chunk * dsub floats each).
   const long long target_ctas = 296;
   long long per = (N * P + target_ctas - 1) / target_ctas;
-  if (per < 64LL * w) per = 64LL * w;
-  const long long max_chunks = (N * D) / (static_cast<long long>(K) * D) + 1;   // N / K + 1
+  if (per < 16LL * w) per = 16LL * w;
+  const long long max_chunks = N / K + 1;
   long long n = (N + per - 1) / per;
   if (n > max_chunks) { n = max_chunks; per = (N + n - 1) / n; }
   *chunk = static_cast<int>(per);
@@ -72,9 +76,9 @@ __global__ void calib_partial_kernel(const CalibArgs a) {
   const long long w1 = w0 + per < r1 ? w0 + per : r1;
   const int nj = (dsub + 31) / 32;                 // coordinates per lane (dsub <= 128)
   const float* rec = a.records + s * dsub;
-  constexpr int U = 4;                             // records in flight per warp
+  constexpr int U = 8;                             // records in flight per warp
   for (long long r = w0; r < w1; r += U) {
-    float x[U][4];
+    float x[U][4], rn[U];
     int code[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -86,26 +90,43 @@ __global__ void calib_partial_kernel(const CalibArgs a) {
         x[u][j] = (ru < w1 && j < nj && c < dsub) ? rec[ru * a.D + c] : 0.f;
       }
     }
+    // Scale each sub-vector by a power of two (exact) that brings its largest
+    // |coordinate| into [0.5, 1), so the sum of squares neither overflows nor
+    // underflows; the eight records' sums proceed side by side.
+    float ss[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      if (code[u] < 0) break;
       float m = 0.f;
 #pragma unroll
       for (int j = 0; j < 4; ++j) m = fmaxf(m, fabsf(x[u][j]));
       const float mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
-      if (mx == 0.f) continue;                     // no direction: not a member
-      float y[4], ss = 0.f;
+      if (mx == 0.f) code[u] = -1;                 // no direction: not a member
+      int ex = 0;
+      frexpf(mx, &ex);
+      ss[u] = 0.f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) { y[j] = __fdiv_rn(x[u][j], mx); ss = __fmaf_rn(y[j], y[j], ss); }
-      const float n = __fsqrt_rn(warp_sum(ss));
+      for (int j = 0; j < 4; ++j) {
+        x[u][j] = ldexpf(x[u][j], -ex);
+        ss[u] = __fmaf_rn(x[u][j], x[u][j], ss[u]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < U; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], o);
+#pragma unroll
+    for (int u = 0; u < U; ++u) rn[u] = code[u] >= 0 ? __frsqrt_rn(ss[u]) : 0.f;
+    // Add the unit vectors to the codewords' rows in record order.
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (code[u] < 0) continue;
       float* row = acc + code[u] * dsub;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int c = lane + 32 * j;
-        if (j < nj && c < dsub) row[c] += __fdiv_rn(y[j], n);
+        if (j < nj && c < dsub) row[c] += x[u][j] * rn[u];
       }
       if (lane == 0) cnt[code[u]] += 1;
-      __syncwarp();
     }
   }
   __syncthreads();
@@ -131,14 +152,28 @@ __global__ void __launch_bounds__(128) calib_finalize_kernel(const CalibArgs a) 
   const int s = gw / a.K, k = gw % a.K;
   float v[4] = {0.f, 0.f, 0.f, 0.f}, old[4];
   int cnt = 0;
-  for (int c = 0; c < a.nchunk; ++c) {
-    const long long row = (static_cast<long long>(s) * a.nchunk + c) * a.K + k;
+  constexpr int G = 8;                             // chunk rows loaded together, added in order
+  for (int c0 = 0; c0 < a.nchunk; c0 += G) {
+    float t[G][4];
+    int tc[G];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int d = lane + 32 * j;
-      if (d < dsub) v[j] += a.part[row * dsub + d];
+    for (int g = 0; g < G; ++g) {
+      const int c = c0 + g;
+      const long long row = (static_cast<long long>(s) * a.nchunk + c) * a.K + k;
+      tc[g] = c < a.nchunk ? a.pcount[row] : 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int d = lane + 32 * j;
+        t[g][j] = (c < a.nchunk && d < dsub) ? a.part[row * dsub + d] : 0.f;
+      }
     }
-    cnt += a.pcount[row];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      if (c0 + g >= a.nchunk) break;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] += t[g][j];
+      cnt += tc[g];
+    }
   }
   float ss = 0.f;
 #pragma unroll
