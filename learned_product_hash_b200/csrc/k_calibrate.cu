@@ -16,8 +16,9 @@
 //                          coordinate is skipped.
 //                          The warps' rows are added in warp order and
 //                          stored per chunk.
-//   calib_finalize_kernel  one warp per (subspace, codeword): adds the
-//                          chunks' sums in chunk order and normalises; a
+//   calib_finalize_kernel  one CTA per (subspace, codeword): warp w adds
+//                          chunks w, w+8, ... in order, the warps' sums are
+//                          added in warp order, then normalised; a
 //                          codeword with no member, or a zero sum, keeps
 //                          the value the round started from.
 //
@@ -144,21 +145,26 @@ __global__ void calib_partial_kernel(const CalibArgs a) {
   }
 }
 
-__global__ void __launch_bounds__(128) calib_finalize_kernel(const CalibArgs a) {
+constexpr int kFinWarps = 8;
+
+__global__ void __launch_bounds__(kFinWarps * 32) calib_finalize_kernel(const CalibArgs a) {
+  __shared__ float wsum[kFinWarps][128];
+  __shared__ int wcnt[kFinWarps];
   grid_dependency_wait();                          // the sums come from the partial kernel
   const int dsub = a.D / a.P;
-  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (gw >= a.P * a.K) return;
-  const int s = gw / a.K, k = gw % a.K;
-  float v[4] = {0.f, 0.f, 0.f, 0.f}, old[4];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int s = blockIdx.x / a.K, k = blockIdx.x % a.K;
+  // Warp w adds chunks w, w + 8, w + 16, ... in increasing order, eight rows
+  // loaded together; the warps' sums are then added in warp order.
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
   int cnt = 0;
-  constexpr int G = 8;                             // chunk rows loaded together, added in order
-  for (int c0 = 0; c0 < a.nchunk; c0 += G) {
+  constexpr int G = 8;
+  for (int c0 = warp; c0 < a.nchunk; c0 += G * kFinWarps) {
     float t[G][4];
     int tc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const int c = c0 + g;
+      const int c = c0 + g * kFinWarps;
       const long long row = (static_cast<long long>(s) * a.nchunk + c) * a.K + k;
       tc[g] = c < a.nchunk ? a.pcount[row] : 0;
 #pragma unroll
@@ -169,16 +175,29 @@ __global__ void __launch_bounds__(128) calib_finalize_kernel(const CalibArgs a) 
     }
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      if (c0 + g >= a.nchunk) break;
+      if (c0 + g * kFinWarps >= a.nchunk) break;
 #pragma unroll
       for (int j = 0; j < 4; ++j) v[j] += t[g][j];
       cnt += tc[g];
     }
   }
-  float ss = 0.f;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int d = lane + 32 * j;
+    if (d < dsub) wsum[warp][d] = v[j];
+  }
+  if (lane == 0) wcnt[warp] = cnt;
+  __syncthreads();
+  if (warp != 0) return;
+  float old[4], ss = 0.f;
+  cnt = 0;
+  for (int w = 0; w < kFinWarps; ++w) cnt += wcnt[w];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int d = lane + 32 * j;
+    v[j] = 0.f;
+    if (d < dsub)
+      for (int w = 0; w < kFinWarps; ++w) v[j] += wsum[w][d];
     old[j] = d < dsub ? a.cb_old[(static_cast<long long>(s) * a.K + k) * dsub + d] : 0.f;
     ss = __fmaf_rn(v[j], v[j], ss);
   }
@@ -201,7 +220,7 @@ cudaError_t launch_calibrate_round(const CalibArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   e = launch_pdl(calib_partial_kernel, dim3(a.nchunk, a.P), dim3(a.warps * 32), smem, st, a);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(calib_finalize_kernel, dim3((a.P * a.K + 3) / 4), dim3(128), 0, st, a);
+  e = launch_pdl(calib_finalize_kernel, dim3(a.P * a.K), dim3(kFinWarps * 32), 0, st, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
