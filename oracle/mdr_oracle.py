@@ -635,3 +635,77 @@ def spherical_objective(records: np.ndarray, codebooks: np.ndarray) -> float:
         ok = n > 0
         tot += float((Xs[ok] / n[ok, None] @ C[s].T).max(axis=1).sum())
     return tot
+
+
+# ---------------------------------------------------------------- 9. backward
+# Gradients of the mixer's output with the route held fixed.  The Article
+# ("The 99.35 Percent Result Does Not Establish Language Quality") notes that
+# hard top-k choices give no ordinary gradient through the chosen index and
+# leaves surrogates to the trainer; so the plainest backward differentiates
+# the selected-set softmax and the rotary embedding only: given dL/d(out),
+# it returns dL/dq, dL/dk, dL/dv, and nothing reaches the codebooks or the
+# block summaries.
+def attend_backward(qr, kr, v, sel, bs: int, scale: float, dout):
+    """dL/dq', dL/dk', dL/dv of attend() for dL/d(out) = dout [B,S,Hq,D].
+
+    Per query block j and head hq, with T = the tokens of the selected
+    blocks, S = scale * q' k'^T masked to s <= t and P = softmax(S):
+      dv[T]  += P^T dout_j
+      dP      = dout_j v[T]^T
+      dS      = P * (dP - rowsum(P * dP))
+      dq'_j   = scale * dS k'[T]
+      dk'[T] += scale * dS^T q'_j
+    Key and value gradients of a KV head add over its query heads.  A query
+    block with no valid selected block has a zero output and gets zero
+    gradients."""
+    B, S, Hq, D = qr.shape
+    Hkv = kr.shape[2]
+    g = Hq // Hkv
+    dq = np.zeros_like(qr, dtype=np.float64)
+    dk = np.zeros(kr.shape, dtype=np.float64)
+    dv = np.zeros(v.shape, dtype=np.float64)
+    nb = S // bs
+    for b in range(B):
+        for hq in range(Hq):
+            h = hq // g
+            for j in range(nb):
+                toks = selected_tokens(sel[b, hq, j], bs)
+                if toks.size == 0:
+                    continue
+                qpos = np.arange(j * bs, (j + 1) * bs)
+                Q, Kt, Vt = qr[b, qpos, hq], kr[b, toks, h], v[b, toks, h]
+                s = (Q @ Kt.T) * scale
+                s[toks[None, :] > qpos[:, None]] = -np.inf
+                s -= s.max(axis=1, keepdims=True)
+                P = np.exp(s)
+                P /= P.sum(axis=1, keepdims=True)
+                dO = dout[b, qpos, hq]
+                dv[b, toks, h] += P.T @ dO
+                dP = dO @ Vt.T
+                dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+                dq[b, qpos, hq] = scale * dS @ Kt
+                dk[b, toks, h] += scale * dS.T @ Q
+    return dq, dk, dv
+
+
+def rope_transpose(y: np.ndarray, base: float) -> np.ndarray:
+    """The transpose of the rotation of section 1 at every position (it is
+    orthogonal, so this is its inverse): y1*cos + y2*sin, y2*cos - y1*sin."""
+    B, S, H, D = y.shape
+    th = rope_angles(S, D, base).astype(np.float64)
+    c, s = np.cos(th)[None, :, None, :], np.sin(th)[None, :, None, :]
+    y1, y2 = y[..., : D // 2], y[..., D // 2:]
+    return np.concatenate([y1 * c + y2 * s, y2 * c - y1 * s], axis=-1)
+
+
+def backward(q, k, v, codebooks, p: Params, dout, sel=None):
+    """dL/dq, dL/dk, dL/dv of forward() for dL/d(out) = dout, with the route
+    of forward() (or the given sel) held fixed.  -> (dq, dk, dv, sel)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    if sel is None:
+        sel = forward(q, k, v, codebooks, p, attention=False).sel
+    qr, kr = rope(q, p.rope_base), rope(k, p.rope_base)
+    dqr, dkr, dv = attend_backward(qr, kr, v, sel, p.block, p.softmax_scale, np.asarray(dout, dtype=np.float64))
+    return rope_transpose(dqr, p.rope_base), rope_transpose(dkr, p.rope_base), dv, sel
