@@ -318,6 +318,34 @@ mdr_status mdr_decode_step(const mdr_config* cfg, int32_t t, const void* q_t,
  * word is nonzero.                                                           */
 mdr_status mdr_read_device_status(const void* ws, int32_t* code, void* stream);
 
+/* ------------------------------------------------------------- backward
+ * Gradients of the attention output with the route held fixed.  The pages
+ * note that hard top-k choices give no ordinary gradient through the chosen
+ * index and leave surrogates to the trainer (Article, "The 99.35 Percent
+ * Result Does Not Establish Language Quality"); this is the gradient of
+ * mdr_attend's output with respect to q, k and v for a given sel:
+ *   for token t of block j and every selected token s <= t,
+ *   P = softmax(scale*<q'_t, k'_s>), dv_s += P dout_t,
+ *   dS = P (<dout_t, v_s> - <dout_t, out_t>),
+ *   dq'_t += scale dS k'_s, dk'_s += scale dS q'_t,
+ *   dq = R(t)^T dq', dk = R(s)^T dk' (the transpose of the rotation);
+ * key and value gradients of a KV head add over its query heads; a query
+ * block with no valid selected block gets zero gradients.  Nothing reaches
+ * the codebooks or the summaries.
+ * q, k, v: device [B,S,H,D] in cfg->dtype (not rotated: the inputs of
+ * mdr_forward); sel: device int32 [B,Hq,nb,R+L] as written by a route call;
+ * dout: device [B,S,Hq,D] in cfg->dtype; dq [B,S,Hq,D], dk and dv
+ * [B,S,Hkv,D]: device float32, written (not accumulated).  Arithmetic is
+ * float32 in a fixed order (deterministic).  ws: device, 256-byte aligned,
+ * at least mdr_backward_workspace_bytes; its first word is the device
+ * status (2: a selected id later than its query block, skipped), read with
+ * mdr_read_device_status.                                                   */
+mdr_status mdr_backward_workspace_bytes(const mdr_config* cfg, size_t* bytes);
+mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void* k,
+                               const void* v, const int32_t* sel, const void* dout,
+                               float* dq, float* dk, float* dv, void* ws,
+                               size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------- codebook calibration
  * Spherical codebook calibration (Report, section Capacity and Figure 3:
  * codebooks calibrated on a training split remove held-out overflow and

@@ -139,4 +139,28 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t st);
 
+// Backward of the selected-set attention (route fixed): dq, dk, dv in float32.
+struct BwdArgs {
+  const void* q;           // [B,S,Hq,D] storage type (not rotated)
+  const void* k;           // [B,S,Hkv,D]
+  const void* v;           // [B,S,Hkv,D]
+  const void* dout;        // [B,S,Hq,D] upstream gradient, storage type
+  const int32_t* sel;      // [B,Hq,nb,nsel]
+  float* qr;               // scratch: rotated q, float32 [B,S,Hq,D]
+  float* kr;               // scratch: rotated k, float32 [B,S,Hkv,D]
+  float* lse;              // scratch: [B,Hq,S] log-sum-exp of the scaled scores
+  float* delta;            // scratch: [B,Hq,S] dout_t . out_t
+  int32_t* rev_off;        // scratch: [B,Hkv,nb+1] reverse-index offsets
+  int32_t* rev;            // scratch: [B,Hkv,(Hq/Hkv)*nb*nsel] (local query head * nb + query block)
+  float* dq;               // [B,S,Hq,D]
+  float* dk;               // [B,S,Hkv,D]
+  float* dv;               // [B,S,Hkv,D]
+  int32_t* status;         // a selected id past its query block sets 2
+  int B, S, Hq, Hkv, D, bs, nb, nsel;
+  float scale;
+  float inv_freq[64];
+};
+size_t bwd_rev_smem(int nb);
+cudaError_t launch_backward(const BwdArgs& a, bool bf16, cudaStream_t st);
+
 }  // namespace mdr

@@ -535,6 +535,60 @@ mdr_status mdr_decode_step(const mdr_config* cfg, int32_t t, const void* q_t, co
   return cuda_status(mdr::launch_decode(d, cfg->dtype == MDR_BF16, s));
 }
 
+// ------------------------------------------------------------------ backward
+struct BwdLayout {
+  size_t status, qr, kr, lse, delta, rev_off, rev, total;
+};
+
+static BwdLayout bwd_layout_of(const mdr_config* c) {
+  BwdLayout l{};
+  const size_t tok = static_cast<size_t>(c->B) * c->S;
+  const size_t nb = static_cast<size_t>(c->S / c->block);
+  size_t o = 0;
+  l.status = o;  o += align_up(16);
+  l.qr = o;      o += align_up(tok * c->Hq * c->D * sizeof(float));
+  l.kr = o;      o += align_up(tok * c->Hkv * c->D * sizeof(float));
+  l.lse = o;     o += align_up(tok * c->Hq * sizeof(float));
+  l.delta = o;   o += align_up(tok * c->Hq * sizeof(float));
+  l.rev_off = o; o += align_up(static_cast<size_t>(c->B) * c->Hkv * (nb + 1) * sizeof(int32_t));
+  l.rev = o;     o += align_up(static_cast<size_t>(c->B) * c->Hq * nb * (c->R + c->L) * sizeof(int32_t));
+  l.total = o;
+  return l;
+}
+
+mdr_status mdr_backward_workspace_bytes(const mdr_config* cfg, size_t* bytes) {
+  MDR_TRY(check(cfg));
+  if (!bytes) return MDR_ERR_INVALID_ARG;
+  *bytes = bwd_layout_of(cfg).total;
+  return MDR_OK;
+}
+
+mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void* k, const void* v,
+                               const int32_t* sel, const void* dout, float* dq, float* dk, float* dv,
+                               void* ws, size_t ws_bytes, void* stream) {
+  MDR_TRY(check(cfg));
+  if (!q || !k || !v || !sel || !dout || !dq || !dk || !dv) return MDR_ERR_INVALID_ARG;
+  const BwdLayout l = bwd_layout_of(cfg);
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % kAlign != 0 || ws_bytes < l.total) return MDR_ERR_WORKSPACE;
+  if (static_cast<long long>(cfg->B) * cfg->Hq * (cfg->S / cfg->block) * (cfg->block / 16) > INT32_MAX)
+    return MDR_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MDR_CUDA(cudaMemsetAsync(at<int32_t>(ws, l.status), 0, sizeof(int32_t), st));
+  mdr::BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.dout = dout; a.sel = sel;
+  a.qr = at<float>(ws, l.qr); a.kr = at<float>(ws, l.kr);
+  a.lse = at<float>(ws, l.lse); a.delta = at<float>(ws, l.delta);
+  a.rev_off = at<int32_t>(ws, l.rev_off); a.rev = at<int32_t>(ws, l.rev);
+  a.dq = dq; a.dk = dk; a.dv = dv; a.status = at<int32_t>(ws, l.status);
+  a.B = cfg->B; a.S = cfg->S; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.bs = cfg->block;
+  a.nb = cfg->S / cfg->block; a.nsel = cfg->R + cfg->L;
+  a.scale = cfg->scale > 0.f ? cfg->scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(cfg->D)));
+  for (int i = 0; i < cfg->D / 2; ++i)
+    a.inv_freq[i] = static_cast<float>(std::pow(static_cast<double>(cfg->rope_base), -2.0 * i / cfg->D));
+  return cuda_status(mdr::launch_backward(a, cfg->dtype == MDR_BF16, st));
+}
+
 // ------------------------------------------------------ codebook calibration
 struct CalibLayout {
   size_t assign, part, pcount, total;

@@ -23,6 +23,7 @@ EXPORTED = (
     "mdr_forward_host", "mdr_read_device_status", "mdr_forward_profiled", "mdr_route_noalloc",
     "mdr_decode_workspace_bytes", "mdr_decode_reset", "mdr_decode_prefill", "mdr_decode_step",
     "mdr_route_forced", "mdr_target_hits", "mdr_calibrate_workspace_bytes", "mdr_calibrate_codebooks",
+    "mdr_backward_workspace_bytes", "mdr_attend_backward",
 )
 
 
@@ -82,6 +83,8 @@ def lib() -> ctypes.CDLL:
             "mdr_route_noalloc": ([cfgp, vp, vp, idxp, vp, vp, vp], i32),
             "mdr_route_forced": ([cfgp, vp, vp, idxp, vp, rtp, vp, sz, vp], i32),
             "mdr_target_hits": ([cfgp, vp, vp, vp, vp, vp], i32),
+            "mdr_backward_workspace_bytes": ([cfgp, ctypes.POINTER(sz)], i32),
+            "mdr_attend_backward": ([cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "mdr_calibrate_workspace_bytes": ([ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.POINTER(sz)], i32),
             "mdr_calibrate_codebooks": ([vp, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
@@ -271,6 +274,26 @@ def mdr_target_hits(cfg, sel, target, counts, hit=None, stream=None):
     target, counts[1] = hits (device int32 [2]); see include/mdr.h."""
     _ok(lib().mdr_target_hits(ctypes.byref(cfg), _ptr(sel), _ptr(target), _ptr(hit), _ptr(counts),
                               _stream(stream)), "mdr_target_hits")
+
+
+# ------------------------------------------------------------------ backward
+def mdr_backward_workspace_bytes(cfg: mdr_config) -> int:
+    n = ctypes.c_size_t(0)
+    _ok(lib().mdr_backward_workspace_bytes(ctypes.byref(cfg), ctypes.byref(n)), "mdr_backward_workspace_bytes")
+    return n.value
+
+
+def backward_workspace(cfg: mdr_config, device=None):
+    import torch
+    return torch.empty(mdr_backward_workspace_bytes(cfg), dtype=torch.uint8, device=device or torch.device("cuda"))
+
+
+def mdr_attend_backward(cfg, q, k, v, sel, dout, dq, dk, dv, ws, stream=None):
+    """dq, dk, dv (float32) of the attention output for upstream gradient
+    dout, with the route sel held fixed; see include/mdr.h."""
+    _ok(lib().mdr_attend_backward(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(dout),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(stream)),
+        "mdr_attend_backward")
 
 
 # ------------------------------------------------------ codebook calibration

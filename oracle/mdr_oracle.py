@@ -645,7 +645,7 @@ def spherical_objective(records: np.ndarray, codebooks: np.ndarray) -> float:
 # the selected-set softmax and the rotary embedding only: given dL/d(out),
 # it returns dL/dq, dL/dk, dL/dv, and nothing reaches the codebooks or the
 # block summaries.
-def attend_backward(qr, kr, v, sel, bs: int, scale: float, dout):
+def attend_backward(qr, kr, v, sel, bs: int, scale: float, dout, rows=None):
     """dL/dq', dL/dk', dL/dv of attend() for dL/d(out) = dout [B,S,Hq,D].
 
     Per query block j and head hq, with T = the tokens of the selected
@@ -657,7 +657,9 @@ def attend_backward(qr, kr, v, sel, bs: int, scale: float, dout):
       dk'[T] += scale * dS^T q'_j
     Key and value gradients of a KV head add over its query heads.  A query
     block with no valid selected block has a zero output and gets zero
-    gradients."""
+    gradients.  rows: optional list of (b, hq, j) to include (dq of the
+    others stays 0, and dk, dv hold only the listed rows' contributions --
+    exact for a key block whose selecting rows are all listed)."""
     B, S, Hq, D = qr.shape
     Hkv = kr.shape[2]
     g = Hq // Hkv
@@ -665,26 +667,25 @@ def attend_backward(qr, kr, v, sel, bs: int, scale: float, dout):
     dk = np.zeros(kr.shape, dtype=np.float64)
     dv = np.zeros(v.shape, dtype=np.float64)
     nb = S // bs
-    for b in range(B):
-        for hq in range(Hq):
-            h = hq // g
-            for j in range(nb):
-                toks = selected_tokens(sel[b, hq, j], bs)
-                if toks.size == 0:
-                    continue
-                qpos = np.arange(j * bs, (j + 1) * bs)
-                Q, Kt, Vt = qr[b, qpos, hq], kr[b, toks, h], v[b, toks, h]
-                s = (Q @ Kt.T) * scale
-                s[toks[None, :] > qpos[:, None]] = -np.inf
-                s -= s.max(axis=1, keepdims=True)
-                P = np.exp(s)
-                P /= P.sum(axis=1, keepdims=True)
-                dO = dout[b, qpos, hq]
-                dv[b, toks, h] += P.T @ dO
-                dP = dO @ Vt.T
-                dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
-                dq[b, qpos, hq] = scale * dS @ Kt
-                dk[b, toks, h] += scale * dS.T @ Q
+    todo = rows if rows is not None else itertools.product(range(B), range(Hq), range(nb))
+    for b, hq, j in todo:
+        h = hq // g
+        toks = selected_tokens(sel[b, hq, j], bs)
+        if toks.size == 0:
+            continue
+        qpos = np.arange(j * bs, (j + 1) * bs)
+        Q, Kt, Vt = qr[b, qpos, hq], kr[b, toks, h], v[b, toks, h]
+        s = (Q @ Kt.T) * scale
+        s[toks[None, :] > qpos[:, None]] = -np.inf
+        s -= s.max(axis=1, keepdims=True)
+        P = np.exp(s)
+        P /= P.sum(axis=1, keepdims=True)
+        dO = dout[b, qpos, hq]
+        dv[b, toks, h] += P.T @ dO
+        dP = dO @ Vt.T
+        dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+        dq[b, qpos, hq] = scale * dS @ Kt
+        dk[b, toks, h] += scale * dS.T @ Q
     return dq, dk, dv
 
 

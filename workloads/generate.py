@@ -32,6 +32,9 @@ the storage type with round-to-nearest-even):
 Codebooks: P sets of K unit vectors of dimension D/P (Gaussian, normalised),
 the seeded untrained-router control.
 
+Upstream gradients (make_grad): dL/d(out) ~ N(0, 1), rounded to the storage
+type like q, k, v.
+
 Calibration records (make_records): rows = one of n_centres unit centres
 times a log-normal length, plus sigma*N(0, I); optional zero rows and exact
 copies of a row (edge cases of the calibration).
@@ -212,3 +215,10 @@ def make_records(N: int, D: int, n_centres: int, sigma: float, seed: int, *,
     if repeat_rows:
         x[r.choice(np.arange(1, N), size=repeat_rows, replace=False)] = x[0]
     return x
+
+
+def make_grad(w: Workload, seed: int):
+    """Upstream gradient dL/d(out) [B,S,Hq,D] ~ N(0, 1): (as stored, widened
+    to float32; in its storage type)."""
+    g = _normal(rng_for(seed, w.name, "dout"), (w.B, w.S, w.Hq, w.D))
+    return _store(g, w.dtype)
