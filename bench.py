@@ -33,7 +33,7 @@ sys.path.insert(0, ROOT)
 
 import numpy as np  # noqa: E402
 
-from workloads import SCALING_SWEEP, ALL, make_codebooks, make_inputs, make_keys  # noqa: E402
+from workloads import SCALING_SWEEP, ALL, make_codebooks, make_grad, make_inputs, make_keys  # noqa: E402
 
 METRIC = "routed-attention fwd tokens/s (index+route+attend) at 32K; % HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
@@ -251,6 +251,23 @@ def config_of(w, args):
             "parallelism": f"one sequence per GPU x {args.gpus}"}
 
 
+FP32_LANES_PER_SM = 128            # B200: 128 FP32 lanes per SM, one FMA (2 flops) each per clock
+
+
+def backward_flops(sel: np.ndarray, bs: int, D: int) -> int:
+    """Flops of the four gradient products of the attention backward (dv =
+    P^T dO, dP = dO V^T, dq = dS K, dk = dS^T Q), 2*D each per visible
+    (query token, key token) pair: bs*bs pairs for a remote block, bs*(bs+1)/2
+    for the query block's own block; -1 entries and ids past the query block
+    add nothing."""
+    nb = sel.shape[2]
+    j = np.arange(nb)[None, None, :, None]
+    full = ((sel >= 0) & (sel < j)).sum()
+    own = (sel == j).sum()
+    pairs = int(full) * bs * bs + int(own) * bs * (bs + 1) // 2
+    return 8 * D * pairs
+
+
 def run_mine(args, w):
     import torch
     from learned_product_hash_b200 import mdr
@@ -442,6 +459,41 @@ def run_mine(args, w):
                        "held_out": held, "capacity": wl.cap}
         del ixl, wsl, cws, rec
 
+    # Backward of the attention with the forward's route held fixed: dq, dk,
+    # dv (float32) for a seeded upstream gradient, timed with CUDA events.
+    backward = None
+    if not args.no_backward:
+        do = torch.from_numpy(make_grad(w, 4000 + rank)[1].view(np.int16)).view(torch.bfloat16).to(dev) \
+            if w.dtype == "bf16" else torch.from_numpy(make_grad(w, 4000 + rank)[1]).to(dev)
+        dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+        dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+        dv = torch.empty(v.shape, dtype=torch.float32, device=dev)
+        bws = mdr.backward_workspace(cfg, dev)
+        for _ in range(2):
+            mdr.mdr_attend_backward(cfg, q, k, v, rt.sel, do, dq, dk, dv, bws)
+        torch.cuda.synchronize()
+        nb_it = 5
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(nb_it):
+            mdr.mdr_attend_backward(cfg, q, k, v, rt.sel, do, dq, dk, dv, bws)
+        b1.record(stream)
+        b1.synchronize()
+        assert mdr.mdr_read_device_status(bws) == 0
+        b_ms = b0.elapsed_time(b1) / nb_it
+        b_ms_max = max_over_ranks(b_ms, dist, world, dev)
+        fl = backward_flops(sel, w.block, w.D)
+        alu_peak = torch.cuda.get_device_properties(dev).multi_processor_count * FP32_LANES_PER_SM * 2 * \
+            (clk.summary() or {}).get("sm_max_mhz", 1965) * 1e6 / 1e12
+        backward = {"metric": "attention backward (dq, dk, dv for a fixed route) at 32K",
+                    "value": throughput(w.B * w.S, world, b_ms_max), "unit": "tokens/s", "ms_per_call": b_ms_max,
+                    "launches_per_call": 4, "arithmetic": "float32 on CUDA cores",
+                    "roofline": {"bound": "alu", "achieved": fl / (b_ms / 1e3) / 1e12, "peak": alu_peak,
+                                 "unit": "TFLOP/s", "frac": fl / (b_ms / 1e3) / 1e12 / alu_peak,
+                                 "peak_kind": "derived: SMs x 128 FP32 lanes x 2 flops x max SM clock",
+                                 "algorithmic_flops_per_call": fl}}
+        del bws, dq, dk, dv, do
+
     # End to end through the C ABI with host buffers.
     e2e = None
     if not args.no_e2e:
@@ -488,7 +540,7 @@ def run_mine(args, w):
                              "kernel": "attend", "algorithmic_bytes_per_launch": attn_bytes},
                 "path_roofline_frac": total_bytes / (ms_max / 1e3) / 1e9 / peak,
                 "kernels_ms": ker, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
-                "controls": controls, "calibration": calibration,
+                "controls": controls, "calibration": calibration, "backward": backward,
                 "gpu_launches": KERNELS_PER_FORWARD * args.steps, "clocks": clk.summary(),
                 "overflow": int(idx.overflow.sum().item()), "selected_blocks": nsel}
         print(json.dumps(line), flush=True)
@@ -508,6 +560,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-controls", action="store_true")
     ap.add_argument("--no-calibration", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()

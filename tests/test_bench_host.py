@@ -58,3 +58,14 @@ def test_clock_sampler_without_nvml_reports_why(monkeypatch):
         pass
     s = clk.summary()
     assert "error" in s and "sm_mhz" not in s
+
+
+def test_backward_flops_counts_visible_pairs():
+    """A 3-block sequence, block size 4, D = 2: query block 0 selects only
+    itself (10 pairs), block 1 nothing, block 2 selects block 0 (remote: 16
+    pairs), block 5 (past it: nothing) and itself (10 pairs).  Four products
+    of 2*D flops per pair."""
+    import numpy as np
+    import bench
+    sel = np.array([[[[-1, -1, 0], [-1, -1, -1], [0, 5, 2]]]])       # [B=1, Hq=1, nb=3, nsel=3]
+    assert bench.backward_flops(sel, 4, 2) == 8 * 2 * (10 + 16 + 10)
