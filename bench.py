@@ -254,6 +254,26 @@ def config_of(w, args):
 FP32_LANES_PER_SM = 128            # B200: 128 FP32 lanes per SM, one FMA (2 flops) each per clock
 
 
+def loglog_exponent(sizes, times) -> float:
+    """Least-squares slope of log(time) against log(size): 1 for linear
+    scaling (the Report's Finite-range scaling fit)."""
+    return float(np.polyfit(np.log(np.asarray(sizes, dtype=np.float64)),
+                            np.log(np.asarray(times, dtype=np.float64)), 1)[0])
+
+
+def oracle_route_seconds(w, seed: int, reps: int = 1) -> list:
+    """Seconds of each of reps calls of the CPU oracle's index build + route
+    (no attention) on the same inputs of workload w."""
+    from oracle import mdr_oracle as O
+    inp = make_inputs(w, seed)
+    out = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        O.forward(inp.q, inp.k, inp.v, inp.codebooks, O.Params.of(w), attention=False)
+        out.append(time.perf_counter() - t0)
+    return out
+
+
 def backward_flops(sel: np.ndarray, bs: int, D: int) -> int:
     """Flops of the four gradient products of the attention backward (dv =
     P^T dO, dP = dO V^T, dq = dS K, dk = dS^T Q), 2*D each per visible
@@ -494,6 +514,56 @@ def run_mine(args, w):
                                  "algorithmic_flops_per_call": fl}}
         del bws, dq, dk, dv, do
 
+    # Scaling of the forward from 4K to 128K tokens (one GPU): the median of
+    # 10 L2-flushed mdr_forward calls per length, inputs drawn on the device
+    # by torch's seeded generator (q, k, v ~ N(0, 1), the recipe of the
+    # scaling workloads), and the log-log slope over 4K-32K (the Report's
+    # range) and 4K-128K; beside it, the CPU oracle's index build + route at
+    # 4K-32K (one warm-up, median of 3, as the Report times it).
+    scaling_obj = None
+    if world == 1 and not args.no_sweep:
+        try:
+            pts = {}
+            for wsw in SCALING_SWEEP:
+                csw = mdr.make_config(wsw)
+                gen = torch.Generator(device=dev)
+                gen.manual_seed(5000 + wsw.S)
+                mk = lambda H: torch.randn(wsw.B, wsw.S, H, wsw.D, generator=gen, device=dev).to(torch.bfloat16)
+                qs_, ks_, vs_ = mk(wsw.Hq), mk(wsw.Hkv), mk(wsw.Hkv)
+                cbs = torch.from_numpy(make_codebooks(wsw, 5000)).to(dev)
+                ixs, rts, wss = mdr.Index.empty(csw, dev), mdr.RouteOut.empty(csw, dev), mdr.workspace(csw, dev)
+                outs = torch.empty_like(qs_)
+                times = []
+                for it in range(13):
+                    flush_l2()
+                    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    s0.record(stream)
+                    mdr.mdr_forward(csw, qs_, ks_, vs_, cbs, ixs, rts, outs, wss)
+                    s1.record(stream)
+                    s1.synchronize()
+                    if it >= 3:
+                        times.append(s0.elapsed_time(s1))
+                assert mdr.mdr_read_device_status(wss) == 0
+                pts[wsw.S] = statistics.median(times)
+                del qs_, ks_, vs_, ixs, rts, wss, outs
+            Ss = sorted(pts)
+            short = [S for S in Ss if S <= 32768]
+            scaling_obj = {"workload": "scaling: B=1, H=8, D=128 bf16, block 64, K=32, cap 64, p=4, R=8, L=2",
+                           "ms_per_forward": {str(S): pts[S] for S in Ss},
+                           "tokens_per_s": {str(S): S / (pts[S] / 1e3) for S in Ss},
+                           "exponent_4k_32k": loglog_exponent(short, [pts[S] for S in short]),
+                           "exponent_4k_128k": loglog_exponent(Ss, [pts[S] for S in Ss])}
+            if rank == 0 and not args.no_cpu:
+                cpu_pts = {}
+                for wsw in [x for x in SCALING_SWEEP if x.S <= 32768]:
+                    cpu_pts[wsw.S] = statistics.median(oracle_route_seconds(wsw, 6000, 4)[1:])   # 1 warm-up, median of 3
+                Sc = sorted(cpu_pts)
+                scaling_obj["cpu_oracle_index_route"] = {
+                    "seconds": {str(S): cpu_pts[S] for S in Sc}, "cores": blas_threads(),
+                    "exponent_4k_32k": loglog_exponent(Sc, [cpu_pts[S] for S in Sc])}
+        except Exception as e:                   # the line still carries every other number
+            scaling_obj = {"error": repr(e)}
+
     # End to end through the C ABI with host buffers.
     e2e = None
     if not args.no_e2e:
@@ -541,6 +611,7 @@ def run_mine(args, w):
                 "path_roofline_frac": total_bytes / (ms_max / 1e3) / 1e9 / peak,
                 "kernels_ms": ker, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
                 "controls": controls, "calibration": calibration, "backward": backward,
+                "scaling_sweep": scaling_obj,
                 "gpu_launches": KERNELS_PER_FORWARD * args.steps, "clocks": clk.summary(),
                 "overflow": int(idx.overflow.sum().item()), "selected_blocks": nsel}
         print(json.dumps(line), flush=True)
@@ -561,6 +632,7 @@ def main():
     ap.add_argument("--no-controls", action="store_true")
     ap.add_argument("--no-calibration", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()

@@ -69,3 +69,17 @@ def test_backward_flops_counts_visible_pairs():
     import bench
     sel = np.array([[[[-1, -1, 0], [-1, -1, -1], [0, 5, 2]]]])       # [B=1, Hq=1, nb=3, nsel=3]
     assert bench.backward_flops(sel, 4, 2) == 8 * 2 * (10 + 16 + 10)
+
+
+def test_loglog_exponent_of_power_laws():
+    import bench
+    S = [4096, 8192, 16384, 32768]
+    assert abs(bench.loglog_exponent(S, [3e-3 * x for x in S]) - 1.0) < 1e-12
+    assert abs(bench.loglog_exponent(S, [2.0 * x ** 1.5 for x in S]) - 1.5) < 1e-12
+
+
+def test_oracle_index_route_timing_runs_on_a_small_workload():
+    import bench
+    from workloads import scaling
+    t = bench.oracle_route_seconds(scaling(4096), 0, 2)
+    assert len(t) == 2 and min(t) > 0
