@@ -339,7 +339,9 @@ mdr_status mdr_read_device_status(const void* ws, int32_t* code, void* stream);
  * float32 in a fixed order (deterministic).  ws: device, 256-byte aligned,
  * at least mdr_backward_workspace_bytes; its first word is the device
  * status (2: a selected id later than its query block, skipped), read with
- * mdr_read_device_status.                                                   */
+ * mdr_read_device_status.  Supported up to 29,000 blocks per sequence
+ * (S/block; the reverse index of a (sequence, KV head) lives in shared
+ * memory), else MDR_ERR_UNSUPPORTED before anything is enqueued.            */
 mdr_status mdr_backward_workspace_bytes(const mdr_config* cfg, size_t* bytes);
 mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void* k,
                                const void* v, const int32_t* sel, const void* dout,

@@ -12,6 +12,7 @@ namespace {
 using mdr::SummarizeArgs;
 
 constexpr size_t kAlign = 256;
+constexpr size_t kMaxDynamicSmem = 227 * 1024;    // per CTA on sm_100a
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -572,6 +573,7 @@ mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void*
   if (!ws || reinterpret_cast<uintptr_t>(ws) % kAlign != 0 || ws_bytes < l.total) return MDR_ERR_WORKSPACE;
   if (static_cast<long long>(cfg->B) * cfg->Hq * (cfg->S / cfg->block) * (cfg->block / 16) > INT32_MAX)
     return MDR_ERR_UNSUPPORTED;
+  if (mdr::bwd_rev_smem(cfg->S / cfg->block) > kMaxDynamicSmem) return MDR_ERR_UNSUPPORTED;   // reverse index
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   MDR_CUDA(cudaMemsetAsync(at<int32_t>(ws, l.status), 0, sizeof(int32_t), st));
   mdr::BwdArgs a;

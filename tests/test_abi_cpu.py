@@ -172,3 +172,21 @@ def test_calibration_entry_points_check_arguments_before_any_gpu_work():
     assert call(cout=ctypes.c_void_p(0x10010)) == mdr.MDR_ERR_INVALID_ARG         # overlaps the input codebooks
     assert call(ws=None) == mdr.MDR_ERR_WORKSPACE
     assert call(ws=ctypes.c_void_p(0x100010)) == mdr.MDR_ERR_WORKSPACE            # not 256-byte aligned
+
+
+def test_backward_entry_point_checks_arguments_before_any_gpu_work():
+    L = mdr.lib()
+    cfg = mdr.make_config(TINY)
+    n = mdr.mdr_backward_workspace_bytes(cfg)
+    assert n > 0
+    fake = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x100000)
+    call = lambda cfg=cfg, dout=fake, ws=ws, nbytes=n: L.mdr_attend_backward(
+        ctypes.byref(cfg), fake, fake, fake, fake, dout, fake, fake, fake, ws, nbytes, None)
+    assert call(dout=None) == mdr.MDR_ERR_INVALID_ARG
+    assert call(ws=None) == mdr.MDR_ERR_WORKSPACE
+    assert call(ws=ctypes.c_void_p(0x100010)) == mdr.MDR_ERR_WORKSPACE       # not 256-byte aligned
+    assert call(nbytes=n - 1) == mdr.MDR_ERR_WORKSPACE
+    big = mdr.make_config(TINY.with_(S=30000 * 16))                           # 30,000 blocks
+    nbig = mdr.mdr_backward_workspace_bytes(big)
+    assert call(cfg=big, nbytes=nbig) == mdr.MDR_ERR_UNSUPPORTED
