@@ -6,7 +6,9 @@
 // hard top-k choices pass no ordinary gradient through the chosen index, so
 // nothing flows to the codebooks or the block summaries.
 //
-// Four kernels, float32 arithmetic, every sum in a fixed order (no atomics):
+// Four kernels, float32 arithmetic, every floating-point sum in a fixed
+// order (the only atomics count list entries in shared memory, whose integer
+// totals do not depend on order), so a call is deterministic:
 //   bwd_rotate_kernel  float32 rotated copies q', k' (the angle of the
 //                      forward: the float32 product t * omega_i, sincosf).
 //   bwd_rev_kernel     one CTA per (sequence, KV head): for every key block,
