@@ -11,7 +11,18 @@ torchrun) runs its own sequence: weak scaling, no collective on the data path.
 L2 is flushed before every step, outside the timed events: a 256 MiB write,
 then a read of the same buffer, so that no dirty lines of the flush are left
 to be written back inside the timed region.
-Rank 0 prints one JSON line.
+Rank 0 prints one JSON line.  Beside the forward's throughput, roofline,
+clocks, CPU baseline and end-to-end number it carries, each measured in the
+same run (each can be left out with its --no-* flag):
+  decode         one-token steps with the incremental index at 32K (latency);
+  controls       target-block hit rates of the planted-block workload: route,
+                 forced route, local-only;
+  calibration    codebook calibration rounds on the long workload's key
+                 summaries, and a held-out sequence's overflow and maximum
+                 load before and after;
+  backward       dq, dk, dv of the attention with the route held fixed at 32K;
+  scaling_sweep  the forward from 4K to 128K tokens with log-log slopes, and
+                 the CPU oracle's index + route slope at 4K-32K (N = 1 only).
 
 --impl reference times the CPU oracle (oracle/mdr_oracle.py) as it stands on
 the host cores, on a bounded sample of the same workload.
