@@ -484,6 +484,7 @@ def run_mine(args, w):
         calibration = {"workload": f"{wl.name}: key summaries of one training sequence ({N} records of {wl.D}), "
                                    f"P={wl.P}, K={wl.K}, {rounds} rounds from random unit codebooks",
                        "us_per_round": c_ms * 1e3, "launches_per_round": 3,
+                       "l2": "not flushed: the 4 MB of records stay in L2 across rounds, as in a calibration loop",
                        "roofline": {"bound": "hbm", "achieved": c_bytes / (c_ms / 1e3) / 1e9, "peak": peak_c,
                                     "unit": "GB/s", "frac": c_bytes / (c_ms / 1e3) / 1e9 / peak_c,
                                     "algorithmic_bytes_per_round": c_bytes},
@@ -519,6 +520,7 @@ def run_mine(args, w):
         backward = {"metric": "attention backward (dq, dk, dv for a fixed route) at 32K",
                     "value": throughput(w.B * w.S, world, b_ms_max), "unit": "tokens/s", "ms_per_call": b_ms_max,
                     "launches_per_call": 4, "arithmetic": "float32 on CUDA cores",
+                    "l2": "not flushed: q, k, v, dout and the float32 rotated copies (~0.5 GB) exceed L2",
                     "roofline": {"bound": "alu", "achieved": fl / (b_ms / 1e3) / 1e12, "peak": alu_peak,
                                  "unit": "TFLOP/s", "frac": fl / (b_ms / 1e3) / 1e12 / alu_peak,
                                  "peak_kind": "derived: SMs x 128 FP32 lanes x 2 flops x max SM clock",
