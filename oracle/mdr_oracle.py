@@ -27,7 +27,12 @@ The forward is index -> route -> attend:
      own values (Report, Mixer; Article).
 And the independent dense selected-mask form of step 6 (Report, Evidence,
 the selected-mask oracle row; Article, "Why Learned Product-Hash Routing
-Matters Now").
+Matters Now").  Beyond the forward (sections 7-9 and the route's options):
+  7. decode: one token at a time with an incremental index;
+  -  controls: a forced target block per route (route_row's force) and the
+     target-block hit count (target_hits);
+  8. codebook calibration: spherical k-means per subspace;
+  9. backward: gradients of the attention output with the route held fixed.
 
 Precision.  Every value is computed in float64 from the stored inputs.  Two
 readings fix what the pages leave open (both recorded with the others in the
