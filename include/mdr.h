@@ -19,7 +19,8 @@
  *   - Every pointer argument named "device" points to GPU memory of the
  *     current device; "host" pointers point to CPU memory (pinned memory
  *     makes the copies asynchronous).  The caller owns every buffer; the
- *     library allocates nothing and keeps no state between calls.
+ *     library allocates nothing and keeps no state between calls, except
+ *     mdr_route_noalloc, whose scratch is an array inside the library.
  *   - Layouts are C-contiguous.  q is [B,S,Hq,D]; k and v are [B,S,Hkv,D];
  *     out is [B,S,Hq,D]; all four have the element type cfg->dtype.
  *     Query head hq reads KV head hq / (Hq/Hkv).
@@ -213,9 +214,14 @@ mdr_status mdr_forward_host(const mdr_config* cfg, const void* q_host,
  * needs B*Hq*nb*(4*D + 4*P*probes) bytes (each part rounded up to 256) and
  * larger calls return MDR_ERR_WORKSPACE before anything is enqueued.  The
  * first call on each device looks up the array's device address with that
- * device current; make it before any stream capture.  Calls share the array,
- * so calls that overlap on the GPU race; nothing in it needs clearing
- * between calls.  Allocates nothing.                                        */
+ * device current; it returns MDR_ERR_INVALID_ARG if the stream is capturing
+ * then, so make it before any stream capture.  Calls share the array and a
+ * device status word, so calls that overlap on the GPU race; the word is
+ * cleared at the start of each call and the array needs no clearing.  If a
+ * bounded wait of the summary step runs out on the device, every sel row is
+ * written as -1 and ncand as -1: sel[b,hq,j,R+L-1] (the query block itself
+ * in a normal route) is then -1, which is how the caller detects it after
+ * synchronising.  Allocates nothing.                                        */
 mdr_status mdr_route_noalloc(const mdr_config* cfg, const void* q,
                              const float* codebooks, const mdr_index* idx,
                              int32_t* sel, int32_t* ncand, void* stream);

@@ -72,6 +72,12 @@ route_kernel(const RouteArgs a) {
   const long long bh = static_cast<long long>(b) * a.Hkv + hkv;
   const int32_t* lists = a.lists + bh * a.A * a.cap;
   const int last = j - a.L;                        // highest eligible block
+  if (a.upstream_status && *reinterpret_cast<const volatile int32_t*>(a.upstream_status) != 0) {
+    // The summaries this route would read may be incomplete: no route.
+    for (int s = lane; s < a.R + a.L; s += 32) a.sel[route * (a.R + a.L) + s] = -1;
+    if (a.ncand && lane == 0) a.ncand[route] = -1;
+    return;
+  }
 
   for (int d = lane; d < a.D; d += 32) qs[d] = a.qbar[route * a.D + d];
   int forced = kForced ? a.force[route] : -1;

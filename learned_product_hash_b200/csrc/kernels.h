@@ -82,6 +82,10 @@ struct RouteArgs {
   int32_t* sel;            // [B,Hq,nb,R+L]
   int32_t* ncand;          // [B,Hq,nb] or null
   const int32_t* force;    // [B,Hq,nb] forced target block per route (-1 none) or null
+  // Status word of the kernels that wrote qbar and qcodes, or null.  When it
+  // is nonzero (a bounded wait there ran out, so the summaries may be
+  // incomplete) every route writes a row of -1 and ncand -1 instead of routing.
+  const int32_t* upstream_status;
   int B, Hq, Hkv, nb, D, P, K, A, probes, cap, R, L;
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);

@@ -6,10 +6,12 @@
 
 #include "mdr.h"
 #include "kernels.h"
+#include "abi_common.h"
 
 namespace {
 
 using mdr::SummarizeArgs;
+using mdr::detail::ipow;
 
 constexpr size_t kAlign = 256;
 constexpr size_t kMaxDynamicSmem = 227 * 1024;    // per CTA on sm_100a
@@ -17,15 +19,6 @@ constexpr size_t kMaxDynamicSmem = 227 * 1024;    // per CTA on sm_100a
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 size_t esize(const mdr_config* c) { return c->dtype == MDR_BF16 ? 2 : 4; }
-
-int ipow(int b, int e) {
-  long long r = 1;
-  for (int i = 0; i < e; ++i) {
-    r *= b;
-    if (r > (1LL << 30)) return -1;
-  }
-  return static_cast<int>(r);
-}
 
 bool is_pow2_in(int x, std::initializer_list<int> allowed) {
   for (int a : allowed)
@@ -123,15 +116,7 @@ mdr_status check_index(const mdr_index* idx) {
 }
 
 void fill_common(SummarizeArgs& a, const mdr_config* c, const float* codebooks) {
-  std::memset(&a, 0, sizeof(a));
-  a.H[0] = c->Hq;
-  a.H[1] = c->Hkv;
-  a.codebooks = codebooks;
-  a.B = c->B; a.S = c->S; a.D = c->D; a.bs = c->block; a.nb = c->S / c->block;
-  a.P = c->P; a.K = c->K; a.probes = c->probes;
-  // omega_i = base^(-2i/D) in double, rounded to float.
-  for (int i = 0; i < c->D / 2; ++i)
-    a.inv_freq[i] = static_cast<float>(std::pow(static_cast<double>(c->rope_base), -2.0 * i / c->D));
+  mdr::detail::fill_summarize_common(a, c, codebooks);
 }
 
 mdr_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MDR_OK : MDR_ERR_CUDA; }
@@ -155,13 +140,7 @@ mdr_status run_lists(const mdr_config* c, const mdr_index* idx, cudaStream_t st)
 mdr_status run_route(const mdr_config* c, const float* qbar, const int32_t* qcodes,
                      const mdr_index* idx, int32_t* sel, int32_t* ncand, cudaStream_t st,
                      const int32_t* force = nullptr) {
-  mdr::RouteArgs ra{};
-  ra.qbar = qbar; ra.qcodes = qcodes; ra.kbar = idx->kbar; ra.lists = idx->lists; ra.load = idx->load;
-  ra.sel = sel; ra.ncand = ncand; ra.force = force;
-  ra.B = c->B; ra.Hq = c->Hq; ra.Hkv = c->Hkv; ra.nb = c->S / c->block; ra.D = c->D;
-  ra.P = c->P; ra.K = c->K; ra.A = ipow(c->K, c->P); ra.probes = c->probes; ra.cap = c->cap;
-  ra.R = c->R; ra.L = c->L;
-  return cuda_status(mdr::launch_route(ra, st));
+  return cuda_status(mdr::launch_route(mdr::detail::route_args(c, qbar, qcodes, idx, sel, ncand, force), st));
 }
 
 mdr_status run_attend(const mdr_config* c, const void* qrot, const void* krot, const void* v,
@@ -170,7 +149,7 @@ mdr_status run_attend(const mdr_config* c, const void* qrot, const void* krot, c
   aa.q = qrot; aa.k = krot; aa.v = v; aa.sel = sel; aa.out = out; aa.status = status;
   aa.B = c->B; aa.S = c->S; aa.Hq = c->Hq; aa.Hkv = c->Hkv; aa.D = c->D; aa.bs = c->block;
   aa.nb = c->S / c->block; aa.nsel = c->R + c->L;
-  aa.scale = c->scale > 0.f ? c->scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(c->D)));
+  aa.scale = mdr::detail::softmax_scale(c);
   if (c->dtype == MDR_BF16) return cuda_status(mdr::launch_attend_tc(aa, st));
   return cuda_status(mdr::launch_attend_simt(aa, false, st));
 }
@@ -530,9 +509,8 @@ mdr_status mdr_decode_step(const mdr_config* cfg, int32_t t, const void* q_t, co
   d.B = cfg->B; d.S = cfg->S; d.Hq = cfg->Hq; d.Hkv = cfg->Hkv; d.D = cfg->D; d.bs = cfg->block;
   d.nb = cfg->S / cfg->block; d.P = cfg->P; d.K = cfg->K; d.A = ipow(cfg->K, cfg->P); d.cap = cfg->cap;
   d.probes = cfg->probes; d.R = cfg->R; d.L = cfg->L;
-  d.scale = cfg->scale > 0.f ? cfg->scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(cfg->D)));
-  for (int i = 0; i < cfg->D / 2; ++i)
-    d.inv_freq[i] = static_cast<float>(std::pow(static_cast<double>(cfg->rope_base), -2.0 * i / cfg->D));
+  d.scale = mdr::detail::softmax_scale(cfg);
+  mdr::detail::fill_inv_freq(d.inv_freq, cfg);
   return cuda_status(mdr::launch_decode(d, cfg->dtype == MDR_BF16, s));
 }
 
@@ -585,9 +563,8 @@ mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void*
   a.dq = dq; a.dk = dk; a.dv = dv; a.status = at<int32_t>(ws, l.status);
   a.B = cfg->B; a.S = cfg->S; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.D = cfg->D; a.bs = cfg->block;
   a.nb = cfg->S / cfg->block; a.nsel = cfg->R + cfg->L;
-  a.scale = cfg->scale > 0.f ? cfg->scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(cfg->D)));
-  for (int i = 0; i < cfg->D / 2; ++i)
-    a.inv_freq[i] = static_cast<float>(std::pow(static_cast<double>(cfg->rope_base), -2.0 * i / cfg->D));
+  a.scale = mdr::detail::softmax_scale(cfg);
+  mdr::detail::fill_inv_freq(a.inv_freq, cfg);
   return cuda_status(mdr::launch_backward(a, cfg->dtype == MDR_BF16, st));
 }
 

@@ -64,6 +64,29 @@ def test_noalloc_route_at_the_benchmark_size():
     assert torch.equal(sel, rt.sel)
 
 
+def test_noalloc_route_allocates_no_device_memory():
+    """After its first call on the device, further calls leave the device's
+    free memory unchanged: the scratch is the library's own array."""
+    import torch
+    from learned_product_hash_b200 import mdr
+    w = scaling(4096)
+    cfg, q, cb, idx, rt = _reference_route(w, make_inputs(w, 4))
+    sel = torch.empty_like(rt.sel)
+    ncand = torch.empty_like(rt.ncand)
+    mdr.mdr_route_noalloc(cfg, q, cb, idx, sel, ncand)          # first call: address lookup
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        mdr.mdr_route_noalloc(cfg, q, cb, idx, sel, ncand)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert torch.equal(sel, rt.sel) and torch.equal(ncand, rt.ncand)
+    # a normal route never writes -1 in a row's last entry (the query block
+    # itself); a call whose summary step failed on the device does
+    assert (sel[..., -1] >= 0).all()
+
+
 def test_noalloc_route_rejects_sizes_beyond_its_scratch():
     from learned_product_hash_b200 import mdr
     big = mdr.make_config(scaling(131072).with_(B=4))        # 4*8*2048 routes * 544 B > 32 MiB
