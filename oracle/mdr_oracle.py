@@ -134,6 +134,12 @@ def assign_codes(kbar: np.ndarray, codebooks: np.ndarray):
     return addr.astype(np.int64), codes.astype(np.int64), margin
 
 
+def code_scale(xbar: np.ndarray, codebooks: np.ndarray) -> np.ndarray:
+    """Largest |codeword score| of each subspace: the |s| that sets the
+    near-tie threshold of a code or probe decision.  -> [..., P]"""
+    return np.abs(codeword_scores(xbar, codebooks)).max(axis=-1)
+
+
 def probe_codes(qbar: np.ndarray, codebooks: np.ndarray, p: int):
     """The p best codewords per subspace for each query block.
 
@@ -188,8 +194,9 @@ class RouteRow:
     sel: np.ndarray          # [R+L]: remote ids ascending, -1 pads, then locals
     slots: np.ndarray        # [p**P, cap] fixed candidate slots (-1 = empty)
     cand: np.ndarray         # eligible candidate ids
-    scores: np.ndarray       # their float32 scores
-    margin: float            # score gap between rank R and R+1 (inf if none)
+    scores: np.ndarray       # float32 scores of the ranked pool (the candidates, less a forced id)
+    margin: float            # score gap between the last kept rank and the next (inf if none)
+    scale: float             # largest |score| in the pool (0 if empty): the near-tie reference
 
 
 def candidate_slots(lists: np.ndarray, probe_addrs: np.ndarray, j: int, L: int) -> np.ndarray:
@@ -239,7 +246,8 @@ def route_row(qbar_j: np.ndarray, kbar_h: np.ndarray, probe_addrs: np.ndarray,
     remote[: top.size] = np.sort(top)
     local = np.arange(j - L + 1, j + 1, dtype=np.int64)
     local[local < 0] = -1
-    return RouteRow(np.concatenate([remote, local]), slots, cand, scores, margin)
+    scale = float(np.abs(scores).max()) if scores.size else 0.0
+    return RouteRow(np.concatenate([remote, local]), slots, cand, scores, margin, scale)
 
 
 # ------------------------------------------------------------------ 6. attend
@@ -362,12 +370,21 @@ class Result:
     ncand: np.ndarray
     out: np.ndarray | None = None
     slots: dict = field(default_factory=dict)
+    sel_scale: np.ndarray | None = None     # [B,Hq,nb] largest |candidate score| per route
+    v: np.ndarray | None = None             # the values, float64 (for re-running attention)
 
 
-def build_index(kr, codebooks, p: Params):
-    """Index of every (sequence, KV head): summaries, addresses, lists."""
+def build_index(kr, codebooks, p: Params, addr=None):
+    """Index of every (sequence, KV head): summaries, addresses, lists.
+
+    ``addr`` [B,Hkv,nb] (or None) replaces the computed addresses when the
+    lists are built: where a code decision is a near tie either codeword is
+    correct, so a check of what follows from another implementation's choice
+    builds the lists from that choice.  codes and margins stay the computed
+    ones."""
     kbar = block_means(kr, p.block)
-    addr, codes, margin = assign_codes(kbar, codebooks)
+    own_addr, codes, margin = assign_codes(kbar, codebooks)
+    addr = own_addr if addr is None else np.asarray(addr, dtype=np.int64)
     B, H, nb = addr.shape
     lists = np.empty((B, H, p.A, p.cap), dtype=np.int64)
     load = np.empty((B, H, p.A), dtype=np.int64)
@@ -379,46 +396,67 @@ def build_index(kr, codebooks, p: Params):
     return kbar, addr, codes, margin, lists, load, overflow, maxload
 
 
-def route(qr, kbar, lists, codebooks, p: Params, keep_slots=False, force=None):
+def route(qr, kbar, lists, codebooks, p: Params, keep_slots=False, force=None, qcodes=None):
     """Route every query block; ``force`` [B,Hq,nb] (or None) holds a forced
-    target block per route, -1 for none (see route_row)."""
+    target block per route, -1 for none (see route_row).  ``qcodes``
+    [B,Hq,nb,P,p] (or None) replaces the computed probe codewords (a near-tie
+    probe decision taken the other way); the returned qcodes and margins are
+    the computed ones.  Returns (qbar, qcodes, qmargin, sel, sel_margin,
+    ncand, slots, sel_scale)."""
     qbar = block_means(qr, p.block)
-    qcodes, qmargin = probe_codes(qbar, codebooks, p.probes)
+    own_qcodes, qmargin = probe_codes(qbar, codebooks, p.probes)
+    use = own_qcodes if qcodes is None else np.asarray(qcodes, dtype=np.int64)
     B, Hq, nb = qbar.shape[:3]
     g = Hq // kbar.shape[1]
     sel = np.empty((B, Hq, nb, p.R + p.L), dtype=np.int64)
     sel_margin = np.empty((B, Hq, nb))
+    sel_scale = np.empty((B, Hq, nb))
     ncand = np.empty((B, Hq, nb), dtype=np.int64)
     slots = {}
     for b in range(B):
         for hq in range(Hq):
             for j in range(nb):
-                pa = probe_addresses(qcodes[b, hq, j], p.K)
+                pa = probe_addresses(use[b, hq, j], p.K)
                 row = route_row(qbar[b, hq, j], kbar[b, hq // g], pa,
                                 lists[b, hq // g], j, p.R, p.L,
                                 -1 if force is None else int(force[b, hq, j]))
                 sel[b, hq, j] = row.sel
                 sel_margin[b, hq, j] = row.margin
+                sel_scale[b, hq, j] = row.scale
                 ncand[b, hq, j] = row.cand.size
                 if keep_slots:
                     slots[(b, hq, j)] = row.slots
-    return qbar, qcodes, qmargin, sel, sel_margin, ncand, slots
+    return qbar, own_qcodes, qmargin, sel, sel_margin, ncand, slots, sel_scale
 
 
 def forward(q, k, v, codebooks, p: Params, *, attention=True, rows=None, keep_slots=False,
-            force=None) -> Result:
+            force=None, addr=None, qcodes=None, sel=None) -> Result:
     """Index -> route -> attend for stored inputs q [B,S,Hq,D], k, v [B,S,Hkv,D];
-    ``force`` as in route."""
+    ``force`` as in route.
+
+    Decision overrides (each None or an array of the decision's shape): where
+    a decision is a near tie, either choice is correct, and the steps after it
+    are checked against the oracle re-run with the other choice --
+      addr   [B,Hkv,nb]      the lists are built from these addresses;
+      qcodes [B,Hq,nb,P,p]   the routes probe these codewords;
+      sel    [B,Hq,nb,R+L]   the attention runs over these selected blocks.
+    The Result's addr, qcodes and sel are the ones used downstream (the
+    overrides where given); the margins are those of the computed decisions,
+    except sel_margin, which belongs to the routes run."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     qr = rope(q, p.rope_base)
     kr = rope(k, p.rope_base)
-    kbar, addr, codes, cmargin, lists, load, overflow, maxload = build_index(kr, codebooks, p)
-    qbar, qcodes, qmargin, sel, smargin, ncand, slots = route(qr, kbar, lists, codebooks, p, keep_slots, force)
-    out = attend(qr, kr, v, sel, p.block, p.softmax_scale, rows) if attention else None
-    return Result(qr, kr, qbar, kbar, addr, codes, cmargin, qcodes, qmargin, lists, load,
-                  overflow, maxload, sel, smargin, ncand, out, slots)
+    kbar, own_addr, codes, cmargin, lists, load, overflow, maxload = build_index(kr, codebooks, p, addr)
+    qbar, own_qcodes, qmargin, rsel, smargin, ncand, slots, sscale = route(
+        qr, kbar, lists, codebooks, p, keep_slots, force, qcodes)
+    use_addr = own_addr if addr is None else np.asarray(addr, dtype=np.int64)
+    use_qcodes = own_qcodes if qcodes is None else np.asarray(qcodes, dtype=np.int64)
+    use_sel = rsel if sel is None else np.asarray(sel, dtype=np.int64)
+    out = attend(qr, kr, v, use_sel, p.block, p.softmax_scale, rows) if attention else None
+    return Result(qr, kr, qbar, kbar, use_addr, codes, cmargin, use_qcodes, qmargin, lists, load,
+                  overflow, maxload, use_sel, smargin, ncand, out, slots, sscale, v)
 
 
 def target_hits(sel: np.ndarray, target: np.ndarray):
@@ -501,13 +539,16 @@ def decode_init(p: Params, B: int) -> DecodeState:
                        np.zeros((B, p.Hkv, p.A), dtype=np.int64))
 
 
-def append_block(st: DecodeState, codebooks: np.ndarray, p: Params, j: int):
+def append_block(st: DecodeState, codebooks: np.ndarray, p: Params, j: int, addr=None):
     """Block j has all its tokens: summarise it, give it an address and append
     it to its list if that list holds fewer than cap blocks (load counts it in
-    any case)."""
+    any case).  ``addr`` [B, Hkv] (or None) replaces the computed address (a
+    near-tie code decision taken the other way).  Returns the computed
+    (addr, codes, margin) of the block."""
     toks = st.kr[:, j * p.block:(j + 1) * p.block]                 # [B, bs, Hkv, D]
     st.kbar[:, :, j] = toks.mean(axis=1)
-    addr, _, _ = assign_codes(st.kbar[:, :, j], codebooks)          # [B, Hkv]
+    own = assign_codes(st.kbar[:, :, j], codebooks)                  # [B, Hkv], ...
+    addr = own[0] if addr is None else np.asarray(addr, dtype=np.int64)
     st.addr[:, :, j] = addr
     B, H = addr.shape
     for b in range(B):
@@ -516,6 +557,7 @@ def append_block(st: DecodeState, codebooks: np.ndarray, p: Params, j: int):
             if st.load[b, h, a] < p.cap:
                 st.lists[b, h, a, st.load[b, h, a]] = j
             st.load[b, h, a] += 1
+    return own
 
 
 @dataclass
@@ -528,26 +570,41 @@ class DecodeOut:
     ncand: np.ndarray        # [B, Hq]
     qcode_scale: np.ndarray  # [B, Hq, P] largest |codeword score| (reference for near ties)
     sel_scale: np.ndarray    # [B, Hq] largest |candidate score| (reference for near ties)
+    # the block completed by this token (None if none): its computed address,
+    # codes, code margins [B, Hkv, P] and largest |codeword score| [B, Hkv, P]
+    key_addr: np.ndarray | None = None
+    key_codes: np.ndarray | None = None
+    key_margin: np.ndarray | None = None
+    key_scale: np.ndarray | None = None
 
 
-def decode_step(st: DecodeState, q_t, k_t, v_t, codebooks, p: Params) -> DecodeOut:
+def decode_step(st: DecodeState, q_t, k_t, v_t, codebooks, p: Params, *, addr=None, sel=None) -> DecodeOut:
     """Token t = st.t of every sequence: store its rotated key and value,
     complete a block if t is its last token, then route the token by its
     rotated query and attend over the selected tokens s <= t.
-    q_t [B, Hq, D], k_t and v_t [B, Hkv, D] (stored inputs)."""
+    q_t [B, Hq, D], k_t and v_t [B, Hkv, D] (stored inputs).
+
+    Decision overrides (near-tie decisions taken the other way, so that what
+    follows is checked against that choice): ``addr`` [B, Hkv] is the address
+    of the block this token completes; ``sel`` [B, Hq, R+L] is the selection
+    the attention runs over.  The returned sel, margins and key decision are
+    the computed ones; out is the attention over the selection used."""
     t = st.t
     q_t, k_t, v_t = (np.asarray(x, dtype=np.float64) for x in (q_t, k_t, v_t))
     st.kr[:, t] = rope_at(k_t, t, p.rope_base)
     st.v[:, t] = v_t
+    key = (None, None, None, None)
     if (t + 1) % p.block == 0:
-        append_block(st, codebooks, p, t // p.block)
+        j_done = t // p.block
+        ka, kc, km = append_block(st, codebooks, p, j_done, addr)
+        key = (ka, kc, km, code_scale(st.kbar[:, :, j_done], codebooks))
     qr = rope_at(q_t, t, p.rope_base)                                # [B, Hq, D]
     qcodes, qmargin = probe_codes(qr, codebooks, p.probes)
-    qscale = np.abs(codeword_scores(qr, codebooks)).max(axis=-1)
+    qscale = code_scale(qr, codebooks)
     B, Hq, D = qr.shape
     g = Hq // p.Hkv
     j = t // p.block
-    sel = np.empty((B, Hq, p.R + p.L), dtype=np.int64)
+    sel_own = np.empty((B, Hq, p.R + p.L), dtype=np.int64)
     smargin = np.empty((B, Hq))
     ncand = np.empty((B, Hq), dtype=np.int64)
     sscale = np.zeros((B, Hq))
@@ -557,15 +614,16 @@ def decode_step(st: DecodeState, q_t, k_t, v_t, codebooks, p: Params) -> DecodeO
             h = hq // g
             row = route_row(qr[b, hq], st.kbar[b, h], probe_addresses(qcodes[b, hq], p.K),
                             st.lists[b, h], j, p.R, p.L)
-            sel[b, hq], smargin[b, hq], ncand[b, hq] = row.sel, row.margin, row.cand.size
-            sscale[b, hq] = np.abs(row.scores).max() if row.scores.size else 0.0
-            toks = selected_tokens(row.sel, p.block)
+            sel_own[b, hq], smargin[b, hq], ncand[b, hq] = row.sel, row.margin, row.cand.size
+            sscale[b, hq] = row.scale
+            use = row.sel if sel is None else np.asarray(sel[b, hq], dtype=np.int64)
+            toks = selected_tokens(use, p.block)
             toks = toks[toks <= t]
             s = (st.kr[b, toks, h] @ qr[b, hq]) * p.softmax_scale
             w = np.exp(s - s.max())
             out[b, hq] = (w @ st.v[b, toks, h]) / w.sum()
     st.t = t + 1
-    return DecodeOut(out, sel, smargin, qcodes, qmargin, ncand, qscale, sscale)
+    return DecodeOut(out, sel_own, smargin, qcodes, qmargin, ncand, qscale, sscale, *key)
 
 
 # ------------------------------------------------------ 8. codebook calibration

@@ -15,6 +15,7 @@ from __future__ import annotations
 import itertools
 import json
 import os
+from fractions import Fraction
 
 import numpy as np
 import torch
@@ -315,6 +316,193 @@ def check_attention_gather_equals_dense_mask():
     assert np.abs(res.out - dense).max() < 1e-12
     # and the selection is genuinely sparse here
     assert (res.sel[..., : p.R] >= 0).sum() < p.nb * p.R * 4
+
+
+# --------------------------------------------------------------- near ties
+# A routing decision (a code, a probe set, a top-R set) is a near tie when the
+# float32 gap at its boundary is below 1e-6*max(1,|s|), |s| the largest score
+# magnitude among the items ranked; there either choice is correct.  These
+# checks pin the margins, the scales and the threshold that decide which
+# disagreements are excused: against a brute-force sorted() of scores
+# computed exactly (rational arithmetic, then rounded to float32), planted
+# exact ties, and gaps just on either side of the threshold.
+
+def _f32_exact_dot(a, b) -> float:
+    """<a, b> of two float32 vectors, summed exactly with rational
+    arithmetic and rounded to float32: the score a float32 kernel aims at,
+    whatever its summation order."""
+    tot = sum(Fraction(float(x)) * Fraction(float(y))
+              for x, y in zip(np.asarray(a, np.float32), np.asarray(b, np.float32)))
+    return float(np.float32(float(tot)))
+
+
+def _ranked(scores):
+    """(score, index) pairs, best first (lower index first on equal scores)."""
+    return [(-ns, i) for ns, i in sorted((-v, i) for i, v in enumerate(scores))]
+
+
+def _close(x, y, ref):
+    """Equal up to two float32 units in the last place at magnitude ref."""
+    return abs(x - y) <= 2 * float(np.spacing(np.float32(max(abs(ref), 1e-30))))
+
+
+def check_code_margin_bruteforce():
+    """Key codes: the margin is the gap between the best and second-best
+    score of the subspace, the scale its largest |score|; a key on a codeword
+    that appears twice in the codebook is an exact tie (margin 0, a near tie)
+    and goes to the lower index; K = 1 has no second choice (margin inf)."""
+    P, K, d = 2, 6, 5
+    cb = _unit_codebooks(P, K, d, 40)
+    cb[1, 4] = cb[1, 2]                               # codewords 2 and 4 of subspace 1 are equal
+    kbar = _rand((1, 2, 12, P * d), 41)
+    kbar[0, 0, 0, d:] = 3.0 * cb[1, 2]                # exactly on the repeated codeword
+    kbar[0, 1, 5, d:] = -0.25 * cb[1, 0] + 0.9 * cb[1, 4]
+    addr, codes, margin = O.assign_codes(kbar, cb)
+    scale = O.code_scale(kbar, cb)
+    ties = 0
+    for h, n, s in itertools.product(range(2), range(12), range(P)):
+        sc = [_f32_exact_dot(kbar[0, h, n, s * d:(s + 1) * d], cb[s, k]) for k in range(K)]
+        r = _ranked(sc)
+        top = max(abs(v) for v in sc)
+        assert codes[0, h, n, s] == r[0][1], (h, n, s)
+        assert _close(margin[0, h, n, s], r[0][0] - r[1][0], top), (h, n, s, margin[0, h, n, s], r[:2])
+        assert _close(scale[0, h, n, s], top, top), (h, n, s)
+        if r[0][0] == r[1][0]:
+            ties += 1
+            assert margin[0, h, n, s] == 0 and O.near_tie(margin[0, h, n, s], scale[0, h, n, s])
+    assert ties >= 2, "the planted exact ties must be seen"
+    assert codes[0, 0, 0, 1] == 2, "an exact tie goes to the lower index"
+    _, _, m1 = O.assign_codes(kbar, cb[:, :1])
+    assert np.isinf(m1).all() and not O.near_tie(m1, 1.0).any()
+
+
+def check_probe_margin_bruteforce():
+    """Probes: the margin is the gap between ranks p and p+1 (the last probed
+    codeword and the first left out); p = K probes everything (margin inf);
+    with one probe and the best codeword repeated, the margin is exactly 0."""
+    P, K, d = 2, 8, 6
+    cb = _unit_codebooks(P, K, d, 42)
+    qbar = _rand((1, 1, 25, P * d), 43)
+    for p in (1, 3, 7):
+        codes, margin = O.probe_codes(qbar, cb, p)
+        for n, s in itertools.product(range(25), range(P)):
+            sc = [_f32_exact_dot(qbar[0, 0, n, s * d:(s + 1) * d], cb[s, k]) for k in range(K)]
+            r = _ranked(sc)
+            assert list(codes[0, 0, n, s]) == [i for _, i in r[:p]]
+            assert _close(margin[0, 0, n, s], r[p - 1][0] - r[p][0], max(abs(v) for v in sc)), (p, n, s)
+    _, mK = O.probe_codes(qbar, cb, K)
+    assert np.isinf(mK).all()
+    cb2 = cb.copy()
+    cb2[0, 6] = cb2[0, 1]
+    q2 = np.concatenate([2.0 * cb2[0, 1], cb2[1, 0]]).astype(np.float64)[None, None, None, :]
+    c2, m2 = O.probe_codes(q2, cb2, 1)
+    assert c2[0, 0, 0, 0, 0] == 1 and m2[0, 0, 0, 0] == 0
+
+
+def _score_rows(scores, D=8):
+    """Query e_0 and one key summary per score: <q, k_i> = scores[i] exactly."""
+    q = np.zeros(D)
+    q[0] = 1.0
+    k = np.zeros((len(scores), D))
+    k[:, 0] = scores
+    k[:, 1] = np.linspace(-3.0, 3.0, len(scores))     # orthogonal to q: no effect on the score
+    return q, k
+
+
+def check_route_margin_bruteforce():
+    """Top-R: with every eligible block a candidate (capacity >= nb, p = K),
+    the margin is the gap between ranks R and R+1 of the eligible scores, the
+    scale their largest |score|, inf with at most R candidates or R = 0; a
+    forced id leaves R-1 places, so the gap moves to ranks R-1 and R."""
+    for (R, L, seed) in [(2, 1, 44), (3, 2, 45), (1, 1, 46)]:
+        p = _p(S=192, block=16, K=4, P=2, cap=12, probes=4, R=R, L=L, D=16)
+        q = _rand((1, p.S, 1, p.D), seed)
+        k = _rand((1, p.S, 1, p.D), seed + 100)
+        res = O.forward(q, k, k, _unit_codebooks(2, 4, 8, seed + 200), p, attention=False)
+        for j in range(p.nb):
+            elig = list(range(0, j - L + 1))
+            sc = [_f32_exact_dot(res.qbar[0, 0, j], res.kbar[0, 0, i]) for i in elig]
+            r = _ranked(sc)
+            top = max((abs(v) for v in sc), default=0.0)
+            m = res.sel_margin[0, 0, j]
+            if len(elig) > R:
+                assert _close(m, r[R - 1][0] - r[R][0], top), (R, j, m)
+            else:
+                assert np.isinf(m), (R, j, m)
+            assert _close(res.sel_scale[0, 0, j], top, top), (R, j)
+    # planted exact tie at the boundary: scores 0.5, 0.9, 0.7, 0.9, 0.1 with R = 1
+    q, k = _score_rows([0.5, 0.9, 0.7, 0.9, 0.1])
+    lists = np.array([[0, 1, 2, 3, 4, -1]])
+    row = O.route_row(q, k, np.array([0]), lists, 6, 1, 1)
+    assert row.sel[0] == 1 and row.margin == 0 and O.near_tie(row.margin, row.scale)
+    assert row.scale == np.float32(0.9)
+    row2 = O.route_row(q, k, np.array([0]), lists, 6, 2, 1)       # R = 2 takes both 0.9s
+    assert list(row2.sel[:2]) == [1, 3] and _close(row2.margin, 0.9 - 0.7, 0.9)
+    row0 = O.route_row(q, k, np.array([0]), lists, 6, 0, 1)
+    assert np.isinf(row0.margin)
+    rowf = O.route_row(q, k, np.array([0]), lists, 6, 2, 1, force=4)   # 4 forced, one place left
+    assert list(rowf.sel[:2]) == [1, 4] and rowf.margin == 0
+
+
+def check_near_tie_threshold():
+    """The threshold is 1e-6*max(1,|s|): at |s| = 2 a gap of 16 float32 steps
+    (1.91e-6) is a tie and 17 steps (2.03e-6) is not; at |s| = 0.5 the
+    threshold is 1e-6, so 33 steps of 2^-25 (9.8e-7) are a tie and 34
+    (1.01e-6) are not.  Codes and routes use the same rule."""
+    d, P = 4, 2
+    cb = np.zeros((P, 2 * d, d), dtype=np.float32)
+    for s in range(P):
+        for i in range(d):
+            cb[s, 2 * i, i], cb[s, 2 * i + 1, i] = 1.0, -1.0
+    for a, step, n_tie in [(2.0, 2.0 ** -23, 16), (0.5, 2.0 ** -25, 33)]:
+        for n, expect in [(n_tie, True), (n_tie + 1, False)]:
+            b = np.float32(a) - np.float32(n * step)
+            kbar = np.zeros((1, 1, 1, P * d))
+            kbar[0, 0, 0, :2] = [a, b]
+            kbar[0, 0, 0, d] = 1.0
+            _, codes, margin = O.assign_codes(kbar, cb)
+            sc = O.code_scale(kbar, cb)
+            assert codes[0, 0, 0, 0] == 0
+            assert margin[0, 0, 0, 0] == np.float32(a) - b
+            assert bool(O.near_tie(margin, sc)[0, 0, 0, 0]) == expect, (a, n)
+            q, k = _score_rows([float(b), a, 0.25])
+            row = O.route_row(q, k, np.array([0]), np.array([[0, 1, 2, -1]]), 3, 1, 1)
+            assert row.sel[0] == 1 and bool(O.near_tie(row.margin, row.scale)) == expect, (a, n)
+
+
+def check_decode_margins_bruteforce():
+    """Decode: a token's probe margins and scales, and its top-R margin and
+    scale over the completed blocks, equal a brute-force sort of its own
+    rotated query's scores."""
+    p = _p(S=128, block=16, K=4, P=2, cap=8, probes=2, R=2, L=1, D=16)
+    B = 2
+    q, k, v = _rand((B, p.S, 1, p.D), 47), _rand((B, p.S, 1, p.D), 48), _rand((B, p.S, 1, p.D), 49)
+    cb = _unit_codebooks(2, 4, 8, 50)
+    st = O.decode_init(p, B)
+    dsub = p.D // p.P
+    for t in range(p.S):
+        o = O.decode_step(st, q[:, t], k[:, t], v[:, t], cb, p)
+        if t % 7:
+            continue
+        qr = O.rope_at(q[:, t], t, p.rope_base)
+        j = t // p.block
+        for b in range(B):
+            for s in range(p.P):
+                sc = [_f32_exact_dot(qr[b, 0, s * dsub:(s + 1) * dsub], cb[s, kk]) for kk in range(p.K)]
+                r = _ranked(sc)
+                top = max(abs(x) for x in sc)
+                assert _close(o.qcode_margin[b, 0, s], r[p.probes - 1][0] - r[p.probes][0], top), (t, b, s)
+                assert _close(o.qcode_scale[b, 0, s], top, top)
+            pa = O.probe_addresses(o.qcodes[b, 0], p.K)
+            cand = sorted(i for i in st.lists[b, 0, pa].ravel() if 0 <= i <= j - p.L)
+            sc = [_f32_exact_dot(qr[b, 0], st.kbar[b, 0, i]) for i in cand]
+            r = _ranked(sc)
+            top = max((abs(x) for x in sc), default=0.0)
+            assert _close(o.sel_scale[b, 0], top, top), (t, b)
+            if len(cand) > p.R:
+                assert _close(o.sel_margin[b, 0], r[p.R - 1][0] - r[p.R][0], top), (t, b)
+            else:
+                assert np.isinf(o.sel_margin[b, 0])
 
 
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

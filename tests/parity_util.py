@@ -5,8 +5,10 @@ The bar (stated once here, used by every parity test):
   * codes, posting lists, loads, overflow, max load, probed codewords,
     candidate counts and selected block ids: bit-exact.  A routing decision
     whose float32 margin in the oracle is below 1e-6*max(1,|s|) is a near tie:
-    there either choice is correct, the GPU's choice must be one of the tied
-    ones, and outputs downstream of it are checked for validity instead.
+    there either choice is correct and the GPU's choice must be one of the
+    tied ones; what follows from it (lists, routes, attention) is compared
+    bit-exactly (or within tolerance) against the oracle re-run with the
+    GPU's choice forced.
   * summaries (float32): |gpu - oracle| <= 1e-5 + 1e-5*|oracle|.
   * attention output: float32 storage, max |gpu - oracle| <= 1e-5; bfloat16
     storage, for every output row (token, head) ||gpu - oracle||_2 <=
@@ -91,7 +93,8 @@ def check_out(w, got, ref, mask_rows=None):
 
 
 def valid_lists(lists, load, addr, cap, nb):
-    """Invariants of one head's lists (used where a near tie changed codes)."""
+    """Invariants of one head's lists (stored <= cap, ascending, each block
+    at most once and under its own address)."""
     A = lists.shape[0]
     stored = lists[lists >= 0]
     assert stored.size == np.unique(stored).size
@@ -103,59 +106,150 @@ def valid_lists(lists, load, addr, cap, nb):
         assert all(addr[i] == a for i in row[:n])
 
 
-def compare(w, g, res, codebooks):
-    """Compare GPU outputs g with the oracle result res.  Returns a report."""
-    rep = {"code_ties": 0, "qcode_ties": 0, "sel_ties": 0}
+def _threshold(scale):
+    return O.TIE_REL * np.maximum(1.0, np.abs(scale))
+
+
+def compare(w, g, res, codebooks, force=None, max_ties=None):
+    """Compare GPU outputs g with the oracle result res (and, where the GPU
+    took a near-tie decision the other way, with the oracle re-run with the
+    GPU's choice forced).  Returns a report with the tie counts.
+
+    Order of the checks, each decision before what follows from it:
+      1. summaries within tolerance;
+      2. key codes: equal outside near ties; inside one, the GPU's codeword
+         must score within the threshold of the best (a valid choice);
+      3. lists, loads, overflow, max load: bit-exact against the oracle's
+         lists built from the GPU's addresses (the oracle's own where they
+         agree);
+      4. probe codewords (a set per subspace): equal outside near ties; inside
+         one, the GPU's set must be a valid top-p within the threshold;
+      5. routes: bit-exact against the oracle's route re-run on the GPU's
+         probes and lists, outside near ties of that route; inside one, the
+         GPU's remote set must be a valid top-R of the route's candidates;
+         candidate counts bit-exact everywhere; causality and layout;
+      6. attention of every computed row against the oracle run on the GPU's
+         selection (rows whose selection differs inside a tie are re-run, not
+         dropped).
+    force: the forced target ids of a forced route (or None).  max_ties: the
+    largest number of decisions that may differ inside near ties."""
+    rep = {"code_ties": 0, "qcode_ties": 0, "sel_ties": 0, "rerun_rows": 0}
     assert g["status"] == 0, f"device status {g['status']}"
     np.testing.assert_allclose(g["kbar"], res.kbar, rtol=1e-5, atol=1e-5)
     np.testing.assert_allclose(g["qbar"], res.qbar, rtol=1e-5, atol=1e-5)
+    P, K, A = w.P, w.K, w.K ** w.P
+    B, Hkv, nb = res.addr.shape
+    gq = w.Hq // w.Hkv
 
-    # key codes
-    best = np.max(np.abs(O.codeword_scores(res.kbar, codebooks)), axis=-1)
-    tie_k = O.near_tie(res.code_margin, best).any(axis=-1)            # [B,Hkv,nb]
-    diff_k = g["addr"] != res.addr
-    assert not (diff_k & ~tie_k).any(), f"{int((diff_k & ~tie_k).sum())} key addresses differ outside near ties"
-    rep["code_ties"] = int((diff_k & tie_k).sum())
-    head_same = ~diff_k.any(axis=-1)                                    # [B,Hkv]
-    B, Hkv = head_same.shape
-    for b in range(B):
-        for h in range(Hkv):
-            if head_same[b, h]:
-                assert np.array_equal(g["lists"][b, h], res.lists[b, h]), (b, h)
-                assert np.array_equal(g["load"][b, h], res.load[b, h]), (b, h)
-                assert g["overflow"][b, h] == res.overflow[b, h] and g["maxload"][b, h] == res.maxload[b, h]
-            else:
-                valid_lists(g["lists"][b, h], g["load"][b, h], g["addr"][b, h], w.cap, w.nb)
+    # 2. key codes, per subspace
+    sc_k = O.codeword_scores(res.kbar, codebooks)                       # [B,Hkv,nb,P,K]
+    scale_k = np.abs(sc_k).max(axis=-1)
+    tie_k = O.near_tie(res.code_margin, scale_k)                        # [B,Hkv,nb,P]
+    g_codes = (g["addr"][..., None] // (K ** np.arange(P - 1, -1, -1))) % K
+    assert (g["addr"] >= 0).all() and (g["addr"] < A).all()
+    diff_ks = g_codes != res.codes
+    assert not (diff_ks & ~tie_k).any(), f"{int((diff_ks & ~tie_k).sum())} key codes differ outside near ties"
+    g_sc = np.take_along_axis(sc_k, g_codes[..., None], axis=-1)[..., 0]
+    assert (sc_k.max(axis=-1) - g_sc < _threshold(scale_k))[diff_ks].all(), "a tied key code is not a tied best"
+    diff_k = diff_ks.any(axis=-1)                                       # [B,Hkv,nb]
+    rep["code_ties"] = int(diff_k.sum())
 
-    # query probes (a set per subspace)
-    qbest = np.max(np.abs(O.codeword_scores(res.qbar, codebooks)), axis=-1)
-    tie_q = O.near_tie(res.qcode_margin, qbest)                         # [B,Hq,nb,P]
+    # 3. lists from the GPU's addresses
+    lists_x, load_x = res.lists.copy(), res.load.copy()
+    ovf_x, mx_x = res.overflow.copy(), res.maxload.copy()
+    head_diff = diff_k.any(axis=-1)                                     # [B,Hkv]
+    for b, h in zip(*np.nonzero(head_diff)):
+        lists_x[b, h], load_x[b, h], ovf_x[b, h], mx_x[b, h] = O.build_lists(g["addr"][b, h], A, w.cap)
+        valid_lists(g["lists"][b, h], g["load"][b, h], g["addr"][b, h], w.cap, w.nb)
+    assert np.array_equal(g["lists"], lists_x), "posting lists differ"
+    assert np.array_equal(g["load"], load_x), "loads differ"
+    assert np.array_equal(g["overflow"], ovf_x) and np.array_equal(g["maxload"], mx_x), "overflow / max load differ"
+
+    # 4. probe codewords (a set per subspace)
+    sc_q = O.codeword_scores(res.qbar, codebooks)                       # [B,Hq,nb,P,K]
+    scale_q = np.abs(sc_q).max(axis=-1)
+    tie_q = O.near_tie(res.qcode_margin, scale_q)                       # [B,Hq,nb,P]
     diff_q = (np.sort(g["qcodes"], axis=-1) != np.sort(res.qcodes, axis=-1)).any(axis=-1)
     assert not (diff_q & ~tie_q).any(), "probed codewords differ outside near ties"
-    rep["qcode_ties"] = int((diff_q & tie_q).sum())
+    if diff_q.any():
+        inset = np.zeros(sc_q.shape, dtype=bool)
+        np.put_along_axis(inset, g["qcodes"], True, axis=-1)
+        assert (inset.sum(axis=-1) == w.probes).all(), "repeated probe codeword"
+        lo_in = np.where(inset, sc_q, np.inf).min(axis=-1)
+        hi_out = np.where(inset, -np.inf, sc_q).max(axis=-1)
+        assert (hi_out - lo_in < _threshold(scale_q))[diff_q].all(), "a tied probe set is not a valid top-p"
+    rep["qcode_ties"] = int(diff_q.any(axis=-1).sum())
 
-    # routes whose inputs are identical on both sides
-    g_ = w.Hq // w.Hkv
-    up_same = head_same[:, np.arange(w.Hq) // g_][:, :, None] & ~diff_q.any(axis=-1)
-    sel_same = (g["sel"] == res.sel).all(axis=-1)
-    tie_s = O.near_tie(res.sel_margin, 1.0)
-    bad = up_same & ~sel_same & ~tie_s
+    # 5. routes: re-run where the GPU's lists or probes differ from the oracle's
+    sel_x, marg_x, scale_x = res.sel.copy(), res.sel_margin.copy(), res.sel_scale.copy()
+    ncand_x = res.ncand.copy()
+    redo = head_diff[:, np.arange(w.Hq) // gq][:, :, None] | diff_q.any(axis=-1)       # [B,Hq,nb]
+    def rerun(b, hq, j):
+        return O.route_row(res.qbar[b, hq, j], res.kbar[b, hq // gq],
+                           O.probe_addresses(g["qcodes"][b, hq, j], K), lists_x[b, hq // gq],
+                           j, w.R, w.L, -1 if force is None else int(force[b, hq, j]))
+    for b, hq, j in zip(*np.nonzero(redo)):
+        row = rerun(b, hq, j)
+        sel_x[b, hq, j], marg_x[b, hq, j], scale_x[b, hq, j] = row.sel, row.margin, row.scale
+        ncand_x[b, hq, j] = row.cand.size
+    assert np.array_equal(g["ncand"], ncand_x), "candidate counts differ"
+    diff_s = (g["sel"] != sel_x).any(axis=-1)
+    tie_s = O.near_tie(marg_x, scale_x)
+    bad = diff_s & ~tie_s
     assert not bad.any(), f"{int(bad.sum())} routes differ outside near ties, first at {np.argwhere(bad)[0]}"
-    rep["sel_ties"] = int((up_same & ~sel_same).sum())
-    assert np.array_equal(g["ncand"][up_same], res.ncand[up_same])
-    # every route, tied or not, obeys causality and the row layout
     R, L = w.R, w.L
+    for b, hq, j in zip(*np.nonzero(diff_s)):
+        row = rerun(b, hq, j)
+        f = -1 if force is None else int(force[b, hq, j])
+        forced = 0 <= f <= j - L and R > 0
+        mine = [int(x) for x in g["sel"][b, hq, j, :R] if x >= 0]
+        pool = dict(zip(row.cand[row.cand != f].tolist() if forced else row.cand.tolist(), row.scores.tolist()))
+        rest = [i for i in mine if i != f] if forced else mine
+        assert len(mine) == len(set(mine)) and set(rest) <= set(pool), (b, hq, j, mine)
+        assert len(rest) == min(R - int(forced), len(pool)) and (not forced or f in mine), (b, hq, j)
+        out_sc = [sc for i, sc in pool.items() if i not in rest]
+        if rest and out_sc:
+            assert max(out_sc) - min(pool[i] for i in rest) < _threshold(row.scale), "a tied route is not a valid top-R"
+    rep["sel_ties"] = int(diff_s.sum())
+    # every route obeys causality and the row layout
     remote = g["sel"][..., :R]
     jj = np.arange(w.nb)[None, None, :, None]
     assert ((remote == -1) | ((remote >= 0) & (remote <= jj - L))).all()
     loc = np.arange(w.nb)[:, None] - L + 1 + np.arange(L)[None, :]
     assert np.array_equal(g["sel"][..., R:], np.broadcast_to(np.where(loc >= 0, loc, -1), g["sel"][..., R:].shape))
 
-    # attention where the selection agrees
-    rowmask = np.repeat(sel_same.transpose(0, 2, 1), w.block, axis=1)   # [B,S,Hq]
-    rep["out_err"] = check_out(w, g["out"], res.out, rowmask)
+    # 6. attention on the GPU's selection: rows whose selection differs from
+    # the oracle's are re-run with the GPU's selection and written into
+    # res.out in place (added to the sampled rows of a full-size run)
+    ref = res.out
+    changed = (g["sel"] != res.sel).any(axis=-1)
+    rows = [tuple(int(x) for x in r) for r in np.argwhere(changed)]
+    if rows:
+        assert res.v is not None, "the oracle result must carry v to re-run attention"
+        p = O.Params.of(w)
+        for b, hq, j in rows:
+            one = O.attend(res.qr[b:b + 1], res.kr[b:b + 1], res.v[b:b + 1], g["sel"][b:b + 1].astype(np.int64),
+                           w.block, p.softmax_scale, [(0, hq, j)])
+            ref[b, j * w.block:(j + 1) * w.block, hq] = one[0, j * w.block:(j + 1) * w.block, hq]
+    rep["rerun_rows"] = len(rows)
+    rep["out_err"] = check_out(w, g["out"], ref)
+    rep["rows_checked"] = int((~np.isnan(ref[..., 0])).sum() // w.block)
     rep["overflow"] = int(g["overflow"].sum())
+    ties = rep["code_ties"] + rep["qcode_ties"] + rep["sel_ties"]
+    if max_ties is not None:
+        assert ties <= max_ties, f"{ties} decisions differ inside near ties (budget {max_ties}): {rep}"
     return rep
+
+
+def full_size_tie_budget(w):
+    """Decisions that may differ inside near ties at full size: 4 plus one in
+    2,000 of the decisions taken (a code per key block and subspace, a probe
+    set per route and subspace, a top-R per route).  A float32 gap below
+    1e-6*max(1,|s|) between two scores spread over ~0.1-1 is rare (about one
+    decision in 10^5 here), so a budget this size is only exceeded when the
+    kernels and the oracle disagree more often than rounding explains."""
+    decisions = w.B * w.Hkv * w.nb * w.P + w.B * w.Hq * w.nb * (w.P + 1)
+    return 4 + decisions // 2000
 
 
 def sampled_rows(w, res, n=12, seed=0):

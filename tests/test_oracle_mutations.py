@@ -1,6 +1,8 @@
 """Plant a plausible mistake in the CPU oracle and require that at least one
 pin check catches it.  Shows that the pins constrain every step of the oracle
-(rotation, summaries, codes, lists, eligibility, rerank, attention)."""
+(rotation, summaries, codes, lists, eligibility, rerank, attention) and the
+near-tie machinery that decides which GPU disagreements are excused
+(margins, scales, threshold)."""
 import itertools
 
 import numpy as np
@@ -79,7 +81,8 @@ def _route_row_lowest_scores(qbar_j, kbar_h, probe_addrs, lists, j, R, L, force=
     remote[: top.size] = np.sort(top)
     local = np.arange(j - L + 1, j + 1)
     local[local < 0] = -1
-    return O.RouteRow(np.concatenate([remote, local]), slots, cand, scores, np.inf)
+    return O.RouteRow(np.concatenate([remote, local]), slots, cand, scores, np.inf,
+                      float(np.abs(scores).max()) if scores.size else 0.0)
 
 
 def _make_attend(scale_mult=1.0, causal=True, kv_map=lambda hq, g, Hkv: hq // g):
@@ -102,7 +105,66 @@ def _make_attend(scale_mult=1.0, causal=True, kv_map=lambda hq, g, Hkv: hq // g)
     return attend
 
 
+# ---- mistakes in the near-tie machinery (margins, scales, threshold): each
+# would excuse real disagreements between the GPU and the oracle
+_REAL_ASSIGN = O.assign_codes
+_REAL_PROBE = O.probe_codes
+_REAL_ROUTE_ROW = O.route_row
+_REAL_NEAR_TIE = O.near_tie
+_REAL_CODE_SCALE = O.code_scale
+
+
+def _code_margin_zero(kbar, codebooks):
+    addr, codes, margin = _REAL_ASSIGN(kbar, codebooks)
+    return addr, codes, np.zeros_like(margin)
+
+
+def _code_margin_wrong_ranks(kbar, codebooks):
+    addr, codes, _ = _REAL_ASSIGN(kbar, codebooks)
+    srt = -np.sort(-O.codeword_scores(kbar, codebooks), axis=-1)
+    return addr, codes, (srt[..., 1] - srt[..., 2]) if srt.shape[-1] > 2 else np.full(srt.shape[:-1], np.inf)
+
+
+def _probe_margin_wrong_ranks(qbar, codebooks, p):
+    codes, _ = _REAL_PROBE(qbar, codebooks, p)
+    srt = -np.sort(-O.codeword_scores(qbar, codebooks), axis=-1)
+    return codes, srt[..., 0] - srt[..., 1]
+
+
+def _route_margin_wrong_ranks(qbar_j, kbar_h, probe_addrs, lists, j, R, L, force=-1):
+    row = _REAL_ROUTE_ROW(qbar_j, kbar_h, probe_addrs, lists, j, R, L, force)
+    srt = np.sort(row.scores)[::-1]
+    row.margin = float(srt[R] - srt[R + 1]) if srt.size > R + 1 else np.inf   # one rank too deep
+    return row
+
+
+def _route_margin_zero(qbar_j, kbar_h, probe_addrs, lists, j, R, L, force=-1):
+    row = _REAL_ROUTE_ROW(qbar_j, kbar_h, probe_addrs, lists, j, R, L, force)
+    row.margin = 0.0
+    return row
+
+
+def _route_scale_zero(qbar_j, kbar_h, probe_addrs, lists, j, R, L, force=-1):
+    row = _REAL_ROUTE_ROW(qbar_j, kbar_h, probe_addrs, lists, j, R, L, force)
+    row.scale = 0.0
+    return row
+
+
+def _code_scale_signed(xbar, codebooks):
+    return O.codeword_scores(xbar, codebooks).max(axis=-1)       # largest score, not |score|
+
+
 MUTATIONS = {
+    "code_margin_always_zero": ("assign_codes", _code_margin_zero),
+    "code_margin_wrong_ranks": ("assign_codes", _code_margin_wrong_ranks),
+    "probe_margin_wrong_ranks": ("probe_codes", _probe_margin_wrong_ranks),
+    "route_margin_wrong_ranks": ("route_row", _route_margin_wrong_ranks),
+    "route_margin_always_zero": ("route_row", _route_margin_zero),
+    "route_scale_zero": ("route_row", _route_scale_zero),
+    "code_scale_signed": ("code_scale", _code_scale_signed),
+    "near_tie_threshold_loose": ("near_tie", lambda m, s: np.asarray(m) < 1e-3 * np.maximum(1.0, np.abs(s))),
+    "near_tie_threshold_absolute": ("near_tie", lambda m, s: np.asarray(m) < 1e-6 + 0 * np.asarray(s)),
+
     "rope_rotates_backwards": ("rope", _rope_wrong_sign),
     "rope_interleaved_pairs": ("rope", _rope_interleaved),
     "summary_is_sum": ("block_means", _means_as_sums),

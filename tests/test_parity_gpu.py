@@ -29,8 +29,8 @@ def test_forward_matches_oracle(w, seed):
     inp = make_inputs(w, seed)
     g = U.run_gpu(w, inp)
     res = U.oracle_for(w, inp)
-    rep = U.compare(w, g, res, inp.codebooks)
-    assert rep["code_ties"] + rep["qcode_ties"] + rep["sel_ties"] <= 2, rep
+    rep = U.compare(w, g, res, inp.codebooks, max_ties=2)
+    print(f"ties {w.name} seed {seed}: {rep}")
 
 
 @pytest.mark.parametrize("w", [TINY, AR.with_(B=8), CAPACITY], ids=lambda w: w.name)
@@ -72,7 +72,8 @@ def test_edge_cases(name):
     inp = make_inputs(w, 5, **kw)
     g = U.run_gpu(w, inp)
     res = U.oracle_for(w, inp)
-    rep = U.compare(w, g, res, inp.codebooks)
+    rep = U.compare(w, g, res, inp.codebooks, max_ties=2)
+    print(f"ties {name}: {rep}")
     if kw.get("zero"):
         assert (g["addr"] == 0).all()
         assert (g["overflow"] == max(0, w.nb - w.cap)).all()
@@ -133,7 +134,8 @@ def test_full_size_sampled(w):
     p = O.Params.of(w)
     res = O.forward(inp.q, inp.k, inp.v, inp.codebooks, p, attention=False)
     rows = U.sampled_rows(w, res)
-    res.out = O.attend(res.qr, res.kr, inp.v.astype(np.float64), res.sel, w.block, p.softmax_scale, rows)
-    rep = U.compare(w, g, res, inp.codebooks)
+    res.out = O.attend(res.qr, res.kr, res.v, res.sel, w.block, p.softmax_scale, rows)
+    rep = U.compare(w, g, res, inp.codebooks, max_ties=U.full_size_tie_budget(w))
+    print(f"ties {w.name}: {rep}")
     if w is LONG:
         assert rep["overflow"] > 0, "the long workload must overflow its lists"
