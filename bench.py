@@ -232,25 +232,42 @@ def blas_threads():
 
 
 def run_reference(args, w):
+    """The CPU oracle as it stands, on the host's cores (BLAS pool = all
+    cores), on this arm's workload: each step is one whole forward of one
+    sequence (all KV-head groups), unless (warm-up + steps) whole forwards
+    would take over REF_BUDGET_S, in which case each step times as many whole
+    KV-head groups as fit and is scaled to the full forward (the line's
+    sample says which)."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
     inp = make_inputs(w, 1000)
+    ncpu = os.cpu_count() or 1
+    t_group = oracle_group_seconds(w, inp, 0)                  # sizing run, not timed
+    groups_total = w.Hkv * w.B
+    per_step = groups_total
+    n_steps = args.warmup + args.steps
+    if n_steps * t_group * groups_total > REF_BUDGET_S:
+        per_step = max(1, int(REF_BUDGET_S / (n_steps * t_group)))
+        per_step = min(per_step, groups_total)
     secs = []
-    for it in range(args.warmup + args.steps):
-        t = oracle_group_seconds(w, inp, it % w.Hkv)
+    for it in range(n_steps):
+        t = sum(oracle_group_seconds(w, inp, (it * per_step + i) % w.Hkv) for i in range(per_step))
         if it >= args.warmup:
             secs.append(t)
-    t_full = statistics.mean(secs) * w.Hkv * w.B
+    t_full = statistics.mean(secs) * groups_total / per_step
     tps = w.B * w.S / t_full
     g = w.Hq // w.Hkv
+    sample = (f"each step: one whole forward of one sequence ({w.Hkv} KV-head groups of {g} query heads, "
+              f"all {w.nb} query blocks)" if per_step == groups_total else
+              f"each step: {per_step} of {groups_total} KV-head groups ({g} query heads, all {w.nb} query "
+              f"blocks each), scaled to the full forward")
     line = {"impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_full * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w, args),
-            "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"each step: one KV-head group ({g} query heads, all {w.nb} query "
-                                       f"blocks) of one sequence; ms_per_step scaled by {w.Hkv * w.B} groups"},
+            "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": ncpu, "kind": "oracle",
+                             "blas_threads": blas_threads(), "sample": sample},
             "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -262,6 +279,7 @@ def config_of(w, args):
             "parallelism": f"one sequence per GPU x {args.gpus}"}
 
 
+REF_BUDGET_S = 240.0               # the reference arm's whole run stays within about four minutes
 FP32_LANES_PER_SM = 128            # B200: 128 FP32 lanes per SM, one FMA (2 flops) each per clock
 
 
@@ -297,6 +315,192 @@ def backward_flops(sel: np.ndarray, bs: int, D: int) -> int:
     own = (sel == j).sum()
     pairs = int(full) * bs * bs + int(own) * bs * (bs + 1) // 2
     return 8 * D * pairs
+
+
+def forward_bytes(w, nsel: int, es: int) -> dict:
+    """Algorithmic bytes of one forward (the survey's byte model): the
+    summary pass reads q and k once; the attention reads q, gathers K and V of
+    every valid selected block and writes the output.  The summary pass's
+    rotated copies (written once, read by the attention) are not algorithmic
+    bytes: they are reported beside, as what this design adds."""
+    routes = w.B * w.Hq * w.nb
+    summ = (w.Hq + w.Hkv) * w.S * w.D * es * w.B
+    attn = routes * 2 * w.block * w.D * es + nsel * w.block * 2 * w.D * es
+    return {"summaries": summ, "attention": attn, "path": summ + attn, "rotated_copies_written": summ}
+
+
+def gqa_union(sel_t, w):
+    """Valid selected ids of a KV-head group's query heads, summed per
+    (sequence, KV head, query block) as the union of the group's rows and as
+    the sum of the rows: how many K/V block gathers one gather per group
+    (instead of one per query head) would save."""
+    import torch
+    g = w.Hq // w.Hkv
+    n = w.R + w.L
+    x = sel_t.view(w.B, w.Hkv, g, w.nb, n).permute(0, 1, 3, 2, 4).reshape(w.B, w.Hkv, w.nb, g * n)
+    xs, _ = torch.sort(x.long(), dim=-1)
+    first = xs[..., :1] >= 0
+    new = (xs[..., 1:] != xs[..., :-1]) & (xs[..., 1:] >= 0)
+    union = int(first.sum().item() + new.sum().item())
+    total = int((x >= 0).sum().item())
+    return {"group_size": g, "per_head_blocks": total, "union_blocks": union,
+            "union_fraction": union / total if total else None}
+
+
+def measure_forward(mdr, w, q, k, v, cb, dev, stream, flush_l2, reps=10, warm=3):
+    """Median of reps L2-flushed mdr_forward calls (CUDA events on the
+    launching stream), per-kernel times from as many calls with an event at
+    every kernel boundary, the §8(d) byte model from the returned selection,
+    overflow and (for grouped heads) the union of each group's selections."""
+    import torch
+    cfg = mdr.make_config(w)
+    idx, rt, ws = mdr.Index.empty(cfg, dev), mdr.RouteOut.empty(cfg, dev), mdr.workspace(cfg, dev)
+    out = torch.empty_like(q)
+    times = []
+    for it in range(warm + reps):
+        flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        mdr.mdr_forward(cfg, q, k, v, cb, idx, rt, out, ws)
+        e1.record(stream)
+        e1.synchronize()
+        if it >= warm:
+            times.append(e0.elapsed_time(e1))
+    assert mdr.mdr_read_device_status(ws) == 0
+    kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(reps)]
+    for e in kevs:
+        flush_l2()
+        mdr.mdr_forward_profiled(cfg, q, k, v, cb, idx, rt, out, ws, e)
+    torch.cuda.synchronize()
+    ker = {n: statistics.median(e[i].elapsed_time(e[i + 1]) for e in kevs)
+           for i, n in enumerate(("summarize", "lists", "route", "attend"))}
+    es = 2 if w.dtype == "bf16" else 4
+    nsel = int((rt.sel >= 0).sum().item())
+    by = forward_bytes(w, nsel, es)
+    ms = statistics.median(times)
+    peak, peak_kind = peaks()
+    res = {"ms_per_forward": ms, "tokens_per_s": w.B * w.S / (ms / 1e3), "selected_blocks": nsel,
+           "selected_blocks_per_route": nsel / (w.B * w.Hq * w.nb),
+           "bytes": by, "path_roofline_frac": by["path"] / (ms / 1e3) / 1e9 / peak,
+           "kernels_ms": ker,
+           "attention_roofline_frac": by["attention"] / (ker["attend"] / 1e3) / 1e9 / peak,
+           "summaries_roofline_frac": by["summaries"] / (ker["summarize"] / 1e3) / 1e9 / peak,
+           "peak_gbs": peak, "peak_kind": peak_kind,
+           "overflow": int(idx.overflow.sum().item()), "max_load": int(idx.maxload.max().item())}
+    if w.Hq != w.Hkv:
+        res["gqa"] = gqa_union(rt.sel, w)
+    del idx, rt, ws, out
+    return res
+
+
+def batched_decode(mdr, w, B, dev, stream, dist, world, peak):
+    """Decode steps with B sequences per GPU of the workload's shape: a
+    prefill of all but the last block (k, v ~ N(0, 1) drawn on the device),
+    then one token of every sequence per step through the last block (no
+    block completes), timed with CUDA events over consecutive steps after
+    three warm-up steps.  Bytes per step: K and V of every selected token
+    (tokens s <= t of the selected blocks, per sequence and query head), the
+    new query, key and value, and the output."""
+    import ctypes
+    import torch
+    if B <= 1:
+        return None
+    wb = w.with_(B=B)
+    cfg = mdr.make_config(wb)
+    S0 = w.S - w.block
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(8000)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    es = 2 if w.dtype == "bf16" else 4
+    cb = torch.from_numpy(make_codebooks(w, 8000)).to(dev)
+    dst = mdr.DecodeState.empty(cfg, dev)
+    dws = mdr.decode_workspace(cfg, dev)
+    k0 = torch.randn(B, S0, w.Hkv, w.D, generator=gen, device=dev).to(dt)
+    v0 = torch.randn(B, S0, w.Hkv, w.D, generator=gen, device=dev).to(dt)
+    mdr.mdr_decode_prefill(cfg, S0, k0, v0, cb, dst, dws)
+    torch.cuda.synchronize()
+    del k0, v0
+    n_dec = min(60, w.block - 1)
+    qs = torch.randn(n_dec, B, w.Hq, w.D, generator=gen, device=dev).to(dt)
+    ks = torch.randn(n_dec, B, w.Hkv, w.D, generator=gen, device=dev).to(dt)
+    vs = torch.randn(n_dec, B, w.Hkv, w.D, generator=gen, device=dev).to(dt)
+    out_t = torch.empty(B, w.Hq, w.D, dtype=dt, device=dev)
+    sel_t = torch.empty(B, w.Hq, w.R + w.L, dtype=torch.int32, device=dev)
+    warm = 3
+    fn = mdr.lib().mdr_decode_step
+    cfg_r, st_r = ctypes.byref(cfg), ctypes.byref(dst.c())
+    sp = stream.cuda_stream
+    calls = [(cfg_r, S0 + i, qs[i].data_ptr(), ks[i].data_ptr(), vs[i].data_ptr(), cb.data_ptr(), st_r,
+              out_t.data_ptr(), sel_t.data_ptr(), None, dws.data_ptr(), dws.numel(), sp) for i in range(n_dec)]
+    for c_args in calls[:warm]:
+        if fn(*c_args) != mdr.MDR_OK:
+            raise RuntimeError("mdr_decode_step failed")
+    torch.cuda.synchronize()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for c_args in calls[warm:]:
+        if fn(*c_args) != mdr.MDR_OK:
+            raise RuntimeError("mdr_decode_step failed")
+    d1.record(stream)
+    d1.synchronize()
+    assert mdr.mdr_read_device_status(dws) == 0
+    n_t = n_dec - warm
+    d_ms = d0.elapsed_time(d1) / n_t
+    t_last = S0 + n_dec - 1
+    sl = sel_t.cpu().numpy()
+    ntok = int(sum(min(w.block, t_last + 1 - int(blk) * w.block) for blk in sl.ravel() if blk >= 0))
+    d_bytes = ntok * 2 * w.D * es + 2 * B * w.Hq * w.D * es + 2 * B * w.Hkv * w.D * es
+    d_ms_max = max_over_ranks(d_ms, dist, world, dev)
+    del dst, dws
+    return {"batch_per_gpu": B, "value": d_ms_max * 1e3, "unit": "us/step",
+            "tokens_per_s": B * world / (d_ms_max / 1e3), "steps": n_t,
+            "position": f"tokens {S0 + warm}..{t_last} ({S0 // w.block} blocks indexed)",
+            "gpu_launches": 3 * n_t, "inputs": "k, v, q ~ N(0, 1) drawn on the device (torch, seeded)",
+            "roofline": {"bound": "hbm", "achieved": d_bytes / (d_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": d_bytes / (d_ms / 1e3) / 1e9 / peak, "algorithmic_bytes_per_step": d_bytes}}
+
+
+def cpu_baseline(w, max_seconds):
+    """The CPU oracle as it stands on this host at 1 thread, 4 threads (the
+    Report's setup) and all cores: its BLAS pool limited by threadpoolctl
+    (the route and attention loops themselves are Python, one thread).  Each
+    setting times whole KV-head groups of one sequence for about
+    max_seconds/3 and scales to the full forward.  value = all cores."""
+    from threadpoolctl import threadpool_limits
+    ncpu = os.cpu_count() or 1
+    by = {}
+    for n in sorted({1, 4, ncpu}):
+        with threadpool_limits(limits=n):
+            tps, secs, groups = oracle_sample(w, 1000, max_seconds=max_seconds / 3)
+        by[str(n)] = {"tokens_per_s": tps, "seconds": secs, "groups_timed": groups}
+    top = by[str(ncpu)]
+    return {"value": top["tokens_per_s"], "unit": "tokens/s", "cores": ncpu, "kind": "oracle", "nproc": ncpu,
+            "by_threads": by,
+            "sample": f"per thread setting, whole KV-head groups (of {w.Hkv}) of one sequence, all {w.nb} query "
+                      f"blocks, about {max_seconds / 3:.0f} s each, scaled to the full forward; threads = the "
+                      f"BLAS pool (threadpoolctl); the oracle's loops run on one Python thread"}
+
+
+def device_inputs(w, seed, dev):
+    """q, v ~ N(0, 1) drawn on the device by torch's seeded generator (the
+    workloads' recipe for q and v, without the host round trip); k by the
+    workload's own key recipe (gaussian or clusters) on the host; codebooks
+    seeded random unit vectors.  Stored as the workload's dtype."""
+    import torch
+    from workloads import make_keys
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q = torch.randn(w.B, w.S, w.Hq, w.D, generator=gen, device=dev).to(dt)
+    v = torch.randn(w.B, w.S, w.Hkv, w.D, generator=gen, device=dev).to(dt)
+    if w.keys == "gaussian":
+        k = torch.randn(w.B, w.S, w.Hkv, w.D, generator=gen, device=dev).to(dt)
+    else:
+        kb = make_keys(w, seed)[1]
+        k = (torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16) if w.dtype == "bf16"
+             else torch.from_numpy(kb)).to(dev)
+    cb = torch.from_numpy(make_codebooks(w, seed)).to(dev)
+    return q, k, v, cb
 
 
 def run_mine(args, w):
@@ -366,11 +570,20 @@ def run_mine(args, w):
     # selected blocks + out write, per (b, hq, j) route.
     sel = rt.sel.cpu().numpy()
     nsel = int((sel >= 0).sum())
-    routes = w.B * w.Hq * w.nb
-    attn_bytes = routes * 2 * w.block * w.D * es + nsel * w.block * 2 * w.D * es
+    by = forward_bytes(w, nsel, es)
+    attn_bytes = by["attention"]
     peak, peak_kind = peaks()
     achieved = attn_bytes / (ker["attend"] / 1e3) / 1e9
-    total_bytes = (w.Hq + w.Hkv) * w.S * w.D * es * w.B + attn_bytes
+    total_bytes = by["path"]
+    kernels = {
+        "summarize": {"ms": ker["summarize"], "algorithmic_bytes": by["summaries"],
+                      "frac": by["summaries"] / (ker["summarize"] / 1e3) / 1e9 / peak,
+                      "also_written_bytes": by["rotated_copies_written"],
+                      "note": "reads q, k once (the byte model); also writes the rotated copies the "
+                              "attention reads, which the byte model does not count"},
+        "lists": {"ms": ker["lists"], "note": "one CTA per (sequence, KV head); < 1 % of the bytes"},
+        "route": {"ms": ker["route"], "note": "reads list slots and key summaries (L2); < 1 % of the bytes"},
+        "attend": {"ms": ker["attend"], "algorithmic_bytes": attn_bytes, "frac": achieved / peak}}
 
     # Decoding: the state of the first nb-1 blocks (prefill), then one token
     # per sequence at a time through the last block, timed with CUDA events
@@ -418,6 +631,7 @@ def run_mine(args, w):
                   "roofline": {"bound": "hbm", "achieved": d_bytes / (d_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
                                "frac": d_bytes / (d_ms / 1e3) / 1e9 / peak, "algorithmic_bytes_per_step": d_bytes}}
         del dst, dws
+        decode["batched"] = batched_decode(mdr, w, args.decode_batch, dev, stream, dist, world, peak)
 
     # Controls on the planted-block workload (untimed): how often the route
     # selects each sequence's planted block for its last query block, with
@@ -536,7 +750,7 @@ def run_mine(args, w):
     scaling_obj = None
     if world == 1 and not args.no_sweep:
         try:
-            pts = {}
+            pts, sweep_bytes = {}, {}
             for wsw in SCALING_SWEEP:
                 csw = mdr.make_config(wsw)
                 gen = torch.Generator(device=dev)
@@ -558,12 +772,20 @@ def run_mine(args, w):
                         times.append(s0.elapsed_time(s1))
                 assert mdr.mdr_read_device_status(wss) == 0
                 pts[wsw.S] = statistics.median(times)
+                nsel_sw = int((rts.sel >= 0).sum().item())
+                by_sw = forward_bytes(wsw, nsel_sw, 2)
+                sweep_bytes[wsw.S] = {"selected_blocks_per_route": nsel_sw / (wsw.B * wsw.Hq * wsw.nb),
+                                      "path_bytes": by_sw["path"],
+                                      "path_roofline_frac": by_sw["path"] / (pts[wsw.S] / 1e3) / 1e9 / peak,
+                                      "kv_bytes": 2 * wsw.B * wsw.S * wsw.Hkv * wsw.D * 2}
                 del qs_, ks_, vs_, ixs, rts, wss, outs
             Ss = sorted(pts)
             short = [S for S in Ss if S <= 32768]
             scaling_obj = {"workload": "scaling: B=1, H=8, D=128 bf16, block 64, K=32, cap 64, p=4, R=8, L=2",
                            "ms_per_forward": {str(S): pts[S] for S in Ss},
                            "tokens_per_s": {str(S): S / (pts[S] / 1e3) for S in Ss},
+                           "per_length": {str(S): sweep_bytes[S] for S in Ss},
+                           "l2_bytes": torch.cuda.get_device_properties(dev).L2_cache_size,
                            "exponent_4k_32k": loglog_exponent(short, [pts[S] for S in short]),
                            "exponent_4k_128k": loglog_exponent(Ss, [pts[S] for S in Ss])}
             if rank == 0 and not args.no_cpu:
@@ -573,9 +795,38 @@ def run_mine(args, w):
                 Sc = sorted(cpu_pts)
                 scaling_obj["cpu_oracle_index_route"] = {
                     "seconds": {str(S): cpu_pts[S] for S in Sc}, "cores": blas_threads(),
+                    "threads": "the BLAS pool as it stands; the route itself is a Python loop (one thread)",
                     "exponent_4k_32k": loglog_exponent(Sc, [cpu_pts[S] for S in Sc])}
         except Exception as e:                   # the line still carries every other number
             scaling_obj = {"error": repr(e)}
+
+    # The forward on the other workload shapes (one GPU): the planted-block,
+    # capacity and long-context workloads, each with its byte model,
+    # roofline fractions, overflow and (grouped heads) the union of each
+    # group's selections.
+    workloads_obj = None
+    if world == 1 and not args.no_workloads:
+        workloads_obj = {}
+        for name in ("ar", "capacity", "long"):
+            try:
+                wx = workload(name)
+                if name == "long":
+                    qx, kx, vx, cbx = device_inputs(wx, 7000, dev)
+                    recipe = "q, v ~ N(0,1) drawn on the device (torch, seeded); keys: the Zipf cluster recipe"
+                else:
+                    ix = make_inputs(wx, 7000)
+                    qx, kx, vx = (conv(x).to(dev) for x in (ix.q_store, ix.k_store, ix.v_store))
+                    cbx = torch.from_numpy(ix.codebooks).to(dev)
+                    recipe = f"the {wx.keys} recipe of the workload generator"
+                r = measure_forward(mdr, wx, qx, kx, vx, cbx, dev, stream, flush_l2)
+                r["config"] = {k_: v_ for k_, v_ in config_of(wx, argparse.Namespace(gpus=1)).items()
+                               if k_ not in ("l2", "parallelism")}
+                r["inputs"] = recipe
+                workloads_obj[name] = r
+                del qx, kx, vx, cbx
+            except Exception as e:                  # the line still carries every other number
+                workloads_obj[name] = {"error": repr(e)}
+        torch.cuda.empty_cache()
 
     # End to end through the C ABI with host buffers.
     e2e = None
@@ -607,10 +858,7 @@ def run_mine(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        tps, secs, groups = oracle_sample(w, 1000, max_seconds=args.cpu_seconds)
-        cpu = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{groups} of {w.Hkv} KV-head groups of one sequence (all {w.nb} query blocks), "
-                         f"{secs:.1f} s, scaled to the full forward"}
+        cpu = cpu_baseline(w, args.cpu_seconds)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -622,9 +870,10 @@ def run_mine(args, w):
                              "peak_kind": peak_kind,
                              "kernel": "attend", "algorithmic_bytes_per_launch": attn_bytes},
                 "path_roofline_frac": total_bytes / (ms_max / 1e3) / 1e9 / peak,
+                "path_bytes": total_bytes, "kernels": kernels,
                 "kernels_ms": ker, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
                 "controls": controls, "calibration": calibration, "backward": backward,
-                "scaling_sweep": scaling_obj,
+                "scaling_sweep": scaling_obj, "workloads": workloads_obj,
                 "gpu_launches": KERNELS_PER_FORWARD * args.steps, "clocks": clk.summary(),
                 "overflow": int(idx.overflow.sum().item()), "selected_blocks": nsel}
         print(json.dumps(line), flush=True)
@@ -647,6 +896,8 @@ def main():
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true")
+    ap.add_argument("--decode-batch", type=int, default=32)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     w = workload(args.workload)

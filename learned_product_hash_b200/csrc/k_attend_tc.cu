@@ -51,6 +51,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
+#include "tmap.h"
 
 namespace mdr {
 
@@ -685,42 +686,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
 namespace {
 
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encoder() {
-  static EncodeTiled fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(p);
-  }
-  return fn;
-}
-
-// [rows, H, D] bf16 viewed as a 3-D tensor (D, H, rows); box (64, 1, BS).
-bool make_map(CUtensorMap* m, const void* ptr, long long rows, int H, int D, int BS) {
-  EncodeTiled enc = encoder();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
-  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(BS)};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int BS, int D>
 cudaError_t launch_tc(const AttendArgs& a, cudaStream_t st) {
   using C = TcCfg<BS, D>;
   CUtensorMap mq, mk, mv;
   const long long rows = static_cast<long long>(a.B) * a.S;
-  if (!make_map(&mq, a.q, rows, a.Hq, D, BS) || !make_map(&mk, a.k, rows, a.Hkv, D, BS) ||
-      !make_map(&mv, a.v, rows, a.Hkv, D, BS))
+  if (!make_tile_map(&mq, a.q, rows, a.Hq, D, BS) || !make_tile_map(&mk, a.k, rows, a.Hkv, D, BS) ||
+      !make_tile_map(&mv, a.v, rows, a.Hkv, D, BS))
     return cudaErrorInvalidValue;
   auto k = attend_tc_kernel<BS, D>;
   cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(k), C::kSmem);

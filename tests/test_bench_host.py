@@ -83,3 +83,59 @@ def test_oracle_index_route_timing_runs_on_a_small_workload():
     from workloads import scaling
     t = bench.oracle_route_seconds(scaling(4096), 0, 2)
     assert len(t) == 2 and min(t) > 0
+
+
+def test_forward_bytes_follow_the_byte_model():
+    """Summary pass: q and k read once; attention: q read, K and V of every
+    valid selected block gathered, output written (per route)."""
+    import bench
+    from workloads import SCALING_32K as w
+    by = bench.forward_bytes(w, 23803, 2)
+    assert by["summaries"] == (8 + 8) * 32768 * 128 * 2
+    assert by["attention"] == 8 * 512 * 2 * 64 * 128 * 2 + 23803 * 64 * 2 * 128 * 2 == 914194432
+    assert by["path"] == by["summaries"] + by["attention"]
+
+
+def test_gqa_union_counts_distinct_blocks_per_group():
+    """Two query heads per KV head: head 0 selects {0, 2}, head 1 selects
+    {2, 3} for query block 3 -> union 3 of 4; -1 pads count in neither."""
+    import types
+    import bench
+    w = types.SimpleNamespace(B=1, Hq=2, Hkv=1, nb=4, R=2, L=1)
+    sel = torch.full((1, 2, 4, 3), -1, dtype=torch.int32)
+    sel[0, 0, 3] = torch.tensor([0, 2, 3])
+    sel[0, 1, 3] = torch.tensor([2, -1, 3])
+    sel[0, 0, 0, 2] = 0
+    sel[0, 1, 0, 2] = 0
+    u = bench.gqa_union(sel, w)
+    assert u == {"group_size": 2, "per_head_blocks": 7, "union_blocks": 4, "union_fraction": 4 / 7}
+
+
+def test_cpu_baseline_reports_each_thread_setting(monkeypatch):
+    import bench
+    from workloads import TINY
+    seen = []
+    monkeypatch.setattr(bench, "oracle_sample", lambda w, seed, max_seconds: (seen.append(1) or (100.0, 0.1, 1)))
+    monkeypatch.setattr(os, "cpu_count", lambda: 16)
+    c = bench.cpu_baseline(TINY, 3.0)
+    assert sorted(c["by_threads"], key=int) == ["1", "4", "16"] and len(seen) == 3
+    assert c["cores"] == 16 and c["kind"] == "oracle" and c["value"] == 100.0
+
+
+def test_reference_arm_prints_whole_steps(monkeypatch, capsys):
+    """Each step of the reference arm is one whole forward (every KV-head
+    group) when warm-up + steps fit the budget, else a scaled sample."""
+    import argparse
+    import json
+    import bench
+    from workloads import TINY
+    calls = []
+    monkeypatch.setattr(bench, "oracle_group_seconds", lambda w, inp, h: (calls.append(h) or 0.5))
+    args = argparse.Namespace(gpus=1, steps=3, warmup=1)
+    bench.run_reference(args, TINY)
+    line = json.loads(capsys.readouterr().out)
+    assert line["impl"] == "reference" and line["ms_per_step"] == 500.0 and "whole forward" in line["cpu_baseline"]["sample"]
+    monkeypatch.setattr(bench, "REF_BUDGET_S", 1.0)
+    bench.run_reference(args, TINY.with_(Hq=8, Hkv=8))
+    line = json.loads(capsys.readouterr().out)
+    assert "scaled" in line["cpu_baseline"]["sample"] and line["ms_per_step"] == 8 * 500.0

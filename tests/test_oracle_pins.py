@@ -32,6 +32,22 @@ def test_planted_block_is_found():
     assert np.mean(hits_route) > 0.3
 
 
+def test_planted_block_mean_cosine_is_the_stated_one():
+    """The planted-block workload states that the planted block's mean key
+    aligns with cosine 0.9 with the last block's mean query: measured here on
+    the rotated block means (the oracle's), averaged over sequences and
+    heads."""
+    w = AR.with_(B=32)
+    inp = make_inputs(w, 0)
+    res = O.forward(inp.q, inp.k, inp.v, inp.codebooks, O.Params.of(w), attention=False)
+    cs = []
+    for b in range(w.B):
+        for h in range(w.Hq):
+            qb, kb = res.qbar[b, h, w.nb - 1], res.kbar[b, h, inp.planted[b]]
+            cs.append(qb @ kb / np.linalg.norm(qb) / np.linalg.norm(kb))
+    assert abs(np.mean(cs) - 0.9) < 0.01, np.mean(cs)
+
+
 def test_capacity_workload_load():
     """The capacity workload has the report's capacity-run shape (8,192
     tokens, capacity 64); its lists stay under capacity."""

@@ -13,12 +13,16 @@ the storage type with round-to-nearest-even):
 * planted  -- as gaussian, plus, per sequence, one planted block b* drawn
               uniformly among the blocks that are remote-eligible for the last
               query block.  Per head, a unit direction u and a unit direction
-              w orthogonal to it are drawn inside the coordinates of the
-              slowest rotary pairs (pair index i in [3D/8, D/2) under the
-              rotate-half pairing, i.e. coordinates i and i + D/2), where
-              rotation over the whole sequence stays small.  The last block's
-              queries get +alpha*u and the planted block's keys get
-              +alpha*(0.9 u + sqrt(0.19) w): their directions have cosine 0.9.
+              w orthogonal to it are drawn inside the coordinates of the two
+              slowest rotary pairs (pair indices D/2-2 and D/2-1 under the
+              rotate-half pairing, i.e. coordinates i and i + D/2), which turn
+              by under 0.07 rad over the whole 384-token sequence.  The last
+              block's queries get +alpha*u and the planted block's keys get
+              +alpha*(c u + sqrt(1-c^2) w).  A block mean of bs standard
+              normals adds noise of squared norm D/bs on average to the planted
+              alpha, so c = 0.9*(alpha^2 + D/bs)/alpha^2 makes the expected
+              cosine between the block-mean query and the block-mean planted
+              key 0.9 (the workload's stated alignment).
 * clusters -- v, q ~ N(0, 1).  Each key block draws one of n_clusters unit
               centres (uniformly, or Zipf(s) over cluster rank when zipf_s >
               0); every key of the block is sigma*N(0, I) plus the centre,
@@ -49,6 +53,8 @@ import numpy as np
 from .configs import Workload
 
 ALPHA_PLANTED = 4.0
+PLANTED_COS = 0.9        # stated alignment of the planted mean key with the last mean query
+PLANTED_PAIRS = 2        # slowest rotary pairs that carry the planted directions
 
 
 def rng_for(seed: int, *tags: str) -> np.random.Generator:
@@ -136,16 +142,17 @@ def make_inputs(w: Workload, seed: int, *, keys: str | None = None,
             last_eligible = nb - 1 - w.L
             assert last_eligible >= 0, "planted recipe needs a remote-eligible block"
             planted = r.integers(0, last_eligible + 1, size=B)
-            coords = slow_pair_coords(D)
+            coords = slow_pair_coords(D, PLANTED_PAIRS)
             m = coords.size
             g = Hq // Hkv
+            c = min(1.0, PLANTED_COS * (ALPHA_PLANTED ** 2 + D / bs) / ALPHA_PLANTED ** 2)
             for b in range(B):
                 for h in range(Hkv):
                     u = _unit(r, (m,))
                     x = r.standard_normal(m)
                     x -= x.dot(u) * u
                     wv = x / np.linalg.norm(x)
-                    key_dir = 0.9 * u + np.sqrt(0.19) * wv
+                    key_dir = c * u + np.sqrt(1.0 - c * c) * wv
                     kb = k[b, planted[b] * bs:(planted[b] + 1) * bs, h]
                     kb[:, coords] += ALPHA_PLANTED * key_dir[None, :]
                     for hq in range(h * g, (h + 1) * g):
