@@ -48,6 +48,7 @@ from workloads import SCALING_SWEEP, ALL, make_codebooks, make_grad, make_inputs
 
 METRIC = "routed-attention fwd tokens/s (index+route+attend) at 32K; % HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def workload(name):
@@ -90,6 +91,18 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 tensor-core peak in TFLOP/s: the measured burst figure (a
+    kernel timed alone), else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured (burst)"
+    return FALLBACK_BF16_TFLOPS, "fallback (burst)"
 
 
 class ClockSampler:
@@ -729,16 +742,30 @@ def run_mine(args, w):
         b_ms = b0.elapsed_time(b1) / nb_it
         b_ms_max = max_over_ranks(b_ms, dist, world, dev)
         fl = backward_flops(sel, w.block, w.D)
-        alu_peak = torch.cuda.get_device_properties(dev).multi_processor_count * FP32_LANES_PER_SM * 2 * \
-            (clk.summary() or {}).get("sm_max_mhz", 1965) * 1e6 / 1e12
+        if w.dtype == "bf16":
+            tpk, tpk_kind = tensor_peak()
+            roof = {"bound": "tensor", "achieved": fl / (b_ms / 1e3) / 1e12, "peak": tpk, "unit": "TFLOP/s",
+                    "frac": fl / (b_ms / 1e3) / 1e12 / tpk, "peak_kind": tpk_kind,
+                    "algorithmic_flops_per_call": fl,
+                    "note": "flops of the four gradient products; the kernels also recompute S twice, "
+                            "dP twice and O once (about 2.25x the algorithmic MMA work)"}
+            arith = "bf16 operands on the tensor cores (tcgen05), float32 accumulation in tensor memory"
+            launches = 4
+        else:
+            alu_peak = torch.cuda.get_device_properties(dev).multi_processor_count * FP32_LANES_PER_SM * 2 * \
+                (clk.summary() or {}).get("sm_max_mhz", 1965) * 1e6 / 1e12
+            roof = {"bound": "alu", "achieved": fl / (b_ms / 1e3) / 1e12, "peak": alu_peak, "unit": "TFLOP/s",
+                    "frac": fl / (b_ms / 1e3) / 1e12 / alu_peak,
+                    "peak_kind": "derived: SMs x 128 FP32 lanes x 2 flops x max SM clock",
+                    "algorithmic_flops_per_call": fl}
+            arith = "float32 on CUDA cores"
+            launches = 4
         backward = {"metric": "attention backward (dq, dk, dv for a fixed route) at 32K",
                     "value": throughput(w.B * w.S, world, b_ms_max), "unit": "tokens/s", "ms_per_call": b_ms_max,
-                    "launches_per_call": 4, "arithmetic": "float32 on CUDA cores",
-                    "l2": "not flushed: q, k, v, dout and the float32 rotated copies (~0.5 GB) exceed L2",
-                    "roofline": {"bound": "alu", "achieved": fl / (b_ms / 1e3) / 1e12, "peak": alu_peak,
-                                 "unit": "TFLOP/s", "frac": fl / (b_ms / 1e3) / 1e12 / alu_peak,
-                                 "peak_kind": "derived: SMs x 128 FP32 lanes x 2 flops x max SM clock",
-                                 "algorithmic_flops_per_call": fl}}
+                    "launches_per_call": launches, "arithmetic": arith,
+                    "l2": "not flushed between calls: q, k, v, dout, the rotated copies and the float32 "
+                          "gradients (~0.8 GB) exceed L2",
+                    "roofline": roof}
         del bws, dq, dk, dv, do
 
     # Scaling of the forward from 4K to 128K tokens (one GPU): the median of

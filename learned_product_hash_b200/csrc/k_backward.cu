@@ -6,7 +6,8 @@
 // hard top-k choices pass no ordinary gradient through the chosen index, so
 // nothing flows to the codebooks or the block summaries.
 //
-// Four kernels, float32 arithmetic, every floating-point sum in a fixed
+// The CUDA-core path (float32 storage; bf16 storage runs on the tensor cores
+// in k_backward_tc.cu).  Four kernels, float32 arithmetic, every floating-point sum in a fixed
 // order (the only atomics count list entries in shared memory, whose integer
 // totals do not depend on order), so a call is deterministic:
 //   bwd_rotate_kernel  float32 rotated copies q', k' (the angle of the
@@ -377,6 +378,13 @@ static cudaError_t launch_grad_for(const BwdArgs& a, cudaStream_t st) {
   }
 }
 
+cudaError_t launch_bwd_rev(const BwdArgs& a, cudaStream_t st) {
+  const size_t smem = bwd_rev_smem(a.nb);
+  cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(bwd_rev_kernel), static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(bwd_rev_kernel, dim3(a.B * a.Hkv), dim3(256), smem, st, a);
+}
+
 cudaError_t launch_backward(const BwdArgs& a, bool bf16, cudaStream_t st) {
   if (a.D != 32 && a.D != 64 && a.D != 128) return cudaErrorInvalidValue;
   const int sms = cached_sm_count();
@@ -387,13 +395,8 @@ cudaError_t launch_backward(const BwdArgs& a, bool bf16, cudaStream_t st) {
     e = launch_pdl(k, dim3(sms * 4), dim3(256), 0, st, a);
     if (e != cudaSuccess) return e;
   }
-  {
-    const size_t smem = bwd_rev_smem(a.nb);
-    e = cached_allow_smem(reinterpret_cast<const void*>(bwd_rev_kernel), static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(bwd_rev_kernel, dim3(a.B * a.Hkv), dim3(256), smem, st, a);
-    if (e != cudaSuccess) return e;
-  }
+  e = launch_bwd_rev(a, st);
+  if (e != cudaSuccess) return e;
   e = bf16 ? launch_grad_for<__nv_bfloat16>(a, st) : launch_grad_for<float>(a, st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

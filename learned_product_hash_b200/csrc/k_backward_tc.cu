@@ -1,0 +1,779 @@
+// Backward of the selected-set attention on the tensor cores (bf16 storage):
+// dL/dq, dL/dk, dL/dv for dL/d(out), the route held fixed.  "Monodratic
+// Claims Learned Routing Can Make Sparse Causal Attention More Selective",
+// section "The 99.35 Percent Result Does Not Establish Language Quality":
+// hard top-k choices pass no ordinary gradient through the chosen index, so
+// the gradient is that of the causal softmax over the selected tokens and of
+// the rotary embedding; nothing reaches the codebooks or the summaries.
+//
+// Inputs are the rotated copies q', k' (bf16, written by the summary kernel
+// exactly as for the forward), v and the upstream gradient dO, all read as
+// 128-byte-swizzled [bs x 64] boxes by TMA; every product runs as a
+// tcgen05.mma (bf16 operands, float32 accumulators in tensor memory).  Scores
+// are kept in log2 units (scale * log2(e) folded in), exponentials are
+// ex2.approx.
+//
+//   bwd_dq_tc_kernel    one query tile (b, hq, j) at a time, persistent.
+//     pass 1, per selected block: S = Q K^T; the running maximum and sum of
+//       each row; P = 2^(S - max) (bf16) into shared memory; O += P V.  At
+//       the end: lse = max + log2(sum) and Delta = <dO, O> / sum per row,
+//       stored for the key-side kernel.
+//     pass 2, per selected block: S = Q K^T and dP = dO V^T; P = 2^(S - lse),
+//       dS = P (dP - Delta) (bf16) into shared memory; dQ += dS K (K read
+//       MN-major from its TMA tile).  Epilogue: dq = R(t)^T (scale dQ).
+//   bwd_dkdv_tc_kernel  one key block (b, hkv, i) at a time, persistent, over
+//     the block's reverse list (the (query head, query block) pairs that
+//     selected it, in a fixed order): S^T = K Q^T and dP^T = V dO^T;
+//     P^T = 2^(S^T - lse_t), dS^T = P^T (dP^T - Delta_t) (bf16); dV += P^T dO,
+//     dK += dS^T Q.  Epilogue: dv = dV, dk = R(s)^T (scale dK).
+// The causal mask applies where the key block is the query block (key s >
+// query t is masked).  Each CTA has four warps; warp w owns TMEM
+// subpartition w (accumulator rows 16w..16w+15 for bs = 64, two threads per
+// row splitting the columns; rows 32w..32w+31 for bs = 128).  Thread 0 issues
+// the TMA loads and the MMAs; the next block's (or entry's) tiles are loaded
+// while the current one is computed.  Sums run in a fixed order and there
+// are no atomics, so a call is deterministic.  Every wait is bounded (2 s of
+// wall time): a wait that runs out writes status 1, the CTA waits (bounded)
+// for its own copies and MMAs, frees its tensor memory and returns.
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+#include "tmap.h"
+
+namespace mdr {
+
+namespace {
+
+constexpr uint64_t kBwWaitNs = 2000000000ull;
+constexpr int kBwThreads = 128;
+
+constexpr int pow2_cols(int c) { return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512; }
+
+template <int BS, int D>
+struct BwCfg {
+  static constexpr bool kHR = (BS == 64);            // rows in lanes 0-15: two threads per row
+  static constexpr int kTile = BS * D * 2;           // bf16 [BS x D]: D/64 regions
+  static constexpr int kRegion = BS * 128;           // one 64-column region of a [BS x *] tile
+  static constexpr int kPTile = BS * BS * 2;         // bf16 [BS x BS]: BS/64 regions
+  static constexpr int kCtl = 1024;                  // barriers, omega, ids, misc
+  // dq kernel: Q, dO, two (K, V) slots, P / dS
+  static constexpr int qOffQ = 0;
+  static constexpr int qOffO = kTile;
+  static constexpr int qOffKV = 2 * kTile;
+  static constexpr int qOffP = qOffKV + 4 * kTile;
+  static constexpr int qOffCtl = qOffP + kPTile;
+  static constexpr int qSmem = qOffCtl + kCtl;
+  static constexpr int qCols = pow2_cols(2 * BS + D);
+  static constexpr int qColS = 0, qColP = BS, qColO = 2 * BS;
+  // dk/dv kernel: K, V, kNE entry slots (Q, dO, lse, Delta), P^T, dS^T
+  static constexpr int kNE = (BS == 128 && D == 128) ? 1 : 3;
+  static constexpr int kSlot = (2 * kTile + 2 * BS * 4 + 1023) / 1024 * 1024;
+  static constexpr int bOffK = 0, bOffV = kTile, bOffE = 2 * kTile;
+  static constexpr int bOffPT = bOffE + kNE * kSlot;
+  static constexpr int bOffDS = bOffPT + kPTile;
+  static constexpr int bOffCtl = bOffDS + kPTile;
+  static constexpr int bSmem = bOffCtl + kCtl;
+  static constexpr int bCols = pow2_cols(2 * BS + 2 * D);
+  static constexpr int bColS = 0, bColP = BS, bColV = 2 * BS, bColK = 2 * BS + D;
+  static_assert(qSmem <= 232448 && bSmem <= 232448, "shared memory per CTA");
+  static_assert(kTile % 1024 == 0 && kPTile % 1024 == 0, "1024-byte aligned tiles");
+  // D-column geometry of a thread: W columns at lo and W at D/2 + lo, NP times.
+  static constexpr int W = kHR ? D / 4 : 32;
+  static constexpr int NP = kHR ? 1 : D / 64;
+  // score-column geometry: NC chunks of 32 columns
+  static constexpr int NC = kHR ? 1 : BS / 32;
+};
+
+// Control block at the end of shared memory.
+struct Ctl {
+  uint64_t bar[16];
+  float om[64];
+  int16_t ids[64];
+  uint32_t tmem;
+  int nblk;
+  int abort;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// K-major operand descriptor of a [rows x D] tile (D/64 regions) at K step kk.
+template <int BS>
+__device__ __forceinline__ uint64_t kmaj(uint32_t s, int kk) {
+  return tc::smem_desc_sw128(s, 16, 1024) + static_cast<uint64_t>(((kk / 4) * (BS * 128) + (kk % 4) * 32) / 16);
+}
+// MN-major operand descriptor (N = D in 64-column regions) at K step kk (16 rows).
+template <int BS>
+__device__ __forceinline__ uint64_t mnmaj(uint32_t s, int kk) {
+  return tc::smem_desc_sw128(s, BS * 128, 1024) + static_cast<uint64_t>(kk * 128);
+}
+
+// Thread geometry over the accumulator rows.
+template <int BS, int D>
+struct Rows {
+  using C = BwCfg<BS, D>;
+  int warp, lane, r, tsub;
+  uint32_t lane_base;
+  __device__ Rows() {
+    warp = threadIdx.x >> 5;
+    lane = threadIdx.x & 31;
+    tsub = C::kHR ? (lane >> 4) : 0;
+    r = C::kHR ? warp * 16 + (lane & 15) : warp * 32 + lane;
+    lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  }
+  // 32 score columns of chunk c (first column returned); all lanes take part.
+  __device__ __forceinline__ int ld_scores(uint32_t tcol, int c, float* v) const {
+    if constexpr (C::kHR) {
+      tc::tmem_ld16x2_32(tcol + lane_base, v);
+      return 32 * tsub;
+    } else {
+      tc::tmem_ld32(tcol + 32 * c + lane_base, v);
+      return 32 * c;
+    }
+  }
+  // W D-columns at offset off (0 or D/2, plus the pair's chunk) of part pp.
+  __device__ __forceinline__ void ld_d(uint32_t tcol, int pp, int half, float* v) const {
+    const uint32_t at = tcol + (half ? D / 2 : 0) + (C::kHR ? 0 : 32 * pp) + lane_base;
+    if constexpr (C::kHR && D == 64) tc::tmem_ld16x2_16(at, v);
+    else if constexpr (C::kHR) tc::tmem_ld16x2_32(at, v);
+    else tc::tmem_ld32(at, v);
+  }
+  __device__ __forceinline__ void st_d(uint32_t tcol, int pp, int half, const float* v) const {
+    const uint32_t at = tcol + (half ? D / 2 : 0) + (C::kHR ? 0 : 32 * pp) + lane_base;
+    if constexpr (C::kHR && D == 64) tc::tmem_st16x2_16(at, v);
+    else if constexpr (C::kHR) tc::tmem_st16x2_32(at, v);
+    else tc::tmem_st32(at, v);
+  }
+  // First D-column of the lower half held for part pp.
+  __device__ __forceinline__ int col_lo(int pp) const { return C::kHR ? C::W * tsub : 32 * pp; }
+  // Sum of a per-thread partial over the row's threads.
+  __device__ __forceinline__ float row_sum(float x) const {
+    if constexpr (C::kHR) x += __shfl_xor_sync(0xffffffffu, x, 16);
+    return x;
+  }
+  __device__ __forceinline__ float row_max(float x) const {
+    if constexpr (C::kHR) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+    return x;
+  }
+};
+
+// Eight bf16 values of row r at columns c0..c0+7 (c0 % 8 == 0) of a
+// K-major, 128-byte-swizzled [BS x *] tile.
+template <int BS>
+__device__ __forceinline__ void st_bf16x8(uint8_t* tile, int r, int c0, const float* x) {
+  const int chunk = ((c0 % 64) / 8) ^ (r & 7);
+  *reinterpret_cast<uint4*>(tile + (c0 / 64) * (BS * 128) + r * 128 + chunk * 16) =
+      make_uint4(pack2(x[0], x[1]), pack2(x[2], x[3]), pack2(x[4], x[5]), pack2(x[6], x[7]));
+}
+
+// Dot product of W float32 values with W bf16 values in global memory.
+template <int W>
+__device__ __forceinline__ float dot_bf16(const float* x, const __nv_bfloat16* g) {
+  float s = 0.f;
+#pragma unroll
+  for (int q = 0; q < W / 8; ++q) {
+    float y[8];
+    Elem<__nv_bfloat16>::load(g + 8 * q, y);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s = __fmaf_rn(x[8 * q + e], y[e], s);
+  }
+  return s;
+}
+
+// y = R(t)^T (scale * x) for the pair (lo, hi) = coordinates (i, i + D/2),
+// i = i0 .. i0 + W - 1, written as float32 to row out at columns i and i + D/2.
+template <int W, int D>
+__device__ __forceinline__ void rotate_store(const float* lo, const float* hi, int i0, int t, float scale,
+                                             const float* om, float* out) {
+#pragma unroll
+  for (int q = 0; q < W / 4; ++q) {
+    float a[4], b[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = i0 + 4 * q + e;
+      float sn, cs;
+      sincosf(static_cast<float>(t) * om[i], &sn, &cs);
+      const float y1 = scale * lo[4 * q + e], y2 = scale * hi[4 * q + e];
+      a[e] = y1 * cs + y2 * sn;
+      b[e] = y2 * cs - y1 * sn;
+    }
+    *reinterpret_cast<float4*>(out + i0 + 4 * q) = make_float4(a[0], a[1], a[2], a[3]);
+    *reinterpret_cast<float4*>(out + D / 2 + i0 + 4 * q) = make_float4(b[0], b[1], b[2], b[3]);
+  }
+}
+
+template <int W>
+__device__ __forceinline__ void store_f32(float* out, const float* x) {
+#pragma unroll
+  for (int q = 0; q < W / 4; ++q)
+    *reinterpret_cast<float4*>(out + 4 * q) = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- dq kernel
+template <int BS, int D>
+__global__ void __launch_bounds__(kBwThreads, 1)
+bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                 const BwdArgs a) {
+  using C = BwCfg<BS, D>;
+  using namespace tc;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicExch(a.status, kDevMisaligned);
+    return;
+  }
+  Ctl& ctl = *reinterpret_cast<Ctl*>(smem + C::qOffCtl);
+  const uint32_t base = smem_u32(smem);
+  const uint32_t sQ = base + C::qOffQ, sO = base + C::qOffO, sKV = base + C::qOffKV, sP = base + C::qOffP;
+  uint8_t* pP = smem + C::qOffP;
+  enum { bQ = 0, bKV0 = 1, bS = 3, bMM = 4, bFin = 5 };
+  auto BAR = [&](int i) { return smem_u32(&ctl.bar[i]); };
+  const Rows<BS, D> R;
+  if (R.warp == 0) {
+    tmem_alloc(smem_u32(&ctl.tmem), C::qCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 6; ++i) mbar_init(BAR(i), 1);
+    fence_mbar_init();
+    ctl.abort = 0;
+  }
+  if (threadIdx.x < D / 2) ctl.om[threadIdx.x] = a.inv_freq[threadIdx.x];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem;
+  grid_dependency_wait();          // q', k' (summary kernel) and the reverse index come from earlier kernels
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmO);
+  }
+
+  constexpr uint32_t idS = idesc_bf16_f32(BS, BS, 0, 0);
+  constexpr uint32_t idPV = idesc_bf16_f32(BS, D, 0, 1);
+  const float sl2 = a.scale * 1.4426950408889634f;
+  const long long ntiles = static_cast<long long>(a.B) * a.Hq * a.nb;
+  const int g = a.Hq / a.Hkv;
+  uint32_t phQ = 0, phS = 0, phMM = 0;
+  long long ld_issue = 0, ld_use = 0;             // (K, V) loads: slot = n & 1, parity (n >> 1) & 1
+  bool mm_pending = false, ok = true, q_pending = false;
+  int mm_step = 0;
+
+  // Wait for a barrier phase in every thread; false (everywhere) if any gave up.
+  auto wait_all = [&](int bar, uint32_t parity) -> bool {
+    const bool w = mbar_wait(BAR(bar), parity, kBwWaitNs);
+    return __syncthreads_and(w) != 0;
+  };
+
+  for (long long tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+    const int j = static_cast<int>(tile % a.nb), hq = static_cast<int>((tile / a.nb) % a.Hq);
+    const int b = static_cast<int>(tile / (static_cast<long long>(a.nb) * a.Hq));
+    const int h = hq / g;
+    __syncthreads();                              // the previous tile's ids are no longer read
+    if (R.warp == 0) {
+      const int32_t* row = a.sel + tile * a.nsel;
+      const int e0 = R.lane < a.nsel ? row[R.lane] : -1, e1 = R.lane + 32 < a.nsel ? row[R.lane + 32] : -1;
+      const bool v0 = e0 >= 0 && e0 <= j, v1 = e1 >= 0 && e1 <= j;
+      if (e0 > j || e1 > j) atomicExch(a.status, kDevBadSelection);
+      const unsigned m0 = __ballot_sync(0xffffffffu, v0), m1 = __ballot_sync(0xffffffffu, v1);
+      const unsigned lt = (1u << R.lane) - 1u;
+      if (v0) ctl.ids[__popc(m0 & lt)] = static_cast<int16_t>(e0);
+      if (v1) ctl.ids[__popc(m0) + __popc(m1 & lt)] = static_cast<int16_t>(e1);
+      if (R.lane == 0) ctl.nblk = __popc(m0) + __popc(m1);
+    }
+    __syncthreads();
+    const int nblk = ctl.nblk;
+    const long long tok0 = static_cast<long long>(b) * a.S + static_cast<long long>(j) * BS;
+    const long long si0 = (static_cast<long long>(b) * a.Hq + hq) * a.S + static_cast<long long>(j) * BS;
+    if (nblk == 0) {                              // nothing selected: zero gradient, no row statistics
+      for (int e = threadIdx.x; e < BS * D; e += kBwThreads)
+        a.dq[((tok0 + e / D) * a.Hq + hq) * D + e % D] = 0.f;
+      for (int t = threadIdx.x; t < BS; t += kBwThreads) {
+        a.lse[si0 + t] = INFINITY;
+        a.delta[si0 + t] = 0.f;
+      }
+      continue;
+    }
+    const int nsteps = 2 * nblk;                  // pass 1 then pass 2 over the same blocks
+    auto issue_kv = [&](int n) {                  // K, V of step n into slot ld_issue & 1
+      if (threadIdx.x == 0) {
+        const int slot = static_cast<int>(ld_issue & 1);
+        const uint32_t bar = BAR(bKV0 + slot), dst = sKV + slot * 2 * C::kTile;
+        const int blk = ctl.ids[n % nblk];
+        mbar_expect_tx(bar, 2 * C::kTile);
+#pragma unroll
+        for (int gg = 0; gg < D / 64; ++gg) {
+          tma_load_3d(dst + gg * C::kRegion, &tmK, bar, gg * 64, h, static_cast<int>(b * a.S + blk * BS));
+          tma_load_3d(dst + C::kTile + gg * C::kRegion, &tmV, bar, gg * 64, h, static_cast<int>(b * a.S + blk * BS));
+        }
+      }
+      ++ld_issue;
+    };
+    // The MMA of step mm_step (PV or dQ) has completed: its slot is free for
+    // step mm_step + 2.
+    auto finish_mm = [&]() -> bool {
+      if (!mm_pending) return true;
+      if (!wait_all(bMM, phMM)) return false;
+      phMM ^= 1;
+      mm_pending = false;
+      if (mm_step + 2 < nsteps) issue_kv(mm_step + 2);
+      return true;
+    };
+    if (threadIdx.x == 0) {
+      mbar_expect_tx(BAR(bQ), 2 * C::kTile);
+#pragma unroll
+      for (int gg = 0; gg < D / 64; ++gg) {
+        tma_load_3d(sQ + gg * C::kRegion, &tmQ, BAR(bQ), gg * 64, hq, static_cast<int>(tok0));
+        tma_load_3d(sO + gg * C::kRegion, &tmO, BAR(bQ), gg * 64, hq, static_cast<int>(tok0));
+      }
+    }
+    q_pending = true;
+    issue_kv(0);
+    issue_kv(1);
+    if (!wait_all(bQ, phQ)) { ok = false; break; }
+    phQ ^= 1;
+    q_pending = false;
+    float m2 = -INFINITY, l = 0.f, lse2 = 0.f, delta = 0.f;
+    for (int n = 0; n < nsteps && ok; ++n) {
+      const bool pass2 = n >= nblk;
+      const int blk = ctl.ids[n % nblk];
+      const int slot = static_cast<int>(ld_use & 1);
+      if (!wait_all(bKV0 + slot, static_cast<uint32_t>((ld_use >> 1) & 1))) { ok = false; break; }
+      ++ld_use;
+      const uint32_t sK = sKV + slot * 2 * C::kTile, sV = sK + C::kTile;
+      if (threadIdx.x == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16(tmem + C::qColS, kmaj<BS>(sQ, kk), kmaj<BS>(sK, kk), idS, kk > 0);
+        if (pass2) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) mma_bf16(tmem + C::qColP, kmaj<BS>(sO, kk), kmaj<BS>(sV, kk), idS, kk > 0);
+        }
+        mma_commit(BAR(bS));
+      }
+      if (!wait_all(bS, phS)) { ok = false; break; }
+      phS ^= 1;
+      if (!finish_mm()) { ok = false; break; }     // O (or dQ) and the P buffer are free
+      tc_fence_after();
+      const bool diag = blk == j;
+      if (!pass2) {
+        // Row maximum of this block, then rescale O and the sum if it grew.
+        float mx = -INFINITY;
+        float sv[C::NC][32];
+#pragma unroll
+        for (int c = 0; c < C::NC; ++c) {
+          const int k0 = R.ld_scores(tmem + C::qColS, c, sv[c]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            sv[c][e] = (diag && k0 + e > R.r) ? -INFINITY : sv[c][e] * sl2;
+            mx = fmaxf(mx, sv[c][e]);
+          }
+        }
+        mx = R.row_max(mx);
+        if (mx > m2) {
+          if (n > 0) {
+            const float alpha = ex2(m2 - mx);
+            l *= alpha;
+#pragma unroll
+            for (int pp = 0; pp < C::NP; ++pp)
+#pragma unroll
+              for (int hf = 0; hf < 2; ++hf) {
+                float o[C::W];
+                R.ld_d(tmem + C::qColO, pp, hf, o);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < C::W; ++e) o[e] *= alpha;
+                R.st_d(tmem + C::qColO, pp, hf, o);
+              }
+            tmem_st_wait();
+          }
+          m2 = mx;
+        }
+        const float mref = m2 == -INFINITY ? 0.f : m2;   // a row with no visible key yet gets P = 0
+#pragma unroll
+        for (int c = 0; c < C::NC; ++c) {
+          const int k0 = C::kHR ? 32 * R.tsub : 32 * c;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float p[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              p[e] = ex2(sv[c][8 * q + e] - mref);
+              l += p[e];
+            }
+            st_bf16x8<BS>(pP, R.r, k0 + 8 * q, p);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < C::NC; ++c) {
+          float sv[32], dp[32];
+          const int k0 = R.ld_scores(tmem + C::qColS, c, sv);
+          R.ld_scores(tmem + C::qColP, c, dp);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float ds[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int k = k0 + 8 * q + e;
+              const float p = (diag && k > R.r) ? 0.f : ex2(sv[8 * q + e] * sl2 - lse2);
+              ds[e] = p * (dp[8 * q + e] - delta);
+            }
+            st_bf16x8<BS>(pP, R.r, k0 + 8 * q, ds);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        tc_fence_after();
+        // pass 1: O += P V (V MN-major); pass 2: dQ += dS K (K MN-major)
+        const uint32_t sB = pass2 ? sK : sV;
+        const bool first = pass2 ? n == nblk : n == 0;
+#pragma unroll
+        for (int kk = 0; kk < BS / 16; ++kk)
+          mma_bf16(tmem + C::qColO, kmaj<BS>(sP, kk), mnmaj<BS>(sB, kk), idPV, (!first || kk > 0) ? 1u : 0u);
+        mma_commit(BAR(bMM));
+      }
+      mm_pending = true;
+      mm_step = n;
+      if (n == nblk - 1) {
+        // End of pass 1: lse and Delta = <dO, O> / sum of each row.
+        if (!finish_mm()) { ok = false; break; }
+        tc_fence_after();
+        const float lt = R.row_sum(l);
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const __nv_bfloat16* dorow = static_cast<const __nv_bfloat16*>(a.dout) + ((tok0 + R.r) * a.Hq + hq) * D;
+        float dsum = 0.f;
+#pragma unroll
+        for (int pp = 0; pp < C::NP; ++pp)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            float o[C::W];
+            R.ld_d(tmem + C::qColO, pp, hf, o);
+            tmem_ld_wait();
+            dsum += dot_bf16<C::W>(o, dorow + (hf ? D / 2 : 0) + R.col_lo(pp));
+          }
+        delta = R.row_sum(dsum) * inv;
+        lse2 = lt > 0.f ? m2 + __log2f(lt) : INFINITY;
+        if (R.tsub == 0) {
+          a.lse[si0 + R.r] = lse2;
+          a.delta[si0 + R.r] = delta;
+        }
+      } else if (n == nsteps - 1) {
+        // End of pass 2: dq = R(t)^T (scale dQ).
+        if (!finish_mm()) { ok = false; break; }
+        tc_fence_after();
+        float* dqrow = a.dq + ((tok0 + R.r) * a.Hq + hq) * D;
+        const int t = j * BS + R.r;
+#pragma unroll
+        for (int pp = 0; pp < C::NP; ++pp) {
+          float lo[C::W], hi[C::W];
+          R.ld_d(tmem + C::qColO, pp, 0, lo);
+          R.ld_d(tmem + C::qColO, pp, 1, hi);
+          tmem_ld_wait();
+          rotate_store<C::W, D>(lo, hi, R.col_lo(pp), t, a.scale, ctl.om, dqrow);
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  if (!ok) {
+    if (threadIdx.x == 0) {
+      atomicExch(a.status, kDevWaitTimeout);
+      mma_commit(BAR(bFin));                      // arrives once every MMA issued so far is done
+      mbar_wait(BAR(bFin), 0, kBwWaitNs);
+      for (long long n = ld_use; n < ld_issue; ++n)
+        mbar_wait(BAR(bKV0 + static_cast<int>(n & 1)), static_cast<uint32_t>((n >> 1) & 1), kBwWaitNs);
+      if (q_pending) mbar_wait(BAR(bQ), phQ, kBwWaitNs);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (R.warp == 0) {
+    __syncwarp();
+    tmem_dealloc(tmem, C::qCols);
+  }
+}
+
+// -------------------------------------------------------------- dk/dv kernel
+template <int BS, int D>
+__global__ void __launch_bounds__(kBwThreads, 1)
+bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const BwdArgs a) {
+  using C = BwCfg<BS, D>;
+  using namespace tc;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicExch(a.status, kDevMisaligned);
+    return;
+  }
+  Ctl& ctl = *reinterpret_cast<Ctl*>(smem + C::bOffCtl);
+  const uint32_t base = smem_u32(smem);
+  const uint32_t sK = base + C::bOffK, sV = base + C::bOffV, sE = base + C::bOffE;
+  const uint32_t sPT = base + C::bOffPT, sDS = base + C::bOffDS;
+  uint8_t* pPT = smem + C::bOffPT;
+  uint8_t* pDS = smem + C::bOffDS;
+  enum { bKV = 0, bS = 1, bMM = 2, bFin = 3, bE0 = 4 };
+  auto BAR = [&](int i) { return smem_u32(&ctl.bar[i]); };
+  const Rows<BS, D> R;
+  if (R.warp == 0) {
+    tmem_alloc(smem_u32(&ctl.tmem), C::bCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < bE0 + C::kNE; ++i) mbar_init(BAR(i), 1);
+    fence_mbar_init();
+  }
+  if (threadIdx.x < D / 2) ctl.om[threadIdx.x] = a.inv_freq[threadIdx.x];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem;
+  grid_dependency_wait();          // lse, Delta (dq kernel) and the reverse index come from earlier kernels
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmO);
+  }
+
+  constexpr uint32_t idS = idesc_bf16_f32(BS, BS, 0, 0);
+  constexpr uint32_t idG = idesc_bf16_f32(BS, D, 0, 1);
+  const float sl2 = a.scale * 1.4426950408889634f;
+  const long long nkt = static_cast<long long>(a.B) * a.Hkv * a.nb;
+  const int g = a.Hq / a.Hkv;
+  uint32_t phKV = 0, phS = 0, phMM = 0;
+  long long e_issue = 0, e_use = 0;               // entry loads: slot = n % kNE, parity (n / kNE) & 1
+  bool mm_pending = false, ok = true, kv_pending = false;
+  int mm_x = 0;
+  auto wait_all = [&](int bar, uint32_t parity) -> bool {
+    const bool w = mbar_wait(BAR(bar), parity, kBwWaitNs);
+    return __syncthreads_and(w) != 0;
+  };
+
+  for (long long kt = blockIdx.x; kt < nkt && ok; kt += gridDim.x) {
+    const int i = static_cast<int>(kt % a.nb);
+    const long long bh = kt / a.nb;
+    const int h = static_cast<int>(bh % a.Hkv), b = static_cast<int>(bh / a.Hkv);
+    const int32_t* roff = a.rev_off + bh * (a.nb + 1);
+    const int32_t* rev = a.rev + bh * (static_cast<long long>(g) * a.nb * a.nsel);
+    const int e0 = roff[i], ne = roff[i + 1] - e0;
+    const long long tok0 = static_cast<long long>(b) * a.S + static_cast<long long>(i) * BS;
+    if (ne == 0) {                                // no query selected this block
+      for (int e = threadIdx.x; e < BS * D; e += kBwThreads) {
+        const long long o = ((tok0 + e / D) * a.Hkv + h) * D + e % D;
+        a.dk[o] = 0.f;
+        a.dv[o] = 0.f;
+      }
+      continue;
+    }
+    auto issue_e = [&](int x) {                   // entry x: Q, dO, lse, Delta of its query tile
+      if (threadIdx.x == 0) {
+        const int slot = static_cast<int>(e_issue % C::kNE);
+        const int code = rev[e0 + x];
+        const int hl = code / a.nb, jq = code - hl * a.nb, hq = h * g + hl;
+        const uint32_t bar = BAR(bE0 + slot), dst = sE + slot * C::kSlot;
+        const int row0 = static_cast<int>(static_cast<long long>(b) * a.S + static_cast<long long>(jq) * BS);
+        const long long si0 = (static_cast<long long>(b) * a.Hq + hq) * a.S + static_cast<long long>(jq) * BS;
+        mbar_expect_tx(bar, 2 * C::kTile + 2 * BS * 4);
+#pragma unroll
+        for (int gg = 0; gg < D / 64; ++gg) {
+          tma_load_3d(dst + gg * C::kRegion, &tmQ, bar, gg * 64, hq, row0);
+          tma_load_3d(dst + C::kTile + gg * C::kRegion, &tmO, bar, gg * 64, hq, row0);
+        }
+        bulk_load(dst + 2 * C::kTile, a.lse + si0, BS * 4, bar);
+        bulk_load(dst + 2 * C::kTile + BS * 4, a.delta + si0, BS * 4, bar);
+      }
+      ++e_issue;
+    };
+    auto finish_mm = [&]() -> bool {
+      if (!mm_pending) return true;
+      if (!wait_all(bMM, phMM)) return false;
+      phMM ^= 1;
+      mm_pending = false;
+      if (mm_x + C::kNE < ne) issue_e(mm_x + C::kNE);
+      return true;
+    };
+    __syncthreads();                              // the previous tile's tensor memory reads are done
+    if (threadIdx.x == 0) {
+      mbar_expect_tx(BAR(bKV), 2 * C::kTile);
+#pragma unroll
+      for (int gg = 0; gg < D / 64; ++gg) {
+        tma_load_3d(sK + gg * C::kRegion, &tmK, BAR(bKV), gg * 64, h, static_cast<int>(tok0));
+        tma_load_3d(sV + gg * C::kRegion, &tmV, BAR(bKV), gg * 64, h, static_cast<int>(tok0));
+      }
+    }
+    kv_pending = true;
+    for (int x = 0; x < C::kNE && x < ne; ++x) issue_e(x);
+    if (!wait_all(bKV, phKV)) { ok = false; break; }
+    phKV ^= 1;
+    kv_pending = false;
+    for (int x = 0; x < ne && ok; ++x) {
+      const int slot = static_cast<int>(e_use % C::kNE);
+      if (!wait_all(bE0 + slot, static_cast<uint32_t>((e_use / C::kNE) & 1))) { ok = false; break; }
+      ++e_use;
+      const int code = rev[e0 + x];
+      const int jq = code % a.nb;
+      const uint32_t sQe = sE + slot * C::kSlot, sOe = sQe + C::kTile;
+      const float* lse_s = reinterpret_cast<const float*>(smem + C::bOffE + slot * C::kSlot + 2 * C::kTile);
+      const float* del_s = lse_s + BS;
+      if (threadIdx.x == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16(tmem + C::bColS, kmaj<BS>(sK, kk), kmaj<BS>(sQe, kk), idS, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) mma_bf16(tmem + C::bColP, kmaj<BS>(sV, kk), kmaj<BS>(sOe, kk), idS, kk > 0);
+        mma_commit(BAR(bS));
+      }
+      if (!wait_all(bS, phS)) { ok = false; break; }
+      phS ^= 1;
+      if (!finish_mm()) { ok = false; break; }     // the P^T, dS^T buffers are free
+      tc_fence_after();
+      const bool diag = jq == i;
+#pragma unroll
+      for (int c = 0; c < C::NC; ++c) {
+        float sv[32], dp[32];
+        const int t0 = R.ld_scores(tmem + C::bColS, c, sv);
+        R.ld_scores(tmem + C::bColP, c, dp);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float p[8], ds[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int t = t0 + 8 * q + e;
+            p[e] = (diag && t < R.r) ? 0.f : ex2(sv[8 * q + e] * sl2 - lse_s[t]);
+            ds[e] = p[e] * (dp[8 * q + e] - del_s[t]);
+          }
+          st_bf16x8<BS>(pPT, R.r, t0 + 8 * q, p);
+          st_bf16x8<BS>(pDS, R.r, t0 + 8 * q, ds);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BS / 16; ++kk)
+          mma_bf16(tmem + C::bColV, kmaj<BS>(sPT, kk), mnmaj<BS>(sOe, kk), idG, (x > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < BS / 16; ++kk)
+          mma_bf16(tmem + C::bColK, kmaj<BS>(sDS, kk), mnmaj<BS>(sQe, kk), idG, (x > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(BAR(bMM));
+      }
+      mm_pending = true;
+      mm_x = x;
+    }
+    if (!ok) break;
+    if (!finish_mm()) { ok = false; break; }
+    tc_fence_after();
+    // dv = dV; dk = R(s)^T (scale dK).
+    const long long krow = (tok0 + R.r) * a.Hkv + h;
+    const int s = i * BS + R.r;
+#pragma unroll
+    for (int pp = 0; pp < C::NP; ++pp) {
+      float lo[C::W], hi[C::W];
+      R.ld_d(tmem + C::bColV, pp, 0, lo);
+      R.ld_d(tmem + C::bColV, pp, 1, hi);
+      tmem_ld_wait();
+      store_f32<C::W>(a.dv + krow * D + R.col_lo(pp), lo);
+      store_f32<C::W>(a.dv + krow * D + D / 2 + R.col_lo(pp), hi);
+      R.ld_d(tmem + C::bColK, pp, 0, lo);
+      R.ld_d(tmem + C::bColK, pp, 1, hi);
+      tmem_ld_wait();
+      rotate_store<C::W, D>(lo, hi, R.col_lo(pp), s, a.scale, ctl.om, a.dk + krow * D);
+    }
+    tc_fence_before();
+  }
+
+  if (!ok) {
+    if (threadIdx.x == 0) {
+      atomicExch(a.status, kDevWaitTimeout);
+      mma_commit(BAR(bFin));
+      mbar_wait(BAR(bFin), 0, kBwWaitNs);
+      if (kv_pending) mbar_wait(BAR(bKV), phKV, kBwWaitNs);
+      for (long long n = e_use; n < e_issue; ++n)
+        mbar_wait(BAR(bE0 + static_cast<int>(n % C::kNE)), static_cast<uint32_t>((n / C::kNE) & 1), kBwWaitNs);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (R.warp == 0) {
+    __syncwarp();
+    tmem_dealloc(tmem, C::bCols);
+  }
+}
+
+namespace {
+
+template <typename K>
+cudaError_t launch_persistent(K kernel, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                              const CUtensorMap& mo, const BwdArgs& a, long long ntiles, int smem, int cols,
+                              cudaStream_t st) {
+  cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(kernel), smem);
+  if (e != cudaSuccess) return e;
+  const int sms = cached_sm_count();
+  int per_sm = cached_occupancy(reinterpret_cast<const void*>(kernel), kBwThreads, smem);
+  if (sms <= 0) return cudaErrorUnknown;
+  per_sm = per_sm < 512 / cols ? per_sm : 512 / cols;    // tensor memory: 512 columns per SM
+  if (per_sm < 1) per_sm = 1;
+  const long long want = static_cast<long long>(sms) * per_sm;
+  const unsigned grid = static_cast<unsigned>(ntiles < want ? ntiles : want);
+  if (grid == 0) return cudaSuccess;
+  return launch_pdl(kernel, dim3(grid), dim3(kBwThreads), static_cast<size_t>(smem), st, mq, mk, mv, mo, a);
+}
+
+template <int BS, int D>
+cudaError_t launch_tc_bwd(const BwdArgs& a, cudaStream_t st) {
+  using C = BwCfg<BS, D>;
+  CUtensorMap mq, mk, mv, mo;
+  const long long rows = static_cast<long long>(a.B) * a.S;
+  if (!make_tile_map(&mq, a.qrot, rows, a.Hq, D, BS) || !make_tile_map(&mk, a.krot, rows, a.Hkv, D, BS) ||
+      !make_tile_map(&mv, a.v, rows, a.Hkv, D, BS) || !make_tile_map(&mo, a.dout, rows, a.Hq, D, BS))
+    return cudaErrorInvalidValue;
+  cudaError_t e = launch_persistent(bwd_dq_tc_kernel<BS, D>, mq, mk, mv, mo, a,
+                                    static_cast<long long>(a.B) * a.Hq * a.nb, C::qSmem, C::qCols, st);
+  if (e != cudaSuccess) return e;
+  return launch_persistent(bwd_dkdv_tc_kernel<BS, D>, mq, mk, mv, mo, a,
+                           static_cast<long long>(a.B) * a.Hkv * a.nb, C::bSmem, C::bCols, st);
+}
+
+}  // namespace
+
+cudaError_t launch_backward_tc(const BwdArgs& a, cudaStream_t st) {
+  cudaError_t e = launch_bwd_rev(a, st);
+  if (e != cudaSuccess) return e;
+  if (a.bs == 64 && a.D == 64) e = launch_tc_bwd<64, 64>(a, st);
+  else if (a.bs == 64 && a.D == 128) e = launch_tc_bwd<64, 128>(a, st);
+  else if (a.bs == 128 && a.D == 64) e = launch_tc_bwd<128, 64>(a, st);
+  else if (a.bs == 128 && a.D == 128) e = launch_tc_bwd<128, 128>(a, st);
+  else return cudaErrorInvalidValue;
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace mdr

@@ -150,8 +150,10 @@ struct BwdArgs {
   const void* v;           // [B,S,Hkv,D]
   const void* dout;        // [B,S,Hq,D] upstream gradient, storage type
   const int32_t* sel;      // [B,Hq,nb,nsel]
-  float* qr;               // scratch: rotated q, float32 [B,S,Hq,D]
-  float* kr;               // scratch: rotated k, float32 [B,S,Hkv,D]
+  float* qr;               // scratch: rotated q, float32 [B,S,Hq,D] (CUDA-core path)
+  float* kr;               // scratch: rotated k, float32 [B,S,Hkv,D] (CUDA-core path)
+  const void* qrot;        // rotated q in the storage type [B,S,Hq,D] (tensor-core path)
+  const void* krot;        // rotated k in the storage type [B,S,Hkv,D] (tensor-core path)
   float* lse;              // scratch: [B,Hq,S] log-sum-exp of the scaled scores
   float* delta;            // scratch: [B,Hq,S] dout_t . out_t
   int32_t* rev_off;        // scratch: [B,Hkv,nb+1] reverse-index offsets
@@ -165,6 +167,12 @@ struct BwdArgs {
   float inv_freq[64];
 };
 size_t bwd_rev_smem(int nb);
+// Float32 storage: rotated float32 copies, reverse index, dq and dk/dv on the CUDA cores.
 cudaError_t launch_backward(const BwdArgs& a, bool bf16, cudaStream_t st);
+// Reverse index of the selection (key block -> selecting (query head, query block)).
+cudaError_t launch_bwd_rev(const BwdArgs& a, cudaStream_t st);
+// Bf16 storage, bs in {64,128}, D in {64,128}: reverse index, then dq and
+// dk/dv on the tensor cores over qrot, krot (written by the summary kernel).
+cudaError_t launch_backward_tc(const BwdArgs& a, cudaStream_t st);
 
 }  // namespace mdr

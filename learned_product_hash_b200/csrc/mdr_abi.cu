@@ -552,6 +552,10 @@ mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void*
   if (static_cast<long long>(cfg->B) * cfg->Hq * (cfg->S / cfg->block) * (cfg->block / 16) > INT32_MAX)
     return MDR_ERR_UNSUPPORTED;
   if (mdr::bwd_rev_smem(cfg->S / cfg->block) > kMaxDynamicSmem) return MDR_ERR_UNSUPPORTED;   // reverse index
+  const bool tc = cfg->dtype == MDR_BF16;          // tensor cores (block and D in {64,128} for bf16)
+  if (tc && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
+             !aligned16(dk) || !aligned16(dv)))
+    return MDR_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   MDR_CUDA(cudaMemsetAsync(at<int32_t>(ws, l.status), 0, sizeof(int32_t), st));
   mdr::BwdArgs a;
@@ -565,7 +569,17 @@ mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void*
   a.nb = cfg->S / cfg->block; a.nsel = cfg->R + cfg->L;
   a.scale = mdr::detail::softmax_scale(cfg);
   mdr::detail::fill_inv_freq(a.inv_freq, cfg);
-  return cuda_status(mdr::launch_backward(a, cfg->dtype == MDR_BF16, st));
+  if (!tc) return cuda_status(mdr::launch_backward(a, false, st));
+  // The rotated copies in the storage type, by the summary kernel (the
+  // operands the forward's attention reads), into the float32 regions.
+  SummarizeArgs sa;
+  fill_common(sa, cfg, nullptr);
+  sa.x[0] = q; sa.x[1] = k;
+  sa.xrot[0] = a.qr; sa.xrot[1] = a.kr;
+  sa.status = a.status;
+  MDR_CUDA(mdr::launch_summarize(sa, true, st));
+  a.qrot = a.qr; a.krot = a.kr;
+  return cuda_status(mdr::launch_backward_tc(a, st));
 }
 
 // ------------------------------------------------------ codebook calibration
