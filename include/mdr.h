@@ -341,8 +341,12 @@ mdr_status mdr_read_device_status(const void* ws, int32_t* code, void* stream);
  * q, k, v: device [B,S,H,D] in cfg->dtype (not rotated: the inputs of
  * mdr_forward); sel: device int32 [B,Hq,nb,R+L] as written by a route call;
  * dout: device [B,S,Hq,D] in cfg->dtype; dq [B,S,Hq,D], dk and dv
- * [B,S,Hkv,D]: device float32, written (not accumulated).  Arithmetic is
- * float32 in a fixed order (deterministic).  ws: device, 256-byte aligned,
+ * [B,S,Hkv,D]: device float32, written (not accumulated).  MDR_BF16: the
+ * four products run on the tensor cores (tcgen05) with bfloat16 operands --
+ * the rotated q', k' the forward uses, and the weights P, dS -- accumulated
+ * in float32 (q, k, v, dout, dq, dk, dv 16-byte aligned, else
+ * MDR_ERR_INVALID_ARG); MDR_F32: float32 on the CUDA cores.  Either way the
+ * sums run in a fixed order (deterministic).  ws: device, 256-byte aligned,
  * at least mdr_backward_workspace_bytes; its first word is the device
  * status (2: a selected id later than its query block, skipped), read with
  * mdr_read_device_status.  Supported up to 29,000 blocks per sequence

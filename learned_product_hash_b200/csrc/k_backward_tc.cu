@@ -48,7 +48,20 @@ namespace mdr {
 namespace {
 
 constexpr uint64_t kBwWaitNs = 2000000000ull;
+constexpr uint64_t kBwBudgetNs = 10000000000ull;  // a CTA gives up after 10 s of wall time in total
 constexpr int kBwThreads = 128;
+
+// Where a CTA gave up, recorded (first one wins) in the second status word:
+// 100 * kernel (1 dq, 2 dk/dv) + site, plus 50 when the CTA's time budget ran
+// out rather than the wait itself; site 90+ are index checks that failed.
+enum BwSite : int {
+  kSiteQ = 1, kSiteKV = 2, kSiteS = 3, kSiteMM = 4, kSiteEntry = 5,
+  kSiteRevRange = 90, kSiteRevCode = 91,
+};
+
+__device__ __forceinline__ void record_site(int32_t* status, int code) {
+  atomicCAS(status + 1, 0, code);
+}
 
 constexpr int pow2_cols(int c) { return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512; }
 
@@ -274,10 +287,14 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   bool mm_pending = false, ok = true, q_pending = false;
   int mm_step = 0;
 
-  // Wait for a barrier phase in every thread; false (everywhere) if any gave up.
-  auto wait_all = [&](int bar, uint32_t parity) -> bool {
+  const uint64_t t_start = globaltimer();
+  // Wait for a barrier phase in every thread; false (everywhere) if any gave
+  // up or the CTA's time budget ran out; the site is recorded.
+  auto wait_all = [&](int bar, uint32_t parity, int site) -> bool {
     const bool w = mbar_wait(BAR(bar), parity, kBwWaitNs);
-    return __syncthreads_and(w) != 0;
+    const bool in_time = globaltimer() - t_start <= kBwBudgetNs;
+    if (!(w && in_time)) record_site(a.status, 100 + site + (w ? 50 : 0));
+    return __syncthreads_and(w && in_time) != 0;
   };
 
   for (long long tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
@@ -328,7 +345,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // step mm_step + 2.
     auto finish_mm = [&]() -> bool {
       if (!mm_pending) return true;
-      if (!wait_all(bMM, phMM)) return false;
+      if (!wait_all(bMM, phMM, kSiteMM)) return false;
       phMM ^= 1;
       mm_pending = false;
       if (mm_step + 2 < nsteps) issue_kv(mm_step + 2);
@@ -345,7 +362,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     q_pending = true;
     issue_kv(0);
     issue_kv(1);
-    if (!wait_all(bQ, phQ)) { ok = false; break; }
+    if (!wait_all(bQ, phQ, kSiteQ)) { ok = false; break; }
     phQ ^= 1;
     q_pending = false;
     float m2 = -INFINITY, l = 0.f, lse2 = 0.f, delta = 0.f;
@@ -353,7 +370,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const bool pass2 = n >= nblk;
       const int blk = ctl.ids[n % nblk];
       const int slot = static_cast<int>(ld_use & 1);
-      if (!wait_all(bKV0 + slot, static_cast<uint32_t>((ld_use >> 1) & 1))) { ok = false; break; }
+      if (!wait_all(bKV0 + slot, static_cast<uint32_t>((ld_use >> 1) & 1), kSiteKV)) { ok = false; break; }
       ++ld_use;
       const uint32_t sK = sKV + slot * 2 * C::kTile, sV = sK + C::kTile;
       if (threadIdx.x == 0) {
@@ -366,7 +383,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         mma_commit(BAR(bS));
       }
-      if (!wait_all(bS, phS)) { ok = false; break; }
+      if (!wait_all(bS, phS, kSiteS)) { ok = false; break; }
       phS ^= 1;
       if (!finish_mm()) { ok = false; break; }     // O (or dQ) and the P buffer are free
       tc_fence_after();
@@ -568,9 +585,12 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   long long e_issue = 0, e_use = 0;               // entry loads: slot = n % kNE, parity (n / kNE) & 1
   bool mm_pending = false, ok = true, kv_pending = false;
   int mm_x = 0;
-  auto wait_all = [&](int bar, uint32_t parity) -> bool {
+  const uint64_t t_start = globaltimer();
+  auto wait_all = [&](int bar, uint32_t parity, int site) -> bool {
     const bool w = mbar_wait(BAR(bar), parity, kBwWaitNs);
-    return __syncthreads_and(w) != 0;
+    const bool in_time = globaltimer() - t_start <= kBwBudgetNs;
+    if (!(w && in_time)) record_site(a.status, 200 + site + (w ? 50 : 0));
+    return __syncthreads_and(w && in_time) != 0;
   };
 
   for (long long kt = blockIdx.x; kt < nkt && ok; kt += gridDim.x) {
@@ -579,7 +599,16 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int h = static_cast<int>(bh % a.Hkv), b = static_cast<int>(bh / a.Hkv);
     const int32_t* roff = a.rev_off + bh * (a.nb + 1);
     const int32_t* rev = a.rev + bh * (static_cast<long long>(g) * a.nb * a.nsel);
-    const int e0 = roff[i], ne = roff[i + 1] - e0;
+    const long long E = static_cast<long long>(g) * a.nb * a.nsel;   // entries of this (b, hkv)
+    const int e0 = roff[i];
+    int ne = roff[i + 1] - e0;
+    if (e0 < 0 || ne < 0 || e0 + static_cast<long long>(ne) > E) {  // never for a reverse index of this call
+      if (threadIdx.x == 0) {
+        atomicExch(a.status, kDevBadSelection);
+        record_site(a.status, 200 + kSiteRevRange);
+      }
+      ne = 0;
+    }
     const long long tok0 = static_cast<long long>(b) * a.S + static_cast<long long>(i) * BS;
     if (ne == 0) {                                // no query selected this block
       for (int e = threadIdx.x; e < BS * D; e += kBwThreads) {
@@ -592,7 +621,12 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     auto issue_e = [&](int x) {                   // entry x: Q, dO, lse, Delta of its query tile
       if (threadIdx.x == 0) {
         const int slot = static_cast<int>(e_issue % C::kNE);
-        const int code = rev[e0 + x];
+        int code = rev[e0 + x];
+        if (code < 0 || code >= g * a.nb) {        // never for a reverse index of this call
+          atomicExch(a.status, kDevBadSelection);
+          record_site(a.status, 200 + kSiteRevCode);
+          code = 0;
+        }
         const int hl = code / a.nb, jq = code - hl * a.nb, hq = h * g + hl;
         const uint32_t bar = BAR(bE0 + slot), dst = sE + slot * C::kSlot;
         const int row0 = static_cast<int>(static_cast<long long>(b) * a.S + static_cast<long long>(jq) * BS);
@@ -610,7 +644,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     };
     auto finish_mm = [&]() -> bool {
       if (!mm_pending) return true;
-      if (!wait_all(bMM, phMM)) return false;
+      if (!wait_all(bMM, phMM, kSiteMM)) return false;
       phMM ^= 1;
       mm_pending = false;
       if (mm_x + C::kNE < ne) issue_e(mm_x + C::kNE);
@@ -627,15 +661,18 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
     kv_pending = true;
     for (int x = 0; x < C::kNE && x < ne; ++x) issue_e(x);
-    if (!wait_all(bKV, phKV)) { ok = false; break; }
+    if (!wait_all(bKV, phKV, kSiteKV)) { ok = false; break; }
     phKV ^= 1;
     kv_pending = false;
     for (int x = 0; x < ne && ok; ++x) {
+      // Entry x is issued when the MMAs of entry x - kNE finish; with a single
+      // slot that is the previous entry's, so wait for them here first.
+      if (e_issue == e_use && !finish_mm()) { ok = false; break; }
       const int slot = static_cast<int>(e_use % C::kNE);
-      if (!wait_all(bE0 + slot, static_cast<uint32_t>((e_use / C::kNE) & 1))) { ok = false; break; }
+      if (!wait_all(bE0 + slot, static_cast<uint32_t>((e_use / C::kNE) & 1), kSiteEntry)) { ok = false; break; }
       ++e_use;
       const int code = rev[e0 + x];
-      const int jq = code % a.nb;
+      const int jq = (code < 0 ? 0 : code) % a.nb;
       const uint32_t sQe = sE + slot * C::kSlot, sOe = sQe + C::kTile;
       const float* lse_s = reinterpret_cast<const float*>(smem + C::bOffE + slot * C::kSlot + 2 * C::kTile);
       const float* del_s = lse_s + BS;
@@ -647,7 +684,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (int kk = 0; kk < D / 16; ++kk) mma_bf16(tmem + C::bColP, kmaj<BS>(sV, kk), kmaj<BS>(sOe, kk), idS, kk > 0);
         mma_commit(BAR(bS));
       }
-      if (!wait_all(bS, phS)) { ok = false; break; }
+      if (!wait_all(bS, phS, kSiteS)) { ok = false; break; }
       phS ^= 1;
       if (!finish_mm()) { ok = false; break; }     // the P^T, dS^T buffers are free
       tc_fence_after();

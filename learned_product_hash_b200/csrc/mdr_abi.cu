@@ -557,7 +557,8 @@ mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void*
              !aligned16(dk) || !aligned16(dv)))
     return MDR_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  MDR_CUDA(cudaMemsetAsync(at<int32_t>(ws, l.status), 0, sizeof(int32_t), st));
+  // the status word and, for the tensor-core kernels, where a CTA gave up
+  MDR_CUDA(cudaMemsetAsync(at<int32_t>(ws, l.status), 0, 4 * sizeof(int32_t), st));
   mdr::BwdArgs a;
   std::memset(&a, 0, sizeof(a));
   a.q = q; a.k = k; a.v = v; a.dout = dout; a.sel = sel;

@@ -190,3 +190,18 @@ def test_backward_entry_point_checks_arguments_before_any_gpu_work():
     big = mdr.make_config(TINY.with_(S=30000 * 16))                           # 30,000 blocks
     nbig = mdr.mdr_backward_workspace_bytes(big)
     assert call(cfg=big, nbytes=nbig) == mdr.MDR_ERR_UNSUPPORTED
+
+
+def test_backward_tensor_core_path_checks_alignment_before_any_gpu_work():
+    """bf16 storage runs on the tensor cores, whose TMA loads need 16-byte
+    aligned tensors: a misaligned input or gradient is refused on the host."""
+    from workloads import AR
+    L = mdr.lib()
+    cfg = mdr.make_config(AR)
+    n = mdr.mdr_backward_workspace_bytes(cfg)
+    ok, bad = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10008)
+    ws = ctypes.c_void_p(0x100000)
+    for i in (0, 1, 2, 4, 5, 6, 7):        # q, k, v, dout, dq, dk, dv (sel may have any alignment)
+        args = [ok] * 8
+        args[i] = bad
+        assert L.mdr_attend_backward(ctypes.byref(cfg), *args, ws, n, None) == mdr.MDR_ERR_INVALID_ARG, i

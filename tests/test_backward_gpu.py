@@ -50,6 +50,8 @@ def gpu_backward(w, inp, dout_store, sel):
     ws = mdr.backward_workspace(cfg)
     mdr.mdr_attend_backward(cfg, q, k, v, s, do, dq, dk, dv, ws)
     status = mdr.mdr_read_device_status(ws)
+    if status != 0:      # the second word says where a tensor-core CTA gave up
+        print(f"backward status {status}, site {int(ws[:16].view(torch.int32)[1].item())}")
     return dq.cpu().numpy(), dk.cpu().numpy(), dv.cpu().numpy(), status
 
 
