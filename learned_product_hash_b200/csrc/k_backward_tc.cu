@@ -403,24 +403,28 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           }
         }
         mx = R.row_max(mx);
-        if (mx > m2) {
-          if (n > 0) {
-            const float alpha = ex2(m2 - mx);
-            l *= alpha;
-#pragma unroll
-            for (int pp = 0; pp < C::NP; ++pp)
-#pragma unroll
-              for (int hf = 0; hf < 2; ++hf) {
-                float o[C::W];
-                R.ld_d(tmem + C::qColO, pp, hf, o);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < C::W; ++e) o[e] *= alpha;
-                R.st_d(tmem + C::qColO, pp, hf, o);
-              }
-            tmem_st_wait();
-          }
+        const bool grow = mx > m2;
+        const float alpha = (grow && n > 0) ? ex2(m2 - mx) : 1.f;   // 1 for rows whose maximum stays
+        if (grow) {
+          l *= alpha;
           m2 = mx;
+        }
+        // tcgen05.ld / tcgen05.st are warp-collective (.sync.aligned): the
+        // whole warp rescales its rows' O when any of them grew, the others
+        // by 1, so no lane skips an instruction another lane executes.
+        if (n > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll
+          for (int pp = 0; pp < C::NP; ++pp)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              float o[C::W];
+              R.ld_d(tmem + C::qColO, pp, hf, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < C::W; ++e) o[e] *= alpha;
+              R.st_d(tmem + C::qColO, pp, hf, o);
+            }
+          tmem_st_wait();
         }
         const float mref = m2 == -INFINITY ? 0.f : m2;   // a row with no visible key yet gets P = 0
 #pragma unroll
