@@ -31,7 +31,7 @@
 // subpartition w (accumulator rows 16w..16w+15 for bs = 64, two threads per
 // row splitting the columns; rows 32w..32w+31 for bs = 128).  Thread 0 issues
 // the TMA loads and the MMAs; the next block's (or entry's) tiles are loaded
-// while the current one is computed.  Sums run in a fixed order and there
+// while the current one is computed (a ring of several slots per CTA).  Sums run in a fixed order and there
 // are no atomics, so a call is deterministic.  Every wait is bounded (2 s of
 // wall time): a wait that runs out writes status 1, the CTA waits (bounded)
 // for its own copies and MMAs, frees its tensor memory and returns.
@@ -72,17 +72,19 @@ struct BwCfg {
   static constexpr int kRegion = BS * 128;           // one 64-column region of a [BS x *] tile
   static constexpr int kPTile = BS * BS * 2;         // bf16 [BS x BS]: BS/64 regions
   static constexpr int kCtl = 1024;                  // barriers, omega, ids, misc
-  // dq kernel: Q, dO, two (K, V) slots, P / dS
+  // dq kernel: Q, dO, NKV (K, V) slots, P / dS.  The slots hold the next
+  // blocks' tiles in flight while the current one computes (one CTA per SM).
+  static constexpr int NKV = (BS == 128 && D == 128) ? 2 : (BS == 64 && D == 64) ? 6 : 5;
   static constexpr int qOffQ = 0;
   static constexpr int qOffO = kTile;
   static constexpr int qOffKV = 2 * kTile;
-  static constexpr int qOffP = qOffKV + 4 * kTile;
+  static constexpr int qOffP = qOffKV + NKV * 2 * kTile;
   static constexpr int qOffCtl = qOffP + kPTile;
   static constexpr int qSmem = qOffCtl + kCtl;
   static constexpr int qCols = pow2_cols(2 * BS + D);
   static constexpr int qColS = 0, qColP = BS, qColO = 2 * BS;
   // dk/dv kernel: K, V, kNE entry slots (Q, dO, lse, Delta), P^T, dS^T
-  static constexpr int kNE = (BS == 128 && D == 128) ? 1 : 3;
+  static constexpr int kNE = (BS == 128 && D == 128) ? 1 : (BS == 128) ? 3 : (D == 64) ? 6 : 5;
   static constexpr int kSlot = (2 * kTile + 2 * BS * 4 + 1023) / 1024 * 1024;
   static constexpr int bOffK = 0, bOffV = kTile, bOffE = 2 * kTile;
   static constexpr int bOffPT = bOffE + kNE * kSlot;
@@ -252,7 +254,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const uint32_t base = smem_u32(smem);
   const uint32_t sQ = base + C::qOffQ, sO = base + C::qOffO, sKV = base + C::qOffKV, sP = base + C::qOffP;
   uint8_t* pP = smem + C::qOffP;
-  enum { bQ = 0, bKV0 = 1, bS = 3, bMM = 4, bFin = 5 };
+  enum { bQ = 0, bS = 1, bMM = 2, bFin = 3, bKV0 = 4 };     // bKV0 .. bKV0 + NKV - 1
+  static_assert(bKV0 + C::NKV <= 16, "barrier space");
   auto BAR = [&](int i) { return smem_u32(&ctl.bar[i]); };
   const Rows<BS, D> R;
   if (R.warp == 0) {
@@ -260,7 +263,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     tmem_relinquish();
   }
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 6; ++i) mbar_init(BAR(i), 1);
+    for (int i = 0; i < bKV0 + C::NKV; ++i) mbar_init(BAR(i), 1);
     fence_mbar_init();
     ctl.abort = 0;
   }
@@ -283,7 +286,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const long long ntiles = static_cast<long long>(a.B) * a.Hq * a.nb;
   const int g = a.Hq / a.Hkv;
   uint32_t phQ = 0, phS = 0, phMM = 0;
-  long long ld_issue = 0, ld_use = 0;             // (K, V) loads: slot = n & 1, parity (n >> 1) & 1
+  long long ld_issue = 0, ld_use = 0;             // (K, V) loads: slot = n % NKV, parity (n / NKV) & 1
   bool mm_pending = false, ok = true, q_pending = false;
   int mm_step = 0;
 
@@ -327,9 +330,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       continue;
     }
     const int nsteps = 2 * nblk;                  // pass 1 then pass 2 over the same blocks
-    auto issue_kv = [&](int n) {                  // K, V of step n into slot ld_issue & 1
+    auto issue_kv = [&](int n) {                  // K, V of step n into slot ld_issue % NKV
       if (threadIdx.x == 0) {
-        const int slot = static_cast<int>(ld_issue & 1);
+        const int slot = static_cast<int>(ld_issue % C::NKV);
         const uint32_t bar = BAR(bKV0 + slot), dst = sKV + slot * 2 * C::kTile;
         const int blk = ctl.ids[n % nblk];
         mbar_expect_tx(bar, 2 * C::kTile);
@@ -342,13 +345,13 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       ++ld_issue;
     };
     // The MMA of step mm_step (PV or dQ) has completed: its slot is free for
-    // step mm_step + 2.
+    // step mm_step + NKV.
     auto finish_mm = [&]() -> bool {
       if (!mm_pending) return true;
       if (!wait_all(bMM, phMM, kSiteMM)) return false;
       phMM ^= 1;
       mm_pending = false;
-      if (mm_step + 2 < nsteps) issue_kv(mm_step + 2);
+      if (mm_step + C::NKV < nsteps) issue_kv(mm_step + C::NKV);
       return true;
     };
     if (threadIdx.x == 0) {
@@ -360,8 +363,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
     }
     q_pending = true;
-    issue_kv(0);
-    issue_kv(1);
+    for (int n = 0; n < C::NKV && n < nsteps; ++n) issue_kv(n);
     if (!wait_all(bQ, phQ, kSiteQ)) { ok = false; break; }
     phQ ^= 1;
     q_pending = false;
@@ -369,8 +371,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     for (int n = 0; n < nsteps && ok; ++n) {
       const bool pass2 = n >= nblk;
       const int blk = ctl.ids[n % nblk];
-      const int slot = static_cast<int>(ld_use & 1);
-      if (!wait_all(bKV0 + slot, static_cast<uint32_t>((ld_use >> 1) & 1), kSiteKV)) { ok = false; break; }
+      const int slot = static_cast<int>(ld_use % C::NKV);
+      if (!wait_all(bKV0 + slot, static_cast<uint32_t>((ld_use / C::NKV) & 1), kSiteKV)) { ok = false; break; }
       ++ld_use;
       const uint32_t sK = sKV + slot * 2 * C::kTile, sV = sK + C::kTile;
       if (threadIdx.x == 0) {
@@ -524,7 +526,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mma_commit(BAR(bFin));                      // arrives once every MMA issued so far is done
       mbar_wait(BAR(bFin), 0, kBwWaitNs);
       for (long long n = ld_use; n < ld_issue; ++n)
-        mbar_wait(BAR(bKV0 + static_cast<int>(n & 1)), static_cast<uint32_t>((n >> 1) & 1), kBwWaitNs);
+        mbar_wait(BAR(bKV0 + static_cast<int>(n % C::NKV)), static_cast<uint32_t>((n / C::NKV) & 1), kBwWaitNs);
       if (q_pending) mbar_wait(BAR(bQ), phQ, kBwWaitNs);
     }
   }
@@ -556,7 +558,8 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const uint32_t sPT = base + C::bOffPT, sDS = base + C::bOffDS;
   uint8_t* pPT = smem + C::bOffPT;
   uint8_t* pDS = smem + C::bOffDS;
-  enum { bKV = 0, bS = 1, bMM = 2, bFin = 3, bE0 = 4 };
+  enum { bKV = 0, bS = 1, bMM = 2, bFin = 3, bE0 = 4 };     // bE0 .. bE0 + kNE - 1
+  static_assert(bE0 + C::kNE <= 16, "barrier space");
   auto BAR = [&](int i) { return smem_u32(&ctl.bar[i]); };
   const Rows<BS, D> R;
   if (R.warp == 0) {
@@ -776,6 +779,11 @@ cudaError_t launch_persistent(K kernel, const CUtensorMap& mq, const CUtensorMap
                               const CUtensorMap& mo, const BwdArgs& a, long long ntiles, int smem, int cols,
                               cudaStream_t st) {
   cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(kernel), smem);
+  if (e != cudaSuccess) return e;
+  // All of the unified L1 / shared storage as shared memory (these kernels
+  // read their operands through TMA, not L1).
+  e = cudaFuncSetAttribute(reinterpret_cast<const void*>(kernel), cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   const int sms = cached_sm_count();
   int per_sm = cached_occupancy(reinterpret_cast<const void*>(kernel), kBwThreads, smem);
