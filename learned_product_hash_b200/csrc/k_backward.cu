@@ -115,16 +115,30 @@ __global__ void __launch_bounds__(256) bwd_rev_kernel(const BwdArgs a) {
   for (int i = threadIdx.x; i <= a.nb; i += blockDim.x) roff[i] = off[i];
   for (int i = threadIdx.x; i < a.nb; i += blockDim.x) cnt[i] = 0;   // reused as fill counters
   __syncthreads();
-  // Stable placement: entries in (hl, j, slot) order, 32 per step.
+  // Stable placement: entries in (hl, j, slot) order, 32 per step; the
+  // selection is read four steps at a time so the loads overlap.
   if (warp == 0) {
     int32_t* rev = a.rev + static_cast<long long>(blockIdx.x) * E;
+    int ahead[4];
     for (long long base = 0; base < E; base += 32) {
+      const int u = static_cast<int>((base >> 5) & 3);
+      if (u == 0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const long long e = base + 32 * q + lane;
+          ahead[q] = e < E ? sel0[e] : -1;
+        }
+      }
+      int loaded = ahead[0];
+#pragma unroll
+      for (int q = 1; q < 4; ++q)
+        if (q == u) loaded = ahead[q];
       const long long e = base + lane;
       int id = -1, j = 0, hl = 0;
       if (e < E) {
         j = static_cast<int>((e / a.nsel) % a.nb);
         hl = static_cast<int>(e / (static_cast<long long>(a.nsel) * a.nb));
-        id = sel0[e];
+        id = loaded;
         if (id > j) id = -1;
       }
       const bool ok = id >= 0;
