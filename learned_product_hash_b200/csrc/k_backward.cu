@@ -80,14 +80,14 @@ __global__ void __launch_bounds__(256) bwd_rev_kernel(const BwdArgs a) {
   int* off = rsm + a.nb;                           // [nb + 1]
   const int b = blockIdx.x / a.Hkv, h = blockIdx.x % a.Hkv;
   const int g = a.Hq / a.Hkv;
-  const long long E = static_cast<long long>(g) * a.nb * a.nsel;   // entries (hl, j, slot)
+  const int E = g * a.nb * a.nsel;                 // entries (hl, j, slot); < 2^31 (checked on the host)
   const int32_t* sel0 = a.sel + (static_cast<long long>(b) * a.Hq + static_cast<long long>(h) * g) * a.nb * a.nsel;
   for (int i = threadIdx.x; i < a.nb; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   grid_dependency_wait();                          // sel may come from the previous kernel
   // Counts (order-free).
-  for (long long e = threadIdx.x; e < E; e += blockDim.x) {
-    const int j = static_cast<int>((e / a.nsel) % a.nb);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int j = (e / a.nsel) % a.nb;
     const int id = sel0[e];
     if (id >= 0 && id <= j) atomicAdd(&cnt[id], 1);
   }
@@ -120,12 +120,13 @@ __global__ void __launch_bounds__(256) bwd_rev_kernel(const BwdArgs a) {
   if (warp == 0) {
     int32_t* rev = a.rev + static_cast<long long>(blockIdx.x) * E;
     int ahead[4];
-    for (long long base = 0; base < E; base += 32) {
-      const int u = static_cast<int>((base >> 5) & 3);
+    const int per_head = a.nsel * a.nb;
+    for (int base = 0; base < E; base += 32) {
+      const int u = (base >> 5) & 3;
       if (u == 0) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const long long e = base + 32 * q + lane;
+          const int e = base + 32 * q + lane;
           ahead[q] = e < E ? sel0[e] : -1;
         }
       }
@@ -133,11 +134,11 @@ __global__ void __launch_bounds__(256) bwd_rev_kernel(const BwdArgs a) {
 #pragma unroll
       for (int q = 1; q < 4; ++q)
         if (q == u) loaded = ahead[q];
-      const long long e = base + lane;
+      const int e = base + lane;
       int id = -1, j = 0, hl = 0;
       if (e < E) {
-        j = static_cast<int>((e / a.nsel) % a.nb);
-        hl = static_cast<int>(e / (static_cast<long long>(a.nsel) * a.nb));
+        hl = e / per_head;
+        j = (e - hl * per_head) / a.nsel;
         id = loaded;
         if (id > j) id = -1;
       }

@@ -73,8 +73,11 @@ struct BwCfg {
   static constexpr int kPTile = BS * BS * 2;         // bf16 [BS x BS]: BS/64 regions
   static constexpr int kCtl = 1024;                  // barriers, omega, ids, misc
   // dq kernel: Q, dO, NKV (K, V) slots, P / dS.  The slots hold the next
-  // blocks' tiles in flight while the current one computes (one CTA per SM).
-  static constexpr int NKV = (BS == 128 && D == 128) ? 2 : (BS == 64 && D == 64) ? 6 : 5;
+  // blocks' tiles in flight while the current one computes.  At bs = 64 the
+  // kernel needs 256 TMEM columns, so two CTAs share an SM (their phases
+  // overlap); shared memory is sized for that.  At bs = 128 one CTA holds
+  // all 512 columns and takes deeper rings instead.
+  static constexpr int NKV = (BS == 64) ? (D == 64 ? 5 : 2) : (D == 128 ? 2 : 5);
   static constexpr int qOffQ = 0;
   static constexpr int qOffO = kTile;
   static constexpr int qOffKV = 2 * kTile;

@@ -552,6 +552,8 @@ mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void*
   if (static_cast<long long>(cfg->B) * cfg->Hq * (cfg->S / cfg->block) * (cfg->block / 16) > INT32_MAX)
     return MDR_ERR_UNSUPPORTED;
   if (mdr::bwd_rev_smem(cfg->S / cfg->block) > kMaxDynamicSmem) return MDR_ERR_UNSUPPORTED;   // reverse index
+  if (static_cast<long long>(cfg->Hq / cfg->Hkv) * (cfg->S / cfg->block) * (cfg->R + cfg->L) > INT32_MAX)
+    return MDR_ERR_UNSUPPORTED;                                 // reverse-index entries of one KV head
   const bool tc = cfg->dtype == MDR_BF16;          // tensor cores (block and D in {64,128} for bf16)
   if (tc && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
              !aligned16(dk) || !aligned16(dv)))
