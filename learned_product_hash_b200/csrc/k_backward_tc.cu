@@ -775,12 +775,353 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   }
 }
 
+// ------------------------------------------- dk/dv kernel, warp-specialised
+// Roles: warps 0-3 compute P^T and dS^T (warp w reads TMEM subpartition w),
+// warp 4 loads by TMA, warp 5 issues the MMAs (and owns the tensor memory).
+// S^T and dP^T of the next entry are computed while the four warps work on
+// the current one (two TMEM buffers at bs = 64); every hand-off is an
+// mbarrier, every wait bounded (2 s, and given up as soon as another role has
+// given up).
+constexpr int kWsThreads = 192;
+
+template <int BS, int D>
+struct WsCfg {
+  using C = BwCfg<BS, D>;
+  static constexpr int NS = (BS == 64) ? 2 : 1;                       // S^T / dP^T / P^T / dS^T buffers
+  static constexpr int NE = (BS == 64) ? (D == 64 ? 8 : 4) : (D == 64 ? 3 : 1);   // entry slots
+  static constexpr int kSlot = C::kSlot;
+  static constexpr int oK = 0, oV = C::kTile, oE = 2 * C::kTile;
+  static constexpr int oPT = oE + NE * kSlot;                          // NS x P^T
+  static constexpr int oDS = oPT + NS * C::kPTile;                     // NS x dS^T
+  static constexpr int oCtl = oDS + NS * C::kPTile;
+  static constexpr int kSmem = oCtl + 1024;
+  static_assert(kSmem <= 232448, "shared memory per CTA");
+  static constexpr int colS = 0, colP = NS * BS, colV = 2 * NS * BS, colK = 2 * NS * BS + D;
+  static constexpr int kCols = pow2_cols(2 * NS * BS + 2 * D);
+  static_assert(2 * NS * BS + 2 * D <= 512, "tensor memory");
+  // barriers
+  static constexpr int bKvF = 0, bKvE = 1, bAF = 2, bAE = 3, bFin = 4;
+  static constexpr int bEF = 5, bEE = bEF + NE;
+  static constexpr int bSF = bEE + NE, bSE = bSF + NS, bPF = bSE + NS, bPE = bPF + NS;
+  static constexpr int kBars = bPE + NS;
+  static_assert(kBars <= 32, "barrier space");
+};
+
+struct WsCtl {
+  uint64_t bar[32];
+  float om[64];
+  uint32_t tmem;
+  int abort;
+};
+
+template <int BS, int D>
+__global__ void __launch_bounds__(kWsThreads, 1)
+bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const BwdArgs a) {
+  using C = BwCfg<BS, D>;
+  using W = WsCfg<BS, D>;
+  using namespace tc;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicExch(a.status, kDevMisaligned);
+    return;
+  }
+  WsCtl& ctl = *reinterpret_cast<WsCtl*>(smem + W::oCtl);
+  const uint32_t base = smem_u32(smem);
+  const uint32_t sK = base + W::oK, sV = base + W::oV, sE = base + W::oE;
+  auto BAR = [&](int i) { return smem_u32(&ctl.bar[i]); };
+  volatile int* abort_flag = &ctl.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 5) {
+    tmem_alloc(smem_u32(&ctl.tmem), W::kCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < W::kBars; ++i) {
+      int count = 1;
+      if (i == W::bAE || (i >= W::bSE && i < W::bSE + W::NS) || (i >= W::bPF && i < W::bPF + W::NS)) count = 4;
+      mbar_init(BAR(i), count);
+    }
+    fence_mbar_init();
+    ctl.abort = 0;
+  }
+  if (threadIdx.x < D / 2) ctl.om[threadIdx.x] = a.inv_freq[threadIdx.x];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem;
+  grid_dependency_wait();          // lse, Delta (dq kernel) and the reverse index come from earlier kernels
+
+  const long long nkt = static_cast<long long>(a.B) * a.Hkv * a.nb;
+  const int g = a.Hq / a.Hkv;
+  const long long E = static_cast<long long>(g) * a.nb * a.nsel;
+  // Entries of key tile kt (0 for a reverse-index range that is out of bounds,
+  // which a reverse index of this call never gives; recorded).
+  auto entries = [&](long long kt, int* e0_out) -> int {
+    const int i = static_cast<int>(kt % a.nb);
+    const long long bh = kt / a.nb;
+    const int32_t* roff = a.rev_off + bh * (a.nb + 1);
+    const int e0 = roff[i], ne = roff[i + 1] - e0;
+    *e0_out = e0;
+    if (e0 < 0 || ne < 0 || e0 + static_cast<long long>(ne) > E) {
+      if (threadIdx.x == 0 || threadIdx.x == 128) {
+        atomicExch(a.status, kDevBadSelection);
+        record_site(a.status, 200 + kSiteRevRange);
+      }
+      return 0;
+    }
+    return ne;
+  };
+  auto code_of = [&](const int32_t* rev, int e) -> int {
+    int code = rev[e];
+    if (code < 0 || code >= g * a.nb) {
+      atomicExch(a.status, kDevBadSelection);
+      record_site(a.status, 200 + kSiteRevCode);
+      code = 0;
+    }
+    return code;
+  };
+  auto fail = [&](int site) {
+    atomicExch(a.status, kDevWaitTimeout);
+    record_site(a.status, 200 + site);
+    *abort_flag = 1;
+  };
+  auto waitb = [&](int bar, uint32_t parity) -> bool {
+    if (mbar_try_wait(BAR(bar), parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+#pragma unroll 1
+      for (int k = 0; k < 32; ++k)
+        if (mbar_try_wait(BAR(bar), parity)) return true;
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kBwWaitNs) return false;
+    }
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ loads
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      prefetch_tmap(&tmO);
+      long long xg = 0, tc_ = 0;
+      bool ok = true;
+      for (long long kt = blockIdx.x; kt < nkt && ok; kt += gridDim.x) {
+        int e0;
+        const int ne = entries(kt, &e0);
+        if (ne == 0) continue;
+        const int i = static_cast<int>(kt % a.nb);
+        const long long bh = kt / a.nb;
+        const int h = static_cast<int>(bh % a.Hkv), b = static_cast<int>(bh / a.Hkv);
+        const int32_t* rev = a.rev + bh * E;
+        if (tc_ > 0 && !waitb(W::bKvE, static_cast<uint32_t>((tc_ - 1) & 1))) { fail(kSiteKV); ok = false; break; }
+        const int row0 = static_cast<int>(static_cast<long long>(b) * a.S + static_cast<long long>(i) * BS);
+        mbar_expect_tx(BAR(W::bKvF), 2 * C::kTile);
+#pragma unroll
+        for (int gg = 0; gg < D / 64; ++gg) {
+          tma_load_3d(sK + gg * C::kRegion, &tmK, BAR(W::bKvF), gg * 64, h, row0);
+          tma_load_3d(sV + gg * C::kRegion, &tmV, BAR(W::bKvF), gg * 64, h, row0);
+        }
+        for (int x = 0; x < ne; ++x, ++xg) {
+          const int slot = static_cast<int>(xg % W::NE);
+          if (xg >= W::NE && !waitb(W::bEE + slot, static_cast<uint32_t>(((xg / W::NE) - 1) & 1))) {
+            fail(kSiteEntry);
+            ok = false;
+            break;
+          }
+          const int code = code_of(rev, e0 + x);
+          const int hl = code / a.nb, jq = code - hl * a.nb, hq = h * g + hl;
+          const uint32_t bar = BAR(W::bEF + slot), dst = sE + slot * W::kSlot;
+          const int q0 = static_cast<int>(static_cast<long long>(b) * a.S + static_cast<long long>(jq) * BS);
+          const long long si0 = (static_cast<long long>(b) * a.Hq + hq) * a.S + static_cast<long long>(jq) * BS;
+          mbar_expect_tx(bar, 2 * C::kTile + 2 * BS * 4);
+#pragma unroll
+          for (int gg = 0; gg < D / 64; ++gg) {
+            tma_load_3d(dst + gg * C::kRegion, &tmQ, bar, gg * 64, hq, q0);
+            tma_load_3d(dst + C::kTile + gg * C::kRegion, &tmO, bar, gg * 64, hq, q0);
+          }
+          bulk_load(dst + 2 * C::kTile, a.lse + si0, BS * 4, bar);
+          bulk_load(dst + 2 * C::kTile + BS * 4, a.delta + si0, BS * 4, bar);
+        }
+        ++tc_;
+      }
+      if (!ok) {
+        // Wait (bounded) for the copies this thread issued and nobody consumed.
+        if (tc_ > 0) mbar_wait(BAR(W::bKvF), static_cast<uint32_t>(tc_ & 1), kBwWaitNs);
+        for (long long n = xg - W::NE > 0 ? xg - W::NE : 0; n < xg; ++n)
+          mbar_wait(BAR(W::bEF + static_cast<int>(n % W::NE)), static_cast<uint32_t>((n / W::NE) & 1), kBwWaitNs);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------- MMAs
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(BS, BS, 0, 0);
+      constexpr uint32_t idG = idesc_bf16_f32(BS, D, 0, 1);
+      long long xg = 0, tc_ = 0;
+      bool ok = true;
+      // dV += P^T dO, dK += dS^T Q for entry yg (x-th of its tile).
+      auto acc = [&](long long yg, int y) -> bool {
+        const int pb = static_cast<int>(yg % W::NS), slot = static_cast<int>(yg % W::NE);
+        if (!waitb(W::bPF + pb, static_cast<uint32_t>((yg / W::NS) & 1))) { fail(kSiteMM); return false; }
+        if (y == 0 && tc_ > 0 && !waitb(W::bAE, static_cast<uint32_t>((tc_ - 1) & 1))) { fail(kSiteMM); return false; }
+        tc_fence_after();
+        const uint32_t sQe = sE + slot * W::kSlot, sOe = sQe + C::kTile;
+        const uint32_t sPT = base + W::oPT + pb * C::kPTile, sDS = base + W::oDS + pb * C::kPTile;
+#pragma unroll
+        for (int kk = 0; kk < BS / 16; ++kk)
+          mma_bf16(tmem + W::colV, kmaj<BS>(sPT, kk), mnmaj<BS>(sOe, kk), idG, (y > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < BS / 16; ++kk)
+          mma_bf16(tmem + W::colK, kmaj<BS>(sDS, kk), mnmaj<BS>(sQe, kk), idG, (y > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(BAR(W::bPE + pb));
+        mma_commit(BAR(W::bEE + slot));
+        return true;
+      };
+      for (long long kt = blockIdx.x; kt < nkt && ok; kt += gridDim.x) {
+        int e0;
+        const int ne = entries(kt, &e0);
+        if (ne == 0) continue;
+        if (!waitb(W::bKvF, static_cast<uint32_t>(tc_ & 1))) { fail(kSiteKV); ok = false; break; }
+        for (int x = 0; x < ne; ++x, ++xg) {
+          const int slot = static_cast<int>(xg % W::NE), sb = static_cast<int>(xg % W::NS);
+          if (!waitb(W::bEF + slot, static_cast<uint32_t>((xg / W::NE) & 1))) { fail(kSiteEntry); ok = false; break; }
+          if (xg >= W::NS && !waitb(W::bSE + sb, static_cast<uint32_t>(((xg / W::NS) - 1) & 1))) {
+            fail(kSiteS);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sQe = sE + slot * W::kSlot, sOe = sQe + C::kTile;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16(tmem + W::colS + sb * BS, kmaj<BS>(sK, kk), kmaj<BS>(sQe, kk), idS, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16(tmem + W::colP + sb * BS, kmaj<BS>(sV, kk), kmaj<BS>(sOe, kk), idS, kk > 0);
+          mma_commit(BAR(W::bSF + sb));
+          if (x > 0 && !acc(xg - 1, x - 1)) { ok = false; break; }
+        }
+        if (!ok) break;
+        if (!acc(xg - 1, ne - 1)) { ok = false; break; }
+        mma_commit(BAR(W::bAF));
+        mma_commit(BAR(W::bKvE));
+        ++tc_;
+      }
+      // Everything this thread issued has completed once bFin fires.
+      mma_commit(BAR(W::bFin));
+      mbar_wait(BAR(W::bFin), 0, kBwWaitNs);
+    }
+  } else {
+    // ---------------------------------------------- P^T, dS^T, epilogue
+    const Rows<BS, D> R;                             // warps 0-3: TMEM subpartitions 0-3
+    const float sl2 = a.scale * 1.4426950408889634f;
+    auto wwait = [&](int bar, uint32_t parity) { return __all_sync(0xffffffffu, waitb(bar, parity)) != 0; };
+    long long xg = 0, tc_ = 0;
+    bool ok = true;
+    for (long long kt = blockIdx.x; kt < nkt && ok; kt += gridDim.x) {
+      int e0;
+      const int ne = entries(kt, &e0);
+      const int i = static_cast<int>(kt % a.nb);
+      const long long bh = kt / a.nb;
+      const int h = static_cast<int>(bh % a.Hkv), b = static_cast<int>(bh / a.Hkv);
+      const long long tok0 = static_cast<long long>(b) * a.S + static_cast<long long>(i) * BS;
+      if (ne == 0) {                                // no query selected this block
+        for (int e = threadIdx.x; e < BS * D; e += 128) {
+          const long long o = ((tok0 + e / D) * a.Hkv + h) * D + e % D;
+          a.dk[o] = 0.f;
+          a.dv[o] = 0.f;
+        }
+        continue;
+      }
+      const int32_t* rev = a.rev + bh * E;
+      for (int x = 0; x < ne; ++x, ++xg) {
+        const int sb = static_cast<int>(xg % W::NS), slot = static_cast<int>(xg % W::NE);
+        if (!wwait(W::bSF + sb, static_cast<uint32_t>((xg / W::NS) & 1))) { ok = false; break; }
+        if (!wwait(W::bEF + slot, static_cast<uint32_t>((xg / W::NE) & 1))) { ok = false; break; }   // lse, Delta landed
+        tc_fence_after();
+        const int code = rev[e0 + x];
+        const int jq = (code < 0 ? 0 : code) % a.nb;
+        const bool diag = jq == i;
+        const float* lse_s = reinterpret_cast<const float*>(smem + W::oE + slot * W::kSlot + 2 * C::kTile);
+        const float* del_s = lse_s + BS;
+        float sv[C::NC][32], dp[C::NC][32];
+#pragma unroll
+        for (int c = 0; c < C::NC; ++c) {
+          R.ld_scores(tmem + W::colS + sb * BS, c, sv[c]);
+          R.ld_scores(tmem + W::colP + sb * BS, c, dp[c]);
+        }
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(W::bSE + sb));            // S^T, dP^T buffer free
+        if (xg >= W::NS && !wwait(W::bPE + sb, static_cast<uint32_t>(((xg / W::NS) - 1) & 1))) { ok = false; break; }
+        uint8_t* pPT = smem + W::oPT + sb * C::kPTile;
+        uint8_t* pDS = smem + W::oDS + sb * C::kPTile;
+#pragma unroll
+        for (int c = 0; c < C::NC; ++c) {
+          const int t0 = C::kHR ? 32 * R.tsub : 32 * c;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float p[8], ds[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int t = t0 + 8 * q + e;
+              p[e] = (diag && t < R.r) ? 0.f : ex2(sv[c][8 * q + e] * sl2 - lse_s[t]);
+              ds[e] = p[e] * (dp[c][8 * q + e] - del_s[t]);
+            }
+            st_bf16x8<BS>(pPT, R.r, t0 + 8 * q, p);
+            st_bf16x8<BS>(pDS, R.r, t0 + 8 * q, ds);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(W::bPF + sb));
+      }
+      if (!ok) break;
+      // dv = dV; dk = R(s)^T (scale dK).
+      if (!wwait(W::bAF, static_cast<uint32_t>(tc_ & 1))) { ok = false; break; }
+      tc_fence_after();
+      const long long krow = (tok0 + R.r) * a.Hkv + h;
+      const int s = i * BS + R.r;
+#pragma unroll
+      for (int pp = 0; pp < C::NP; ++pp) {
+        float lo[C::W], hi[C::W];
+        R.ld_d(tmem + W::colV, pp, 0, lo);
+        R.ld_d(tmem + W::colV, pp, 1, hi);
+        tmem_ld_wait();
+        store_f32<C::W>(a.dv + krow * D + R.col_lo(pp), lo);
+        store_f32<C::W>(a.dv + krow * D + D / 2 + R.col_lo(pp), hi);
+        R.ld_d(tmem + W::colK, pp, 0, lo);
+        R.ld_d(tmem + W::colK, pp, 1, hi);
+        tmem_ld_wait();
+        rotate_store<C::W, D>(lo, hi, R.col_lo(pp), s, a.scale, ctl.om, a.dk + krow * D);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(W::bAE));
+      ++tc_;
+    }
+    if (!ok && lane == 0) fail(kSiteS);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) {
+    __syncwarp();
+    tmem_dealloc(tmem, W::kCols);
+  }
+}
+
 namespace {
 
 template <typename K>
 cudaError_t launch_persistent(K kernel, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                               const CUtensorMap& mo, const BwdArgs& a, long long ntiles, int smem, int cols,
-                              cudaStream_t st) {
+                              int threads, cudaStream_t st) {
   cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(kernel), smem);
   if (e != cudaSuccess) return e;
   // All of the unified L1 / shared storage as shared memory (these kernels
@@ -789,14 +1130,32 @@ cudaError_t launch_persistent(K kernel, const CUtensorMap& mq, const CUtensorMap
                            cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   const int sms = cached_sm_count();
-  int per_sm = cached_occupancy(reinterpret_cast<const void*>(kernel), kBwThreads, smem);
+  int per_sm = cached_occupancy(reinterpret_cast<const void*>(kernel), threads, smem);
   if (sms <= 0) return cudaErrorUnknown;
+  // Residency from the kernel's own registers and shared memory (the larger
+  // of this and the occupancy query; a CTA that does not fit waits for one
+  // to finish, so an overestimate costs nothing).
+  {
+    int dev = 0, regs_sm = 0, smem_sm = 0, reserved = 0;
+    cudaFuncAttributes fa{};
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kernel)) == cudaSuccess &&
+        cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) == cudaSuccess) {
+      const int warps = (threads + 31) / 32;
+      const int regs_warp = (fa.numRegs * 32 + 255) / 256 * 256;
+      const int by_regs = regs_sm / (regs_warp * warps);
+      const int by_smem = smem_sm / (smem + static_cast<int>(fa.sharedSizeBytes) + reserved);
+      int est = by_regs < by_smem ? by_regs : by_smem;
+      if (est > per_sm) per_sm = est;
+    }
+  }
   per_sm = per_sm < 512 / cols ? per_sm : 512 / cols;    // tensor memory: 512 columns per SM
   if (per_sm < 1) per_sm = 1;
   const long long want = static_cast<long long>(sms) * per_sm;
   const unsigned grid = static_cast<unsigned>(ntiles < want ? ntiles : want);
   if (grid == 0) return cudaSuccess;
-  return launch_pdl(kernel, dim3(grid), dim3(kBwThreads), static_cast<size_t>(smem), st, mq, mk, mv, mo, a);
+  return launch_pdl(kernel, dim3(grid), dim3(threads), static_cast<size_t>(smem), st, mq, mk, mv, mo, a);
 }
 
 template <int BS, int D>
@@ -808,10 +1167,11 @@ cudaError_t launch_tc_bwd(const BwdArgs& a, cudaStream_t st) {
       !make_tile_map(&mv, a.v, rows, a.Hkv, D, BS) || !make_tile_map(&mo, a.dout, rows, a.Hq, D, BS))
     return cudaErrorInvalidValue;
   cudaError_t e = launch_persistent(bwd_dq_tc_kernel<BS, D>, mq, mk, mv, mo, a,
-                                    static_cast<long long>(a.B) * a.Hq * a.nb, C::qSmem, C::qCols, st);
+                                    static_cast<long long>(a.B) * a.Hq * a.nb, C::qSmem, C::qCols, kBwThreads, st);
   if (e != cudaSuccess) return e;
-  return launch_persistent(bwd_dkdv_tc_kernel<BS, D>, mq, mk, mv, mo, a,
-                           static_cast<long long>(a.B) * a.Hkv * a.nb, C::bSmem, C::bCols, st);
+  using W = WsCfg<BS, D>;
+  return launch_persistent(bwd_dkdv_ws_kernel<BS, D>, mq, mk, mv, mo, a,
+                           static_cast<long long>(a.B) * a.Hkv * a.nb, W::kSmem, W::kCols, kWsThreads, st);
 }
 
 }  // namespace
