@@ -986,6 +986,9 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (!waitb(W::bKvF, static_cast<uint32_t>(tc_ & 1))) { fail(kSiteKV); ok = false; break; }
         for (int x = 0; x < ne; ++x, ++xg) {
           const int slot = static_cast<int>(xg % W::NE), sb = static_cast<int>(xg % W::NS);
+          // With a single entry slot, entry x loads only once entry x-1's
+          // products have read the slot: issue those first.
+          if (W::NE == 1 && x > 0 && !acc(xg - 1, x - 1)) { ok = false; break; }
           if (!waitb(W::bEF + slot, static_cast<uint32_t>((xg / W::NE) & 1))) { fail(kSiteEntry); ok = false; break; }
           if (xg >= W::NS && !waitb(W::bSE + sb, static_cast<uint32_t>(((xg / W::NS) - 1) & 1))) {
             fail(kSiteS);
@@ -1001,7 +1004,7 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           for (int kk = 0; kk < D / 16; ++kk)
             mma_bf16(tmem + W::colP + sb * BS, kmaj<BS>(sV, kk), kmaj<BS>(sOe, kk), idS, kk > 0);
           mma_commit(BAR(W::bSF + sb));
-          if (x > 0 && !acc(xg - 1, x - 1)) { ok = false; break; }
+          if (W::NE > 1 && x > 0 && !acc(xg - 1, x - 1)) { ok = false; break; }
         }
         if (!ok) break;
         if (!acc(xg - 1, ne - 1)) { ok = false; break; }
