@@ -21,17 +21,19 @@
 //     pass 2, per selected block: S = Q K^T and dP = dO V^T; P = 2^(S - lse),
 //       dS = P (dP - Delta) (bf16) into shared memory; dQ += dS K (K read
 //       MN-major from its TMA tile).  Epilogue: dq = R(t)^T (scale dQ).
-//   bwd_dkdv_tc_kernel  one key block (b, hkv, i) at a time, persistent, over
+//   bwd_dkdv_ws_kernel  one key block (b, hkv, i) at a time, persistent, over
 //     the block's reverse list (the (query head, query block) pairs that
 //     selected it, in a fixed order): S^T = K Q^T and dP^T = V dO^T;
 //     P^T = 2^(S^T - lse_t), dS^T = P^T (dP^T - Delta_t) (bf16); dV += P^T dO,
-//     dK += dS^T Q.  Epilogue: dv = dV, dk = R(s)^T (scale dK).
+//     dK += dS^T Q.  Epilogue: dv = dV, dk = R(s)^T (scale dK).  Warp-
+//     specialised (see the kernel).
 // The causal mask applies where the key block is the query block (key s >
-// query t is masked).  Each CTA has four warps; warp w owns TMEM
-// subpartition w (accumulator rows 16w..16w+15 for bs = 64, two threads per
-// row splitting the columns; rows 32w..32w+31 for bs = 128).  Thread 0 issues
-// the TMA loads and the MMAs; the next block's (or entry's) tiles are loaded
-// while the current one is computed (a ring of several slots per CTA).  Sums run in a fixed order and there
+// query t is masked).  Warp w of the four that read accumulators owns TMEM
+// subpartition w (rows 16w..16w+15 for bs = 64, two threads per row
+// splitting the columns; rows 32w..32w+31 for bs = 128).  In the dq kernel
+// thread 0 issues the TMA loads and the MMAs and the next blocks' tiles load
+// into a ring of slots while the current one is computed; the dk/dv kernel
+// has a TMA warp and an MMA warp of its own.  Sums run in a fixed order and there
 // are no atomics, so a call is deterministic.  Every wait is bounded (2 s of
 // wall time): a wait that runs out writes status 1, the CTA waits (bounded)
 // for its own copies and MMAs, frees its tensor memory and returns.
@@ -86,17 +88,9 @@ struct BwCfg {
   static constexpr int qSmem = qOffCtl + kCtl;
   static constexpr int qCols = pow2_cols(2 * BS + D);
   static constexpr int qColS = 0, qColP = BS, qColO = 2 * BS;
-  // dk/dv kernel: K, V, kNE entry slots (Q, dO, lse, Delta), P^T, dS^T
-  static constexpr int kNE = (BS == 128 && D == 128) ? 1 : (BS == 128) ? 3 : (D == 64) ? 6 : 5;
+  // dk/dv kernel: an entry slot holds a query tile's Q, dO, lse and Delta
   static constexpr int kSlot = (2 * kTile + 2 * BS * 4 + 1023) / 1024 * 1024;
-  static constexpr int bOffK = 0, bOffV = kTile, bOffE = 2 * kTile;
-  static constexpr int bOffPT = bOffE + kNE * kSlot;
-  static constexpr int bOffDS = bOffPT + kPTile;
-  static constexpr int bOffCtl = bOffDS + kPTile;
-  static constexpr int bSmem = bOffCtl + kCtl;
-  static constexpr int bCols = pow2_cols(2 * BS + 2 * D);
-  static constexpr int bColS = 0, bColP = BS, bColV = 2 * BS, bColK = 2 * BS + D;
-  static_assert(qSmem <= 232448 && bSmem <= 232448, "shared memory per CTA");
+  static_assert(qSmem <= 232448, "shared memory per CTA");
   static_assert(kTile % 1024 == 0 && kPTile % 1024 == 0, "1024-byte aligned tiles");
   // D-column geometry of a thread: W columns at lo and W at D/2 + lo, NP times.
   static constexpr int W = kHR ? D / 4 : 32;
@@ -542,239 +536,6 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   }
 }
 
-// -------------------------------------------------------------- dk/dv kernel
-template <int BS, int D>
-__global__ void __launch_bounds__(kBwThreads, 1)
-bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                   const BwdArgs a) {
-  using C = BwCfg<BS, D>;
-  using namespace tc;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  if ((smem_u32(smem) & 1023u) != 0) {
-    if (threadIdx.x == 0) atomicExch(a.status, kDevMisaligned);
-    return;
-  }
-  Ctl& ctl = *reinterpret_cast<Ctl*>(smem + C::bOffCtl);
-  const uint32_t base = smem_u32(smem);
-  const uint32_t sK = base + C::bOffK, sV = base + C::bOffV, sE = base + C::bOffE;
-  const uint32_t sPT = base + C::bOffPT, sDS = base + C::bOffDS;
-  uint8_t* pPT = smem + C::bOffPT;
-  uint8_t* pDS = smem + C::bOffDS;
-  enum { bKV = 0, bS = 1, bMM = 2, bFin = 3, bE0 = 4 };     // bE0 .. bE0 + kNE - 1
-  static_assert(bE0 + C::kNE <= 16, "barrier space");
-  auto BAR = [&](int i) { return smem_u32(&ctl.bar[i]); };
-  const Rows<BS, D> R;
-  if (R.warp == 0) {
-    tmem_alloc(smem_u32(&ctl.tmem), C::bCols);
-    tmem_relinquish();
-  }
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < bE0 + C::kNE; ++i) mbar_init(BAR(i), 1);
-    fence_mbar_init();
-  }
-  if (threadIdx.x < D / 2) ctl.om[threadIdx.x] = a.inv_freq[threadIdx.x];
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = ctl.tmem;
-  grid_dependency_wait();          // lse, Delta (dq kernel) and the reverse index come from earlier kernels
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&tmQ);
-    prefetch_tmap(&tmK);
-    prefetch_tmap(&tmV);
-    prefetch_tmap(&tmO);
-  }
-
-  constexpr uint32_t idS = idesc_bf16_f32(BS, BS, 0, 0);
-  constexpr uint32_t idG = idesc_bf16_f32(BS, D, 0, 1);
-  const float sl2 = a.scale * 1.4426950408889634f;
-  const long long nkt = static_cast<long long>(a.B) * a.Hkv * a.nb;
-  const int g = a.Hq / a.Hkv;
-  uint32_t phKV = 0, phS = 0, phMM = 0;
-  long long e_issue = 0, e_use = 0;               // entry loads: slot = n % kNE, parity (n / kNE) & 1
-  bool mm_pending = false, ok = true, kv_pending = false;
-  int mm_x = 0;
-  const uint64_t t_start = globaltimer();
-  auto wait_all = [&](int bar, uint32_t parity, int site) -> bool {
-    const bool w = mbar_wait(BAR(bar), parity, kBwWaitNs);
-    const bool in_time = globaltimer() - t_start <= kBwBudgetNs;
-    if (!(w && in_time)) record_site(a.status, 200 + site + (w ? 50 : 0));
-    return __syncthreads_and(w && in_time) != 0;
-  };
-
-  for (long long kt = blockIdx.x; kt < nkt && ok; kt += gridDim.x) {
-    const int i = static_cast<int>(kt % a.nb);
-    const long long bh = kt / a.nb;
-    const int h = static_cast<int>(bh % a.Hkv), b = static_cast<int>(bh / a.Hkv);
-    const int32_t* roff = a.rev_off + bh * (a.nb + 1);
-    const int32_t* rev = a.rev + bh * (static_cast<long long>(g) * a.nb * a.nsel);
-    const long long E = static_cast<long long>(g) * a.nb * a.nsel;   // entries of this (b, hkv)
-    const int e0 = roff[i];
-    int ne = roff[i + 1] - e0;
-    if (e0 < 0 || ne < 0 || e0 + static_cast<long long>(ne) > E) {  // never for a reverse index of this call
-      if (threadIdx.x == 0) {
-        atomicExch(a.status, kDevBadSelection);
-        record_site(a.status, 200 + kSiteRevRange);
-      }
-      ne = 0;
-    }
-    const long long tok0 = static_cast<long long>(b) * a.S + static_cast<long long>(i) * BS;
-    if (ne == 0) {                                // no query selected this block
-      for (int e = threadIdx.x; e < BS * D; e += kBwThreads) {
-        const long long o = ((tok0 + e / D) * a.Hkv + h) * D + e % D;
-        a.dk[o] = 0.f;
-        a.dv[o] = 0.f;
-      }
-      continue;
-    }
-    auto issue_e = [&](int x) {                   // entry x: Q, dO, lse, Delta of its query tile
-      if (threadIdx.x == 0) {
-        const int slot = static_cast<int>(e_issue % C::kNE);
-        int code = rev[e0 + x];
-        if (code < 0 || code >= g * a.nb) {        // never for a reverse index of this call
-          atomicExch(a.status, kDevBadSelection);
-          record_site(a.status, 200 + kSiteRevCode);
-          code = 0;
-        }
-        const int hl = code / a.nb, jq = code - hl * a.nb, hq = h * g + hl;
-        const uint32_t bar = BAR(bE0 + slot), dst = sE + slot * C::kSlot;
-        const int row0 = static_cast<int>(static_cast<long long>(b) * a.S + static_cast<long long>(jq) * BS);
-        const long long si0 = (static_cast<long long>(b) * a.Hq + hq) * a.S + static_cast<long long>(jq) * BS;
-        mbar_expect_tx(bar, 2 * C::kTile + 2 * BS * 4);
-#pragma unroll
-        for (int gg = 0; gg < D / 64; ++gg) {
-          tma_load_3d(dst + gg * C::kRegion, &tmQ, bar, gg * 64, hq, row0);
-          tma_load_3d(dst + C::kTile + gg * C::kRegion, &tmO, bar, gg * 64, hq, row0);
-        }
-        bulk_load(dst + 2 * C::kTile, a.lse + si0, BS * 4, bar);
-        bulk_load(dst + 2 * C::kTile + BS * 4, a.delta + si0, BS * 4, bar);
-      }
-      ++e_issue;
-    };
-    auto finish_mm = [&]() -> bool {
-      if (!mm_pending) return true;
-      if (!wait_all(bMM, phMM, kSiteMM)) return false;
-      phMM ^= 1;
-      mm_pending = false;
-      if (mm_x + C::kNE < ne) issue_e(mm_x + C::kNE);
-      return true;
-    };
-    __syncthreads();                              // the previous tile's tensor memory reads are done
-    if (threadIdx.x == 0) {
-      mbar_expect_tx(BAR(bKV), 2 * C::kTile);
-#pragma unroll
-      for (int gg = 0; gg < D / 64; ++gg) {
-        tma_load_3d(sK + gg * C::kRegion, &tmK, BAR(bKV), gg * 64, h, static_cast<int>(tok0));
-        tma_load_3d(sV + gg * C::kRegion, &tmV, BAR(bKV), gg * 64, h, static_cast<int>(tok0));
-      }
-    }
-    kv_pending = true;
-    for (int x = 0; x < C::kNE && x < ne; ++x) issue_e(x);
-    if (!wait_all(bKV, phKV, kSiteKV)) { ok = false; break; }
-    phKV ^= 1;
-    kv_pending = false;
-    for (int x = 0; x < ne && ok; ++x) {
-      // Entry x is issued when the MMAs of entry x - kNE finish; with a single
-      // slot that is the previous entry's, so wait for them here first.
-      if (e_issue == e_use && !finish_mm()) { ok = false; break; }
-      const int slot = static_cast<int>(e_use % C::kNE);
-      if (!wait_all(bE0 + slot, static_cast<uint32_t>((e_use / C::kNE) & 1), kSiteEntry)) { ok = false; break; }
-      ++e_use;
-      const int code = rev[e0 + x];
-      const int jq = (code < 0 ? 0 : code) % a.nb;
-      const uint32_t sQe = sE + slot * C::kSlot, sOe = sQe + C::kTile;
-      const float* lse_s = reinterpret_cast<const float*>(smem + C::bOffE + slot * C::kSlot + 2 * C::kTile);
-      const float* del_s = lse_s + BS;
-      if (threadIdx.x == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) mma_bf16(tmem + C::bColS, kmaj<BS>(sK, kk), kmaj<BS>(sQe, kk), idS, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) mma_bf16(tmem + C::bColP, kmaj<BS>(sV, kk), kmaj<BS>(sOe, kk), idS, kk > 0);
-        mma_commit(BAR(bS));
-      }
-      if (!wait_all(bS, phS, kSiteS)) { ok = false; break; }
-      phS ^= 1;
-      if (!finish_mm()) { ok = false; break; }     // the P^T, dS^T buffers are free
-      tc_fence_after();
-      const bool diag = jq == i;
-#pragma unroll
-      for (int c = 0; c < C::NC; ++c) {
-        float sv[32], dp[32];
-        const int t0 = R.ld_scores(tmem + C::bColS, c, sv);
-        R.ld_scores(tmem + C::bColP, c, dp);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float p[8], ds[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int t = t0 + 8 * q + e;
-            p[e] = (diag && t < R.r) ? 0.f : ex2(sv[8 * q + e] * sl2 - lse_s[t]);
-            ds[e] = p[e] * (dp[8 * q + e] - del_s[t]);
-          }
-          st_bf16x8<BS>(pPT, R.r, t0 + 8 * q, p);
-          st_bf16x8<BS>(pDS, R.r, t0 + 8 * q, ds);
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BS / 16; ++kk)
-          mma_bf16(tmem + C::bColV, kmaj<BS>(sPT, kk), mnmaj<BS>(sOe, kk), idG, (x > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < BS / 16; ++kk)
-          mma_bf16(tmem + C::bColK, kmaj<BS>(sDS, kk), mnmaj<BS>(sQe, kk), idG, (x > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(BAR(bMM));
-      }
-      mm_pending = true;
-      mm_x = x;
-    }
-    if (!ok) break;
-    if (!finish_mm()) { ok = false; break; }
-    tc_fence_after();
-    // dv = dV; dk = R(s)^T (scale dK).
-    const long long krow = (tok0 + R.r) * a.Hkv + h;
-    const int s = i * BS + R.r;
-#pragma unroll
-    for (int pp = 0; pp < C::NP; ++pp) {
-      float lo[C::W], hi[C::W];
-      R.ld_d(tmem + C::bColV, pp, 0, lo);
-      R.ld_d(tmem + C::bColV, pp, 1, hi);
-      tmem_ld_wait();
-      store_f32<C::W>(a.dv + krow * D + R.col_lo(pp), lo);
-      store_f32<C::W>(a.dv + krow * D + D / 2 + R.col_lo(pp), hi);
-      R.ld_d(tmem + C::bColK, pp, 0, lo);
-      R.ld_d(tmem + C::bColK, pp, 1, hi);
-      tmem_ld_wait();
-      rotate_store<C::W, D>(lo, hi, R.col_lo(pp), s, a.scale, ctl.om, a.dk + krow * D);
-    }
-    tc_fence_before();
-  }
-
-  if (!ok) {
-    if (threadIdx.x == 0) {
-      atomicExch(a.status, kDevWaitTimeout);
-      mma_commit(BAR(bFin));
-      mbar_wait(BAR(bFin), 0, kBwWaitNs);
-      if (kv_pending) mbar_wait(BAR(bKV), phKV, kBwWaitNs);
-      for (long long n = e_use; n < e_issue; ++n)
-        mbar_wait(BAR(bE0 + static_cast<int>(n % C::kNE)), static_cast<uint32_t>((n / C::kNE) & 1), kBwWaitNs);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (R.warp == 0) {
-    __syncwarp();
-    tmem_dealloc(tmem, C::bCols);
-  }
-}
-
 // ------------------------------------------- dk/dv kernel, warp-specialised
 // Roles: warps 0-3 compute P^T and dS^T (warp w reads TMEM subpartition w),
 // warp 4 loads by TMA, warp 5 issues the MMAs (and owns the tensor memory).
@@ -1049,34 +810,49 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const bool diag = jq == i;
         const float* lse_s = reinterpret_cast<const float*>(smem + W::oE + slot * W::kSlot + 2 * C::kTile);
         const float* del_s = lse_s + BS;
-        float sv[C::NC][32], dp[C::NC][32];
-#pragma unroll
-        for (int c = 0; c < C::NC; ++c) {
-          R.ld_scores(tmem + W::colS + sb * BS, c, sv[c]);
-          R.ld_scores(tmem + W::colP + sb * BS, c, dp[c]);
-        }
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(W::bSE + sb));            // S^T, dP^T buffer free
-        if (xg >= W::NS && !wwait(W::bPE + sb, static_cast<uint32_t>(((xg / W::NS) - 1) & 1))) { ok = false; break; }
         uint8_t* pPT = smem + W::oPT + sb * C::kPTile;
         uint8_t* pDS = smem + W::oDS + sb * C::kPTile;
-#pragma unroll
-        for (int c = 0; c < C::NC; ++c) {
-          const int t0 = C::kHR ? 32 * R.tsub : 32 * c;
+        // P^T, dS^T of one 32-column chunk into the shared-memory operands.
+        auto chunk_out = [&](const float* sv, const float* dp, int t0) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             float p[8], ds[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const int t = t0 + 8 * q + e;
-              p[e] = (diag && t < R.r) ? 0.f : ex2(sv[c][8 * q + e] * sl2 - lse_s[t]);
-              ds[e] = p[e] * (dp[c][8 * q + e] - del_s[t]);
+              p[e] = (diag && t < R.r) ? 0.f : ex2(sv[8 * q + e] * sl2 - lse_s[t]);
+              ds[e] = p[e] * (dp[8 * q + e] - del_s[t]);
             }
             st_bf16x8<BS>(pPT, R.r, t0 + 8 * q, p);
             st_bf16x8<BS>(pDS, R.r, t0 + 8 * q, ds);
           }
+        };
+        if constexpr (C::NC == 1) {
+          // bs = 64: one chunk; free the S^T, dP^T buffer before waiting for
+          // the P^T, dS^T buffer, so the next entry's products can start.
+          float sv[32], dp[32];
+          const int t0 = R.ld_scores(tmem + W::colS + sb * BS, 0, sv);
+          R.ld_scores(tmem + W::colP + sb * BS, 0, dp);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(W::bSE + sb));          // S^T, dP^T buffer free
+          if (xg >= W::NS && !wwait(W::bPE + sb, static_cast<uint32_t>(((xg / W::NS) - 1) & 1))) { ok = false; break; }
+          chunk_out(sv, dp, t0);
+        } else {
+          // bs = 128 (one buffer): chunk by chunk, 64 values in registers.
+          if (xg >= W::NS && !wwait(W::bPE + sb, static_cast<uint32_t>(((xg / W::NS) - 1) & 1))) { ok = false; break; }
+#pragma unroll 1
+          for (int c = 0; c < C::NC; ++c) {
+            float sv[32], dp[32];
+            const int t0 = R.ld_scores(tmem + W::colS + sb * BS, c, sv);
+            R.ld_scores(tmem + W::colP + sb * BS, c, dp);
+            tmem_ld_wait();
+            chunk_out(sv, dp, t0);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(W::bSE + sb));          // S^T, dP^T buffer free
         }
         fence_proxy_async_smem();
         tc_fence_before();
