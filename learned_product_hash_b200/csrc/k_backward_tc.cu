@@ -40,6 +40,8 @@
 
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -140,9 +142,10 @@ struct Rows {
   __device__ Rows() {
     warp = threadIdx.x >> 5;
     lane = threadIdx.x & 31;
+    const int sp = warp & 3;                         // TMEM subpartition of this warp
     tsub = C::kHR ? (lane >> 4) : 0;
-    r = C::kHR ? warp * 16 + (lane & 15) : warp * 32 + lane;
-    lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    r = C::kHR ? sp * 16 + (lane & 15) : sp * 32 + lane;
+    lane_base = static_cast<uint32_t>(sp * 32) << 16;
   }
   // 32 score columns of chunk c (first column returned); all lanes take part.
   __device__ __forceinline__ int ld_scores(uint32_t tcol, int c, float* v) const {
@@ -537,13 +540,16 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 }
 
 // ------------------------------------------- dk/dv kernel, warp-specialised
-// Roles: warps 0-3 compute P^T and dS^T (warp w reads TMEM subpartition w),
-// warp 4 loads by TMA, warp 5 issues the MMAs (and owns the tensor memory).
+// Roles: warps 0-7 compute P^T and dS^T (warp w reads TMEM subpartition
+// w % 4 and half w / 4 of each entry's columns; warps 0-3 also run the
+// epilogue), warp 8 loads by TMA, warp 9 issues the MMAs (and owns the
+// tensor memory).
 // S^T and dP^T of the next entry are computed while the four warps work on
 // the current one (two TMEM buffers at bs = 64); every hand-off is an
 // mbarrier, every wait bounded (2 s, and given up as soon as another role has
 // given up).
-constexpr int kWsThreads = 192;
+constexpr int kWsThreads = 320;                  // 8 elementwise warps, a TMA warp, an MMA warp
+constexpr int kWsEw = 8;                         // elementwise warps: two per TMEM subpartition
 
 template <int BS, int D>
 struct WsCfg {
@@ -594,14 +600,15 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   auto BAR = [&](int i) { return smem_u32(&ctl.bar[i]); };
   volatile int* abort_flag = &ctl.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp == 5) {
+  if (warp == kWsEw + 1) {
     tmem_alloc(smem_u32(&ctl.tmem), W::kCols);
     tmem_relinquish();
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < W::kBars; ++i) {
       int count = 1;
-      if (i == W::bAE || (i >= W::bSE && i < W::bSE + W::NS) || (i >= W::bPF && i < W::bPF + W::NS)) count = 4;
+      if (i == W::bAE) count = 4;                                        // the epilogue warps
+      if ((i >= W::bSE && i < W::bSE + W::NS) || (i >= W::bPF && i < W::bPF + W::NS)) count = kWsEw;
       mbar_init(BAR(i), count);
     }
     fence_mbar_init();
@@ -626,7 +633,7 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int e0 = roff[i], ne = roff[i + 1] - e0;
     *e0_out = e0;
     if (e0 < 0 || ne < 0 || e0 + static_cast<long long>(ne) > E) {
-      if (threadIdx.x == 0 || threadIdx.x == 128) {
+      if (threadIdx.x == 0 || threadIdx.x == 32 * kWsEw) {
         atomicExch(a.status, kDevBadSelection);
         record_site(a.status, 200 + kSiteRevRange);
       }
@@ -660,7 +667,7 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
   };
 
-  if (warp == 4) {
+  if (warp == kWsEw) {
     // ------------------------------------------------------------ loads
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -715,7 +722,7 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           mbar_wait(BAR(W::bEF + static_cast<int>(n % W::NE)), static_cast<uint32_t>((n / W::NE) & 1), kBwWaitNs);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kWsEw + 1) {
     // ------------------------------------------------------------- MMAs
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(BS, BS, 0, 0);
@@ -779,7 +786,8 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
   } else {
     // ---------------------------------------------- P^T, dS^T, epilogue
-    const Rows<BS, D> R;                             // warps 0-3: TMEM subpartitions 0-3
+    const Rows<BS, D> R;                             // TMEM subpartition warp % 4
+    const int ch = warp >> 2;                        // which half of an entry's columns
     const float sl2 = a.scale * 1.4426950408889634f;
     auto wwait = [&](int bar, uint32_t parity) { return __all_sync(0xffffffffu, waitb(bar, parity)) != 0; };
     long long xg = 0, tc_ = 0;
@@ -792,7 +800,7 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int h = static_cast<int>(bh % a.Hkv), b = static_cast<int>(bh / a.Hkv);
       const long long tok0 = static_cast<long long>(b) * a.S + static_cast<long long>(i) * BS;
       if (ne == 0) {                                // no query selected this block
-        for (int e = threadIdx.x; e < BS * D; e += 128) {
+        for (int e = threadIdx.x; e < BS * D; e += 32 * kWsEw) {
           const long long o = ((tok0 + e / D) * a.Hkv + h) * D + e % D;
           a.dk[o] = 0.f;
           a.dv[o] = 0.f;
@@ -812,10 +820,11 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const float* del_s = lse_s + BS;
         uint8_t* pPT = smem + W::oPT + sb * C::kPTile;
         uint8_t* pDS = smem + W::oDS + sb * C::kPTile;
-        // P^T, dS^T of one 32-column chunk into the shared-memory operands.
-        auto chunk_out = [&](const float* sv, const float* dp, int t0) {
+        // P^T, dS^T of NW columns from t0 into the shared-memory operands.
+        auto cols_out = [&](const float* sv, const float* dp, int t0, auto nw) {
+          constexpr int NW = decltype(nw)::value;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < NW / 8; ++q) {
             float p[8], ds[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -828,27 +837,28 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           }
         };
         if constexpr (C::NC == 1) {
-          // bs = 64: one chunk; free the S^T, dP^T buffer before waiting for
-          // the P^T, dS^T buffer, so the next entry's products can start.
-          float sv[32], dp[32];
-          const int t0 = R.ld_scores(tmem + W::colS + sb * BS, 0, sv);
-          R.ld_scores(tmem + W::colP + sb * BS, 0, dp);
+          // bs = 64: 16 columns a thread (32 ch + 16 tsub ..); free the S^T,
+          // dP^T buffer before waiting for the P^T, dS^T buffer, so the next
+          // entry's products can start.
+          float sv[16], dp[16];
+          tmem_ld16x2_16(tmem + W::colS + sb * BS + 32 * ch + R.lane_base, sv);
+          tmem_ld16x2_16(tmem + W::colP + sb * BS + 32 * ch + R.lane_base, dp);
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(BAR(W::bSE + sb));          // S^T, dP^T buffer free
           if (xg >= W::NS && !wwait(W::bPE + sb, static_cast<uint32_t>(((xg / W::NS) - 1) & 1))) { ok = false; break; }
-          chunk_out(sv, dp, t0);
+          cols_out(sv, dp, 32 * ch + 16 * R.tsub, std::integral_constant<int, 16>{});
         } else {
-          // bs = 128 (one buffer): chunk by chunk, 64 values in registers.
+          // bs = 128 (one buffer): chunks 2 ch and 2 ch + 1 of 32 columns.
           if (xg >= W::NS && !wwait(W::bPE + sb, static_cast<uint32_t>(((xg / W::NS) - 1) & 1))) { ok = false; break; }
 #pragma unroll 1
-          for (int c = 0; c < C::NC; ++c) {
+          for (int c = 2 * ch; c < 2 * ch + 2; ++c) {
             float sv[32], dp[32];
             const int t0 = R.ld_scores(tmem + W::colS + sb * BS, c, sv);
             R.ld_scores(tmem + W::colP + sb * BS, c, dp);
             tmem_ld_wait();
-            chunk_out(sv, dp, t0);
+            cols_out(sv, dp, t0, std::integral_constant<int, 32>{});
           }
           tc_fence_before();
           __syncwarp();
@@ -860,8 +870,10 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (lane == 0) mbar_arrive(BAR(W::bPF + sb));
       }
       if (!ok) break;
+      ++tc_;
+      if (ch != 0) continue;                           // the epilogue: warps 0-3
       // dv = dV; dk = R(s)^T (scale dK).
-      if (!wwait(W::bAF, static_cast<uint32_t>(tc_ & 1))) { ok = false; break; }
+      if (!wwait(W::bAF, static_cast<uint32_t>((tc_ - 1) & 1))) { ok = false; break; }
       tc_fence_after();
       const long long krow = (tok0 + R.r) * a.Hkv + h;
       const int s = i * BS + R.r;
@@ -881,7 +893,6 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(W::bAE));
-      ++tc_;
     }
     if (!ok && lane == 0) fail(kSiteS);
   }
@@ -889,7 +900,7 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) {
+  if (warp == kWsEw + 1) {
     __syncwarp();
     tmem_dealloc(tmem, W::kCols);
   }
