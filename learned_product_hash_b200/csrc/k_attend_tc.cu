@@ -6,9 +6,12 @@
 // section Mixer: exact causal softmax over the selected set, with the
 // selected values themselves).
 //
-// Persistent, warp-specialised kernel, one CTA per SM.  A CTA walks the
-// (b, hq, j) tiles blockIdx.x, blockIdx.x + gridDim.x, ... (consecutive CTAs
-// take consecutive query blocks of one head, so that head's K/V stays in L2).
+// Persistent, warp-specialised kernel, one CTA per SM.  The CTAs take
+// (b, hq, j) tiles from a global counter, head by head and within a head from
+// the last query block down: the CTAs running at any time work on
+// neighbouring query blocks of one head (that head's K/V stays in L2), and
+// the last tiles handed out are the first query blocks, which select the
+// fewest blocks, so the CTAs finish close together.
 // The selected blocks of a tile are taken in groups of 128 keys: two
 // consecutive 64-token blocks, or one 128-token block.
 //   warp 0        reads each sel row once (warp-parallel, ballot compaction)
@@ -185,7 +188,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = a.B * a.Hq * a.nb;
   const int g = a.Hq / a.Hkv;
-  const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
   if (warp == 1) {
     tmem_alloc(smem_u32(&tmem_base_s), C::kCols);
@@ -230,15 +232,26 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     int itv = 0, G = 0;                        // non-empty tiles, groups issued
     int last_q[2] = {-1, -1};                  // last tile whose Q each buffer received
     bool ok = true;
-    for (int it = 0; it < my_tiles && ok; ++it) {
-      const int tile = blockIdx.x + it * gridDim.x;
-      const int j = tile % a.nb, hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq);
+    for (int it = 0; ok; ++it) {
       const int slot = it % kSlots;
       if (it >= kSlots &&
           !__all_sync(0xffffffffu, wait_bar(BAR(C::bTEmpty + slot), ((it / kSlots) - 1) & 1, abort_flag))) {
         ok = false;
         break;
       }
+      int t = 0;
+      if (lane == 0) t = atomicAdd(a.tile_counter, 1);
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (t >= ntiles) {                       // no tiles left: tile -1 ends every role's loop
+        if (lane == 0) {
+          slot_tile(slot) = -1;
+          __threadfence_block();
+          mbar_arrive(BAR(C::bTFull + slot));
+        }
+        break;
+      }
+      const int tile = (t / a.nb) * a.nb + (a.nb - 1 - t % a.nb);
+      const int j = tile % a.nb, hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq);
       const int32_t* row = a.sel + static_cast<size_t>(tile) * a.nsel;
       const int e0 = lane < a.nsel ? row[lane] : -1, e1 = lane + 32 < a.nsel ? row[lane + 32] : -1;
       const bool v0 = valid_id(e0, j), v1 = valid_id(e1, j);
@@ -311,10 +324,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       prefetch_tmap(&tmV);
       int G = 0;
       bool ok = true;
-      for (int it = 0; it < my_tiles && ok; ++it) {
-        const int tile = blockIdx.x + it * gridDim.x;
+      for (int it = 0; ok; ++it) {
         const int slot = it % kSlots;
         if (!wait_bar(BAR(C::bTFull + slot), (it / kSlots) & 1, abort_flag)) { ok = false; break; }
+        const int tile = slot_tile(slot);
+        if (tile < 0) break;
         const int nblk = slot_s16(slot, 0);
         const int hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq), hkv = hq / g, tok0 = b * a.S;
         for (int n = 0; n < nblk && ok; ++G) {
@@ -360,7 +374,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       int q_nblk[4], q_g0[4], q_itv[4];
       int nring = 0, head = 0;
       int next_it = 0, next_itv = 0, next_g0 = 0;
-      bool ok = true;
+      bool ok = true, tiles_left = true;
       auto get = [&](const int* arr, int qi) {
         int v = arr[0];
 #pragma unroll
@@ -372,11 +386,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       // producer publishes a tile only after loading the previous tile's K,
       // which needs this lane's S MMAs.
       auto fetch = [&](bool block) {
-        while (next_it < my_tiles && ok && nring < 4) {
+        while (tiles_left && ok && nring < 4) {
           const int slot = next_it % kSlots;
           const uint32_t par = (next_it / kSlots) & 1;
           if (!block && !mbar_try_wait(BAR(C::bTFull + slot), par)) return;
           if (block && !wait_bar(BAR(C::bTFull + slot), par, abort_flag)) { ok = false; return; }
+          if (slot_tile(slot) < 0) { tiles_left = false; return; }
           ++next_it;
           const int nblk = slot_s16(slot, 0);
           mbar_arrive(BAR(C::bTEmpty + slot));   // nothing else is read from the slot
@@ -553,10 +568,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     };
     int itv = 0, g0 = 0, G = 0;
     bool ok = true;
-    for (int it = 0; it < my_tiles && ok; ++it) {
+    for (int it = 0; ok; ++it) {
       const int slot = it % kSlots;
       if (!wwait(C::bTFull + slot, (it / kSlots) & 1)) { ok = false; break; }
       const int tile = slot_tile(slot), nblk = slot_s16(slot, 0), diag = slot_s16(slot, 1);
+      if (tile < 0) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::bTEmpty + slot));
       const int j = tile % a.nb, hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq);
@@ -706,6 +722,8 @@ cudaError_t launch_tc(const AttendArgs& a, cudaStream_t st) {
   const long long ntiles = static_cast<long long>(a.B) * a.Hq * a.nb;
   const long long want = static_cast<long long>(sms) * per_sm;
   const unsigned grid = static_cast<unsigned>(ntiles < want ? ntiles : want);
+  // Every CTA takes one tile number past the last: the counter reaches ntiles + grid.
+  if (!a.tile_counter || ntiles + grid > 0x7fffffffLL) return cudaErrorInvalidValue;
   e = launch_pdl(k, dim3(grid), dim3(kThreads), C::kSmem, st, mq, mk, mv, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -109,6 +109,7 @@ struct AttendArgs {
   const int32_t* sel;      // [B,Hq,nb,R+L]
   void* out;               // [B,S,Hq,D]
   int32_t* status;         // device status word
+  int32_t* tile_counter;   // tensor-core kernel: zero at launch; tiles are handed out from it
   int B, S, Hq, Hkv, D, bs, nb, nsel;
   float scale;
 };

@@ -17,6 +17,10 @@ constexpr size_t kAlign = 256;
 constexpr size_t kMaxDynamicSmem = 227 * 1024;    // per CTA on sm_100a
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+// The forward workspace starts with four int32 words, zeroed by every call
+// before its first kernel: [0] the status word, [2] the attention kernel's
+// tile counter.
+constexpr size_t kStatusBytes = 4 * sizeof(int32_t);
 
 size_t esize(const mdr_config* c) { return c->dtype == MDR_BF16 ? 2 : 4; }
 
@@ -62,7 +66,7 @@ Layout layout_of(const mdr_config* c) {
   const size_t tok = static_cast<size_t>(c->B) * c->S;
   Layout l{};
   size_t o = 0;
-  l.status = o; o += align_up(16);
+  l.status = o; o += align_up(kStatusBytes);
   l.qrot = o;   o += align_up(tok * c->Hq * c->D * esize(c));
   l.krot = o;   o += align_up(tok * c->Hkv * c->D * esize(c));
   l.qbar = o;   o += align_up(static_cast<size_t>(c->B) * c->Hq * nb * c->D * sizeof(float));
@@ -147,6 +151,7 @@ mdr_status run_attend(const mdr_config* c, const void* qrot, const void* krot, c
                       const int32_t* sel, void* out, int32_t* status, cudaStream_t st) {
   mdr::AttendArgs aa{};
   aa.q = qrot; aa.k = krot; aa.v = v; aa.sel = sel; aa.out = out; aa.status = status;
+  aa.tile_counter = status + 2;
   aa.B = c->B; aa.S = c->S; aa.Hq = c->Hq; aa.Hkv = c->Hkv; aa.D = c->D; aa.bs = c->block;
   aa.nb = c->S / c->block; aa.nsel = c->R + c->L;
   aa.scale = mdr::detail::softmax_scale(c);
@@ -253,7 +258,7 @@ mdr_status mdr_attend(const mdr_config* cfg, const void* q, const void* k, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Layout l = layout_of(cfg);
   int32_t* status = at<int32_t>(ws, l.status);
-  MDR_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+  MDR_CUDA(cudaMemsetAsync(status, 0, kStatusBytes, st));
   SummarizeArgs a;
   fill_common(a, cfg, nullptr);
   a.x[0] = q; a.x[1] = k;
@@ -283,7 +288,7 @@ static mdr_status forward_impl(const mdr_config* cfg, const void* q, const void*
   int32_t* status = at<int32_t>(ws, l.status);
   float* qbar = rt->qbar ? rt->qbar : at<float>(ws, l.qbar);
   int32_t* qcodes = rt->qcodes ? rt->qcodes : at<int32_t>(ws, l.qcodes);
-  MDR_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+  MDR_CUDA(cudaMemsetAsync(status, 0, kStatusBytes, st));
   SummarizeArgs a;
   fill_common(a, cfg, codebooks);
   a.x[0] = q; a.x[1] = k;
