@@ -51,6 +51,7 @@
 
 #include <cuda.h>
 
+#include "attend_tc_common.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -60,7 +61,11 @@ namespace mdr {
 
 namespace {
 
-constexpr uint64_t kWaitNs = 2000000000ull;
+using atc::kWaitNs;
+using atc::valid_id;
+using atc::wait_bar;
+using atc::ex2_approx;
+using atc::pack_bf16;
 constexpr int kThreads = 352;   // 11 warps
 constexpr int kSlots = 4;       // tile descriptors in flight
 constexpr int kSlotBytes = 144; // int32 tile; int16 nblk, diag; int16 ids[64]
@@ -118,40 +123,11 @@ struct TcCfg {
   static_assert(kTile % 1024 == 0 && kPBytes % 1024 == 0 && kGRegion % 1024 == 0, "1024-byte aligned tiles");
 };
 
-// Valid entries of a sel row are ids in [0, j]; everything else is skipped.
-__device__ __forceinline__ bool valid_id(int id, int j) { return id >= 0 && id <= j; }
-
 // Size of the group that starts at block n (0-based, in the tile's list) of
 // a tile with nblk selected blocks: blocks 0-1, 2-3, ... pair up for bs = 64.
 template <bool kPair>
 __device__ __forceinline__ int group_size(int n, int nblk) {
   return (kPair && (n & 1) == 0 && n + 1 < nblk) ? 2 : 1;
-}
-
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  using namespace tc;
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > kWaitNs) return false;
-  }
-}
-
-// 2^x on the special-function unit (ex2.approx.ftz: about 2 ulp, subnormal
-// results flush to zero, which the softmax weights tolerate).
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 }  // namespace
@@ -732,6 +708,7 @@ cudaError_t launch_tc(const AttendArgs& a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t st) {
+  if (a.bs == 128 && a.Hkv > 0 && a.Hq / a.Hkv >= 2) return launch_attend_union(a, st);
   if (a.bs == 64 && a.D == 64) return launch_tc<64, 64>(a, st);
   if (a.bs == 64 && a.D == 128) return launch_tc<64, 128>(a, st);
   if (a.bs == 128 && a.D == 64) return launch_tc<128, 64>(a, st);

@@ -115,6 +115,9 @@ struct AttendArgs {
 };
 cudaError_t launch_attend_simt(const AttendArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t st);
+// Block 128 with two or more query heads per KV head: one unit per pair of
+// query heads, the union of their selected blocks gathered once.
+cudaError_t launch_attend_union(const AttendArgs& a, cudaStream_t st);
 
 // K6: one decode step (token t of every sequence) on a caller-owned state.
 struct DecodeArgs {

@@ -149,6 +149,27 @@ __device__ __forceinline__ void mma_bf16_c(uint32_t d_tmem, uint64_t adesc, uint
   }
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc], bf16 inputs, f32 accumulate.  A is
+// read from tensor memory: row i of the M rows in lane i, two bf16 of
+// consecutive K per 32-bit column (the lower K in the low half), K = 16 per
+// instruction, so 8 columns from a_tmem on.
+template <bool kAccumulate>
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc) {
+  if constexpr (kAccumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.eq.u32 p, 1, 1;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.eq.u32 p, 1, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc)
+        : "memory");
+  }
+}
+
 // The mbarrier gets one arrive when every tcgen05 operation this thread
 // issued before has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {

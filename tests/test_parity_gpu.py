@@ -63,6 +63,11 @@ EDGE = {
     "many_heads_bf16": (AR.with_(B=1, S=256, Hq=72, Hkv=72, D=128, keys="gaussian"), {}),
     # odd head count: token groups that do not tile the 512 summary threads
     "three_heads_bf16": (AR.with_(B=2, S=512, Hq=3, Hkv=3, D=128, block=128, keys="gaussian"), {}),
+    # block 128 with grouped query heads: pairs of heads share one gather of
+    # their selections' union (two and four heads per KV head, D 128 and 64)
+    "union_g2_d128": (CAPACITY.with_(S=12 * 128, block=128, D=128, Hq=4, Hkv=2, K=8, cap=16, R=4, L=2), {}),
+    "union_g4_long": (LONG.with_(B=2, S=24 * 128), {}),
+    "union_g2_d64": (CAPACITY.with_(S=10 * 128, block=128, Hq=2, Hkv=1, K=8, cap=16, R=5, L=1), {}),
 }
 
 
@@ -101,6 +106,50 @@ def test_bad_selection_sets_device_status():
     rows = np.ones((1, w.S, 1), dtype=bool)
     rows[0, 32:48] = False
     U.check_out(w, out.cpu().numpy(), res.out, rows)
+
+
+def test_union_attend_caller_selections():
+    """Block 128, two query heads per KV head (one unit per head pair, the
+    union of the pair's blocks gathered once), on selections a route never
+    writes: one head of a pair with nothing selected while the other has
+    blocks, both heads empty, disjoint and identical rows, ids in any order,
+    and an id past its query block (skipped, status 2)."""
+    import torch
+    from learned_product_hash_b200 import mdr
+    w = CAPACITY.with_(S=9 * 128, block=128, D=128, Hq=4, Hkv=2, K=8, cap=16, R=4, L=2)
+    inp = make_inputs(w, 21)
+    cfg = mdr.make_config(w)
+    q, k, v, _ = U.to_device(inp, w)
+    rng = np.random.default_rng(22)
+    sel = np.full((w.B, w.Hq, w.nb, w.R + w.L), -1, dtype=np.int32)
+    for hq in range(w.Hq):
+        for j in range(w.nb):
+            n = int(rng.integers(1, min(j + 1, w.R + w.L) + 1))
+            sel[0, hq, j, :n] = rng.permutation(j + 1)[:n]          # distinct, any order
+    sel[0, 0, 5] = -1                                              # head 0 empty, head 1 not
+    sel[0, 1, 7] = -1                                              # head 1 empty, head 0 not
+    sel[0, 2, 3] = -1                                              # both heads of a pair empty
+    sel[0, 3, 3] = -1
+    sel[0, 3, 6] = sel[0, 2, 6]                                    # identical rows
+    sel[0, 2, 8, :] = [0, 2, 4, 6, 8, -1]                          # disjoint rows
+    sel[0, 3, 8, :] = [1, 3, 5, 7, -1, -1]
+    sel[0, 1, 4, -1] = 6                                           # later than block 4
+    out = torch.empty_like(q)
+    ws = mdr.workspace(cfg)
+    mdr.mdr_attend(cfg, q, k, v, torch.from_numpy(sel).cuda(), out, ws)
+    assert mdr.mdr_read_device_status(ws) == 2
+    got = U.out_to_numpy(out, w)
+    p = O.Params.of(w)
+    qr, kr = O.rope(inp.q.astype(np.float64), p.rope_base), O.rope(inp.k.astype(np.float64), p.rope_base)
+    jj = np.arange(w.nb)[None, None, :, None]
+    clean = np.where((sel >= 0) & (sel <= jj), sel, -1)
+    has = (clean >= 0).any(axis=-1)
+    rows = [(0, hq, j) for hq in range(w.Hq) for j in range(w.nb) if has[0, hq, j]]
+    ref = O.attend(qr, kr, inp.v.astype(np.float64), clean, w.block, p.softmax_scale, rows)
+    for hq, j in ((0, 5), (1, 7), (2, 3), (3, 3)):
+        assert not has[0, hq, j]
+        assert (got[0, j * w.block:(j + 1) * w.block, hq] == 0).all()
+    U.check_out(w, got, ref)
 
 
 def test_host_entry_point_matches_device():
