@@ -179,7 +179,8 @@ class ClockSampler:
 # sources they were taken from, and the workload they were taken on.
 PROFILED_TRAFFIC = {
     "attend": ("profiles/attend_tc_scaling32k.txt", "scaling32k",
-               ("learned_product_hash_b200/csrc/k_attend_tc.cu", "learned_product_hash_b200/csrc/tc_ptx.cuh")),
+               ("learned_product_hash_b200/csrc/k_attend_tc.cu", "learned_product_hash_b200/csrc/attend_tc_common.cuh",
+                "learned_product_hash_b200/csrc/tc_ptx.cuh")),
 }
 
 
