@@ -191,11 +191,18 @@ mdr_status mdr_forward_profiled(const mdr_config* cfg, const void* q,
 mdr_status mdr_host_workspace_bytes(const mdr_config* cfg, size_t* bytes);
 
 /* The forward from host buffers: copies q, k, v, codebooks to the device
- * workspace, runs mdr_forward there, copies out, sel, overflow and maxload
- * back, and synchronises the stream before returning.  q, k, v, codebooks,
- * out: host; sel_host [B,Hq,nb,R+L], overflow_host and maxload_host [B,Hkv]:
- * host int32 (each may be NULL to skip its copy).  dev_ws: device, at least
- * mdr_host_workspace_bytes.                                                 */
+ * workspace, runs the forward there, copies out, sel, overflow and maxload
+ * back, and synchronises before returning.  The forward is causal (block j's
+ * output needs the inputs of blocks <= j only), so it runs in up to eight
+ * chunks of query blocks: a chunk's inputs are copied in on one internal
+ * stream, its blocks summarised, appended to the posting lists, routed and
+ * attended on `stream`, and its output copied out on another internal
+ * stream while the next chunk's inputs come in.  The results are
+ * bit-identical to mdr_forward.  The copies overlap only from pinned host
+ * memory.  q, k, v, codebooks, out: host; sel_host [B,Hq,nb,R+L],
+ * overflow_host and maxload_host [B,Hkv]: host int32 (each may be NULL to
+ * skip its copy).  dev_ws: device, at least mdr_host_workspace_bytes.  Work
+ * enqueued on `stream` before the call comes first.                         */
 mdr_status mdr_forward_host(const mdr_config* cfg, const void* q_host,
                             const void* k_host, const void* v_host,
                             const float* codebooks_host, void* out_host,

@@ -24,10 +24,12 @@ attend_simt_kernel(const AttendArgs a) {
   __shared__ int32_t blocks[kMaxSel];
   __shared__ int nblk;
   grid_dependency_wait();
-  const int tile = blockIdx.x;
-  const int j = tile % a.nb;
-  const int hq = (tile / a.nb) % a.Hq;
-  const int b = tile / (a.nb * a.Hq);
+  const int nbr = a.nbr > 0 ? a.nbr : a.nb;         // query blocks a.j0 .. a.j0 + nbr - 1
+  const int bhq = blockIdx.x / nbr;
+  const int j = a.j0 + static_cast<int>(blockIdx.x - bhq * nbr);
+  const int hq = bhq % a.Hq;
+  const int b = bhq / a.Hq;
+  const int tile = bhq * a.nb + j;
   const int hkv = hq / (a.Hq / a.Hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const T* q = static_cast<const T*>(a.q);
@@ -91,7 +93,9 @@ attend_simt_kernel(const AttendArgs a) {
 }
 
 cudaError_t launch_attend_simt(const AttendArgs& a, bool bf16, cudaStream_t st) {
-  const unsigned grid = static_cast<unsigned>(a.B) * a.Hq * a.nb;
+  const int nbr = a.nbr > 0 ? a.nbr : a.nb;
+  if (a.j0 < 0 || a.j0 + nbr > a.nb || (a.nbr <= 0 && a.j0 != 0)) return cudaErrorInvalidValue;
+  const unsigned grid = static_cast<unsigned>(a.B) * a.Hq * nbr;
   const cudaError_t e = bf16 ? launch_pdl(attend_simt_kernel<__nv_bfloat16>, dim3(grid), dim3(128), 0, st, a)
                              : launch_pdl(attend_simt_kernel<float>, dim3(grid), dim3(128), 0, st, a);
   if (e != cudaSuccess) return e;

@@ -162,7 +162,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   // slot_s16(s, 0) = nblk, (s, 1) = diag, (s, 2 + n) = id n
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntiles = a.B * a.Hq * a.nb;
+  const int nbr = a.nbr > 0 ? a.nbr : a.nb;         // query blocks a.j0 .. a.j0 + nbr - 1
+  const int ntiles = a.B * a.Hq * nbr;
   const int g = a.Hq / a.Hkv;
 
   if (warp == 1) {
@@ -226,7 +227,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         break;
       }
-      const int tile = (t / a.nb) * a.nb + (a.nb - 1 - t % a.nb);
+      const int tile = (t / nbr) * a.nb + (a.j0 + nbr - 1 - t % nbr);
       const int j = tile % a.nb, hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq);
       const int32_t* row = a.sel + static_cast<size_t>(tile) * a.nsel;
       const int e0 = lane < a.nsel ? row[lane] : -1, e1 = lane + 32 < a.nsel ? row[lane + 32] : -1;
@@ -695,7 +696,9 @@ cudaError_t launch_tc(const AttendArgs& a, cudaStream_t st) {
   // Tensor memory: at most 512 columns per SM.
   per_sm = per_sm < 512 / C::kCols ? per_sm : 512 / C::kCols;
   if (per_sm < 1) per_sm = 1;
-  const long long ntiles = static_cast<long long>(a.B) * a.Hq * a.nb;
+  const int nbr = a.nbr > 0 ? a.nbr : a.nb;
+  if (a.j0 < 0 || a.j0 + nbr > a.nb || (a.nbr <= 0 && a.j0 != 0)) return cudaErrorInvalidValue;
+  const long long ntiles = static_cast<long long>(a.B) * a.Hq * nbr;
   const long long want = static_cast<long long>(sms) * per_sm;
   const unsigned grid = static_cast<unsigned>(ntiles < want ? ntiles : want);
   // Every CTA takes one tile number past the last: the counter reaches ntiles + grid.

@@ -160,7 +160,8 @@ attend_union_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = a.Hq / a.Hkv;
   const int npair = (g + 1) / 2;
-  const int nunits = a.B * a.Hkv * npair * a.nb;
+  const int nbr = a.nbr > 0 ? a.nbr : a.nb;         // query blocks a.j0 .. a.j0 + nbr - 1
+  const int nunits = a.B * a.Hkv * npair * nbr;
 
   if (warp == 1) {
     tmem_alloc(smem_u32(&tmem_base_s), C::kCols);
@@ -197,8 +198,8 @@ attend_union_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   };
   // Unit t -> (b, hkv, pair p, j): pairs in order, query blocks from the last.
   auto decode = [&](int t, int& b, int& hkv, int& p, int& j) {
-    const int bp = t / a.nb;
-    j = a.nb - 1 - (t - bp * a.nb);
+    const int bp = t / nbr;
+    j = a.j0 + nbr - 1 - (t - bp * nbr);
     p = bp % npair;
     const int bh = bp / npair;
     hkv = bh % a.Hkv;
@@ -763,7 +764,9 @@ cudaError_t launch_union(const AttendArgs& a, cudaStream_t st) {
   const int sms = cached_sm_count();
   if (sms <= 0) return cudaErrorUnknown;
   const int g = a.Hq / a.Hkv;
-  const long long nunits = static_cast<long long>(a.B) * a.Hkv * ((g + 1) / 2) * a.nb;
+  const int nbr = a.nbr > 0 ? a.nbr : a.nb;
+  if (a.j0 < 0 || a.j0 + nbr > a.nb || (a.nbr <= 0 && a.j0 != 0)) return cudaErrorInvalidValue;
+  const long long nunits = static_cast<long long>(a.B) * a.Hkv * ((g + 1) / 2) * nbr;
   // 512 tensor-memory columns: one CTA per SM.
   const unsigned grid = static_cast<unsigned>(nunits < sms ? nunits : sms);
   // Every CTA takes one unit number past the last: the counter reaches nunits + grid.

@@ -59,12 +59,14 @@ codes_kernel(const __grid_constant__ CodesArgs a) {
   __syncthreads();
   if (!a.codebooks_written_before) grid_dependency_wait();   // the summaries come from the previous kernel
 
-  const long long rows0 = a.xbar[0] ? static_cast<long long>(a.B) * a.H[0] * a.nb : 0;
-  const long long rows1 = a.xbar[1] ? static_cast<long long>(a.B) * a.H[1] * a.nb : 0;
+  const int nbr = a.nbr > 0 ? a.nbr : a.nb;         // blocks a.j0 .. a.j0 + nbr - 1
+  const long long rows0 = a.xbar[0] ? static_cast<long long>(a.B) * a.H[0] * nbr : 0;
+  const long long rows1 = a.xbar[1] ? static_cast<long long>(a.B) * a.H[1] * nbr : 0;
   const long long nwarps = static_cast<long long>(gridDim.x) * kCodeWarps;
   for (long long row = static_cast<long long>(blockIdx.x) * kCodeWarps + warp; row < rows0 + rows1; row += nwarps) {
     const int side = row < rows0 ? 0 : 1;
-    const long long rr = side ? row - rows0 : row;             // (b * H + h) * nb + j
+    const long long rl = side ? row - rows0 : row;
+    const long long rr = (rl / nbr) * a.nb + a.j0 + rl % nbr;  // (b * H + h) * nb + j
     const float* xb = a.xbar[side] + rr * D;
     for (int d4 = lane; d4 < D / 4; d4 += 32)
       reinterpret_cast<float4*>(xs)[d4] = __ldg(reinterpret_cast<const float4*>(xb) + d4);
@@ -119,8 +121,10 @@ codes_kernel(const __grid_constant__ CodesArgs a) {
 }
 
 cudaError_t launch_codes(const CodesArgs& a, cudaStream_t st) {
-  const long long rows = (a.xbar[0] ? static_cast<long long>(a.B) * a.H[0] * a.nb : 0) +
-                         (a.xbar[1] ? static_cast<long long>(a.B) * a.H[1] * a.nb : 0);
+  const int nbr = a.nbr > 0 ? a.nbr : a.nb;
+  if (a.j0 < 0 || a.j0 + nbr > a.nb || (a.nbr <= 0 && a.j0 != 0)) return cudaErrorInvalidValue;
+  const long long rows = (a.xbar[0] ? static_cast<long long>(a.B) * a.H[0] * nbr : 0) +
+                         (a.xbar[1] ? static_cast<long long>(a.B) * a.H[1] * nbr : 0);
   if (rows == 0) return cudaSuccess;
   if (a.K > kMaxK || a.P > 4) return cudaErrorInvalidValue;
   const size_t smem =

@@ -33,29 +33,32 @@ lists_kernel(const ListsArgs a) {
   grid_dependency_wait();
   const int bh = blockIdx.x;
   int32_t* lists = a.lists + static_cast<size_t>(bh) * static_cast<size_t>(a.A) * a.cap;
-  const int32_t* addr = a.addr + static_cast<size_t>(bh) * a.nb;
+  const int j0 = a.j0, j1 = a.j1 > 0 ? a.j1 : a.nb, n = j1 - j0;   // blocks added
+  const int32_t* addr = a.addr + static_cast<size_t>(bh) * a.nb + j0;
   const int tid = threadIdx.x, lane = tid & 31;
   int32_t* saddr = cnt + a.A;
+  int32_t* load = a.load + static_cast<size_t>(bh) * a.A;
 
-  for (int x = tid; x < a.A; x += kListThreads) cnt[x] = 0;
-  for (int x = tid; x < a.nb; x += kListThreads) saddr[x] = addr[x];   // one coalesced read
+  // Counts so far: none, or the lists of blocks < j0.
+  for (int x = tid; x < a.A; x += kListThreads) cnt[x] = j0 == 0 ? 0 : load[x];
+  for (int x = tid; x < n; x += kListThreads) saddr[x] = addr[x];      // one coalesced read
   if (tid == 0) { s_ovf = 0; s_max = 0; }
   __syncthreads();
 
   if (tid < 32) {
     const unsigned lower = (1u << lane) - 1u;
-    int ad_next = lane < a.nb ? saddr[lane] : -1;
-    for (int c0 = 0; c0 < a.nb; c0 += 32) {
+    int ad_next = lane < n ? saddr[lane] : -1;
+    for (int c0 = 0; c0 < n; c0 += 32) {
       const int i = c0 + lane;
       const int ad = ad_next;
-      ad_next = i + 32 < a.nb ? saddr[i + 32] : -1;
-      const bool valid = i < a.nb;
+      ad_next = i + 32 < n ? saddr[i + 32] : -1;
+      const bool valid = i < n;
       const unsigned vm = __ballot_sync(0xffffffffu, valid);
       if (valid) {
         const unsigned peers = __match_any_sync(vm, ad);
         const int base = cnt[ad];
         const int rank = base + __popc(peers & lower);
-        if (rank < a.cap) lists[static_cast<size_t>(ad) * a.cap + rank] = i;
+        if (rank < a.cap) lists[static_cast<size_t>(ad) * a.cap + rank] = j0 + i;
         __syncwarp(vm);                            // every peer read the old count
         if ((peers & lower) == 0) cnt[ad] = base + __popc(peers);
       }
@@ -65,7 +68,6 @@ lists_kernel(const ListsArgs a) {
   __syncthreads();
 
   int ovf = 0, mx = 0;
-  int32_t* load = a.load + static_cast<size_t>(bh) * a.A;
   for (int x = tid; x < a.A; x += kListThreads) {
     const int c = cnt[x];
     load[x] = c;
@@ -83,7 +85,9 @@ lists_kernel(const ListsArgs a) {
 }
 
 cudaError_t launch_lists(const ListsArgs& a, cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(a.A + a.nb) * sizeof(int32_t);
+  const int j1 = a.j1 > 0 ? a.j1 : a.nb;
+  if (a.j0 < 0 || a.j0 >= j1 || j1 > a.nb) return cudaErrorInvalidValue;
+  const size_t smem = static_cast<size_t>(a.A + (j1 - a.j0)) * sizeof(int32_t);
   cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(lists_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   e = launch_pdl(lists_kernel, dim3(a.B * a.H), dim3(kListThreads), smem, st, a);

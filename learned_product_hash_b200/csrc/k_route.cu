@@ -62,12 +62,14 @@ route_kernel(const RouteArgs a) {
   int32_t* cand = offs + 68;                       // [kBatch) batch, [kBatch, kBatch+R) winners
   float* score = reinterpret_cast<float*>(cand + kBatch + 32);
 
-  const long long route = static_cast<long long>(blockIdx.x) * kRouteWarps + warp;
-  const long long nroutes = static_cast<long long>(a.B) * a.Hq * a.nb;
-  if (route >= nroutes) return;
-  const int j = static_cast<int>(route % a.nb);
-  const int hq = static_cast<int>((route / a.nb) % a.Hq);
-  const int b = static_cast<int>(route / (static_cast<long long>(a.nb) * a.Hq));
+  const int nbr = a.nbr > 0 ? a.nbr : a.nb;         // query blocks a.j0 .. a.j0 + nbr - 1
+  const long long rl = static_cast<long long>(blockIdx.x) * kRouteWarps + warp;
+  if (rl >= static_cast<long long>(a.B) * a.Hq * nbr) return;
+  const long long bhq = rl / nbr;
+  const int j = a.j0 + static_cast<int>(rl - bhq * nbr);
+  const int hq = static_cast<int>(bhq % a.Hq);
+  const int b = static_cast<int>(bhq / a.Hq);
+  const long long route = bhq * a.nb + j;           // (b, hq, j) in the [B,Hq,nb] grid
   const int hkv = hq / (a.Hq / a.Hkv);
   const long long bh = static_cast<long long>(b) * a.Hkv + hkv;
   const int32_t* lists = a.lists + bh * a.A * a.cap;
@@ -276,7 +278,9 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   const auto kern = a.force ? route_kernel<true> : route_kernel<false>;
   cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const long long nroutes = static_cast<long long>(a.B) * a.Hq * a.nb;
+  const int nbr = a.nbr > 0 ? a.nbr : a.nb;
+  if (a.j0 < 0 || a.j0 + nbr > a.nb || (a.nbr <= 0 && a.j0 != 0)) return cudaErrorInvalidValue;
+  const long long nroutes = static_cast<long long>(a.B) * a.Hq * nbr;
   const unsigned grid = static_cast<unsigned>((nroutes + kRouteWarps - 1) / kRouteWarps);
   e = launch_pdl(kern, dim3(grid), dim3(kRouteWarps * 32), smem, st, a);
   if (e != cudaSuccess) return e;

@@ -109,12 +109,13 @@ summarize_kernel(const __grid_constant__ SummarizeArgs a, const SumPlan pl) {
   struct Unit {
     int b, j, side, h0, HGa, rowbytes, TPC, nch;
   };
+  const int nbr = a.nbr > 0 ? a.nbr : a.nb;        // blocks a.j0 .. a.j0 + nbr - 1
   auto unit_of = [&](int u) {
     Unit x;
     const int bj = u / pl.NG;
     const int sg = u - bj * pl.NG;
-    x.b = bj / a.nb;
-    x.j = bj - x.b * a.nb;
+    x.b = bj / nbr;
+    x.j = a.j0 + (bj - x.b * nbr);
     x.side = sg < pl.ng[0] ? 0 : 1;
     const int hg = x.side ? sg - pl.ng[0] : sg;
     const int H = a.H[x.side];
@@ -335,7 +336,9 @@ bool make_plan(const SummarizeArgs& a, bool bf16, SumPlan& pl) {
     if (rowbytes > kMaxRowBytes || rowbytes % 16 != 0) return false;
   }
   pl.NG = pl.ng[0] + pl.ng[1];
-  const long long nunits = static_cast<long long>(a.B) * a.nb * pl.NG;
+  const int nbr = a.nbr > 0 ? a.nbr : a.nb;
+  if (a.j0 < 0 || a.j0 + nbr > a.nb || (a.nbr <= 0 && a.j0 != 0)) return false;
+  const long long nunits = static_cast<long long>(a.B) * nbr * pl.NG;
   if (nunits > 0x7fffffffLL) return false;
   pl.nunits = static_cast<int>(nunits);
   auto up = [](size_t x) { return (x + 127) / 128 * 128; };
@@ -392,6 +395,7 @@ cudaError_t launch_summarize(const SummarizeArgs& a, bool bf16, cudaStream_t st)
   c.H[0] = a.H[0]; c.H[1] = a.H[1];
   c.qcodes = a.qcodes; c.addr = a.addr; c.codebooks = a.codebooks;
   c.B = a.B; c.nb = a.nb; c.D = a.D; c.P = a.P; c.K = a.K; c.probes = a.probes;
+  c.j0 = a.j0; c.nbr = a.nbr;
   return launch_codes(c, st);
 }
 

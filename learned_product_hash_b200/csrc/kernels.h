@@ -26,6 +26,7 @@ struct SummarizeArgs {
   int32_t* lists_fill;     // posting lists [B, Hkv*A*cap] padded with -1 by the key side; null = skip
   size_t lists_per_seq;    // Hkv*A*cap
   int32_t* status;         // device status word (a wait that ran out writes 1); null = none
+  int j0, nbr;             // blocks j0 .. j0 + nbr - 1 only (nbr = 0: every block, j0 = 0)
 };
 size_t summarize_smem_bytes(int bs, int D, int Hq, int Hkv);
 // Launches K1 (rotation, summaries) and, when qcodes or addr is given, K2.
@@ -40,6 +41,7 @@ struct CodesArgs {
   const float* codebooks;  // [P,K,D/P]
   int B, nb, D, P, K, probes;
   bool codebooks_written_before;   // the previous kernel on the stream writes the codebooks
+  int j0, nbr;             // rows of blocks j0 .. j0 + nbr - 1 only (nbr = 0: every block)
 };
 cudaError_t launch_codes(const CodesArgs& a, cudaStream_t st);
 
@@ -69,6 +71,10 @@ struct ListsArgs {
   int32_t* overflow;       // [B,Hkv]
   int32_t* maxload;        // [B,Hkv]
   int B, H, nb, A, cap;
+  // Blocks j0 .. j1 - 1 are added, in order.  j0 = 0 starts from empty
+  // lists; j0 > 0 continues from the counts in load (the lists of blocks
+  // < j0 already built).  j1 = 0: every block.
+  int j0, j1;
 };
 cudaError_t launch_lists(const ListsArgs& a, cudaStream_t st);
 
@@ -87,6 +93,7 @@ struct RouteArgs {
   // incomplete) every route writes a row of -1 and ncand -1 instead of routing.
   const int32_t* upstream_status;
   int B, Hq, Hkv, nb, D, P, K, A, probes, cap, R, L;
+  int j0, nbr;             // query blocks j0 .. j0 + nbr - 1 only (nbr = 0: every block)
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 
@@ -112,6 +119,7 @@ struct AttendArgs {
   int32_t* tile_counter;   // tensor-core kernel: zero at launch; tiles are handed out from it
   int B, S, Hq, Hkv, D, bs, nb, nsel;
   float scale;
+  int j0, nbr;             // query blocks j0 .. j0 + nbr - 1 only (nbr = 0: every block)
 };
 cudaError_t launch_attend_simt(const AttendArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t st);

@@ -133,23 +133,29 @@ mdr_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MDR_OK : MDR_E
 
 #define MDR_CUDA(x) MDR_TRY(cuda_status(x))
 
-mdr_status run_lists(const mdr_config* c, const mdr_index* idx, cudaStream_t st) {
+// The list, route and attention steps over query / key blocks j0 .. j1 - 1
+// (j1 = 0: every block).
+mdr_status run_lists(const mdr_config* c, const mdr_index* idx, cudaStream_t st, int j0 = 0, int j1 = 0) {
   mdr::ListsArgs la{};
   la.addr = idx->addr; la.lists = idx->lists; la.load = idx->load;
   la.overflow = idx->overflow; la.maxload = idx->maxload;
   la.B = c->B; la.H = c->Hkv; la.nb = c->S / c->block; la.A = ipow(c->K, c->P); la.cap = c->cap;
+  la.j0 = j0; la.j1 = j1;
   return cuda_status(mdr::launch_lists(la, st));
 }
 
 mdr_status run_route(const mdr_config* c, const float* qbar, const int32_t* qcodes,
                      const mdr_index* idx, int32_t* sel, int32_t* ncand, cudaStream_t st,
-                     const int32_t* force = nullptr) {
-  return cuda_status(mdr::launch_route(mdr::detail::route_args(c, qbar, qcodes, idx, sel, ncand, force), st));
+                     const int32_t* force = nullptr, int j0 = 0, int j1 = 0) {
+  mdr::RouteArgs ra = mdr::detail::route_args(c, qbar, qcodes, idx, sel, ncand, force);
+  ra.j0 = j0; ra.nbr = j1 > 0 ? j1 - j0 : 0;
+  return cuda_status(mdr::launch_route(ra, st));
 }
 
 mdr_status run_attend(const mdr_config* c, const void* qrot, const void* krot, const void* v,
-                      const int32_t* sel, void* out, int32_t* status, cudaStream_t st) {
+                      const int32_t* sel, void* out, int32_t* status, cudaStream_t st, int j0 = 0, int j1 = 0) {
   mdr::AttendArgs aa{};
+  aa.j0 = j0; aa.nbr = j1 > 0 ? j1 - j0 : 0;
   aa.q = qrot; aa.k = krot; aa.v = v; aa.sel = sel; aa.out = out; aa.status = status;
   aa.tile_counter = status + 2;
   aa.B = c->B; aa.S = c->S; aa.Hq = c->Hq; aa.Hkv = c->Hkv; aa.D = c->D; aa.bs = c->block;
@@ -347,7 +353,128 @@ HostLayout host_layout_of(const mdr_config* c) {
   h.total = o;
   return h;
 }
+
+// Streams and events of one mdr_forward_host call: the input copies run on
+// `in`, the kernels on the caller's stream, the output copies on `out`, so
+// that chunk c's output copy overlaps chunk c+1's input copy (the link is
+// full duplex).
+struct HostPipeline {
+  static constexpr int kMaxChunks = 8;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, in_done[kMaxChunks] = {}, comp_done[kMaxChunks] = {};
+  cudaError_t init(cudaStream_t st) {
+    cudaError_t e;
+    if ((e = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&start, cudaEventDisableTiming)) != cudaSuccess) return e;
+    for (int c = 0; c < kMaxChunks; ++c) {
+      if ((e = cudaEventCreateWithFlags(&in_done[c], cudaEventDisableTiming)) != cudaSuccess) return e;
+      if ((e = cudaEventCreateWithFlags(&comp_done[c], cudaEventDisableTiming)) != cudaSuccess) return e;
+    }
+    // The copies start after whatever the caller enqueued before.
+    if ((e = cudaEventRecord(start, st)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(in, start, 0)) != cudaSuccess) return e;
+    return cudaStreamWaitEvent(out, start, 0);
+  }
+  // Waits for all three streams, then releases the streams and events.
+  cudaError_t finish(cudaStream_t st) {
+    cudaError_t r = cudaSuccess, e;
+    for (cudaStream_t s : {in, st, out})
+      if ((s == st || s) && (e = cudaStreamSynchronize(s)) != cudaSuccess && r == cudaSuccess) r = e;
+    if (in) cudaStreamDestroy(in);
+    if (out) cudaStreamDestroy(out);
+    if (start) cudaEventDestroy(start);
+    for (int c = 0; c < kMaxChunks; ++c) {
+      if (in_done[c]) cudaEventDestroy(in_done[c]);
+      if (comp_done[c]) cudaEventDestroy(comp_done[c]);
+    }
+    in = out = nullptr;
+    return r;
+  }
+};
+
+// Rows t0 .. t1 - 1 of every sequence of a [B,S,...] tensor with row_bytes
+// per token, one strided copy.
+cudaError_t copy_rows(void* dst, const void* src, size_t row_bytes, int B, int S, int t0, int t1,
+                      cudaMemcpyKind kind, cudaStream_t st) {
+  const size_t pitch = row_bytes * S, off = row_bytes * t0;
+  return cudaMemcpy2DAsync(static_cast<char*>(dst) + off, pitch, static_cast<const char*>(src) + off, pitch,
+                           row_bytes * (t1 - t0), B, kind, st);
+}
+
 }  // namespace
+
+// The forward is causal: query block j's output needs the inputs of blocks
+// <= j only (its summary, the index of key blocks <= j, the K/V of its
+// selected blocks), and the posting lists of blocks < j are the same whether
+// or not later blocks exist (each list keeps its first cap blocks in
+// ascending order).  So the sequence runs in chunks of query blocks: chunk
+// c's inputs are copied in, its blocks summarised, appended to the lists,
+// routed and attended, and its output copied out while chunk c+1 comes in.
+// The result is bit-identical to mdr_forward on the whole sequence.
+static mdr_status forward_host_chunked(const mdr_config* cfg, const HostLayout& h, const void* q_host,
+                                       const void* k_host, const void* v_host, const float* codebooks_host,
+                                       void* out_host, int32_t* sel_host, int32_t* overflow_host,
+                                       int32_t* maxload_host, void* dev_ws, cudaStream_t st, HostPipeline& pl) {
+  const int nb = cfg->S / cfg->block, nsel = cfg->R + cfg->L;
+  const size_t es = esize(cfg);
+  const size_t qrow = static_cast<size_t>(cfg->Hq) * cfg->D * es, krow = static_cast<size_t>(cfg->Hkv) * cfg->D * es;
+  const int nchunk = nb < HostPipeline::kMaxChunks ? nb : HostPipeline::kMaxChunks;
+  const Layout l = layout_of(cfg);
+  void* ws = at<void>(dev_ws, h.dev);
+  int32_t* status = at<int32_t>(ws, l.status);
+  float* qbar = at<float>(ws, l.qbar);
+  int32_t* qcodes = at<int32_t>(ws, l.qcodes);
+  void *q = at<void>(dev_ws, h.q), *k = at<void>(dev_ws, h.k), *v = at<void>(dev_ws, h.v);
+  void* out = at<void>(dev_ws, h.out);
+  const float* cb = at<float>(dev_ws, h.cb);
+  mdr_index idx{at<float>(dev_ws, h.kbar), at<int32_t>(dev_ws, h.addr), at<int32_t>(dev_ws, h.lists),
+                at<int32_t>(dev_ws, h.load), at<int32_t>(dev_ws, h.ovf), at<int32_t>(dev_ws, h.maxl)};
+  int32_t* sel = at<int32_t>(dev_ws, h.sel);
+  const size_t lists_bytes = static_cast<size_t>(cfg->B) * cfg->Hkv * ipow(cfg->K, cfg->P) * cfg->cap * sizeof(int32_t);
+
+  MDR_CUDA(cudaMemcpyAsync(at<void>(dev_ws, h.cb), codebooks_host, static_cast<size_t>(cfg->K) * cfg->D * sizeof(float),
+                           cudaMemcpyHostToDevice, pl.in));
+  MDR_CUDA(cudaMemsetAsync(status, 0, kStatusBytes, st));
+  MDR_CUDA(cudaMemsetAsync(idx.lists, 0xff, lists_bytes, st));   // every list empty (-1)
+  for (int c = 0; c < nchunk; ++c) {
+    const int j0 = static_cast<int>(static_cast<long long>(nb) * c / nchunk);
+    const int j1 = static_cast<int>(static_cast<long long>(nb) * (c + 1) / nchunk);
+    const int t0 = j0 * cfg->block, t1 = j1 * cfg->block;
+    MDR_CUDA(copy_rows(q, q_host, qrow, cfg->B, cfg->S, t0, t1, cudaMemcpyHostToDevice, pl.in));
+    MDR_CUDA(copy_rows(k, k_host, krow, cfg->B, cfg->S, t0, t1, cudaMemcpyHostToDevice, pl.in));
+    MDR_CUDA(copy_rows(v, v_host, krow, cfg->B, cfg->S, t0, t1, cudaMemcpyHostToDevice, pl.in));
+    MDR_CUDA(cudaEventRecord(pl.in_done[c], pl.in));
+    MDR_CUDA(cudaStreamWaitEvent(st, pl.in_done[c], 0));
+    MDR_CUDA(cudaMemsetAsync(status + 2, 0, sizeof(int32_t), st));   // the attention's tile counter
+    SummarizeArgs a;
+    fill_common(a, cfg, cb);
+    a.x[0] = q; a.x[1] = k;
+    a.xrot[0] = at<void>(ws, l.qrot); a.xrot[1] = at<void>(ws, l.krot);
+    a.xbar[0] = qbar; a.xbar[1] = idx.kbar;
+    a.qcodes = qcodes; a.addr = idx.addr;
+    a.status = status;
+    a.j0 = j0; a.nbr = j1 - j0;
+    MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
+    MDR_TRY(run_lists(cfg, &idx, st, j0, j1));
+    MDR_TRY(run_route(cfg, qbar, qcodes, &idx, sel, nullptr, st, nullptr, j0, j1));
+    MDR_TRY(run_attend(cfg, at<void>(ws, l.qrot), at<void>(ws, l.krot), v, sel, out, status, st, j0, j1));
+    MDR_CUDA(cudaEventRecord(pl.comp_done[c], st));
+    MDR_CUDA(cudaStreamWaitEvent(pl.out, pl.comp_done[c], 0));
+    MDR_CUDA(copy_rows(out_host, out, qrow, cfg->B, cfg->S, t0, t1, cudaMemcpyDeviceToHost, pl.out));
+    if (sel_host) {
+      const size_t row = static_cast<size_t>(nsel) * sizeof(int32_t);
+      MDR_CUDA(cudaMemcpy2DAsync(sel_host + static_cast<size_t>(j0) * nsel, nb * row, sel + static_cast<size_t>(j0) * nsel,
+                                 nb * row, (j1 - j0) * row, static_cast<size_t>(cfg->B) * cfg->Hq,
+                                 cudaMemcpyDeviceToHost, pl.out));
+    }
+  }
+  const size_t bh = static_cast<size_t>(cfg->B) * cfg->Hkv * sizeof(int32_t);
+  if (overflow_host) MDR_CUDA(cudaMemcpyAsync(overflow_host, idx.overflow, bh, cudaMemcpyDeviceToHost, pl.out));
+  if (maxload_host) MDR_CUDA(cudaMemcpyAsync(maxload_host, idx.maxload, bh, cudaMemcpyDeviceToHost, pl.out));
+  return MDR_OK;
+}
+
 
 mdr_status mdr_host_workspace_bytes(const mdr_config* cfg, size_t* bytes) {
   MDR_TRY(check(cfg));
@@ -366,30 +493,14 @@ mdr_status mdr_forward_host(const mdr_config* cfg, const void* q_host, const voi
   if (!dev_ws || reinterpret_cast<uintptr_t>(dev_ws) % kAlign != 0 || dev_ws_bytes < h.total)
     return MDR_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t nb = cfg->S / cfg->block, tok = static_cast<size_t>(cfg->B) * cfg->S;
-  const size_t qb = tok * cfg->Hq * cfg->D * esize(cfg), kb = tok * cfg->Hkv * cfg->D * esize(cfg);
-  MDR_CUDA(cudaMemcpyAsync(at<void>(dev_ws, h.q), q_host, qb, cudaMemcpyHostToDevice, st));
-  MDR_CUDA(cudaMemcpyAsync(at<void>(dev_ws, h.k), k_host, kb, cudaMemcpyHostToDevice, st));
-  MDR_CUDA(cudaMemcpyAsync(at<void>(dev_ws, h.v), v_host, kb, cudaMemcpyHostToDevice, st));
-  MDR_CUDA(cudaMemcpyAsync(at<void>(dev_ws, h.cb), codebooks_host,
-                           static_cast<size_t>(cfg->K) * cfg->D * sizeof(float), cudaMemcpyHostToDevice, st));
-  mdr_index idx{at<float>(dev_ws, h.kbar), at<int32_t>(dev_ws, h.addr), at<int32_t>(dev_ws, h.lists),
-                at<int32_t>(dev_ws, h.load), at<int32_t>(dev_ws, h.ovf), at<int32_t>(dev_ws, h.maxl)};
-  mdr_route_out rt{at<int32_t>(dev_ws, h.sel), nullptr, nullptr, nullptr};
-  MDR_TRY(mdr_forward(cfg, at<void>(dev_ws, h.q), at<void>(dev_ws, h.k), at<void>(dev_ws, h.v),
-                      at<float>(dev_ws, h.cb), &idx, &rt, at<void>(dev_ws, h.out),
-                      at<void>(dev_ws, h.dev), layout_of(cfg).total, stream));
-  MDR_CUDA(cudaMemcpyAsync(out_host, at<void>(dev_ws, h.out), qb, cudaMemcpyDeviceToHost, st));
-  if (sel_host)
-    MDR_CUDA(cudaMemcpyAsync(sel_host, rt.sel, static_cast<size_t>(cfg->B) * cfg->Hq * nb * (cfg->R + cfg->L) * sizeof(int32_t),
-                             cudaMemcpyDeviceToHost, st));
-  if (overflow_host)
-    MDR_CUDA(cudaMemcpyAsync(overflow_host, idx.overflow, static_cast<size_t>(cfg->B) * cfg->Hkv * sizeof(int32_t),
-                             cudaMemcpyDeviceToHost, st));
-  if (maxload_host)
-    MDR_CUDA(cudaMemcpyAsync(maxload_host, idx.maxload, static_cast<size_t>(cfg->B) * cfg->Hkv * sizeof(int32_t),
-                             cudaMemcpyDeviceToHost, st));
-  MDR_CUDA(cudaStreamSynchronize(st));
+  HostPipeline pl;
+  MDR_CUDA(pl.init(st));
+  const mdr_status s = forward_host_chunked(cfg, h, q_host, k_host, v_host, codebooks_host, out_host, sel_host,
+                                            overflow_host, maxload_host, dev_ws, st, pl);
+  // Whatever was enqueued finishes before the streams and events go.
+  const cudaError_t e = pl.finish(st);
+  MDR_TRY(s);
+  MDR_CUDA(e);
   int32_t code = 0;
   MDR_CUDA(cudaMemcpy(&code, at<int32_t>(dev_ws, h.dev), sizeof(int32_t), cudaMemcpyDeviceToHost));
   return code == 0 ? MDR_OK : MDR_ERR_DEVICE;

@@ -152,10 +152,23 @@ def test_union_attend_caller_selections():
     U.check_out(w, got, ref)
 
 
-def test_host_entry_point_matches_device():
+HOST_CASES = {
+    "ar_b4": AR.with_(B=4),                                          # 6 blocks: one chunk per block
+    "scaling4k": scaling(4096),                                      # 64 blocks in 8 chunks
+    "overflow_heavy": scaling(4096).with_(cap=1, probes=1, K=4, L=4),  # lists overflow across chunks
+    "union_g2_d128": CAPACITY.with_(S=12 * 128, block=128, D=128, Hq=4, Hkv=2, K=8, cap=16, R=4, L=2, B=2),
+    "tiny_f32": TINY,
+}
+
+
+@pytest.mark.parametrize("name", sorted(HOST_CASES))
+def test_host_entry_point_matches_device(name):
+    """mdr_forward_host runs the sequence in chunks of query blocks (copies of
+    one chunk overlapping the kernels and copies of the others); its out,
+    sel, overflow and maxload are bit-identical to mdr_forward's."""
     import torch
     from learned_product_hash_b200 import mdr
-    w = AR.with_(B=4)
+    w = HOST_CASES[name]
     inp = make_inputs(w, 7)
     g = U.run_gpu(w, inp)
     cfg = mdr.make_config(w)
@@ -170,7 +183,7 @@ def test_host_entry_point_matches_device():
     mdr.mdr_forward_host(cfg, q, k, v, cb, out, sel, ovf, mx, dws)
     assert np.array_equal(sel.numpy(), g["sel"])
     assert np.array_equal(ovf.numpy(), g["overflow"]) and np.array_equal(mx.numpy(), g["maxload"])
-    got = out.view(torch.bfloat16).float().numpy()
+    got = out.view(torch.bfloat16).float().numpy() if w.dtype == "bf16" else out.numpy()
     assert np.array_equal(got, g["out"])
 
 
