@@ -193,7 +193,7 @@ mdr_status mdr_host_workspace_bytes(const mdr_config* cfg, size_t* bytes);
 /* The forward from host buffers: copies q, k, v, codebooks to the device
  * workspace, runs the forward there, copies out, sel, overflow and maxload
  * back, and synchronises before returning.  The forward is causal (block j's
- * output needs the inputs of blocks <= j only), so it runs in up to eight
+ * output needs the inputs of blocks <= j only), so it runs in up to four
  * chunks of query blocks: a chunk's inputs are copied in on one internal
  * stream, its blocks summarised, appended to the posting lists, routed and
  * attended on `stream`, and its output copied out on another internal

@@ -3,6 +3,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "mdr.h"
 #include "kernels.h"
@@ -358,11 +359,20 @@ HostLayout host_layout_of(const mdr_config* c) {
 // `in`, the kernels on the caller's stream, the output copies on `out`, so
 // that chunk c's output copy overlaps chunk c+1's input copy (the link is
 // full duplex).
+// Created on a device's first call and kept (one set per device; calls on a
+// device hold its mutex, so they run one at a time).
 struct HostPipeline {
-  static constexpr int kMaxChunks = 8;
+  // Four chunks: each more chunk costs ~20 us of launches and waits, each
+  // fewer makes the last chunk's output copy, which nothing overlaps, longer
+  // (32K workload on B200: 4.40 ms with 4 chunks, 4.49 with 8, 4.66 with 16;
+  // the input copy alone takes 3.66 ms at 55 GB/s).
+  static constexpr int kMaxChunks = 4;
   cudaStream_t in = nullptr, out = nullptr;
   cudaEvent_t start = nullptr, in_done[kMaxChunks] = {}, comp_done[kMaxChunks] = {};
-  cudaError_t init(cudaStream_t st) {
+  bool ready = false;
+  std::mutex mu;
+  cudaError_t create() {
+    if (ready) return cudaSuccess;
     cudaError_t e;
     if ((e = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking)) != cudaSuccess) return e;
     if ((e = cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking)) != cudaSuccess) return e;
@@ -371,27 +381,32 @@ struct HostPipeline {
       if ((e = cudaEventCreateWithFlags(&in_done[c], cudaEventDisableTiming)) != cudaSuccess) return e;
       if ((e = cudaEventCreateWithFlags(&comp_done[c], cudaEventDisableTiming)) != cudaSuccess) return e;
     }
-    // The copies start after whatever the caller enqueued before.
+    ready = true;
+    return cudaSuccess;
+  }
+  // The copies start after whatever the caller enqueued before.
+  cudaError_t begin(cudaStream_t st) {
+    cudaError_t e = create();
+    if (e != cudaSuccess) return e;
     if ((e = cudaEventRecord(start, st)) != cudaSuccess) return e;
     if ((e = cudaStreamWaitEvent(in, start, 0)) != cudaSuccess) return e;
     return cudaStreamWaitEvent(out, start, 0);
   }
-  // Waits for all three streams, then releases the streams and events.
+  // Waits for the three streams.
   cudaError_t finish(cudaStream_t st) {
     cudaError_t r = cudaSuccess, e;
-    for (cudaStream_t s : {in, st, out})
-      if ((s == st || s) && (e = cudaStreamSynchronize(s)) != cudaSuccess && r == cudaSuccess) r = e;
-    if (in) cudaStreamDestroy(in);
-    if (out) cudaStreamDestroy(out);
-    if (start) cudaEventDestroy(start);
-    for (int c = 0; c < kMaxChunks; ++c) {
-      if (in_done[c]) cudaEventDestroy(in_done[c]);
-      if (comp_done[c]) cudaEventDestroy(comp_done[c]);
-    }
-    in = out = nullptr;
+    if (ready && (e = cudaStreamSynchronize(in)) != cudaSuccess) r = e;
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess && r == cudaSuccess) r = e;
+    if (ready && (e = cudaStreamSynchronize(out)) != cudaSuccess && r == cudaSuccess) r = e;
     return r;
   }
 };
+
+HostPipeline* host_pipeline(int device) {
+  constexpr int kMaxDevices = 64;
+  static HostPipeline pipes[kMaxDevices];
+  return device >= 0 && device < kMaxDevices ? &pipes[device] : nullptr;
+}
 
 // Rows t0 .. t1 - 1 of every sequence of a [B,S,...] tensor with row_bytes
 // per token, one strided copy.
@@ -493,12 +508,16 @@ mdr_status mdr_forward_host(const mdr_config* cfg, const void* q_host, const voi
   if (!dev_ws || reinterpret_cast<uintptr_t>(dev_ws) % kAlign != 0 || dev_ws_bytes < h.total)
     return MDR_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  HostPipeline pl;
-  MDR_CUDA(pl.init(st));
+  int device = -1;
+  MDR_CUDA(cudaGetDevice(&device));
+  HostPipeline* pl = host_pipeline(device);
+  if (!pl) return MDR_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(pl->mu);
+  MDR_CUDA(pl->begin(st));
   const mdr_status s = forward_host_chunked(cfg, h, q_host, k_host, v_host, codebooks_host, out_host, sel_host,
-                                            overflow_host, maxload_host, dev_ws, st, pl);
-  // Whatever was enqueued finishes before the streams and events go.
-  const cudaError_t e = pl.finish(st);
+                                            overflow_host, maxload_host, dev_ws, st, *pl);
+  // Whatever was enqueued finishes before the call returns.
+  const cudaError_t e = pl->finish(st);
   MDR_TRY(s);
   MDR_CUDA(e);
   int32_t code = 0;
