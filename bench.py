@@ -331,6 +331,20 @@ def backward_flops(sel: np.ndarray, bs: int, D: int) -> int:
     return 8 * D * pairs
 
 
+def backward_bytes(w, sel: np.ndarray, es: int) -> int:
+    """Algorithmic bytes of one attention backward, the forward's byte model
+    carried over: q, k, v and dout read once, dq, dk, dv written once in
+    float32, and per valid (route, selected block) pair the four tiles the
+    gradient needs -- the block's K and V (for dq) and the query block's Q and
+    dO (for dk, dv), bs x D each."""
+    nb = sel.shape[2]
+    j = np.arange(nb)[None, None, :, None]
+    pairs = int(((sel >= 0) & (sel <= j)).sum())
+    tok = w.B * w.S
+    once = tok * w.D * (2 * w.Hq + 2 * w.Hkv) * es + tok * w.D * (w.Hq + 2 * w.Hkv) * 4
+    return once + pairs * 4 * w.block * w.D * es
+
+
 def forward_bytes(w, nsel: int, es: int) -> dict:
     """Algorithmic bytes of one forward (the survey's byte model): the
     summary pass reads q and k once; the attention reads q, gathers K and V of
@@ -761,12 +775,20 @@ def run_mine(args, w):
                     "algorithmic_flops_per_call": fl}
             arith = "float32 on CUDA cores"
             launches = 4
+        bb = backward_bytes(w, sel, es)
+        hpk, hpk_kind = peaks()
+        roof_bytes = {"bound": "hbm", "achieved": bb / (b_ms / 1e3) / 1e9, "peak": hpk, "unit": "GB/s",
+                      "frac": bb / (b_ms / 1e3) / 1e9 / hpk, "peak_kind": hpk_kind,
+                      "algorithmic_bytes_per_call": bb,
+                      "note": "the bytes side of the same call: at ~34 flops per byte the gradient sits far below "
+                              "the ridge of either peak; the kernels take in ~2.7 GB (the dq kernel gathers K, V "
+                              "twice: a statistics pass and a gradient pass)"}
         backward = {"metric": "attention backward (dq, dk, dv for a fixed route) at 32K",
                     "value": throughput(w.B * w.S, world, b_ms_max), "unit": "tokens/s", "ms_per_call": b_ms_max,
                     "launches_per_call": launches, "arithmetic": arith,
                     "l2": "not flushed between calls: q, k, v, dout, the rotated copies and the float32 "
                           "gradients (~0.8 GB) exceed L2",
-                    "roofline": roof}
+                    "roofline": roof, "roofline_bytes": roof_bytes}
         del bws, dq, dk, dv, do
 
     # Scaling of the forward from 4K to 128K tokens (one GPU): the median of
