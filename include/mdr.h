@@ -20,7 +20,9 @@
  *     current device; "host" pointers point to CPU memory (pinned memory
  *     makes the copies asynchronous).  The caller owns every buffer; the
  *     library allocates nothing and keeps no state between calls, except
- *     mdr_route_noalloc, whose scratch is an array inside the library.
+ *     mdr_route_noalloc, whose scratch is an array inside the library, and
+ *     mdr_forward_host, which keeps two streams and nine events per device
+ *     from its first call on (calls on one device run one at a time).
  *   - Layouts are C-contiguous.  q is [B,S,Hq,D]; k and v are [B,S,Hkv,D];
  *     out is [B,S,Hq,D]; all four have the element type cfg->dtype.
  *     Query head hq reads KV head hq / (Hq/Hkv).
