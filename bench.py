@@ -775,6 +775,30 @@ def run_mine(args, w):
                     "algorithmic_flops_per_call": fl}
             arith = "float32 on CUDA cores"
             launches = 4
+        # With the forward's output and row normalisers saved (training: the
+        # forward ran mdr_forward_train), the dq kernel skips its statistics pass.
+        saved = None
+        if w.dtype == "bf16":
+            o_s = torch.empty_like(q)
+            lse_s = torch.empty(w.B, w.Hq, w.S, dtype=torch.float32, device=dev)
+            mdr.mdr_attend_train(cfg, q, k, v, rt.sel, o_s, lse_s, ws)
+            for _ in range(2):
+                mdr.mdr_attend_backward_saved(cfg, q, k, v, rt.sel, o_s, lse_s, do, dq, dk, dv, bws)
+            torch.cuda.synchronize()
+            b0.record(stream)
+            for _ in range(nb_it):
+                mdr.mdr_attend_backward_saved(cfg, q, k, v, rt.sel, o_s, lse_s, do, dq, dk, dv, bws)
+            b1.record(stream)
+            b1.synchronize()
+            assert mdr.mdr_read_device_status(bws) == 0
+            s_ms = max_over_ranks(b0.elapsed_time(b1) / nb_it, dist, world, dev)
+            tpk_s, tpk_kind_s = tensor_peak()
+            saved = {"entry_point": "mdr_attend_backward_saved (output and row normalisers of mdr_attend_train)",
+                     "ms_per_call": s_ms, "value": throughput(w.B * w.S, world, s_ms), "unit": "tokens/s",
+                     "roofline": {"bound": "tensor", "achieved": fl / (s_ms / 1e3) / 1e12, "peak": tpk_s,
+                                  "unit": "TFLOP/s", "frac": fl / (s_ms / 1e3) / 1e12 / tpk_s,
+                                  "peak_kind": tpk_kind_s}}
+            del o_s, lse_s
         bb = backward_bytes(w, sel, es)
         hpk, hpk_kind = peaks()
         roof_bytes = {"bound": "hbm", "achieved": bb / (b_ms / 1e3) / 1e9, "peak": hpk, "unit": "GB/s",
@@ -788,7 +812,7 @@ def run_mine(args, w):
                     "launches_per_call": launches, "arithmetic": arith,
                     "l2": "not flushed between calls: q, k, v, dout, the rotated copies and the float32 "
                           "gradients (~0.8 GB) exceed L2",
-                    "roofline": roof, "roofline_bytes": roof_bytes}
+                    "roofline": roof, "roofline_bytes": roof_bytes, "saved_statistics": saved}
         del bws, dq, dk, dv, do
 
     # Scaling of the forward from 4K to 128K tokens (one GPU): the median of

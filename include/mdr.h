@@ -176,6 +176,20 @@ mdr_status mdr_forward(const mdr_config* cfg, const void* q, const void* k,
                        const mdr_index* idx, const mdr_route_out* rt,
                        void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* mdr_attend / mdr_forward for training: the same output, and besides it
+ * each row's softmax normaliser, lse[b,hq,t] = log of the sum over the
+ * row's visible keys s of exp(scale*<q'_t, k'_s>) (natural log; -inf for a
+ * query block with no valid selected block), which mdr_attend_backward_saved
+ * reuses.  lse: device float32 [B,Hq,S], required.                          */
+mdr_status mdr_attend_train(const mdr_config* cfg, const void* q, const void* k,
+                            const void* v, const int32_t* sel, void* out,
+                            float* lse, void* ws, size_t ws_bytes, void* stream);
+mdr_status mdr_forward_train(const mdr_config* cfg, const void* q, const void* k,
+                             const void* v, const float* codebooks,
+                             const mdr_index* idx, const mdr_route_out* rt,
+                             void* out, float* lse, void* ws, size_t ws_bytes,
+                             void* stream);
+
 /* mdr_forward that also records CUDA events at the kernel boundaries, for
  * timing each kernel on the stream it runs on.  events: host array of
  * n_events cudaEvent_t (as void*), each NULL to skip; events[0] before the
@@ -366,6 +380,20 @@ mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void*
                                const void* v, const int32_t* sel, const void* dout,
                                float* dq, float* dk, float* dv, void* ws,
                                size_t ws_bytes, void* stream);
+
+/* mdr_attend_backward with the forward's output and row normalisers saved
+ * by mdr_attend_train / mdr_forward_train (out: device [B,S,Hq,D] in
+ * cfg->dtype, 16-byte aligned for MDR_BF16; lse: device float32 [B,Hq,S];
+ * both required, both from the same sel).  MDR_BF16 takes
+ * Delta_t = <dout_t, out_t> and the normalisers from them and so skips the
+ * first of its two passes over the selected blocks; MDR_F32 recomputes them
+ * as mdr_attend_backward does.  Same outputs, workspace and status.         */
+mdr_status mdr_attend_backward_saved(const mdr_config* cfg, const void* q,
+                                     const void* k, const void* v,
+                                     const int32_t* sel, const void* out,
+                                     const float* lse, const void* dout,
+                                     float* dq, float* dk, float* dv, void* ws,
+                                     size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------- codebook calibration
  * Spherical codebook calibration (Report, section Capacity and Figure 3:

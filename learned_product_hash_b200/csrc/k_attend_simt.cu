@@ -82,6 +82,8 @@ attend_simt_kernel(const AttendArgs a) {
       }
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;   // nothing selected: zero output
+    if (a.lse && lane == 0)
+      a.lse[(static_cast<size_t>(b) * a.Hq + hq) * a.S + t] = l > 0.f ? mx + logf(l) : -INFINITY;
     const size_t ooff = ((static_cast<size_t>(b) * a.S + t) * a.Hq + hq) * a.D;
 #pragma unroll
     for (int m = 0; m < 4; ++m)

@@ -511,8 +511,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     };
     bool pend = false;
     int pend_itv = 0;
-    float pend_l = 0.f;
+    float pend_l = 0.f, pend_m = 0.f;
     __nv_bfloat16* pend_out = nullptr;
+    float* pend_lse = nullptr;                       // this row's normaliser, when asked for
     auto epilogue = [&]() -> bool {
       if (!wwait(C::bOFull + (pend_itv & 1), (pend_itv >> 1) & 1)) return false;
       // Row sum: the two threads of a row, then the partner warp.
@@ -521,6 +522,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       if (writer) xl[half * BS + r] = l;
       if (!exchange()) return false;
       l += xl[(1 - half) * BS + r];
+      if (pend_lse && writer && half == 0) *pend_lse = (pend_m + __log2f(l)) * 0.6931471805599453f;
       tc_fence_after();
       const uint32_t tO = tmem + C::kColO + (pend_itv & 1) * D + lane_base;
       const float inv = 1.f / l;
@@ -555,9 +557,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const int j = tile % a.nb, hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq);
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
                            ((static_cast<size_t>(b) * a.S + static_cast<size_t>(j) * BS + r) * a.Hq + hq) * D;
+      float* lse = a.lse ? a.lse + (static_cast<size_t>(b) * a.Hq + hq) * a.S + static_cast<size_t>(j) * BS + r : nullptr;
       if (nblk == 0) {                                 // nothing selected: zero output
         for (int i = 0; i < kOParts; ++i)
           for (int q8 = 0; q8 < kOW / 8; ++q8) *reinterpret_cast<uint4*>(out + o_col(i) + q8 * 8) = make_uint4(0, 0, 0, 0);
+        if (lse && writer && half == 0) *lse = -INFINITY;
         continue;
       }
       const uint32_t tO = tmem + C::kColO + (itv & 1) * D + lane_base;
@@ -660,7 +664,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       pend = true;
       pend_itv = itv;
       pend_l = l_sum;
+      pend_m = m_used;
       pend_out = out;
+      pend_lse = lse;
       g0 = gend;
       ++itv;
     }

@@ -565,9 +565,10 @@ attend_union_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     };
     bool pend = false;
     int pend_itv = 0;
-    float pend_l0 = 0.f, pend_l1 = 0.f;
+    float pend_l0 = 0.f, pend_l1 = 0.f, pend_m0 = 0.f, pend_m1 = 0.f;
     bool pend_has0 = false, pend_has1 = false;
     __nv_bfloat16* pend_out = nullptr;                // the first head's row; the second's is + D
+    float* pend_lse = nullptr;                        // the first head's normaliser; the second's is + S
     auto epilogue = [&]() -> bool {
       if (!wwait(C::bOFull, pend_itv & 1)) return false;
       xl[(0 * 2 + half) * BS + r] = pend_l0;
@@ -587,6 +588,8 @@ attend_union_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (!(x == 0 ? pend_has0 : pend_has1)) continue;
         const float l = (x == 0 ? pend_l0 : pend_l1) + xl[(x * 2 + 1 - half) * BS + r];
         const float inv = 1.f / l;
+        if (pend_lse && half == 0)
+          pend_lse[static_cast<size_t>(x) * a.S] = ((x == 0 ? pend_m0 : pend_m1) + __log2f(l)) * 0.6931471805599453f;
         const uint32_t tO = tmem + lane_base + C::kColO + x * D + (D / 2) * half;
         uint4 w[kChunks];
 #pragma unroll
@@ -641,8 +644,14 @@ attend_union_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       const bool hasB = 2 * p + 1 < g;
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
                            ((static_cast<size_t>(b) * a.S + static_cast<size_t>(j) * BS + r) * a.Hq + hqA) * D;
+      float* lse = a.lse ? a.lse + (static_cast<size_t>(b) * a.Hq + hqA) * a.S + static_cast<size_t>(j) * BS + r
+                         : nullptr;
       if (nA == 0) zero_row(out);                     // a head with nothing selected: zero output
       if (hasB && nB == 0) zero_row(out + D);
+      if (lse && half == 0) {
+        if (nA == 0) lse[0] = -INFINITY;
+        if (hasB && nB == 0) lse[a.S] = -INFINITY;
+      }
       if (nu == 0) {
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::bTEmpty + slot));
@@ -730,6 +739,9 @@ attend_union_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       pend_itv = itv;
       pend_l0 = l0;
       pend_l1 = l1;
+      pend_m0 = m0;
+      pend_m1 = m1;
+      pend_lse = lse;
       pend_has0 = nA > 0;
       pend_has1 = hasB && nB > 0;
       pend_out = out;

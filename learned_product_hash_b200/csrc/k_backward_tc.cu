@@ -329,7 +329,11 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       continue;
     }
-    const int nsteps = 2 * nblk;                  // pass 1 then pass 2 over the same blocks
+    // Pass 1 then pass 2 over the same blocks; with the forward's output and
+    // row normalisers given, pass 2 alone.
+    const bool given = a.lse_in != nullptr;
+    const int p2 = given ? 0 : nblk;
+    const int nsteps = p2 + nblk;
     auto issue_kv = [&](int n) {                  // K, V of step n into slot ld_issue % NKV
       if (threadIdx.x == 0) {
         const int slot = static_cast<int>(ld_issue % C::NKV);
@@ -368,8 +372,31 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     phQ ^= 1;
     q_pending = false;
     float m2 = -INFINITY, l = 0.f, lse2 = 0.f, delta = 0.f;
+    if (given) {
+      // Delta = <dO, out> of the saved (normalised) output; lse in log2 units.
+      const __nv_bfloat16* dorow = static_cast<const __nv_bfloat16*>(a.dout) + ((tok0 + R.r) * a.Hq + hq) * D;
+      const __nv_bfloat16* orow = static_cast<const __nv_bfloat16*>(a.out_in) + ((tok0 + R.r) * a.Hq + hq) * D;
+      float dsum = 0.f;
+#pragma unroll
+      for (int pp = 0; pp < C::NP; ++pp)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int c0 = (hf ? D / 2 : 0) + R.col_lo(pp);
+          float o[C::W];
+#pragma unroll
+          for (int q = 0; q < C::W / 8; ++q) Elem<__nv_bfloat16>::load(orow + c0 + 8 * q, o + 8 * q);
+          dsum += dot_bf16<C::W>(o, dorow + c0);
+        }
+      delta = R.row_sum(dsum);
+      const float ln = a.lse_in[si0 + R.r];
+      lse2 = ln > -INFINITY ? ln * 1.4426950408889634f : INFINITY;
+      if (R.tsub == 0) {
+        a.lse[si0 + R.r] = lse2;
+        a.delta[si0 + R.r] = delta;
+      }
+    }
     for (int n = 0; n < nsteps && ok; ++n) {
-      const bool pass2 = n >= nblk;
+      const bool pass2 = n >= p2;
       const int blk = ctl.ids[n % nblk];
       const int slot = static_cast<int>(ld_use % C::NKV);
       if (!wait_all(bKV0 + slot, static_cast<uint32_t>((ld_use / C::NKV) & 1), kSiteKV)) { ok = false; break; }
@@ -470,7 +497,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tc_fence_after();
         // pass 1: O += P V (V MN-major); pass 2: dQ += dS K (K MN-major)
         const uint32_t sB = pass2 ? sK : sV;
-        const bool first = pass2 ? n == nblk : n == 0;
+        const bool first = n == (pass2 ? p2 : 0);
 #pragma unroll
         for (int kk = 0; kk < BS / 16; ++kk)
           mma_bf16(tmem + C::qColO, kmaj<BS>(sP, kk), mnmaj<BS>(sB, kk), idPV, (!first || kk > 0) ? 1u : 0u);
@@ -478,7 +505,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       mm_pending = true;
       mm_step = n;
-      if (n == nblk - 1) {
+      if (!given && n == nblk - 1) {
         // End of pass 1: lse and Delta = <dO, O> / sum of each row.
         if (!finish_mm()) { ok = false; break; }
         tc_fence_after();

@@ -117,6 +117,8 @@ struct AttendArgs {
   void* out;               // [B,S,Hq,D]
   int32_t* status;         // device status word
   int32_t* tile_counter;   // tensor-core kernel: zero at launch; tiles are handed out from it
+  float* lse;              // [B,Hq,S] natural-log normaliser of each row's softmax
+                           // (-inf for a row with nothing selected), or null
   int B, S, Hq, Hkv, D, bs, nb, nsel;
   float scale;
   int j0, nbr;             // query blocks j0 .. j0 + nbr - 1 only (nbr = 0: every block)
@@ -168,6 +170,12 @@ struct BwdArgs {
   const void* krot;        // rotated k in the storage type [B,S,Hkv,D] (tensor-core path)
   float* lse;              // scratch: [B,Hq,S] log-sum-exp of the scaled scores
   float* delta;            // scratch: [B,Hq,S] dout_t . out_t
+  // Saved by the forward (both or neither; tensor-core path): its output
+  // [B,S,Hq,D] and row normalisers [B,Hq,S] (natural log).  Given, the dq
+  // kernel takes Delta = dout . out and the log-sum-exp from them instead of
+  // a first pass over the selected blocks.
+  const void* out_in;
+  const float* lse_in;
   int32_t* rev_off;        // scratch: [B,Hkv,nb+1] reverse-index offsets
   int32_t* rev;            // scratch: [B,Hkv,(Hq/Hkv)*nb*nsel] (local query head * nb + query block)
   float* dq;               // [B,S,Hq,D]

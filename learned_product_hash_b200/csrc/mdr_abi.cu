@@ -154,8 +154,10 @@ mdr_status run_route(const mdr_config* c, const float* qbar, const int32_t* qcod
 }
 
 mdr_status run_attend(const mdr_config* c, const void* qrot, const void* krot, const void* v,
-                      const int32_t* sel, void* out, int32_t* status, cudaStream_t st, int j0 = 0, int j1 = 0) {
+                      const int32_t* sel, void* out, int32_t* status, cudaStream_t st, int j0 = 0, int j1 = 0,
+                      float* lse = nullptr) {
   mdr::AttendArgs aa{};
+  aa.lse = lse;
   aa.j0 = j0; aa.nbr = j1 > 0 ? j1 - j0 : 0;
   aa.q = qrot; aa.k = krot; aa.v = v; aa.sel = sel; aa.out = out; aa.status = status;
   aa.tile_counter = status + 2;
@@ -256,8 +258,8 @@ mdr_status mdr_target_hits(const mdr_config* cfg, const int32_t* sel, const int3
   return cuda_status(mdr::launch_hits(ha, static_cast<cudaStream_t>(stream)));
 }
 
-mdr_status mdr_attend(const mdr_config* cfg, const void* q, const void* k, const void* v,
-                      const int32_t* sel, void* out, void* ws, size_t ws_bytes, void* stream) {
+static mdr_status attend_impl(const mdr_config* cfg, const void* q, const void* k, const void* v,
+                              const int32_t* sel, void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
   MDR_TRY(check(cfg));
   if (!q || !k || !v || !sel || !out) return MDR_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MDR_ERR_INVALID_ARG;
@@ -272,13 +274,24 @@ mdr_status mdr_attend(const mdr_config* cfg, const void* q, const void* k, const
   a.xrot[0] = at<void>(ws, l.qrot); a.xrot[1] = at<void>(ws, l.krot);
   a.status = status;
   MDR_CUDA(mdr::launch_summarize(a, cfg->dtype == MDR_BF16, st));
-  return run_attend(cfg, at<void>(ws, l.qrot), at<void>(ws, l.krot), v, sel, out, status, st);
+  return run_attend(cfg, at<void>(ws, l.qrot), at<void>(ws, l.krot), v, sel, out, status, st, 0, 0, lse);
+}
+
+mdr_status mdr_attend(const mdr_config* cfg, const void* q, const void* k, const void* v,
+                      const int32_t* sel, void* out, void* ws, size_t ws_bytes, void* stream) {
+  return attend_impl(cfg, q, k, v, sel, out, nullptr, ws, ws_bytes, stream);
+}
+
+mdr_status mdr_attend_train(const mdr_config* cfg, const void* q, const void* k, const void* v,
+                            const int32_t* sel, void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!lse) return MDR_ERR_INVALID_ARG;
+  return attend_impl(cfg, q, k, v, sel, out, lse, ws, ws_bytes, stream);
 }
 
 static mdr_status forward_impl(const mdr_config* cfg, const void* q, const void* k, const void* v,
                                const float* codebooks, const mdr_index* idx, const mdr_route_out* rt,
                                void* out, void* ws, size_t ws_bytes, void* stream,
-                               void* const* events, int32_t n_events) {
+                               void* const* events, int32_t n_events, float* lse = nullptr) {
   MDR_TRY(check(cfg));
   if (!q || !k || !v || !codebooks || !out || !rt || !rt->sel) return MDR_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MDR_ERR_INVALID_ARG;
@@ -312,7 +325,7 @@ static mdr_status forward_impl(const mdr_config* cfg, const void* q, const void*
   MDR_TRY(mark(2));
   MDR_TRY(run_route(cfg, qbar, qcodes, idx, rt->sel, rt->ncand, st));
   MDR_TRY(mark(3));
-  MDR_TRY(run_attend(cfg, at<void>(ws, l.qrot), at<void>(ws, l.krot), v, rt->sel, out, status, st));
+  MDR_TRY(run_attend(cfg, at<void>(ws, l.qrot), at<void>(ws, l.krot), v, rt->sel, out, status, st, 0, 0, lse));
   return mark(4);
 }
 
@@ -320,6 +333,13 @@ mdr_status mdr_forward(const mdr_config* cfg, const void* q, const void* k, cons
                        const float* codebooks, const mdr_index* idx, const mdr_route_out* rt,
                        void* out, void* ws, size_t ws_bytes, void* stream) {
   return forward_impl(cfg, q, k, v, codebooks, idx, rt, out, ws, ws_bytes, stream, nullptr, 0);
+}
+
+mdr_status mdr_forward_train(const mdr_config* cfg, const void* q, const void* k, const void* v,
+                             const float* codebooks, const mdr_index* idx, const mdr_route_out* rt,
+                             void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!lse) return MDR_ERR_INVALID_ARG;
+  return forward_impl(cfg, q, k, v, codebooks, idx, rt, out, ws, ws_bytes, stream, nullptr, 0, lse);
 }
 
 mdr_status mdr_forward_profiled(const mdr_config* cfg, const void* q, const void* k, const void* v,
@@ -677,11 +697,12 @@ mdr_status mdr_backward_workspace_bytes(const mdr_config* cfg, size_t* bytes) {
   return MDR_OK;
 }
 
-mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void* k, const void* v,
-                               const int32_t* sel, const void* dout, float* dq, float* dk, float* dv,
-                               void* ws, size_t ws_bytes, void* stream) {
+static mdr_status backward_impl(const mdr_config* cfg, const void* q, const void* k, const void* v,
+                                const int32_t* sel, const void* out, const float* lse, const void* dout,
+                                float* dq, float* dk, float* dv, void* ws, size_t ws_bytes, void* stream) {
   MDR_TRY(check(cfg));
   if (!q || !k || !v || !sel || !dout || !dq || !dk || !dv) return MDR_ERR_INVALID_ARG;
+  if ((out == nullptr) != (lse == nullptr)) return MDR_ERR_INVALID_ARG;
   const BwdLayout l = bwd_layout_of(cfg);
   if (!ws || reinterpret_cast<uintptr_t>(ws) % kAlign != 0 || ws_bytes < l.total) return MDR_ERR_WORKSPACE;
   if (static_cast<long long>(cfg->B) * cfg->Hq * (cfg->S / cfg->block) * (cfg->block / 16) > INT32_MAX)
@@ -707,7 +728,8 @@ mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void*
   a.nb = cfg->S / cfg->block; a.nsel = cfg->R + cfg->L;
   a.scale = mdr::detail::softmax_scale(cfg);
   mdr::detail::fill_inv_freq(a.inv_freq, cfg);
-  if (!tc) return cuda_status(mdr::launch_backward(a, false, st));
+  if (!tc) return cuda_status(mdr::launch_backward(a, false, st));   // float32 recomputes the statistics
+  a.out_in = out; a.lse_in = lse;
   // The rotated copies in the storage type, by the summary kernel (the
   // operands the forward's attention reads), into the float32 regions.
   SummarizeArgs sa;
@@ -718,6 +740,20 @@ mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void*
   MDR_CUDA(mdr::launch_summarize(sa, true, st));
   a.qrot = a.qr; a.krot = a.kr;
   return cuda_status(mdr::launch_backward_tc(a, st));
+}
+
+mdr_status mdr_attend_backward(const mdr_config* cfg, const void* q, const void* k, const void* v,
+                               const int32_t* sel, const void* dout, float* dq, float* dk, float* dv,
+                               void* ws, size_t ws_bytes, void* stream) {
+  return backward_impl(cfg, q, k, v, sel, nullptr, nullptr, dout, dq, dk, dv, ws, ws_bytes, stream);
+}
+
+mdr_status mdr_attend_backward_saved(const mdr_config* cfg, const void* q, const void* k, const void* v,
+                                     const int32_t* sel, const void* out, const float* lse, const void* dout,
+                                     float* dq, float* dk, float* dv, void* ws, size_t ws_bytes, void* stream) {
+  if (!out || !lse) return MDR_ERR_INVALID_ARG;
+  if (cfg && cfg->dtype == MDR_BF16 && !aligned16(out)) return MDR_ERR_INVALID_ARG;
+  return backward_impl(cfg, q, k, v, sel, out, lse, dout, dq, dk, dv, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------ codebook calibration

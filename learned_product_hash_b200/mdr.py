@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
             "mdr_route": ([cfgp, vp, vp, idxp, rtp, vp, sz, vp], i32),
             "mdr_attend": ([cfgp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "mdr_forward": ([cfgp, vp, vp, vp, vp, idxp, rtp, vp, vp, sz, vp], i32),
+            "mdr_attend_train": ([cfgp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "mdr_forward_train": ([cfgp, vp, vp, vp, vp, idxp, rtp, vp, vp, vp, sz, vp], i32),
             "mdr_host_workspace_bytes": ([cfgp, ctypes.POINTER(sz)], i32),
             "mdr_forward_host": ([cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "mdr_read_device_status": ([vp, ctypes.POINTER(ctypes.c_int32), vp], i32),
@@ -85,6 +87,7 @@ def lib() -> ctypes.CDLL:
             "mdr_target_hits": ([cfgp, vp, vp, vp, vp, vp], i32),
             "mdr_backward_workspace_bytes": ([cfgp, ctypes.POINTER(sz)], i32),
             "mdr_attend_backward": ([cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "mdr_attend_backward_saved": ([cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "mdr_calibrate_workspace_bytes": ([ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.POINTER(sz)], i32),
             "mdr_calibrate_codebooks": ([vp, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
@@ -225,6 +228,20 @@ def mdr_forward(cfg, q, k, v, codebooks, idx: Index, rt: RouteOut, out, ws, stre
                           ws.numel(), _stream(stream)), "mdr_forward")
 
 
+def mdr_attend_train(cfg, q, k, v, sel, out, lse, ws, stream=None):
+    """mdr_attend that also writes each row's softmax normaliser lse
+    (float32 [B,Hq,S], natural log) for mdr_attend_backward_saved."""
+    _ok(lib().mdr_attend_train(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(out), _ptr(lse),
+                               _ptr(ws), ws.numel(), _stream(stream)), "mdr_attend_train")
+
+
+def mdr_forward_train(cfg, q, k, v, codebooks, idx: Index, rt: RouteOut, out, lse, ws, stream=None):
+    """mdr_forward that also writes each row's softmax normaliser lse."""
+    _ok(lib().mdr_forward_train(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(codebooks),
+                                ctypes.byref(idx.c()), ctypes.byref(rt.c()), _ptr(out), _ptr(lse), _ptr(ws),
+                                ws.numel(), _stream(stream)), "mdr_forward_train")
+
+
 def mdr_forward_profiled(cfg, q, k, v, codebooks, idx: Index, rt: RouteOut, out, ws, events, stream=None):
     """events: list of torch.cuda.Event(enable_timing=True) (or None), recorded
     before K1 and after K1, K3, K4, K5."""
@@ -294,6 +311,14 @@ def mdr_attend_backward(cfg, q, k, v, sel, dout, dq, dk, dv, ws, stream=None):
     _ok(lib().mdr_attend_backward(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(dout),
                                   _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(stream)),
         "mdr_attend_backward")
+
+
+def mdr_attend_backward_saved(cfg, q, k, v, sel, out, lse, dout, dq, dk, dv, ws, stream=None):
+    """mdr_attend_backward reusing the forward's output and row normalisers
+    (from mdr_attend_train / mdr_forward_train)."""
+    _ok(lib().mdr_attend_backward_saved(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(out),
+                                        _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
+                                        _stream(stream)), "mdr_attend_backward_saved")
 
 
 # ------------------------------------------------------ codebook calibration

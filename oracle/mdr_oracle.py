@@ -285,6 +285,31 @@ def attend(qr, kr, v, sel, bs: int, scale: float, rows=None) -> np.ndarray:
     return out
 
 
+def softmax_lse(qr, kr, sel, bs: int, scale: float, rows=None) -> np.ndarray:
+    """Log of the denominator of the softmax `attend` takes: for token t of
+    query block j, head hq, log of the sum over every token s <= t of the
+    selected blocks of exp(scale * <q'_t, k'_s>) (natural log; -inf when no
+    block is selected).  The saved statistic a backward reuses (Report,
+    Mixer: the exact causal softmax over the selected set).  rows: optional
+    list of (b, hq, j); the others stay NaN.  -> [B,Hq,S] float64.
+    """
+    B, S, Hq, D = qr.shape
+    g = Hq // kr.shape[2]
+    out = np.full((B, Hq, S), np.nan)
+    nb = S // bs
+    todo = rows if rows is not None else itertools.product(range(B), range(Hq), range(nb))
+    for b, hq, j in todo:
+        toks = selected_tokens(sel[b, hq, j], bs)
+        qpos = np.arange(j * bs, (j + 1) * bs)
+        s = (qr[b, qpos, hq] @ kr[b, toks, hq // g].T) * scale
+        s[toks[None, :] > qpos[:, None]] = -np.inf
+        m = s.max(axis=1, initial=-np.inf)
+        finite = np.isfinite(m)
+        tot = np.where(finite[:, None], np.exp(s - np.where(finite, m, 0.0)[:, None]), 0.0).sum(axis=1)
+        out[b, hq, qpos] = np.where(finite, m + np.log(np.where(finite, tot, 1.0)), -np.inf)
+    return out
+
+
 def selected_mask(sel_bh: np.ndarray, S: int, bs: int) -> np.ndarray:
     """Dense boolean [S, S] mask of one (sequence, head): M[t, s] is true when
     s's block is selected for t's block and s <= t."""
@@ -708,7 +733,7 @@ def spherical_objective(records: np.ndarray, codebooks: np.ndarray) -> float:
 # the selected-set softmax and the rotary embedding only: given dL/d(out),
 # it returns dL/dq, dL/dk, dL/dv, and nothing reaches the codebooks or the
 # block summaries.
-def attend_backward(qr, kr, v, sel, bs: int, scale: float, dout, rows=None):
+def attend_backward(qr, kr, v, sel, bs: int, scale: float, dout, rows=None, saved_out=None):
     """dL/dq', dL/dk', dL/dv of attend() for dL/d(out) = dout [B,S,Hq,D].
 
     Per query block j and head hq, with T = the tokens of the selected
@@ -722,7 +747,11 @@ def attend_backward(qr, kr, v, sel, bs: int, scale: float, dout, rows=None):
     block with no valid selected block has a zero output and gets zero
     gradients.  rows: optional list of (b, hq, j) to include (dq of the
     others stays 0, and dk, dv hold only the listed rows' contributions --
-    exact for a key block whose selecting rows are all listed)."""
+    exact for a key block whose selecting rows are all listed).
+    saved_out: optional [B,S,Hq,D] output saved by a forward; the row term
+    rowsum(P * dP) = <dout_t, out_t> is then taken from it (equal to the
+    above when the saved output is attend()'s own; a rounded copy gives the
+    gradient a backward reusing that copy computes)."""
     B, S, Hq, D = qr.shape
     Hkv = kr.shape[2]
     g = Hq // Hkv
@@ -746,7 +775,11 @@ def attend_backward(qr, kr, v, sel, bs: int, scale: float, dout, rows=None):
         dO = dout[b, qpos, hq]
         dv[b, toks, h] += P.T @ dO
         dP = dO @ Vt.T
-        dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+        if saved_out is None:
+            delta = (P * dP).sum(axis=1, keepdims=True)
+        else:
+            delta = (dO * saved_out[b, qpos, hq]).sum(axis=1, keepdims=True)
+        dS = P * (dP - delta)
         dq[b, qpos, hq] = scale * dS @ Kt
         dk[b, toks, h] += scale * dS.T @ Q
     return dq, dk, dv

@@ -318,6 +318,46 @@ def check_attention_gather_equals_dense_mask():
     assert (res.sel[..., : p.R] >= 0).sum() < p.nb * p.R * 4
 
 
+def check_softmax_lse_bruteforce():
+    """The row normaliser against scipy's logsumexp of the dense score matrix
+    under the selected-position mask; a query block with nothing selected is
+    -inf; a row that sees only itself has the normaliser scale*<q'_t, k'_t>."""
+    from scipy.special import logsumexp
+    p = _p(S=96, block=16, K=3, P=2, cap=2, probes=2, R=2, L=1, Hq=2, Hkv=1, D=16)
+    q, k, v = _rand((1, p.S, 2, p.D), 36), _rand((1, p.S, 1, p.D), 37), _rand((1, p.S, 1, p.D), 38)
+    res = O.forward(q, k, v, _unit_codebooks(2, 3, 8, 39), p, attention=False)
+    sel = res.sel.copy()
+    sel[0, 1, 3] = -1                                   # nothing selected for (head 1, block 3)
+    lse = O.softmax_lse(res.qr, res.kr, sel, p.block, p.softmax_scale)
+    for hq in range(2):
+        mask = O.selected_mask(sel[0, hq], p.S, p.block)
+        sc = (res.qr[0, :, hq] @ res.kr[0, :, 0].T) * p.softmax_scale
+        ref = logsumexp(np.where(mask, sc, -np.inf), axis=1)
+        assert np.allclose(lse[0, hq], ref, rtol=0, atol=1e-12, equal_nan=False)
+    assert np.isneginf(lse[0, 1, 3 * p.block:4 * p.block]).all()
+    # local-only rows: token 0 of a block that selected only itself sees only itself
+    own = O.softmax_lse(res.qr, res.kr, np.zeros_like(sel)[..., :1] + np.arange(p.nb)[None, None, :, None],
+                        p.block, p.softmax_scale)
+    t = 5 * p.block
+    assert abs(own[0, 0, t] - p.softmax_scale * res.qr[0, t, 0] @ res.kr[0, t, 0]) < 1e-12
+
+
+def check_backward_saved_output_identity():
+    """The backward's row term rowsum(P * dP) equals <dout_t, out_t>: given
+    attend()'s own output as the saved one, the gradients are unchanged."""
+    p = _p(S=96, block=16, K=3, P=2, cap=2, probes=2, R=2, L=1, Hq=2, Hkv=1, D=16)
+    q, k, v = _rand((1, p.S, 2, p.D), 40), _rand((1, p.S, 1, p.D), 41), _rand((1, p.S, 1, p.D), 42)
+    res = O.forward(q, k, v, _unit_codebooks(2, 3, 8, 43), p)
+    dout = _rand((1, p.S, 2, p.D), 44)
+    a = O.attend_backward(res.qr, res.kr, v, res.sel, p.block, p.softmax_scale, dout)
+    b = O.attend_backward(res.qr, res.kr, v, res.sel, p.block, p.softmax_scale, dout, saved_out=res.out)
+    for x, y in zip(a, b):
+        assert np.abs(x - y).max() < 1e-12
+    # a perturbed saved output moves dq, dk but not dv
+    c = O.attend_backward(res.qr, res.kr, v, res.sel, p.block, p.softmax_scale, dout, saved_out=res.out * 1.01)
+    assert np.abs(c[2] - a[2]).max() < 1e-12 and np.abs(c[0] - a[0]).max() > 1e-6
+
+
 # --------------------------------------------------------------- near ties
 # A routing decision (a code, a probe set, a top-R set) is a near tie when the
 # float32 gap at its boundary is below 1e-6*max(1,|s|), |s| the largest score

@@ -57,11 +57,11 @@ def gpu_backward(w, inp, dout_store, sel):
     return dq.cpu().numpy(), dk.cpu().numpy(), dv.cpu().numpy(), status
 
 
-def oracle_backward(w, inp, dout, sel, rows=None):
+def oracle_backward(w, inp, dout, sel, rows=None, saved_out=None):
     p = O.Params.of(w)
     qr, kr = O.rope(inp.q.astype(np.float64), p.rope_base), O.rope(inp.k.astype(np.float64), p.rope_base)
     dqr, dkr, dv = O.attend_backward(qr, kr, inp.v.astype(np.float64), sel, w.block, p.softmax_scale,
-                                     dout.astype(np.float64), rows)
+                                     dout.astype(np.float64), rows, saved_out)
     return O.rope_transpose(dqr, p.rope_base), O.rope_transpose(dkr, p.rope_base), dv
 
 
@@ -210,3 +210,81 @@ def test_backward_full_size_sampled():
     errs = [_close("dq", dq, rq, qmask, w.dtype), _close("dk", dk, rk, kmask, w.dtype),
             _close("dv", dv, rv, kmask, w.dtype)]
     print(f"backward {w.name} sampled: {errs}")
+
+
+def gpu_attend_train(w, inp, sel):
+    """mdr_attend_train on the given selection: the output (device tensor in
+    the storage type) and the row normalisers (numpy [B,Hq,S])."""
+    import torch
+    from learned_product_hash_b200 import mdr
+    cfg = mdr.make_config(w)
+    q, k, v = (_dev(x, w) for x in (inp.q_store, inp.k_store, inp.v_store))
+    s = torch.from_numpy(np.ascontiguousarray(sel, dtype=np.int32)).cuda()
+    out = torch.empty_like(q)
+    lse = torch.full((w.B, w.Hq, w.S), np.nan, dtype=torch.float32, device="cuda")
+    ws = mdr.workspace(cfg)
+    mdr.mdr_attend_train(cfg, q, k, v, s, out, lse, ws)
+    assert mdr.mdr_read_device_status(ws) == 0
+    return out, lse.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_forward_lse_matches_oracle(name):
+    """The row normalisers written with the forward output (per-head tiles,
+    grouped-query units at block 128, float32 rows) against the oracle's.
+    Bar: |gpu - oracle| <= 2^-7 * scale * |q'_t| * max_s |k'_s| per
+    row: the normaliser moves by at most the largest change of a score, and
+    a bf16 q' or k' moves a score by at most 2^-8 of that product; plus
+    2e-5 + 2e-6 |lse| for the float32 sums and logarithm."""
+    w = CASES[name]
+    inp = make_inputs(w, 31)
+    p = O.Params.of(w)
+    sel = O.forward(inp.q, inp.k, inp.v, inp.codebooks, p, attention=False).sel
+    _, lse = gpu_attend_train(w, inp, sel)
+    qr, kr = O.rope(inp.q.astype(np.float64), p.rope_base), O.rope(inp.k.astype(np.float64), p.rope_base)
+    ref = O.softmax_lse(qr, kr, sel, w.block, p.softmax_scale)
+    assert np.isneginf(ref).sum() == np.isneginf(lse).sum() and (np.isneginf(ref) == np.isneginf(lse)).all()
+    fin = np.isfinite(ref)
+    qn = np.linalg.norm(qr, axis=-1).transpose(0, 2, 1)                      # [B,Hq,S]
+    kmax = np.linalg.norm(kr, axis=-1).max()
+    tol = (2.0 ** -7 * p.softmax_scale * qn * kmax if w.dtype == "bf16" else 0.0) + 2e-5 + 2e-6 * np.abs(
+        np.where(fin, ref, 0.0))
+    err = np.abs(lse - ref)
+    assert (err[fin] <= tol[fin]).all(), f"{name}: worst lse error {err[fin].max():.3g}"
+    print(f"lse {name}: max error {err[fin].max():.3g}")
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_backward_saved_matches_oracle(name):
+    """mdr_attend_backward_saved, fed the output and row normalisers of
+    mdr_attend_train on the same selection (tensor cores: no statistics
+    pass), against the oracle's gradients given that saved output, at the
+    same bar as the backward that recomputes them.  (Against the exact
+    output the row term <dout_t, out_t> carries the output's bf16 rounding,
+    2^-9 of sum_d |dout_td out_td|, which dS = P (dP - Delta) can magnify
+    where dP and Delta nearly cancel.)"""
+    import torch
+    from learned_product_hash_b200 import mdr
+    w = CASES[name]
+    inp = make_inputs(w, 7)
+    dout, dout_store = make_grad(w, 8)
+    sel = O.forward(inp.q, inp.k, inp.v, inp.codebooks, O.Params.of(w), attention=False).sel
+    out, lse = gpu_attend_train(w, inp, sel)
+    cfg = mdr.make_config(w)
+    q, k, v = (_dev(x, w) for x in (inp.q_store, inp.k_store, inp.v_store))
+    do = _dev(dout_store, w)
+    s = torch.from_numpy(np.ascontiguousarray(sel, dtype=np.int32)).cuda()
+    dq = torch.full(q.shape, np.nan, dtype=torch.float32, device="cuda")
+    dk = torch.full(k.shape, np.nan, dtype=torch.float32, device="cuda")
+    dv = torch.full(v.shape, np.nan, dtype=torch.float32, device="cuda")
+    ws = mdr.backward_workspace(cfg)
+    mdr.mdr_attend_backward_saved(cfg, q, k, v, s, out, torch.from_numpy(lse).cuda(), do, dq, dk, dv, ws)
+    assert mdr.mdr_read_device_status(ws) == 0
+    # The reference is the gradient given the saved output: the oracle takes
+    # <dout_t, out_t> from the GPU forward's (rounded) output, as the kernel does.
+    saved = out.float().cpu().numpy().astype(np.float64)
+    rq, rk, rv = oracle_backward(w, inp, dout, sel, saved_out=saved)
+    qz, kz = structural_zeros(w, sel)
+    errs = [_close(n, x.cpu().numpy(), y, dtype=w.dtype, zeros=z)
+            for n, x, y, z in (("dq", dq, rq, qz), ("dk", dk, rk, kz), ("dv", dv, rv, kz))]
+    print(f"backward saved {name}: {errs}")
