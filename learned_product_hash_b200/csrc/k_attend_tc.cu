@@ -132,7 +132,9 @@ __device__ __forceinline__ int group_size(int n, int nblk) {
 
 }  // namespace
 
-template <int BS, int D>
+// kLse: also write each row's softmax normaliser (a separate instantiation,
+// so that the plain forward carries none of it).
+template <int BS, int D, bool kLse>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const AttendArgs a) {
@@ -522,7 +524,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       if (writer) xl[half * BS + r] = l;
       if (!exchange()) return false;
       l += xl[(1 - half) * BS + r];
-      if (pend_lse && writer && half == 0) *pend_lse = (pend_m + __log2f(l)) * 0.6931471805599453f;
+      if constexpr (kLse)
+        if (writer && half == 0) *pend_lse = (pend_m + __log2f(l)) * 0.6931471805599453f;
       tc_fence_after();
       const uint32_t tO = tmem + C::kColO + (pend_itv & 1) * D + lane_base;
       const float inv = 1.f / l;
@@ -557,11 +560,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const int j = tile % a.nb, hq = (tile / a.nb) % a.Hq, b = tile / (a.nb * a.Hq);
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
                            ((static_cast<size_t>(b) * a.S + static_cast<size_t>(j) * BS + r) * a.Hq + hq) * D;
-      float* lse = a.lse ? a.lse + (static_cast<size_t>(b) * a.Hq + hq) * a.S + static_cast<size_t>(j) * BS + r : nullptr;
+      float* lse = kLse ? a.lse + (static_cast<size_t>(b) * a.Hq + hq) * a.S + static_cast<size_t>(j) * BS + r : nullptr;
       if (nblk == 0) {                                 // nothing selected: zero output
         for (int i = 0; i < kOParts; ++i)
           for (int q8 = 0; q8 < kOW / 8; ++q8) *reinterpret_cast<uint4*>(out + o_col(i) + q8 * 8) = make_uint4(0, 0, 0, 0);
-        if (lse && writer && half == 0) *lse = -INFINITY;
+        if constexpr (kLse)
+          if (writer && half == 0) *lse = -INFINITY;
         continue;
       }
       const uint32_t tO = tmem + C::kColO + (itv & 1) * D + lane_base;
@@ -693,7 +697,7 @@ cudaError_t launch_tc(const AttendArgs& a, cudaStream_t st) {
   if (!make_tile_map(&mq, a.q, rows, a.Hq, D, BS) || !make_tile_map(&mk, a.k, rows, a.Hkv, D, BS) ||
       !make_tile_map(&mv, a.v, rows, a.Hkv, D, BS))
     return cudaErrorInvalidValue;
-  auto k = attend_tc_kernel<BS, D>;
+  auto k = a.lse ? attend_tc_kernel<BS, D, true> : attend_tc_kernel<BS, D, false>;
   cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(k), C::kSmem);
   if (e != cudaSuccess) return e;
   const int sms = cached_sm_count();

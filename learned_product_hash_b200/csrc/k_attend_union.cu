@@ -128,7 +128,8 @@ struct Step {
 
 }  // namespace
 
-template <int D>
+// kLse: also write each row's softmax normaliser (a separate instantiation).
+template <int D, bool kLse>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_union_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttendArgs a) {
@@ -588,8 +589,9 @@ attend_union_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (!(x == 0 ? pend_has0 : pend_has1)) continue;
         const float l = (x == 0 ? pend_l0 : pend_l1) + xl[(x * 2 + 1 - half) * BS + r];
         const float inv = 1.f / l;
-        if (pend_lse && half == 0)
-          pend_lse[static_cast<size_t>(x) * a.S] = ((x == 0 ? pend_m0 : pend_m1) + __log2f(l)) * 0.6931471805599453f;
+        if constexpr (kLse)
+          if (half == 0)
+            pend_lse[static_cast<size_t>(x) * a.S] = ((x == 0 ? pend_m0 : pend_m1) + __log2f(l)) * 0.6931471805599453f;
         const uint32_t tO = tmem + lane_base + C::kColO + x * D + (D / 2) * half;
         uint4 w[kChunks];
 #pragma unroll
@@ -644,11 +646,11 @@ attend_union_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       const bool hasB = 2 * p + 1 < g;
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
                            ((static_cast<size_t>(b) * a.S + static_cast<size_t>(j) * BS + r) * a.Hq + hqA) * D;
-      float* lse = a.lse ? a.lse + (static_cast<size_t>(b) * a.Hq + hqA) * a.S + static_cast<size_t>(j) * BS + r
-                         : nullptr;
+      float* lse = kLse ? a.lse + (static_cast<size_t>(b) * a.Hq + hqA) * a.S + static_cast<size_t>(j) * BS + r
+                        : nullptr;
       if (nA == 0) zero_row(out);                     // a head with nothing selected: zero output
       if (hasB && nB == 0) zero_row(out + D);
-      if (lse && half == 0) {
+      if (kLse && half == 0) {
         if (nA == 0) lse[0] = -INFINITY;
         if (hasB && nB == 0) lse[a.S] = -INFINITY;
       }
@@ -770,7 +772,7 @@ cudaError_t launch_union(const AttendArgs& a, cudaStream_t st) {
   if (!make_tile_map(&mq, a.q, rows, a.Hq, D, C::BS) || !make_tile_map(&mk, a.k, rows, a.Hkv, D, C::BS) ||
       !make_tile_map(&mv, a.v, rows, a.Hkv, D, C::BS))
     return cudaErrorInvalidValue;
-  auto k = attend_union_kernel<D>;
+  auto k = a.lse ? attend_union_kernel<D, true> : attend_union_kernel<D, false>;
   cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(k), C::kSmem);
   if (e != cudaSuccess) return e;
   const int sms = cached_sm_count();
