@@ -473,8 +473,15 @@ static mdr_status forward_host_chunked(const mdr_config* cfg, const HostLayout& 
   MDR_CUDA(cudaMemsetAsync(status, 0, kStatusBytes, st));
   MDR_CUDA(cudaMemsetAsync(idx.lists, 0xff, lists_bytes, st));   // every list empty (-1)
   for (int c = 0; c < nchunk; ++c) {
-    const int j0 = static_cast<int>(static_cast<long long>(nb) * c / nchunk);
-    const int j1 = static_cast<int>(static_cast<long long>(nb) * (c + 1) / nchunk);
+    // Decreasing chunks (4, 3, 2, 1 tenths of the blocks): the last chunk's
+    // kernels and output copy, which nothing overlaps, are the shortest
+    // (32K workload: 4.25 ms per call against 4.79 with equal chunks).
+    static constexpr int kEdge[5] = {0, 4, 7, 9, 10};
+    const int j0 = nchunk == 4 ? static_cast<int>(static_cast<long long>(nb) * kEdge[c] / 10)
+                               : static_cast<int>(static_cast<long long>(nb) * c / nchunk);
+    const int j1 = nchunk == 4 ? static_cast<int>(static_cast<long long>(nb) * kEdge[c + 1] / 10)
+                               : static_cast<int>(static_cast<long long>(nb) * (c + 1) / nchunk);
+    if (j1 <= j0) continue;
     const int t0 = j0 * cfg->block, t1 = j1 * cfg->block;
     MDR_CUDA(copy_rows(q, q_host, qrow, cfg->B, cfg->S, t0, t1, cudaMemcpyHostToDevice, pl.in));
     MDR_CUDA(copy_rows(k, k_host, krow, cfg->B, cfg->S, t0, t1, cudaMemcpyHostToDevice, pl.in));
