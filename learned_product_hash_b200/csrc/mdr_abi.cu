@@ -404,11 +404,20 @@ struct HostPipeline {
     ready = true;
     return cudaSuccess;
   }
-  // The copies start after whatever the caller enqueued before.
+  // The copies start after whatever the caller enqueued before.  Streams
+  // and events made in a context the caller has since reset are made anew.
   cudaError_t begin(cudaStream_t st) {
     cudaError_t e = create();
+    if (e == cudaSuccess) e = cudaEventRecord(start, st);
+    if (e == cudaErrorInvalidResourceHandle || e == cudaErrorContextIsDestroyed) {
+      (void)cudaGetLastError();
+      in = out = nullptr;                          // the old handles died with their context
+      start = nullptr;
+      for (int c = 0; c < kMaxChunks; ++c) in_done[c] = comp_done[c] = nullptr;
+      ready = false;
+      if ((e = create()) == cudaSuccess) e = cudaEventRecord(start, st);
+    }
     if (e != cudaSuccess) return e;
-    if ((e = cudaEventRecord(start, st)) != cudaSuccess) return e;
     if ((e = cudaStreamWaitEvent(in, start, 0)) != cudaSuccess) return e;
     return cudaStreamWaitEvent(out, start, 0);
   }
