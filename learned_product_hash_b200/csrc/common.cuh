@@ -74,6 +74,13 @@ template <> struct Elem<__nv_bfloat16> {
 // global memory it executes grid_dependency_wait(), which returns once the
 // previous kernel has completed and its writes are visible.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel on the stream start before this one completes (its
+// grid_dependency_wait() still waits for this kernel's completion and
+// writes).  Called after this kernel's own grid_dependency_wait(), so what
+// the next kernel reads before its wait was complete before this kernel ran.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,

@@ -11,7 +11,9 @@
 // same lists); the new token is routed by its own rotated query (a block of
 // one token) and attends causally over the selected tokens.
 //
-// Three kernels, chained by programmatic dependent launch:
+// Three kernels, chained by programmatic dependent launch (the key kernel
+// lets the route kernel start at once, so the query's rotation and probe
+// codes, which need nothing the key kernel writes, overlap it):
 //   decode_keys_kernel    one CTA per (b, KV head): rotate k_t into the key
 //                         cache, copy v_t, add the rotated key (float32) to
 //                         the running sum of the block; when t completes its
@@ -63,30 +65,26 @@ template <typename T> __device__ __forceinline__ T st_f(float x);
 template <> __device__ __forceinline__ float st_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 st_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
-// vpl (1, 2 or 4) consecutive elements at p (aligned to vpl elements) as floats.
-__device__ __forceinline__ void ld_vec(const float* p, int vpl, float* o) {
-  if (vpl == 4) {
-    const float4 f = *reinterpret_cast<const float4*>(p);
-    o[0] = f.x; o[1] = f.y; o[2] = f.z; o[3] = f.w;
-  } else if (vpl == 2) {
-    const float2 f = *reinterpret_cast<const float2*>(p);
-    o[0] = f.x; o[1] = f.y;
-  } else {
-    o[0] = *p;
+// 16 bytes of a row (4 float32 or 8 bf16 coordinates) as floats.
+template <typename T> struct Row16;
+template <> struct Row16<float> {
+  static constexpr int kN = 4;
+  static __device__ __forceinline__ void unpack(const uint4& r, float* o) {
+    o[0] = __uint_as_float(r.x); o[1] = __uint_as_float(r.y);
+    o[2] = __uint_as_float(r.z); o[3] = __uint_as_float(r.w);
   }
-}
-__device__ __forceinline__ void ld_vec(const __nv_bfloat16* p, int vpl, float* o) {
-  if (vpl == 4) {
-    const uint2 r = *reinterpret_cast<const uint2*>(p);
-    o[0] = __uint_as_float(r.x << 16); o[1] = __uint_as_float(r.x & 0xffff0000u);
-    o[2] = __uint_as_float(r.y << 16); o[3] = __uint_as_float(r.y & 0xffff0000u);
-  } else if (vpl == 2) {
-    const uint32_t r = *reinterpret_cast<const uint32_t*>(p);
-    o[0] = __uint_as_float(r << 16); o[1] = __uint_as_float(r & 0xffff0000u);
-  } else {
-    o[0] = __bfloat162float(*p);
+};
+template <> struct Row16<__nv_bfloat16> {
+  static constexpr int kN = 8;
+  static __device__ __forceinline__ void unpack(const uint4& r, float* o) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      o[2 * i] = __uint_as_float(w[i] << 16);             // the element at the lower address
+      o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
   }
-}
+};
 
 // Score of codeword k of subspace sdx against xs (dsub floats, shared
 // memory): four float32 partial sums over d mod 4, added pairwise.
@@ -124,6 +122,7 @@ decode_keys_kernel(const __grid_constant__ DecodeArgs a) {
   __shared__ int widx[kKeyThreads / 32];
   __shared__ int code[4];
   grid_dependency_wait();
+  grid_launch_dependents();          // the route kernel rotates its query and probes meanwhile
   const int b = blockIdx.x / a.Hkv, h = blockIdx.x % a.Hkv;
   const int D = a.D, half = D / 2, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t bh = static_cast<size_t>(b) * a.Hkv + h;
@@ -211,7 +210,6 @@ decode_route_kernel(const __grid_constant__ DecodeArgs a) {
   int* cand = reinterpret_cast<int*>(dsm + kDecCand);
   uint32_t* ckey = reinterpret_cast<uint32_t*>(dsm + kDecKey);
   __shared__ int s_ncand;
-  grid_dependency_wait();            // the key kernel of this step wrote token t
   const int b = blockIdx.x / a.Hq, hq = blockIdx.x % a.Hq, h = hq / (a.Hq / a.Hkv);
   const size_t bh = static_cast<size_t>(b) * a.Hkv + h, bq = static_cast<size_t>(b) * a.Hq + hq;
   const int t = a.t, j = t / a.bs, D = a.D, half = D / 2, dsub = D / a.P;
@@ -254,6 +252,9 @@ decode_route_kernel(const __grid_constant__ DecodeArgs a) {
     }
   }
   __syncthreads();
+  // Steps 1 and 2 read only the step's query and the codebooks; from here on
+  // the index, which the key kernel of this step may have appended to.
+  grid_dependency_wait();
 
   // 3. route (warp 0).
   if (warp == 0) {
@@ -397,73 +398,114 @@ decode_route_kernel(const __grid_constant__ DecodeArgs a) {
 }
 
 // Attention of token t over one selected block: CTA (b*Hq + hq, slot) takes
-// block sel[slot] (tokens s <= t), four warps with a float32 online softmax
-// each (lanes hold D/32 coordinates of the rows they read, eight tokens in
-// flight), merged into the block's (max, sum, output); the last CTA of a
-// (b, hq) to finish merges all blocks, in slot order, into the output.
-template <typename T>
+// block sel[slot] (tokens s <= t).  A row of the cache is read as 16-byte
+// pieces by kLpr consecutive lanes, so a warp reads 32/kLpr rows per load
+// and each lane keeps eight loads of K and eight of V in flight at once (one
+// memory round trip per 8*32/kLpr rows).  Scores are summed over the lanes
+// of a row; the warp shares one running maximum (float32 online softmax) and
+// each lane accumulates its coordinates over its own rows; the row groups of
+// a warp, then the four warps, are merged into the block's (max, sum,
+// output).  The last CTA of a (b, hq) to finish merges all blocks, in slot
+// order, into the output, reading every block's partial result in one
+// parallel round.
+template <typename T, int kLpr>
 __global__ void __launch_bounds__(128)
 decode_partial_kernel(const __grid_constant__ DecodeArgs a) {
+  constexpr int kEpl = Row16<T>::kN;       // coordinates per lane
+  constexpr int kRpi = 32 / kLpr;          // rows per warp load
+  constexpr int kSteps = 8;                // loads of K (and of V) in flight per lane
+  constexpr int kRowsWarp = kSteps * kRpi;
+  constexpr int kRowsPass = 4 * kRowsWarp;
+  constexpr int kMaxSlots = 64;            // R + L <= 64 (the configuration check)
   __shared__ float wm[4], wl[4];
   __shared__ float wo[4][128];
+  __shared__ float s_m[kMaxSlots], s_l[kMaxSlots], s_f[kMaxSlots];
   __shared__ int s_last;
   grid_dependency_wait();            // sel and the rotated query of this step
   const int bq = blockIdx.x, slot = blockIdx.y, nsl = a.R + a.L;
   const int b = bq / a.Hq, hq = bq % a.Hq, h = hq / (a.Hq / a.Hkv);
-  const int t = a.t, D = a.D, vpl = D / 32;
+  const int t = a.t, D = a.D;        // D == kLpr * kEpl
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = lane / kLpr, col = (lane % kLpr) * kEpl;
   const int blk = a.sel_t[static_cast<size_t>(bq) * nsl + slot];
-  float m = -INFINITY, l = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+  float m = -INFINITY, l = 0.f, o[kEpl];
+#pragma unroll
+  for (int e = 0; e < kEpl; ++e) o[e] = 0.f;
   if (blk >= 0) {
     const int first = blk * a.bs, ntok = min(a.bs, t + 1 - first);
-    float qv[4];
+    float qv[kEpl];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) qv[e] = e < vpl ? a.qrot_t[static_cast<size_t>(bq) * D + lane * vpl + e] * a.scale : 0.f;
-    const int per = (ntok + 3) / 4, u0 = warp * per, u1 = min(ntok, u0 + per);
-    constexpr int kTok = 8;
-    for (int u = u0; u < u1; u += kTok) {
-      float sc[kTok], vv[kTok][4], kv[kTok][4];
+    for (int e = 0; e < kEpl; ++e) qv[e] = a.qrot_t[static_cast<size_t>(bq) * D + col + e] * a.scale;
+    const size_t rs = static_cast<size_t>(a.Hkv) * D;                 // elements from one token to the next
+    const size_t base = (static_cast<size_t>(b) * a.S + first) * rs + static_cast<size_t>(h) * D + col;
+    const T* kb = static_cast<const T*>(a.krot) + base;
+    const T* vb = static_cast<const T*>(a.v) + base;
+    for (int r0 = 0; r0 < ntok; r0 += kRowsPass) {
+      const int rw = r0 + warp * kRowsWarp + grp;                      // row of step 0; step s adds s*kRpi
+      uint4 kr[kSteps], vr[kSteps];
 #pragma unroll
-      for (int x = 0; x < kTok; ++x) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) { vv[x][e] = 0.f; kv[x][e] = 0.f; }
-        if (u + x < u1) {
-          const size_t off = ((static_cast<size_t>(b) * a.S + first + u + x) * a.Hkv + h) * D + lane * vpl;
-          ld_vec(static_cast<const T*>(a.krot) + off, vpl, kv[x]);
-          ld_vec(static_cast<const T*>(a.v) + off, vpl, vv[x]);
+      for (int s = 0; s < kSteps; ++s) {
+        const int r = rw + s * kRpi;
+        if (r < ntok) {
+          kr[s] = *reinterpret_cast<const uint4*>(kb + r * rs);
+          vr[s] = *reinterpret_cast<const uint4*>(vb + r * rs);
+        } else {
+          kr[s] = make_uint4(0u, 0u, 0u, 0u);
+          vr[s] = make_uint4(0u, 0u, 0u, 0u);
         }
       }
+      float sc[kSteps];
 #pragma unroll
-      for (int x = 0; x < kTok; ++x) {
-        sc[x] = 0.f;
+      for (int s = 0; s < kSteps; ++s) {
+        float kf[kEpl];
+        Row16<T>::unpack(kr[s], kf);
+        float d = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sc[x] = __fmaf_rn(qv[e], kv[x][e], sc[x]);
+        for (int e = 0; e < kEpl; ++e) d = __fmaf_rn(qv[e], kf[e], d);
+        sc[s] = d;
       }
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1)
+      for (int off = kLpr / 2; off > 0; off >>= 1)
 #pragma unroll
-        for (int x = 0; x < kTok; ++x) sc[x] = __fadd_rn(sc[x], __shfl_xor_sync(0xffffffffu, sc[x], off));
+        for (int s = 0; s < kSteps; ++s) sc[s] = __fadd_rn(sc[s], __shfl_xor_sync(0xffffffffu, sc[s], off));
+      float pm = -INFINITY;
 #pragma unroll
-      for (int x = 0; x < kTok; ++x) {
-        if (u + x >= u1) break;
-        if (sc[x] > m) {
-          const float alpha = expf(m - sc[x]);
-          l *= alpha;
+      for (int s = 0; s < kSteps; ++s) {
+        if (rw + s * kRpi >= ntok) sc[s] = -INFINITY;
+        pm = fmaxf(pm, sc[s]);
+      }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) o[e] *= alpha;
-          m = sc[x];
-        }
-        const float p = expf(sc[x] - m);
+      for (int off = kLpr; off < 32; off <<= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, off));
+      if (pm == -INFINITY) break;      // warp-uniform: this warp has no row left in the block
+      const float mn = fmaxf(m, pm);
+      const float alpha = expf(m - mn);
+      l *= alpha;
+#pragma unroll
+      for (int e = 0; e < kEpl; ++e) o[e] *= alpha;
+#pragma unroll
+      for (int s = 0; s < kSteps; ++s) {
+        const float p = expf(sc[s] - mn);
         l += p;
+        float vf[kEpl];
+        Row16<T>::unpack(vr[s], vf);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[e] = __fmaf_rn(p, vv[x][e], o[e]);
+        for (int e = 0; e < kEpl; ++e) o[e] = __fmaf_rn(p, vf[e], o[e]);
       }
+      m = mn;
+    }
+    // The warp's row groups share m: add their sums and outputs.
+#pragma unroll
+    for (int off = kLpr; off < 32; off <<= 1) {
+      l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, off));
+#pragma unroll
+      for (int e = 0; e < kEpl; ++e) o[e] = __fadd_rn(o[e], __shfl_xor_sync(0xffffffffu, o[e], off));
     }
   }
   if (lane == 0) { wm[warp] = m; wl[warp] = l; }
+  if (lane < kLpr) {
 #pragma unroll
-  for (int e = 0; e < 4; ++e)
-    if (e < vpl) wo[warp][lane * vpl + e] = o[e];
+    for (int e = 0; e < kEpl; ++e) wo[warp][col + e] = o[e];
+  }
   __syncthreads();
   // This block's (max, sum, output) over its four warps.
   float* pp = a.part + (static_cast<size_t>(bq) * nsl + slot) * (2 + D);
@@ -488,27 +530,44 @@ decode_partial_kernel(const __grid_constant__ DecodeArgs a) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // Last block of this (b, hq): merge the blocks in slot order.
+  // Last block of this (b, hq): every block's max and sum in one round, then
+  // the outputs weighted in slot order.
   const float* pb = a.part + static_cast<size_t>(bq) * nsl * (2 + D);
+  if (tid < nsl) {
+    s_m[tid] = __ldcg(pb + tid * (2 + D));
+    s_l[tid] = __ldcg(pb + tid * (2 + D) + 1);
+  }
+  __syncthreads();
   float MM = -INFINITY;
-  for (int s = 0; s < nsl; ++s) MM = fmaxf(MM, __ldcg(pb + s * (2 + D)));
+  for (int s = 0; s < nsl; ++s) MM = fmaxf(MM, s_m[s]);
+  if (tid < nsl) s_f[tid] = s_m[tid] == -INFINITY ? 0.f : expf(s_m[tid] - MM);
+  __syncthreads();
+  float den = 0.f;
+  for (int s = 0; s < nsl; ++s) den = __fmaf_rn(s_f[s], s_l[s], den);
   T* out = static_cast<T*>(a.out_t) + static_cast<size_t>(bq) * D;
   for (int i = tid; i < D; i += 128) {
-    float num = 0.f, den = 0.f;
-    for (int s = 0; s < nsl; ++s) {
-      const float ms = __ldcg(pb + s * (2 + D));
-      if (ms == -INFINITY) continue;
-      const float f = expf(ms - MM);
-      num = __fmaf_rn(f, __ldcg(pb + s * (2 + D) + 2 + i), num);
-      den = __fmaf_rn(f, __ldcg(pb + s * (2 + D) + 1), den);
-    }
+    float num = 0.f;
+#pragma unroll 8
+    for (int s = 0; s < nsl; ++s) num = __fmaf_rn(s_f[s], __ldcg(pb + s * (2 + D) + 2 + i), num);
     out[i] = st_f<T>(num / den);
   }
   if (tid == 0) a.done[bq] = 0;
 }
 
+template <typename T>
+cudaError_t launch_partial(const DecodeArgs& a, cudaStream_t st) {
+  const dim3 grid(a.B * a.Hq, a.R + a.L);
+  const int lpr = a.D * static_cast<int>(sizeof(T)) / 16;   // lanes per row (D is 32, 64 or 128)
+  if (lpr == 8) return launch_pdl(decode_partial_kernel<T, 8>, grid, dim3(128), 0, st, a);
+  if (lpr == 16) return launch_pdl(decode_partial_kernel<T, 16>, grid, dim3(128), 0, st, a);
+  if constexpr (sizeof(T) == 4) {
+    if (lpr == 32) return launch_pdl(decode_partial_kernel<T, 32>, grid, dim3(128), 0, st, a);
+  }
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t st) {
-  if (a.D > 128 || a.D % 32 != 0 || a.K > 128 || a.P > 4) return cudaErrorInvalidValue;
+  if (a.D > 128 || a.D % 32 != 0 || a.K > 128 || a.P > 4 || a.R + a.L > 64) return cudaErrorInvalidValue;
   cudaError_t e = bf16 ? launch_pdl(decode_keys_kernel<__nv_bfloat16>, dim3(a.B * a.Hkv), dim3(kKeyThreads), 0, st, a)
                        : launch_pdl(decode_keys_kernel<float>, dim3(a.B * a.Hkv), dim3(kKeyThreads), 0, st, a);
   if (e != cudaSuccess) return e;
@@ -516,8 +575,7 @@ cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t st) {
   void (*k)(DecodeArgs) = bf16 ? decode_route_kernel<__nv_bfloat16> : decode_route_kernel<float>;
   if ((e = cached_allow_smem(reinterpret_cast<const void*>(k), static_cast<int>(smem))) != cudaSuccess) return e;
   if ((e = launch_pdl(k, dim3(a.B * a.Hq), dim3(kAttWarps * 32), smem, st, a)) != cudaSuccess) return e;
-  void (*kp)(DecodeArgs) = bf16 ? decode_partial_kernel<__nv_bfloat16> : decode_partial_kernel<float>;
-  if ((e = launch_pdl(kp, dim3(a.B * a.Hq, a.R + a.L), dim3(128), 0, st, a)) != cudaSuccess) return e;
+  if ((e = bf16 ? launch_partial<__nv_bfloat16>(a, st) : launch_partial<float>(a, st)) != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -150,6 +150,26 @@ def test_decode_local_only_f32():
     _compare(w, inp, 32, w.S)
 
 
+def test_decode_block128_gqa_bf16():
+    """Blocks of 128 tokens at D = 128 with four query heads per KV head (the
+    long workload's head shape, shortened): a selected block is read in two
+    passes of 64 rows, so the running maximum is rescaled between passes; a
+    block completes during decoding."""
+    from workloads import LONG
+    w = LONG.with_(S=2048, Hq=8, Hkv=2, keys="gaussian")
+    inp = make_inputs(w, 6)
+    _compare(w, inp, 1536, 1536 + 129)
+
+
+@pytest.mark.parametrize("D,block,S", [(64, 32, 192), (128, 64, 384)])
+def test_decode_f32_wide_rows(D, block, S):
+    """float32 rows of 64 and 128 coordinates (16 and 32 lanes per row; at
+    D = 128 a block of 64 rows takes two passes)."""
+    w = TINY.with_(D=D, block=block, S=S)
+    inp = make_inputs(w, 7)
+    _compare(w, inp, S // 2, S)
+
+
 def test_prefill_state_equals_oracle_index():
     """mdr_decode_prefill of a prefix holds the oracle's index of that prefix
     (the batch build), in the state's own strides (capacity larger than the
