@@ -524,12 +524,18 @@ decode_partial_kernel(const __grid_constant__ DecodeArgs a) {
     pp[0] = M;
     pp[1] = den;
   }
-  __threadfence();
+  // Publish: the barrier orders the CTA's stores before thread 0's fence
+  // and counter increment (a release, cumulative over the barrier); the last
+  // block's thread 0 fences again (acquire) before the barrier after which
+  // its threads read the other blocks' partial results.
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(a.done + bq, 1) == nsl - 1;
+  if (tid == 0) {
+    __threadfence();
+    s_last = atomicAdd(a.done + bq, 1) == nsl - 1;
+    if (s_last) __threadfence();
+  }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   // Last block of this (b, hq): every block's max and sum in one round, then
   // the outputs weighted in slot order.
   const float* pb = a.part + static_cast<size_t>(bq) * nsl * (2 + D);

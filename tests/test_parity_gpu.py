@@ -63,6 +63,9 @@ EDGE = {
     "many_heads_bf16": (AR.with_(B=1, S=256, Hq=72, Hkv=72, D=128, keys="gaussian"), {}),
     # odd head count: token groups that do not tile the 512 summary threads
     "three_heads_bf16": (AR.with_(B=2, S=512, Hq=3, Hkv=3, D=128, block=128, keys="gaussian"), {}),
+    # block 128 at D = 64, one query head per KV head: the per-head kernel
+    # rotates 128-row Q tiles whose pairs share one 64-column region
+    "block128_d64_bf16": (AR.with_(B=2, S=640, Hq=2, Hkv=2, block=128, keys="gaussian"), {}),
     # block 128 with grouped query heads: pairs of heads share one gather of
     # their selections' union (two and four heads per KV head, D 128 and 64)
     "union_g2_d128": (CAPACITY.with_(S=12 * 128, block=128, D=128, Hq=4, Hkv=2, K=8, cap=16, R=4, L=2), {}),
