@@ -70,9 +70,9 @@ template <> struct Elem<__nv_bfloat16> {
 
 // Programmatic dependent launch.  Every libmdr kernel is launched with
 // launch_pdl, so it may start (set up shared memory, barriers, tensor memory)
-// while the previous kernel on the stream drains; before it reads anything in
-// global memory it executes grid_dependency_wait(), which returns once the
-// previous kernel has completed and its writes are visible.
+// while the previous kernel on the stream drains; before it reads anything an
+// earlier kernel wrote it executes grid_dependency_wait(), which returns once
+// the previous kernel has completed and its writes are visible.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // Lets the next kernel on the stream start before this one completes (its
 // grid_dependency_wait() still waits for this kernel's completion and
