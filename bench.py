@@ -19,7 +19,7 @@ same run (each can be left out with its --no-* flag):
                  forced route, local-only;
   calibration    codebook calibration rounds on the long workload's key
                  summaries, and a held-out sequence's overflow and maximum
-                 load before and after;
+                 load before and after; the same rounds on 2^20 records;
   backward       dq, dk, dv of the attention with the route held fixed at 32K;
   scaling_sweep  the forward from 4K to 128K tokens with log-log slopes, and
                  the CPU oracle's index + route slope at 4K-32K (N = 1 only).
@@ -732,6 +732,29 @@ def run_mine(args, w):
                                     "algorithmic_bytes_per_round": c_bytes},
                        "held_out": held, "capacity": wl.cap}
         del ixl, wsl, cws, rec
+        # The same rounds on a record set far larger than L2 (2^20 unit
+        # records, 512 MB): the bandwidth regime, where the 8K-record loop
+        # above is bound by its three launches per round.
+        NL, rounds_l = 1 << 20, 5
+        gl = torch.Generator(device=dev)
+        gl.manual_seed(3100 + rank)
+        recl = torch.randn(NL, wl.D, generator=gl, device=dev)
+        recl /= recl.norm(dim=1, keepdim=True)
+        cwl = mdr.calibrate_workspace(NL, wl.D, wl.P, wl.K, dev)
+        mdr.mdr_calibrate_codebooks(recl, cb0, cb1, 1, cwl)      # warm-up
+        c0.record(stream)
+        mdr.mdr_calibrate_codebooks(recl, cb0, cb1, rounds_l, cwl)
+        c1.record(stream)
+        c1.synchronize()
+        cl_ms = c0.elapsed_time(c1) / rounds_l
+        cl_bytes = 2 * NL * wl.D * 4 + 2 * NL * wl.P * 4
+        calibration["large"] = {
+            "records": NL, "rounds": rounds_l, "us_per_round": cl_ms * 1e3,
+            "inputs": "unit vectors (torch's seeded generator on the device, normalised)",
+            "l2": "the records (512 MB) exceed L2",
+            "roofline": {"bound": "hbm", "achieved": cl_bytes / (cl_ms / 1e3) / 1e9, "peak": peak_c, "unit": "GB/s",
+                         "frac": cl_bytes / (cl_ms / 1e3) / 1e9 / peak_c, "algorithmic_bytes_per_round": cl_bytes}}
+        del recl, cwl
 
     # Backward of the attention with the forward's route held fixed: dq, dk,
     # dv (float32) for a seeded upstream gradient, timed with CUDA events.
