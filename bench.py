@@ -346,7 +346,7 @@ def backward_bytes(w, sel: np.ndarray, es: int) -> int:
 
 
 def forward_bytes(w, nsel: int, es: int) -> dict:
-    """Algorithmic bytes of one forward (the survey's byte model): the
+    """Algorithmic bytes of one forward (the path's byte model): the
     summary pass reads q and k once; the attention reads q, gathers K and V of
     every valid selected block and writes the output.  The summary pass's
     rotated copies (written once, read by the attention) are not algorithmic
