@@ -27,9 +27,10 @@
 //                         first); route (warp 0): all probes' list lengths at
 //                         once, slots read 32 at a time and filtered to
 //                         i <= j - L; candidates scored <q'_t, kbar_i> in
-//                         float32 by all warps; top R by rounds of warp
-//                         arg-max (higher score, lower id), remote ids
-//                         ascending, then the locals.
+//                         float32 by all warps; top R (higher score, lower
+//                         id) by one ranking pass over at most 32
+//                         candidates, else by rounds of warp arg-max;
+//                         remote ids ascending, then the locals.
 //   decode_partial_kernel one CTA per (b, query head, selected block): the
 //                         block's tokens s <= t with a float32 online softmax
 //                         (split-K over the selected blocks, so that a
@@ -359,7 +360,38 @@ decode_route_kernel(const __grid_constant__ DecodeArgs a) {
   }
   __syncthreads();
 
-  if (warp == 0) {
+  if (warp == 0 && s_ncand <= 32) {
+    // At most 32 candidates: lane l ranks candidate l against all the others
+    // in one pass (higher score first, lower id on equal scores); the best R
+    // are written in ascending id order, -1 after them -- the same selection
+    // as the rounds below, without their chain of dependent reductions.
+    const int n = s_ncand;
+    const bool have = lane < n;
+    const uint32_t k = have ? ckey[lane] : 0u;
+    const int id = have ? cand[lane] : INT_MAX;
+    int better = 0;
+    for (int m = 0; m < n; ++m) {
+      const uint32_t km = __shfl_sync(0xffffffffu, k, m);
+      const int im = __shfl_sync(0xffffffffu, id, m);
+      better += (km > k || (km == k && im < id)) ? 1 : 0;
+    }
+    const bool win = have && better < a.R;
+    const unsigned wmask = __ballot_sync(0xffffffffu, win);
+    int pos = 0;                                  // winners with a lower id
+    for (int m = 0; m < n; ++m) {
+      const int im = __shfl_sync(0xffffffffu, id, m);
+      pos += (((wmask >> m) & 1u) && im < id) ? 1 : 0;
+    }
+    int32_t* srow = a.sel_t + bq * (a.R + a.L);
+    const int nwin = __popc(wmask);
+    if (win) srow[pos] = id;
+    if (lane >= nwin && lane < a.R) srow[lane] = -1;
+    if (lane < a.L) {
+      const int lid = j - a.L + 1 + lane;
+      srow[a.R + lane] = lid >= 0 ? lid : -1;
+    }
+    if (a.ncand_t && lane == 0) a.ncand_t[bq] = n;
+  } else if (warp == 0) {
     const int n = s_ncand;
     int mine = INT_MAX;                           // lane r: the r-th winner
     for (int r = 0; r < a.R; ++r) {

@@ -150,6 +150,16 @@ def test_decode_local_only_f32():
     _compare(w, inp, 32, w.S)
 
 
+def test_decode_many_candidates_bf16():
+    """Four codewords per subspace (16 addresses) probed four deep: every
+    list is probed, so a token sees every eligible block as a candidate
+    (more than 32): the route takes its best R by rounds of arg-max rather
+    than by the one-pass ranking used for at most 32."""
+    w = AR.with_(B=1, S=4096, K=4, probes=4, cap=16, R=8, L=2, keys="gaussian")
+    inp = make_inputs(w, 8)
+    _compare(w, inp, 3072, 3072 + 66)
+
+
 def test_decode_block128_gqa_bf16():
     """Blocks of 128 tokens at D = 128 with four query heads per KV head (the
     long workload's head shape, shortened): a selected block is read in two
