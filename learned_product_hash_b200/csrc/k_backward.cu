@@ -16,8 +16,11 @@
 //                      the (query head, query block) pairs whose selection
 //                      holds it, in (head, block, slot) order -- a stable
 //                      counting sort of the selection (counts, prefix sums,
-//                      then one warp places the entries 32 at a time with
-//                      __match_any_sync ranks).
+//                      then rounds of 32 entries per warp: ranks within a
+//                      warp by __match_any_sync, each warp's starting rank
+//                      per key block by a prefix over a [warps][nb] count
+//                      table; one warp walks the entries when the table does
+//                      not fit in shared memory).
 //   bwd_dq_kernel      one or more CTAs per (sequence, query head, query
 //                      block), thread = (query token, 16 coordinates):
 //                      pass 1 over the selected blocks (K, V staged in shared
@@ -74,26 +77,30 @@ __global__ void bwd_rotate_kernel(const BwdArgs a) {
   }
 }
 
-__global__ void __launch_bounds__(256) bwd_rev_kernel(const BwdArgs a) {
+constexpr int kRevThreads = 512;
+
+__global__ void __launch_bounds__(kRevThreads) bwd_rev_kernel(const BwdArgs a, const int nw) {
   extern __shared__ int rsm[];
   int* cnt = rsm;                                  // [nb]
   int* off = rsm + a.nb;                           // [nb + 1]
+  int* cw = off + a.nb + 1;                        // [nw][nb] when nw > 0
   const int b = blockIdx.x / a.Hkv, h = blockIdx.x % a.Hkv;
   const int g = a.Hq / a.Hkv;
   const int E = g * a.nb * a.nsel;                 // entries (hl, j, slot); < 2^31 (checked on the host)
   const int32_t* sel0 = a.sel + (static_cast<long long>(b) * a.Hq + static_cast<long long>(h) * g) * a.nb * a.nsel;
-  for (int i = threadIdx.x; i < a.nb; i += blockDim.x) cnt[i] = 0;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < a.nb; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   grid_dependency_wait();                          // sel may come from the previous kernel
   // Counts (order-free).
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+  for (int e = tid; e < E; e += blockDim.x) {
     const int j = (e / a.nsel) % a.nb;
     const int id = sel0[e];
     if (id >= 0 && id <= j) atomicAdd(&cnt[id], 1);
   }
   __syncthreads();
   // Exclusive prefix sums by warp 0, 32 blocks at a time.
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = tid >> 5, lane = tid & 31;
   if (warp == 0) {
     int run = 0;
     for (int base = 0; base < a.nb; base += 32) {
@@ -112,15 +119,59 @@ __global__ void __launch_bounds__(256) bwd_rev_kernel(const BwdArgs a) {
   }
   __syncthreads();
   int32_t* roff = a.rev_off + static_cast<long long>(blockIdx.x) * (a.nb + 1);
-  for (int i = threadIdx.x; i <= a.nb; i += blockDim.x) roff[i] = off[i];
-  for (int i = threadIdx.x; i < a.nb; i += blockDim.x) cnt[i] = 0;   // reused as fill counters
+  for (int i = tid; i <= a.nb; i += blockDim.x) roff[i] = off[i];
+  for (int i = tid; i < a.nb; i += blockDim.x) cnt[i] = 0;   // reused as running counts
   __syncthreads();
-  // Stable placement: entries in (hl, j, slot) order, 32 per step; the
-  // selection is read four steps at a time so the loads overlap.
-  if (warp == 0) {
-    int32_t* rev = a.rev + static_cast<long long>(blockIdx.x) * E;
+  int32_t* rev = a.rev + static_cast<long long>(blockIdx.x) * E;
+  const int per_head = a.nsel * a.nb;
+  if (nw > 0) {
+    // Stable placement in rounds of nw * 32 entries: (1) ranks within each
+    // warp's 32 consecutive entries, the lowest peer recording its group's
+    // size in the warp's row of the table; (2) per key block, a prefix over
+    // the warps gives each warp's starting rank and advances the running
+    // count; (3) each entry lands at its block's offset + starting rank +
+    // rank within the warp.
+    const unsigned lower = (1u << lane) - 1u;
+    for (int r0 = 0; r0 < E; r0 += nw * 32) {
+      for (int x = tid; x < nw * a.nb; x += blockDim.x) cw[x] = 0;
+      __syncthreads();
+      const int e = r0 + warp * 32 + lane;
+      int id = -1, code = 0;
+      if (warp < nw && e < E) {
+        const int hl = e / per_head, j = (e - hl * per_head) / a.nsel;
+        const int v = sel0[e];
+        if (v >= 0 && v <= j) {
+          id = v;
+          code = hl * a.nb + j;
+        }
+      }
+      int rk = 0;
+      if (warp < nw) {
+        const unsigned vm = __ballot_sync(0xffffffffu, id >= 0);
+        if (id >= 0) {
+          const unsigned peers = __match_any_sync(vm, id);
+          rk = __popc(peers & lower);
+          if (rk == 0) cw[warp * a.nb + id] = __popc(peers);
+        }
+      }
+      __syncthreads();
+      for (int x = tid; x < a.nb; x += blockDim.x) {
+        int run = cnt[x];
+        for (int w = 0; w < nw; ++w) {
+          const int t = cw[w * a.nb + x];
+          cw[w * a.nb + x] = run;
+          run += t;
+        }
+        cnt[x] = run;
+      }
+      __syncthreads();
+      if (id >= 0) rev[off[id] + cw[warp * a.nb + id] + rk] = code;
+      __syncthreads();                             // the table is cleared for the next round
+    }
+  } else if (warp == 0) {
+    // One warp walks the entries 32 at a time; the selection is read four
+    // steps ahead so the loads overlap.
     int ahead[4];
-    const int per_head = a.nsel * a.nb;
     for (int base = 0; base < E; base += 32) {
       const int u = (base >> 5) & 3;
       if (u == 0) {
@@ -394,10 +445,17 @@ static cudaError_t launch_grad_for(const BwdArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_bwd_rev(const BwdArgs& a, cudaStream_t st) {
-  const size_t smem = bwd_rev_smem(a.nb);
+  // As many warp rows of the placement table as fit beside the counts and
+  // offsets (none: one warp walks the entries).
+  constexpr int kSmemInts = 227 * 1024 / 4 - 64;
+  const long long base_ints = 2LL * a.nb + 1;
+  long long nw = a.nb > 0 ? (kSmemInts - base_ints) / a.nb : 0;
+  nw = nw < kRevThreads / 32 ? nw : kRevThreads / 32;
+  if (nw < 2) nw = 0;
+  const size_t smem = bwd_rev_smem(a.nb) + static_cast<size_t>(nw) * a.nb * sizeof(int);
   cudaError_t e = cached_allow_smem(reinterpret_cast<const void*>(bwd_rev_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(bwd_rev_kernel, dim3(a.B * a.Hkv), dim3(256), smem, st, a);
+  return launch_pdl(bwd_rev_kernel, dim3(a.B * a.Hkv), dim3(kRevThreads), smem, st, a, static_cast<int>(nw));
 }
 
 cudaError_t launch_backward(const BwdArgs& a, bool bf16, cudaStream_t st) {
