@@ -90,8 +90,8 @@ struct BwCfg {
   static constexpr int qSmem = qOffCtl + kCtl;
   static constexpr int qCols = pow2_cols(2 * BS + D);
   static constexpr int qColS = 0, qColP = BS, qColO = 2 * BS;
-  // dk/dv kernel: an entry slot holds a query tile's Q, dO, lse and Delta
-  static constexpr int kSlot = (2 * kTile + 2 * BS * 4 + 1023) / 1024 * 1024;
+  // dk/dv kernel: an entry slot holds a query tile's Q, dO, lse and Delta, and a header (its query block)
+  static constexpr int kSlot = (2 * kTile + 2 * BS * 4 + 16 + 1023) / 1024 * 1024;   // + a 16-byte header
   static_assert(qSmem <= 232448, "shared memory per CTA");
   static_assert(kTile % 1024 == 0 && kPTile % 1024 == 0, "1024-byte aligned tiles");
   // D-column geometry of a thread: W columns at lo and W at D/2 + lo, NP times.
@@ -572,7 +572,10 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // epilogue), warp 8 loads by TMA, warp 9 issues the MMAs (and owns the
 // tensor memory).
 // S^T and dP^T of the next entry are computed while the four warps work on
-// the current one (two TMEM buffers at bs = 64); every hand-off is an
+// the current one (two TMEM buffers at bs = 64); the next key tile's K and V
+// load into a second buffer during the current tile (not at bs = D = 128),
+// and at bs = 64 the epilogue hands the accumulators back as soon as it has
+// read them; every hand-off is an
 // mbarrier, every wait bounded (2 s, and given up as soon as another role has
 // given up).
 constexpr int kWsThreads = 320;                  // 8 elementwise warps, a TMA warp, an MMA warp
@@ -582,9 +585,15 @@ template <int BS, int D>
 struct WsCfg {
   using C = BwCfg<BS, D>;
   static constexpr int NS = (BS == 64) ? 2 : 1;                       // S^T / dP^T / P^T / dS^T buffers
-  static constexpr int NE = (BS == 64) ? (D == 64 ? 8 : 4) : (D == 64 ? 3 : 1);   // entry slots
+  static constexpr int NE = (BS == 64) ? (D == 64 ? 8 : 3) : (D == 64 ? 2 : 1);   // entry slots
+  // (K, V) tile buffers: two, so that the next key tile's K and V (and, behind
+  // them, its entries) load while the current tile is processed; one at
+  // bs = D = 128, where a second does not fit.
+  static constexpr int NKV = (BS == 128 && D == 128) ? 1 : 2;
   static constexpr int kSlot = C::kSlot;
-  static constexpr int oK = 0, oV = C::kTile, oE = 2 * C::kTile;
+  static constexpr int kHdr = 2 * C::kTile + 2 * BS * 4;               // the entry's query block (int)
+  static_assert(kHdr + 4 <= kSlot, "entry slot header");
+  static constexpr int oKV = 0, oE = NKV * 2 * C::kTile;
   static constexpr int oPT = oE + NE * kSlot;                          // NS x P^T
   static constexpr int oDS = oPT + NS * C::kPTile;                     // NS x dS^T
   static constexpr int oCtl = oDS + NS * C::kPTile;
@@ -594,8 +603,8 @@ struct WsCfg {
   static constexpr int kCols = pow2_cols(2 * NS * BS + 2 * D);
   static_assert(2 * NS * BS + 2 * D <= 512, "tensor memory");
   // barriers
-  static constexpr int bKvF = 0, bKvE = 1, bAF = 2, bAE = 3, bFin = 4;
-  static constexpr int bEF = 5, bEE = bEF + NE;
+  static constexpr int bKvF = 0, bKvE = 2, bAF = 4, bAE = 5, bFin = 6;   // bKvF, bKvE: NKV each
+  static constexpr int bEF = 7, bEE = bEF + NE;
   static constexpr int bSF = bEE + NE, bSE = bSF + NS, bPF = bSE + NS, bPE = bPF + NS;
   static constexpr int kBars = bPE + NS;
   static_assert(kBars <= 32, "barrier space");
@@ -623,7 +632,7 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   }
   WsCtl& ctl = *reinterpret_cast<WsCtl*>(smem + W::oCtl);
   const uint32_t base = smem_u32(smem);
-  const uint32_t sK = base + W::oK, sV = base + W::oV, sE = base + W::oE;
+  const uint32_t sKV = base + W::oKV, sE = base + W::oE;
   auto BAR = [&](int i) { return smem_u32(&ctl.bar[i]); };
   volatile int* abort_flag = &ctl.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -701,7 +710,7 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       prefetch_tmap(&tmO);
-      long long xg = 0, tc_ = 0;
+      long long xg = 0, tc_ = 0, kv_issued = 0;   // entries, key tiles, key tiles whose K, V were issued
       bool ok = true;
       for (long long kt = blockIdx.x; kt < nkt && ok; kt += gridDim.x) {
         int e0;
@@ -711,13 +720,17 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const long long bh = kt / a.nb;
         const int h = static_cast<int>(bh % a.Hkv), b = static_cast<int>(bh / a.Hkv);
         const int32_t* rev = a.rev + bh * E;
-        if (tc_ > 0 && !waitb(W::bKvE, static_cast<uint32_t>((tc_ - 1) & 1))) { fail(kSiteKV); ok = false; break; }
+        const int kv = static_cast<int>(tc_ % W::NKV);
+        if (tc_ >= W::NKV &&
+            !waitb(W::bKvE + kv, static_cast<uint32_t>(((tc_ / W::NKV) - 1) & 1))) { fail(kSiteKV); ok = false; break; }
         const int row0 = static_cast<int>(static_cast<long long>(b) * a.S + static_cast<long long>(i) * BS);
-        mbar_expect_tx(BAR(W::bKvF), 2 * C::kTile);
+        const uint32_t sKb = sKV + kv * 2 * C::kTile, kvbar = BAR(W::bKvF + kv);
+        mbar_expect_tx(kvbar, 2 * C::kTile);
+        kv_issued = tc_ + 1;
 #pragma unroll
         for (int gg = 0; gg < D / 64; ++gg) {
-          tma_load_3d(sK + gg * C::kRegion, &tmK, BAR(W::bKvF), gg * 64, h, row0);
-          tma_load_3d(sV + gg * C::kRegion, &tmV, BAR(W::bKvF), gg * 64, h, row0);
+          tma_load_3d(sKb + gg * C::kRegion, &tmK, kvbar, gg * 64, h, row0);
+          tma_load_3d(sKb + C::kTile + gg * C::kRegion, &tmV, kvbar, gg * 64, h, row0);
         }
         for (int x = 0; x < ne; ++x, ++xg) {
           const int slot = static_cast<int>(xg % W::NE);
@@ -731,6 +744,9 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           const uint32_t bar = BAR(W::bEF + slot), dst = sE + slot * W::kSlot;
           const int q0 = static_cast<int>(static_cast<long long>(b) * a.S + static_cast<long long>(jq) * BS);
           const long long si0 = (static_cast<long long>(b) * a.Hq + hq) * a.S + static_cast<long long>(jq) * BS;
+          // The entry's query block, for the elementwise warps: published by
+          // the full barrier's arrive below.
+          *reinterpret_cast<volatile int*>(smem + W::oE + slot * W::kSlot + W::kHdr) = jq;
           mbar_expect_tx(bar, 2 * C::kTile + 2 * BS * 4);
 #pragma unroll
           for (int gg = 0; gg < D / 64; ++gg) {
@@ -744,7 +760,8 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       if (!ok) {
         // Wait (bounded) for the copies this thread issued and nobody consumed.
-        if (tc_ > 0) mbar_wait(BAR(W::bKvF), static_cast<uint32_t>(tc_ & 1), kBwWaitNs);
+        for (long long n = kv_issued - W::NKV > 0 ? kv_issued - W::NKV : 0; n < kv_issued; ++n)
+          mbar_wait(BAR(W::bKvF + static_cast<int>(n % W::NKV)), static_cast<uint32_t>((n / W::NKV) & 1), kBwWaitNs);
         for (long long n = xg - W::NE > 0 ? xg - W::NE : 0; n < xg; ++n)
           mbar_wait(BAR(W::bEF + static_cast<int>(n % W::NE)), static_cast<uint32_t>((n / W::NE) & 1), kBwWaitNs);
       }
@@ -774,11 +791,25 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         mma_commit(BAR(W::bEE + slot));
         return true;
       };
+      // The next tile's reverse-list offsets are read a tile ahead, so that
+      // their latency does not sit between two tiles' products.
+      auto offsets = [&](long long kt, int* lo, int* hi) {
+        if (kt >= nkt) { *lo = *hi = 0; return; }
+        const int32_t* roff = a.rev_off + (kt / a.nb) * (a.nb + 1) + kt % a.nb;
+        *lo = roff[0];
+        *hi = roff[1];
+      };
+      int nlo, nhi;
+      offsets(blockIdx.x, &nlo, &nhi);
       for (long long kt = blockIdx.x; kt < nkt && ok; kt += gridDim.x) {
-        int e0;
-        const int ne = entries(kt, &e0);
+        const int e0 = nlo, e1 = nhi;
+        offsets(kt + gridDim.x, &nlo, &nhi);
+        // The same range checks as entries(), which the other roles run.
+        const int ne = (e0 < 0 || e1 < e0 || e1 > E) ? 0 : e1 - e0;
         if (ne == 0) continue;
-        if (!waitb(W::bKvF, static_cast<uint32_t>(tc_ & 1))) { fail(kSiteKV); ok = false; break; }
+        const int kv = static_cast<int>(tc_ % W::NKV);
+        if (!waitb(W::bKvF + kv, static_cast<uint32_t>((tc_ / W::NKV) & 1))) { fail(kSiteKV); ok = false; break; }
+        const uint32_t sK = sKV + kv * 2 * C::kTile, sV = sK + C::kTile;
         for (int x = 0; x < ne; ++x, ++xg) {
           const int slot = static_cast<int>(xg % W::NE), sb = static_cast<int>(xg % W::NS);
           // With a single entry slot, entry x loads only once entry x-1's
@@ -804,7 +835,7 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (!ok) break;
         if (!acc(xg - 1, ne - 1)) { ok = false; break; }
         mma_commit(BAR(W::bAF));
-        mma_commit(BAR(W::bKvE));
+        mma_commit(BAR(W::bKvE + static_cast<int>(tc_ % W::NKV)));
         ++tc_;
       }
       // Everything this thread issued has completed once bFin fires.
@@ -834,14 +865,12 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
         continue;
       }
-      const int32_t* rev = a.rev + bh * E;
       for (int x = 0; x < ne; ++x, ++xg) {
         const int sb = static_cast<int>(xg % W::NS), slot = static_cast<int>(xg % W::NE);
         if (!wwait(W::bSF + sb, static_cast<uint32_t>((xg / W::NS) & 1))) { ok = false; break; }
         if (!wwait(W::bEF + slot, static_cast<uint32_t>((xg / W::NE) & 1))) { ok = false; break; }   // lse, Delta landed
         tc_fence_after();
-        const int code = rev[e0 + x];
-        const int jq = (code < 0 ? 0 : code) % a.nb;
+        const int jq = *reinterpret_cast<volatile const int*>(smem + W::oE + slot * W::kSlot + W::kHdr);
         const bool diag = jq == i;
         const float* lse_s = reinterpret_cast<const float*>(smem + W::oE + slot * W::kSlot + 2 * C::kTile);
         const float* del_s = lse_s + BS;
@@ -904,22 +933,39 @@ bwd_dkdv_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc_fence_after();
       const long long krow = (tok0 + R.r) * a.Hkv + h;
       const int s = i * BS + R.r;
+      if constexpr (C::NP == 1) {
+        // One part per thread: read both accumulators, hand them back to the
+        // MMA lane at once (the next tile's products may start), then store.
+        float vlo[C::W], vhi[C::W], klo[C::W], khi[C::W];
+        R.ld_d(tmem + W::colV, 0, 0, vlo);
+        R.ld_d(tmem + W::colV, 0, 1, vhi);
+        R.ld_d(tmem + W::colK, 0, 0, klo);
+        R.ld_d(tmem + W::colK, 0, 1, khi);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(W::bAE));
+        store_f32<C::W>(a.dv + krow * D + R.col_lo(0), vlo);
+        store_f32<C::W>(a.dv + krow * D + D / 2 + R.col_lo(0), vhi);
+        rotate_store<C::W, D>(klo, khi, R.col_lo(0), s, a.scale, ctl.om, a.dk + krow * D);
+      } else {
 #pragma unroll
-      for (int pp = 0; pp < C::NP; ++pp) {
-        float lo[C::W], hi[C::W];
-        R.ld_d(tmem + W::colV, pp, 0, lo);
-        R.ld_d(tmem + W::colV, pp, 1, hi);
-        tmem_ld_wait();
-        store_f32<C::W>(a.dv + krow * D + R.col_lo(pp), lo);
-        store_f32<C::W>(a.dv + krow * D + D / 2 + R.col_lo(pp), hi);
-        R.ld_d(tmem + W::colK, pp, 0, lo);
-        R.ld_d(tmem + W::colK, pp, 1, hi);
-        tmem_ld_wait();
-        rotate_store<C::W, D>(lo, hi, R.col_lo(pp), s, a.scale, ctl.om, a.dk + krow * D);
+        for (int pp = 0; pp < C::NP; ++pp) {
+          float lo[C::W], hi[C::W];
+          R.ld_d(tmem + W::colV, pp, 0, lo);
+          R.ld_d(tmem + W::colV, pp, 1, hi);
+          tmem_ld_wait();
+          store_f32<C::W>(a.dv + krow * D + R.col_lo(pp), lo);
+          store_f32<C::W>(a.dv + krow * D + D / 2 + R.col_lo(pp), hi);
+          R.ld_d(tmem + W::colK, pp, 0, lo);
+          R.ld_d(tmem + W::colK, pp, 1, hi);
+          tmem_ld_wait();
+          rotate_store<C::W, D>(lo, hi, R.col_lo(pp), s, a.scale, ctl.om, a.dk + krow * D);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(W::bAE));
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(W::bAE));
     }
     if (!ok && lane == 0) fail(kSiteS);
   }
