@@ -440,8 +440,9 @@ decode_route_kernel(const __grid_constant__ DecodeArgs a) {
 // output).  The last CTA of a (b, hq) to finish merges all blocks, in slot
 // order, into the output, reading every block's partial result in one
 // parallel round.
+// Five CTAs per SM (96 registers): more blocks' loads in flight per SM.
 template <typename T, int kLpr>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 5)
 decode_partial_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int kEpl = Row16<T>::kN;       // coordinates per lane
   constexpr int kRpi = 32 / kLpr;          // rows per warp load
