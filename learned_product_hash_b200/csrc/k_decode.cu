@@ -113,6 +113,23 @@ __device__ __forceinline__ float codeword_score(const float* xs, const float* co
   return v == v ? v : -INFINITY;
 }
 
+// The same score with the codeword row in shared memory (rows padded to
+// dsub + 4 words, so that 32 lanes reading 32 codewords hit distinct banks).
+__device__ __forceinline__ float codeword_score_s(const float* xs, const float* cw_row, int dsub) {
+  const float4* cw = reinterpret_cast<const float4*>(cw_row);
+  const float4* x4 = reinterpret_cast<const float4*>(xs);
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  for (int c = 0; c < dsub / 4; ++c) {
+    const float4 xv = x4[c], cv = cw[c];
+    a0 = __fmaf_rn(xv.x, cv.x, a0);
+    a1 = __fmaf_rn(xv.y, cv.y, a1);
+    a2 = __fmaf_rn(xv.z, cv.z, a2);
+    a3 = __fmaf_rn(xv.w, cv.w, a3);
+  }
+  const float v = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
+  return v == v ? v : -INFINITY;
+}
+
 }  // namespace
 
 template <typename T>
@@ -198,7 +215,7 @@ constexpr int kDecPAddr = kDecCode + 64;          // probed addresses [<= 64]
 constexpr int kDecOffs = kDecPAddr + 64;          // slot offsets [<= 65]
 constexpr int kDecCand = kDecOffs + 68;          // candidate ids [kMaxCand]
 constexpr int kDecKey = kDecCand + kMaxCand;      // candidate score keys [kMaxCand]
-constexpr int kDecWords = kDecKey + kMaxCand;
+constexpr int kDecWords = kDecKey + kMaxCand;    // then the codebooks [P][K][dsub + 4]
 
 template <typename T>
 __global__ void __launch_bounds__(kAttWarps * 32)
@@ -215,6 +232,18 @@ decode_route_kernel(const __grid_constant__ DecodeArgs a) {
   const size_t bh = static_cast<size_t>(b) * a.Hkv + h, bq = static_cast<size_t>(b) * a.Hq + hq;
   const int t = a.t, j = t / a.bs, D = a.D, half = D / 2, dsub = D / a.P;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // 0. the codebooks into shared memory (an input: no wait needed); the
+  // barrier after the rotation covers these stores too.
+  float* cbs = dsm + kDecWords;
+  {
+    const int dsub0 = D / a.P, RS = dsub0 + 4;
+    const float4* cb4 = reinterpret_cast<const float4*>(a.codebooks);
+    for (int i4 = tid; i4 < a.P * a.K * dsub0 / 4; i4 += kAttWarps * 32) {
+      const int i = 4 * i4, row = i / dsub0, d = i - row * dsub0;   // row = sdx * K + k
+      *reinterpret_cast<float4*>(cbs + row * RS + d) = cb4[i4];
+    }
+  }
 
   // 1. rotated query.
   const T* qt = static_cast<const T*>(a.q_t) + bq * D;
@@ -235,7 +264,7 @@ decode_route_kernel(const __grid_constant__ DecodeArgs a) {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int k = lane + 32 * m;
-      key[m] = k < a.K ? dec_ordered(codeword_score(qs + sdx * dsub, a.codebooks, sdx, k, a.K, dsub)) : 0u;
+      key[m] = k < a.K ? dec_ordered(codeword_score_s(qs + sdx * dsub, cbs + (sdx * a.K + k) * (dsub + 4), dsub)) : 0u;
     }
     for (int rnd = 0; rnd < a.probes; ++rnd) {
       uint32_t lk = key[0];
@@ -610,7 +639,7 @@ cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t st) {
   cudaError_t e = bf16 ? launch_pdl(decode_keys_kernel<__nv_bfloat16>, dim3(a.B * a.Hkv), dim3(kKeyThreads), 0, st, a)
                        : launch_pdl(decode_keys_kernel<float>, dim3(a.B * a.Hkv), dim3(kKeyThreads), 0, st, a);
   if (e != cudaSuccess) return e;
-  const size_t smem = static_cast<size_t>(kDecWords) * sizeof(float);
+  const size_t smem = (static_cast<size_t>(kDecWords) + static_cast<size_t>(a.K) * (a.D + 4 * a.P)) * sizeof(float);
   void (*k)(DecodeArgs) = bf16 ? decode_route_kernel<__nv_bfloat16> : decode_route_kernel<float>;
   if ((e = cached_allow_smem(reinterpret_cast<const void*>(k), static_cast<int>(smem))) != cudaSuccess) return e;
   if ((e = launch_pdl(k, dim3(a.B * a.Hq), dim3(kAttWarps * 32), smem, st, a)) != cudaSuccess) return e;
